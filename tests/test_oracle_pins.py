@@ -1,0 +1,358 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each test pins one oracle function to a library conversion, a closed form, a
+hand-worked example, brute force on tiny inputs, or a property the method's
+pages state (ScaleSweep summary sec. 2, Lemma 4.1 / 4.3; H-Scale summary
+sec. 3 and B).  No GPU needed.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def bf16(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.uint16).numpy()
+
+
+# ------------------------------------------------------------------ E4M3 table
+
+def test_e4m3_table_matches_torch_float8(orc):
+    """Codes 0..126 decode exactly as torch's float8_e4m3fn does (library)."""
+    tab = orc.e4m3_table()
+    ref = torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(tab, ref)
+
+
+def test_e4m3_table_shape_facts(orc):
+    """126 positive finite codes, strictly increasing, max 448, min 2^-9; 127 excluded."""
+    tab = orc.e4m3_table()
+    pos = tab[1:]
+    assert len(pos) == 126 and tab[0] == 0.0
+    assert np.all(np.diff(tab) > 0)
+    assert pos.max() == 448.0 and pos.min() == 2.0 ** -9
+    assert orc.e4m3_value(127) == -1.0 and orc.e4m3_value(-1) == -1.0
+    # octave identity for normal codes: code c+8 is exactly twice code c
+    for c in range(8, 119):
+        assert tab[c + 8] == 2 * tab[c]
+
+
+def test_e4m3_nearest_matches_torch_rne(orc):
+    """Round-to-nearest-even to E4M3 agrees with torch's float8_e4m3fn cast
+    on random floats and on every midpoint (+-1 ulp) below the overflow point."""
+    rng = np.random.default_rng(0)
+    tab = orc.e4m3_table()
+    mids = (tab[:-1] + tab[1:]) / 2
+    vals = [np.float32(m) for m in mids]
+    vals += [np.nextafter(np.float32(m), np.float32(0)) for m in mids]
+    vals += [np.nextafter(np.float32(m), np.float32(1e9)) for m in mids]
+    vals += list(np.float32(np.exp(rng.uniform(math.log(1e-4), math.log(460), 4000))))
+    vals += list(tab.astype(np.float32))
+    vals = np.array(vals, dtype=np.float32)
+    vals = vals[vals < 464.0]          # torch turns >= 464 into NaN (no saturation)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy().astype(int)
+    got = np.array([orc.e4m3_nearest(float(v)) for v in vals])
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_e4m3_nearest_saturates(orc):
+    for v in [448.0, 463.99, 464.0, 1000.0, 3.0e38]:
+        assert orc.e4m3_nearest(v) == 126
+    assert orc.e4m3_nearest(0.0) == 0
+    assert orc.e4m3_nearest(2.0 ** -10) == 0          # tie 0 / 2^-9: even code 0
+    assert orc.e4m3_nearest(float("nan")) == -1
+
+
+# ------------------------------------------------------------------- E2M1 RNE
+
+@pytest.mark.parametrize("vS", [1.0, 0.375, 3.0e-3])
+def test_e2m1_midpoints_ties_to_even(orc, vS):
+    """Textbook RNE on the grid {0,.5,1,1.5,2,3,4,6}: an exact midpoint goes to
+    the even index, one ulp either side goes to the nearer point."""
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    for i, m in enumerate(mids):
+        t = m * vS
+        even = i if i % 2 == 0 else i + 1
+        assert orc.e2m1_index(t, vS) == even, (m, vS)
+        assert orc.e2m1_index(np.nextafter(t, 0.0), vS) == i
+        assert orc.e2m1_index(np.nextafter(t, 1e30), vS) == i + 1
+    # saturation: 7 is the tie 6|8 -> 8 -> saturates to 6 (index 7); far above too
+    assert orc.e2m1_index(7.0 * vS, vS) == 7
+    assert orc.e2m1_index(1e6 * vS, vS) == 7
+    assert orc.e2m1_index(0.0, vS) == 0
+
+
+def test_e2m1_index_brute_force_nearest(orc):
+    """Against a brute-force nearest-grid search (argmin over the 8 values)."""
+    rng = np.random.default_rng(1)
+    g = np.array(GRID)
+    for _ in range(3000):
+        vS = float(np.float32(rng.uniform(0.01, 10)))
+        a = float(np.float32(rng.uniform(0, 8)) * vS)
+        x = a / vS
+        d = np.abs(x - g)
+        k = int(np.argmin(d))
+        if np.sort(d)[1] - d[k] < 1e-9:   # too close to a midpoint for the float check
+            continue
+        assert orc.e2m1_index(a, vS) == k
+
+
+# ----------------------------------------------------------- objective, loss
+
+def test_group_loss_hand_example(orc):
+    """S = 1, code 56 (value 1.0), h = [1,2,3,4,0,...]:
+    |w| = 3/16 -> 0 (err 3/16); 19/16 -> 1 (err 3/16); 21/8 -> 3 (err 3/8);
+    7 -> tie 6|8 -> 8 -> saturated 6 (err 1).  L = 9/256 + 18/256 + 27/64 + 4."""
+    w = bf16([0.1875, -1.1875, 2.625, 7.0] + [0.0] * 12)
+    h = np.array([1, 2, 3, 4] + [0] * 12, np.float32)
+    assert orc.e4m3_value(56) == 1.0
+    L = orc.group_loss(w, h, 1.0, 56)
+    assert L == 9 / 256 + 18 / 256 + 27 / 64 + 4.0 == 4.52734375
+
+
+def test_group_loss_zero_for_grid_values(orc):
+    """Weights exactly on the grid at scale v*S reconstruct with zero loss."""
+    S = float(np.float32(0.0078125))
+    v = orc.e4m3_value(60)   # 1.5
+    w = bf16([g * v * S * s for g in GRID for s in (1, -1)])
+    assert orc.group_loss(w, None, S, 60) == 0.0
+
+
+def test_group_loss_weighting_is_linear(orc):
+    """Doubling h doubles the loss; h == 1 equals h == NULL (plain MSE)."""
+    rng = np.random.default_rng(2)
+    w = bf16(rng.normal(0, 1, 16))
+    h = np.float32(rng.uniform(0.1, 3, 16))
+    for code in (40, 56, 77):
+        a = orc.group_loss(w, h, 0.01, code)
+        assert orc.group_loss(w, 2 * h, 0.01, code) == 2 * a
+        assert orc.group_loss(w, np.ones(16, np.float32), 0.01, code) == orc.group_loss(w, None, 0.01, code)
+
+
+# ------------------------------------------------------------ diag Hessian
+
+def test_diag_hessian_closed_forms(orc):
+    T, n = 37, 48
+    ones = torch.ones(T, n, dtype=torch.bfloat16)
+    np.testing.assert_array_equal(orc.diag_hessian(ones), np.full(n, T, np.float32))
+    X = torch.zeros(T, n, dtype=torch.bfloat16)
+    row = torch.linspace(-3, 3, n).to(torch.bfloat16)
+    X[5] = row
+    np.testing.assert_array_equal(orc.diag_hessian(X), (row.float() ** 2).numpy())
+    empty = torch.zeros(0, n, dtype=torch.bfloat16)
+    np.testing.assert_array_equal(orc.diag_hessian(empty), np.zeros(n, np.float32))
+    h0 = np.arange(n, dtype=np.float32)
+    np.testing.assert_array_equal(orc.diag_hessian(empty, h0, accumulate=True), h0)
+    np.testing.assert_array_equal(orc.diag_hessian(ones, h0, accumulate=True), h0 + T)
+
+
+def test_diag_hessian_matches_numpy(orc):
+    X = (torch.randn(300, 64, generator=torch.Generator().manual_seed(3)) * 5).to(torch.bfloat16)
+    ref = (X.double().numpy() ** 2).sum(0).astype(np.float32)
+    np.testing.assert_allclose(orc.diag_hessian(X), ref, rtol=1e-7)
+    np.testing.assert_array_equal(orc.parallel_diag_hessian(X, threads=3), orc.diag_hessian(X))
+
+
+# ------------------------------------------------------------- global scale
+
+def test_global_scale_closed_form(orc):
+    W = torch.zeros(8, 32, dtype=torch.bfloat16)
+    W[3, 7] = -5.25
+    W[6, 1] = 2.0
+    S, am, st = orc.global_scale(W, 448.0)
+    assert st == 0 and am == np.float32(5.25)
+    assert S == np.float32(5.25) / np.float32(2688.0)
+    S, am, st = orc.global_scale(W, 256.0)
+    assert S == np.float32(5.25) / np.float32(1536.0)
+    S, am, st = orc.global_scale(torch.zeros(4, 16, dtype=torch.bfloat16))
+    assert S == 0.0 and am == 0.0 and st == 0
+    W[0, 0] = float("inf")
+    assert orc.global_scale(W)[2] == -5
+    W[0, 0] = float("nan")
+    assert orc.global_scale(W)[2] == -5
+
+
+# ------------------------------------------------------------------- sweep
+
+def test_sweep_hand_example_ties_to_lowest_offset(orc):
+    """All |w| = 6, S = 1: base code 56 (v = 1) reconstructs exactly, and so does
+    code 60 (v = 1.5, x = 4).  The tie goes to the lower offset: code 56,
+    offset 0.  Every element has index 7 (value 6); signs alternate."""
+    w = bf16([6.0, -6.0] * 8)
+    codes, scales, offs, loss = orc.sweep_groups(w, None, 1.0, -9, 6)
+    assert scales[0] == 56 and offs[0] == 0 and loss[0] == 0.0
+    assert list(codes[0]) == [0xF7] * 8
+
+
+def test_sweep_pack_layout_hand_example(orc):
+    """Window [0,0] keeps the base code.  w = [6, -3, 0.5, -0.0, 1.75, 2.5, ...],
+    S = 1 -> b = 56 (v = 1); indices 7, 5(neg), 1, 0, 4 (1.75 ties up to 2),
+    4 (2.5 ties down to 2), rest 0.  Low nibble = even element."""
+    w = bf16([6.0, -3.0, 0.5, -0.0, 1.75, 2.5] + [0.0] * 10)
+    codes, scales, offs, _ = orc.sweep_groups(w, None, 1.0, 0, 0)
+    assert scales[0] == 56
+    assert list(codes[0]) == [0xD7, 0x01, 0x44, 0, 0, 0, 0, 0]
+
+
+def test_sweep_zero_groups(orc):
+    W = torch.zeros(4, 64, dtype=torch.bfloat16)
+    W[1, 20] = 0.5
+    W[2, :16] = -0.0
+    codes, scales, offs = orc.sweep_quantize(W, None, 0.5 / 2688, -9, 6)
+    assert scales[0].tolist() == [0, 0, 0, 0] and scales[2].tolist() == [0, 0, 0, 0]
+    assert scales[1].tolist()[1] == 126 and scales[1].tolist()[0] == 0
+    assert not codes[0].any() and not codes[2].any() and not codes[3].any()
+    # output size: 4.5 bits per value (codes + one E4M3 byte per 16)
+    assert codes.nbytes + scales.nbytes == W.numel() * (0.5 + 1 / 16)
+
+
+def _random_groups(n, seed):
+    """Mixed group shapes: Gaussian, heavy outliers, near-constant, tiny, sparse."""
+    rng = np.random.default_rng(seed)
+    w = rng.normal(0, 1, (n, 16))
+    kind = rng.integers(0, 5, n)
+    w[kind == 1] *= np.where(rng.random((np.sum(kind == 1), 16)) < 0.1, 10, 1)
+    w[kind == 2] = rng.normal(3, 0.01, (np.sum(kind == 2), 16))
+    w[kind == 3] *= 1e-3
+    w[kind == 4] *= rng.random((np.sum(kind == 4), 16)) < 0.3
+    w *= np.exp(rng.normal(0, 1, (n, 1)))
+    return bf16(w.reshape(-1)).reshape(n, 16)
+
+
+def _all_code_losses(orc, w, h, S):
+    n = w.shape[0]
+    L = np.empty((n, 127))
+    for c in range(127):
+        L[:, c] = orc.group_losses(w, h, S, np.full(n, c, np.uint8))
+    return L
+
+
+def test_window_contains_global_mse_optimum(orc):
+    """ScaleSweep Lemma 4.1 / 4.3: for plain MSE with S = amax/(256*6), the
+    window [-3,+7] around the FP8-rounded max-abs code contains a global optimum
+    over all 126 positive codes.  Compare losses (ties may pick other codes)."""
+    w = _random_groups(20000, 4)
+    amax = np.abs(w.view(np.uint16).astype(np.uint32) << 16).view(np.float32).max()
+    S = float(np.float32(amax) / np.float32(1536.0))
+    _, _, _, lw = orc.sweep_groups(w, None, S, -3, 7)
+    L = _all_code_losses(orc, w, None, S)[:, 1:]
+    base = np.array([orc.base_code(w[i], S) for i in range(len(w))])
+    # The lemmas speak of ratios of scales; "+7 / -3 codes" equals those ratios
+    # only where the codes are normal (exponent field > 0, base code >= 8).  In
+    # the subnormal range the codes are evenly spaced and the window can miss
+    # the optimum (a finding, kept visible below rather than patched).
+    normal = base >= 8
+    assert normal.sum() > 10000
+    assert np.all(lw[normal] == L[normal].min(axis=1))
+    miss = np.flatnonzero(lw != L.min(axis=1))
+    assert np.all(base[miss] < 8)
+
+
+def test_upper_bound_lemma_any_weights(orc):
+    """Lemma 4.1 (a scale above 12/7 s_base never beats half of it; the argument
+    is per element, so it holds for any non-negative weights): with a window up
+    to +15 the chosen offset never exceeds +7, for MSE and for WMSE."""
+    w = _random_groups(5000, 5)
+    rng = np.random.default_rng(6)
+    h = np.float32(np.exp(rng.normal(0, 2, w.shape)))
+    for hh in (None, h):
+        _, _, offs, _ = orc.sweep_groups(w, hh, 1e-3, -16, 15)
+        assert offs.max() <= 7
+
+
+def test_sweep_brute_force_small(orc):
+    """Brute force: evaluate every code in the clamped window with a separate
+    nearest-grid search in numpy (argmin over the 8 grid values) and keep the
+    first strict minimum in offset order; the oracle must pick the same code."""
+    rng = np.random.default_rng(7)
+    w = _random_groups(400, 8)
+    h = np.float32(np.exp(rng.normal(0, 1.5, w.shape)))
+    S = float(np.float32(2.5e-3))     # the global scale is an FP32 number
+    tab = orc.e4m3_table()
+    codes, scales, offs, _ = orc.sweep_groups(w, h, S, -9, 6)
+    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    g = np.array(GRID)
+    for i in range(w.shape[0]):
+        a = np.abs(wf[i])
+        if a.max() == 0:
+            assert scales[i] == 0
+            continue
+        u = np.float32(np.float32(a.max()) / np.float32(6.0)) / np.float32(S)
+        d = np.abs(tab - float(u))
+        near = np.flatnonzero(d == d.min())          # one code, or two on a tie
+        b = int(near[0] if len(near) == 1 or near[0] % 2 == 0 else near[1])
+        b = min(max(b, 1), 126)
+        best, bc = np.inf, None
+        for k in range(-9, 7):
+            c = min(max(b + k, 1), 126)
+            vS = tab[c] * S
+            q = g[np.argmin(np.abs(a[:, None] / vS - g[None, :]), axis=1)]
+            L = float(np.sum(h[i].astype(np.float64) * (a - q * vS) ** 2))
+            if L < best:
+                best, bc = L, c
+        assert scales[i] == bc, i
+
+
+def test_sweep_never_worse_than_base(orc):
+    """The base (offset 0) is in every window, so the chosen loss never exceeds
+    the max-abs (Min-Max) initialisation's loss under the same objective."""
+    w = _random_groups(5000, 9)
+    rng = np.random.default_rng(10)
+    h = np.float32(np.exp(rng.normal(0, 1, w.shape)))
+    S = 1e-3
+    for hh, (lo, hi) in ((None, (-3, 7)), (h, (-8, 7)), (h, (-9, 6))):
+        _, scales, _, loss = orc.sweep_groups(w, hh, S, lo, hi)
+        base = np.array([orc.base_code(w[i], S) for i in range(len(w))], np.uint8)
+        lb = orc.group_losses(w, hh, S, base)
+        assert np.all(loss <= lb)
+        np.testing.assert_array_equal(orc.group_losses(w, hh, S, scales), loss)
+
+
+def test_sweep_unit_h_equals_mse(orc):
+    W = torch.from_numpy(_random_groups(64, 11).view(np.int16)).view(torch.bfloat16).reshape(16, 64)
+    a = orc.sweep_quantize(W, None, 3e-3, -9, 6)
+    b = orc.sweep_quantize(W, np.ones(64, np.float32), 3e-3, -9, 6)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    c = orc.parallel_sweep_quantize(W, np.ones(64, np.float32), 3e-3, -9, 6, threads=4)
+    for x, y in zip(a, c):
+        np.testing.assert_array_equal(x, y)
+
+
+# --------------------------------------------------------------- dequantize
+
+def test_dequantize_closed_form(orc):
+    codes = np.array([[0xD7, 0x01, 0x44, 0, 0, 0, 0, 0]], np.uint8)
+    scales = np.array([[56]], np.uint8)
+    out = orc.dequantize(codes, scales, 0.5)
+    exp = np.array([6, -3, 0.5, 0, 2, 2] + [0] * 10, np.float32) * 0.5
+    np.testing.assert_array_equal(out[0], exp)
+    out = orc.dequantize(codes, np.array([[0]], np.uint8), 0.5)
+    assert not out.any()
+
+
+def test_dequantize_round_trip_never_worse_than_base_rtn(orc):
+    """dequantize(quantize(W)) has a weighted error no larger than max-abs RTN
+    (window [0,0]) under the same objective, up to the float rounding of the
+    dequantized values; every unsaturated element sits within half a grid step
+    of its reconstruction."""
+    rng = np.random.default_rng(12)
+    w = _random_groups(256, 12)
+    W = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).reshape(16, 256)
+    h = np.float32(np.exp(rng.normal(0, 1, 256)))
+    S = float(np.float32(2e-3))
+    Wf = W.double().numpy()
+    errs = []
+    for lo, hi in ((-9, 6), (0, 0)):
+        codes, scales, _ = orc.sweep_quantize(W, h, S, lo, hi)
+        Wq = orc.dequantize(codes, scales, S).astype(np.float64)
+        errs.append(((Wf - Wq) ** 2 * h.astype(np.float64)).reshape(16, 16, 16).sum(-1))
+        step = np.repeat(orc.e4m3_table()[scales], 16, axis=1) * S
+        a = np.abs(Wf)
+        unsat = a <= 6 * step
+        half = np.where(a < 2 * step, 0.25, np.where(a < 4 * step, 0.5, 1.0)) * step
+        assert np.all(np.abs(Wf - Wq)[unsat] <= half[unsat] * (1 + 1e-6) + 1e-30)
+    assert np.all(errs[0] <= errs[1] * (1 + 1e-5) + 1e-30)
