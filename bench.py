@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Benchmark: Hessian-weighted NVFP4 block-scale selection on B200.
+
+One step = the whole hot path over one synthetic 70B-shaped MLP layer
+(gate/up 28672x8192, down 8192x28672 bf16; calibration X of 65536 tokens per
+input site): diagonal Hessian of both X, global scale of the three weights,
+windowed [-9,+6] h-weighted scale sweep + pack of the three weights.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+N > 1 runs under torchrun, one rank per GPU: every rank quantizes its own
+layer (different seeds), there is no data-path collective, and the step time
+is the max over ranks (weak scaling).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 weight elems/s quantized + calib GB/s (diag-H), % of B200 HBM roofline"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+LO, HI = -9, 6
+SWEEP_BYTES_PER_ELEM = 2 + 0.5 + 1 / 16   # read bf16 W; write 4-bit code + 1/16 E4M3 byte
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured", d
+    return FALLBACK_HBM_GBS, "fallback", {}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- workload
+
+def build_layer(rank: int, device):
+    import torch
+    import workloads
+    wl = workloads.llama33_70b_mlp(seed_offset=rank)
+    Ws = {m.name: m.make(device) for m in wl.matrices}
+    Xs = {k: c.make(device) for k, c in wl.calibs.items()}
+    torch.cuda.synchronize()
+    return wl, Ws, Xs
+
+
+class Step:
+    """Preallocated buffers + one pass of the hot path through the C ABI."""
+
+    def __init__(self, nv, wl, Ws, Xs, device):
+        import torch
+        self.nv, self.wl, self.Ws, self.Xs = nv, wl, Ws, Xs
+        self.h = {k: torch.empty(X.shape[1], dtype=torch.float32, device=device) for k, X in Xs.items()}
+        self.hws = {k: torch.empty(nv.nvfp4_diag_hessian_workspace_size(*X.shape), dtype=torch.uint8,
+                                   device=device) for k, X in Xs.items()}
+        self.S = {n: torch.empty(1, dtype=torch.float32, device=device) for n in Ws}
+        self.amax = {n: torch.empty(1, dtype=torch.float32, device=device) for n in Ws}
+        self.status = {n: torch.empty(1, dtype=torch.int32, device=device) for n in Ws}
+        self.gws = {n: torch.empty(max(16, nv.nvfp4_global_scale_workspace_size(*W.shape)),
+                                   dtype=torch.uint8, device=device) for n, W in Ws.items()}
+        self.codes = {n: torch.empty(W.shape[0], W.shape[1] // 2, dtype=torch.uint8, device=device)
+                      for n, W in Ws.items()}
+        self.scales = {n: torch.empty(W.shape[0], W.shape[1] // 16, dtype=torch.uint8, device=device)
+                       for n, W in Ws.items()}
+        self.x_of = {m.name: m.x_key for m in wl.matrices}
+        self.launches_per_step = 2 * len(Xs) + 2 * len(Ws) + len(Ws)
+
+    def run(self, ev=None):
+        """ev: optional dict kind -> list of (start, end) event pairs to record."""
+        import torch
+        nv = self.nv
+        stream = torch.cuda.current_stream()
+
+        def rec(kind, fn):
+            if ev is None:
+                fn()
+                return
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev.setdefault(kind, []).append((a, b))
+
+        for k, X in self.Xs.items():
+            ws = self.hws[k]
+            rec("diag_hessian", lambda X=X, k=k, ws=ws: nv.nvfp4_diag_hessian(
+                X, X.shape[0], X.shape[1], X.stride(0), self.h[k], 0, ws, ws.numel(), stream))
+        for n, W in self.Ws.items():
+            ws = self.gws[n]
+            rec("global_scale", lambda W=W, n=n, ws=ws: nv.nvfp4_global_scale(
+                W, W.shape[0], W.shape[1], W.stride(0), self.wl.q_max, self.S[n], self.amax[n],
+                self.status[n], ws, ws.numel(), stream))
+        for n, W in self.Ws.items():
+            rec("scale_sweep", lambda W=W, n=n: nv.nvfp4_scale_sweep_quantize(
+                W, W.shape[0], W.shape[1], W.stride(0), self.h[self.x_of[n]], self.S[n], LO, HI,
+                self.codes[n], self.scales[n], None, stream))
+
+
+def kernel_bytes(wl):
+    wel = wl.weight_elems
+    return {"diag_hessian": wl.calib_bytes + 4 * sum(c.inp for c in wl.calibs.values()),
+            "global_scale": 2 * wel,
+            "scale_sweep": SWEEP_BYTES_PER_ELEM * wel}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_sample_rate(wl, Ws, Xs, threads=None, budget_rows=None):
+    """Time the CPU oracle on a bounded sample of this workload and extrapolate
+    to whole-job weight elements per second.  Returns (rate, info)."""
+    import numpy as np
+    import torch
+    import oracle
+    threads = threads or oracle.default_threads()
+    rows = budget_rows or {"gate": 192, "up": 192, "down": 64}
+    t_sweep = t_abs = t_h = 0.0
+    el_sweep = el_abs = 0
+    xel = 0
+    hs = {}
+    for k, X in Xs.items():
+        n_tok = 256
+        sub = X[:n_tok].cpu()
+        t0 = time.perf_counter()
+        hs[k] = oracle.parallel_diag_hessian(sub, threads=threads)
+        t_h += time.perf_counter() - t0
+        xel += sub.numel()
+    for m in wl.matrices:
+        W = Ws[m.name]
+        r = rows.get(m.name, 64)
+        sub = W[:r].cpu().view(torch.uint16).numpy()
+        t0 = time.perf_counter()
+        S, _, _ = oracle.global_scale(sub, wl.q_max)
+        t_abs += time.perf_counter() - t0
+        el_abs += sub.size
+        h = hs[m.x_key]
+        t0 = time.perf_counter()
+        oracle.parallel_sweep_quantize(sub, h, float(S) if S > 0 else 1e-3, LO, HI, threads=threads)
+        t_sweep += time.perf_counter() - t0
+        el_sweep += sub.size
+    wel = wl.weight_elems
+    x_total = sum(c.tokens * c.inp for c in wl.calibs.values())
+    t_full = t_sweep * wel / el_sweep + t_abs * wel / el_abs + t_h * x_total / xel
+    info = {"sample": (f"oracle on {el_sweep} of {wel} weight elements "
+                       f"(rows {rows}) and 256 of {wl.calibs['gu'].tokens} tokens per X; "
+                       f"extrapolated linearly to the full layer"),
+            "cores": threads, "t_sample_s": round(t_sweep + t_abs + t_h, 3),
+            "t_full_est_s": round(t_full, 2)}
+    return wel / t_full, info
+
+
+# ------------------------------------------------------------------ main
+
+def init_dist():
+    import torch
+    import torch.distributed as dist
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local}"))
+    return rank, local, ws
+
+
+def barrier(ws):
+    import torch
+    import torch.distributed as dist
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    import torch
+    import torch.distributed as dist
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, per-step bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    dev = "cuda:0" if torch.cuda.is_available() else "cpu"
+    wl, Ws, Xs = build_layer(0, dev)
+    for _ in range(args.warmup):
+        oracle_sample_rate(wl, Ws, Xs, budget_rows={"gate": 16, "up": 16, "down": 8})
+    rates, info = [], None
+    for _ in range(args.steps):
+        r, info = oracle_sample_rate(wl, Ws, Xs, budget_rows={"gate": 64, "up": 64, "down": 16})
+        rates.append(r)
+    v = statistics.median(rates)
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "elem/s",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic",
+           "config": {"workload": "llama33_70b_mlp gate/up 28672x8192, down 8192x28672; "
+                                  "X 65536 tokens; window [-9,+6]; Q=448",
+                      "impl": "CPU oracle (plain C, fp64), sampled and extrapolated"},
+           "cpu_baseline": {"value": v, "unit": "elem/s", "cores": info["cores"], "kind": "oracle",
+                            "sample": info["sample"]},
+           "e2e": {"value": v, "unit": "elem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import block_scale_search_b200 as nv
+    nv.lib()  # fails loudly if the CUDA library is missing
+    rank, local, ws = init_dist()
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    wl, Ws, Xs = build_layer(rank, dev)
+    step = Step(nv, wl, Ws, Xs, dev)
+
+    for _ in range(args.warmup):
+        step.run()
+    barrier(ws)
+
+    # ---- device-resident timed region (events on the launch stream)
+    stream = torch.cuda.current_stream()
+    ev = {}
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(ws)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step.run(ev)
+    t1.record(stream)
+    barrier(ws)
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    ms_max = max_over_ranks(ms, ws)
+
+    kern = {}
+    kb = kernel_bytes(wl)
+    peak, peak_kind, peaks = measured_peaks()
+    for kind, pairs in ev.items():
+        tot = sum(a.elapsed_time(b) for a, b in pairs) / args.steps   # ms per step
+        gbs = kb[kind] / (tot * 1e-3) / 1e9
+        kern[kind] = {"ms_per_step": round(tot, 4), "launch_pairs_per_step": len(pairs) // args.steps,
+                      "algorithmic_bytes_per_step": int(kb[kind]), "gbs": round(gbs, 1),
+                      f"frac_of_{peak_kind}": round(gbs / peak, 4),
+                      "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)}
+    wel = wl.weight_elems
+    value = wel * ws / (ms_max * 1e-3)
+
+    # ---- status of the quantized tensors (non-finite check) and sanity
+    for n in Ws:
+        assert int(step.status[n].item()) == 0, f"non-finite weights in {n}"
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hostW = {n: W.cpu().pin_memory() for n, W in Ws.items()}
+        hostX = {k: X.cpu().pin_memory() for k, X in Xs.items()}
+        hostC = {n: torch.empty_like(c, device="cpu").pin_memory() for n, c in step.codes.items()}
+        hostS = {n: torch.empty_like(s, device="cpu").pin_memory() for n, s in step.scales.items()}
+
+        def e2e_step():
+            for k in Xs:
+                Xs[k].copy_(hostX[k], non_blocking=True)
+            for n in Ws:
+                Ws[n].copy_(hostW[n], non_blocking=True)
+            step.run()
+            for n in Ws:
+                hostC[n].copy_(step.codes[n], non_blocking=True)
+                hostS[n].copy_(step.scales[n], non_blocking=True)
+
+        e2e_step()
+        barrier(ws)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        barrier(ws)
+        e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, ws)
+        h2d = sum(t.numel() * t.element_size() for t in list(hostW.values()) + list(hostX.values()))
+        d2h = sum(t.numel() for t in list(hostC.values()) + list(hostS.values()))
+        e2e = {"value": wel * ws / (e_ms * 1e-3), "unit": "elem/s", "ms_per_step": round(e_ms, 3),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps}
+        del hostW, hostX
+
+    # ---- roofline of the dominant kernel
+    dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
+    per_launch_ms = kern[dom]["ms_per_step"] / kern[dom]["launch_pairs_per_step"]
+    achieved = kb[dom] / kern[dom]["launch_pairs_per_step"] / (per_launch_ms * 1e-3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS copy)", "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                "traffic": None}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rate, info = oracle_sample_rate(wl, Ws, Xs)
+        cpu = {"value": rate, "unit": "elem/s", "cores": info["cores"], "kind": "oracle",
+               "sample": info["sample"], "t_full_est_s": info["t_full_est_s"]}
+
+    if rank == 0:
+        xbytes = wl.calib_bytes
+        out = {
+            "metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "llama33_70b_mlp: gate/up 28672x8192, down 8192x28672 bf16 "
+                                   "N(0,0.015) 0.1% x10 outliers; X 65536 tokens x {8192, 28672} "
+                                   "bf16 lognormal(1.5) channel scales",
+                       "window": [LO, HI], "q_max": wl.q_max, "weighted": True,
+                       "l2": "inputs 6.2 GB per rank > 126 MB L2; no flush",
+                       "parallelism": f"weak: {ws} rank(s), one independent layer per rank"},
+            "calib_gbs": round(xbytes / (kern["diag_hessian"]["ms_per_step"] * 1e-3) / 1e9, 1),
+            "quantize_elems_per_s": wel / ((kern["global_scale"]["ms_per_step"] +
+                                            kern["scale_sweep"]["ms_per_step"]) * 1e-3),
+            "kernels": kern, "roofline": roofline, "e2e": e2e,
+            "gpu_launches": step.launches_per_step * args.steps,
+            "cpu_baseline": cpu, "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

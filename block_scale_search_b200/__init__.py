@@ -1,0 +1,210 @@
+"""Python binding of libnvfp4hs (Hessian-weighted NVFP4 block-scale selection).
+
+Argument marshalling only: every step runs in the CUDA kernels behind the C
+ABI declared in ``include/nvfp4hs.h``.  PyTorch provides device memory and the
+current stream.  The ``nvfp4_*`` functions mirror the C entry points one to
+one; the lower-case helpers below them allocate outputs and workspaces with
+torch and call those entry points.  There is no CPU fallback: if the shared
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+import torch
+
+from . import _build
+
+__all__ = [
+    "NVFP4Error", "lib", "nvfp4_version", "nvfp4_diag_hessian_workspace_size",
+    "nvfp4_diag_hessian", "nvfp4_global_scale_workspace_size", "nvfp4_global_scale",
+    "nvfp4_scale_sweep_quantize", "nvfp4_dequantize",
+    "diag_hessian", "global_scale", "scale_sweep_quantize", "dequantize", "quantize_layer",
+]
+
+STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_INVALID_ARG", -2: "NVFP4_ERR_SHAPE",
+          -3: "NVFP4_ERR_ALIGN", -4: "NVFP4_ERR_WINDOW", -5: "NVFP4_ERR_NONFINITE",
+          -6: "NVFP4_ERR_CUDA", -7: "NVFP4_ERR_WORKSPACE"}
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, fn: str, status: int, cuda_error: int = 0):
+        self.status = status
+        msg = f"{fn} returned {status} ({STATUS.get(status, '?')})"
+        if status == -6:
+            msg += f", cudaError {cuda_error}"
+        super().__init__(msg)
+
+
+_lock = threading.Lock()
+_lib = None
+LIB_PATH = _build.LIB
+
+_vp, _i64, _sz, _int, _f32 = C.c_void_p, C.c_int64, C.c_size_t, C.c_int, C.c_float
+_SIGS = {
+    "nvfp4_version": ([], _int),
+    "nvfp4_last_cuda_error": ([], _int),
+    "nvfp4_diag_hessian_workspace_size": ([_i64, _i64], _sz),
+    "nvfp4_diag_hessian": ([_vp, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp], _int),
+    "nvfp4_global_scale_workspace_size": ([_i64, _i64], _sz),
+    "nvfp4_global_scale": ([_vp, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _vp, _sz, _vp], _int),
+    "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
+                                    _vp], _int),
+    "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
+}
+
+
+def lib(path: str | None = None):
+    """Load the shared library (built in-tree by ``__graft_entry__.build()``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            p = path or LIB_PATH
+            if not os.path.exists(p):
+                raise ImportError(f"libnvfp4hs.so not built at {p}; run __graft_entry__.build()")
+            L = C.CDLL(p)
+            for name, (args, res) in _SIGS.items():
+                fn = getattr(L, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = L
+    return _lib
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise NVFP4Error(fn, st, lib().nvfp4_last_cuda_error() if st == -6 else 0)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+# ------------------------------------------------------------- raw C mirrors
+# Same names and argument order as the C entry points; tensors (or None) stand
+# in for pointers, and `stream` defaults to torch's current stream.
+
+def nvfp4_version() -> int:
+    return lib().nvfp4_version()
+
+
+def nvfp4_diag_hessian_workspace_size(tokens: int, inp: int) -> int:
+    return lib().nvfp4_diag_hessian_workspace_size(tokens, inp)
+
+
+def nvfp4_diag_hessian(X, tokens, inp, ldx, h, accumulate, workspace, workspace_bytes, stream=None):
+    _check("nvfp4_diag_hessian", lib().nvfp4_diag_hessian(
+        _ptr(X), tokens, inp, ldx, _ptr(h), int(accumulate), _ptr(workspace), workspace_bytes,
+        _stream(stream)))
+
+
+def nvfp4_global_scale_workspace_size(out: int, inp: int) -> int:
+    return lib().nvfp4_global_scale_workspace_size(out, inp)
+
+
+def nvfp4_global_scale(W, out, inp, ldw, q_max, S, amax, status, workspace, workspace_bytes,
+                       stream=None):
+    _check("nvfp4_global_scale", lib().nvfp4_global_scale(
+        _ptr(W), out, inp, ldw, float(q_max), _ptr(S), _ptr(amax), _ptr(status), _ptr(workspace),
+        workspace_bytes, _stream(stream)))
+
+
+def nvfp4_scale_sweep_quantize(W, out, inp, ldw, h, S, lo, hi, codes, scales, chosen_offset,
+                               stream=None):
+    _check("nvfp4_scale_sweep_quantize", lib().nvfp4_scale_sweep_quantize(
+        _ptr(W), out, inp, ldw, _ptr(h), _ptr(S), int(lo), int(hi), _ptr(codes), _ptr(scales),
+        _ptr(chosen_offset), _stream(stream)))
+
+
+def nvfp4_dequantize(codes, scales, S, out, inp, W_out, stream=None):
+    _check("nvfp4_dequantize", lib().nvfp4_dequantize(
+        _ptr(codes), _ptr(scales), _ptr(S), out, inp, _ptr(W_out), _stream(stream)))
+
+
+# -------------------------------------------------------- tensor conveniences
+
+def _bf16_2d(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_cuda:
+        raise ValueError(f"{name} must be a 2-D bf16 CUDA tensor")
+    if t.stride(1) != 1:
+        raise ValueError(f"{name} must have unit stride along its last dimension")
+    return t
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def diag_hessian(X: torch.Tensor, h: torch.Tensor | None = None, accumulate: bool = False,
+                 workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """h[in] (+)= sum_t X[t, :]^2 (float32)."""
+    X = _bf16_2d(X, "X")
+    T, n = X.shape
+    if h is None:
+        h = torch.empty(n, dtype=torch.float32, device=X.device)
+    nb = nvfp4_diag_hessian_workspace_size(T, n)
+    if nb == 0:
+        raise NVFP4Error("nvfp4_diag_hessian_workspace_size", -1)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, X.device)
+    nvfp4_diag_hessian(X, T, n, X.stride(0), h, accumulate, ws, ws.numel(), stream)
+    return h
+
+
+def global_scale(W: torch.Tensor, q_max: float = 448.0, workspace: torch.Tensor | None = None,
+                 stream=None):
+    """Returns device tensors (S[1], amax[1], status[1] int32)."""
+    W = _bf16_2d(W, "W")
+    o, n = W.shape
+    dev = W.device
+    S = torch.empty(1, dtype=torch.float32, device=dev)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    nb = nvfp4_global_scale_workspace_size(o, n)
+    if nb == 0:
+        raise NVFP4Error("nvfp4_global_scale_workspace_size", -1)
+    ws = workspace if workspace is not None and workspace.numel() >= nb else _workspace(nb, dev)
+    nvfp4_global_scale(W, o, n, W.stride(0), q_max, S, amax, status, ws, ws.numel(), stream)
+    return S, amax, status
+
+
+def scale_sweep_quantize(W: torch.Tensor, h: torch.Tensor | None, S: torch.Tensor, lo: int = -9,
+                         hi: int = 6, want_offsets: bool = False, out=None, stream=None):
+    """Returns (codes[out, in/2] u8, scales[out, in/16] u8, offsets or None)."""
+    W = _bf16_2d(W, "W")
+    o, n = W.shape
+    dev = W.device
+    if out is None:
+        codes = torch.empty(o, n // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(o, n // 16, dtype=torch.uint8, device=dev)
+        offs = torch.empty(o, n // 16, dtype=torch.int8, device=dev) if want_offsets else None
+    else:
+        codes, scales, offs = out
+    nvfp4_scale_sweep_quantize(W, o, n, W.stride(0), h, S, lo, hi, codes, scales, offs, stream)
+    return codes, scales, offs
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, S: torch.Tensor, stream=None):
+    o, half = codes.shape
+    W = torch.empty(o, half * 2, dtype=torch.float32, device=codes.device)
+    nvfp4_dequantize(codes, scales, S, o, half * 2, W, stream)
+    return W
+
+
+def quantize_layer(W: torch.Tensor, X: torch.Tensor | None, q_max: float = 448.0, lo: int = -9,
+                   hi: int = 6, stream=None):
+    """The whole path for one layer: h from X (None = plain MSE), S from W,
+    then the windowed sweep.  Returns (codes, scales, S, h)."""
+    h = diag_hessian(X, stream=stream) if X is not None else None
+    S, _, _ = global_scale(W, q_max, stream=stream)
+    codes, scales, _ = scale_sweep_quantize(W, h, S, lo, hi, stream=stream)
+    return codes, scales, S, h

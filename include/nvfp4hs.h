@@ -1,0 +1,142 @@
+/*
+ * nvfp4hs.h -- C ABI of the B200 (sm_100a) library for Hessian-weighted NVFP4
+ * block-scale selection.
+ *
+ * The method (H-Scale summary, sec. 3 "Method" and sec. B "Implementation
+ * Pseudocode"; ScaleSweep summary, sec. 2 "Theoretical Bounds" and sec. 3
+ * "Implementation"): for a weight matrix W[out, in] quantized to NVFP4 (16
+ * E2M1 values share one E4M3 scale, one FP32 scale per tensor),
+ *   1. h_j = sum_t x_tj^2 over calibration activations X[tokens, in]
+ *      (the diagonal of X^T X, the per-channel second-order proxy);
+ *   2. S = amax(|W|) / (Q * 6), Q = 448 (standard) or 256 (ScaleSweep);
+ *   3. per 16-element group along `in`: base code b = E4M3(absmax / 6 / S);
+ *      candidate codes b+lo .. b+hi (clamped to the 126 positive finite E4M3
+ *      codes), each scored by sum_j h_j (w_j - q_j)^2 with q the E2M1
+ *      round-to-nearest-even reconstruction at that scale; the smallest score
+ *      wins, ties to the lowest offset;
+ *   4. the group is quantized once with the winner and packed.
+ *
+ * Conventions shared by every call
+ *   - All array pointers are DEVICE pointers owned by the caller, except where
+ *     a parameter says "host".  The library allocates nothing.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work and returns; results are valid
+ *     once the stream has reached that point.
+ *   - bf16 inputs are raw bfloat16 bit patterns (uint16), row-major with a
+ *     leading dimension in ELEMENTS.
+ *   - Arguments are checked on the host before anything is enqueued; a failed
+ *     check enqueues nothing and returns a negative nvfp4_status.  A CUDA
+ *     launch error returns NVFP4_ERR_CUDA.  No C++ exception crosses the ABI.
+ *   - Calls are re-entrant: concurrent calls on different streams are safe as
+ *     long as they do not share output or workspace buffers.
+ *   - Packed layout: codes[r, j/2] holds element j of row r in its low nibble
+ *     when j is even and in its high nibble when j is odd; a nibble is
+ *     (sign << 3) | k with k the E2M1 magnitude index (0,0.5,1,1.5,2,3,4,6) and
+ *     the sign bit set only for a negative nonzero value.  scales[r, j/16] is
+ *     the E4M3 bit pattern of group j/16 (0 for an all-zero group).  This is
+ *     4.5 bits per weight (Replay-the-Curvature summary, sec. 1).
+ */
+#ifndef NVFP4HS_H
+#define NVFP4HS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nvfp4_status {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = -1,  /* NULL where not allowed, negative size, bad q_max/flag */
+    NVFP4_ERR_SHAPE = -2,        /* in % 16 != 0, leading dimension < in, too large     */
+    NVFP4_ERR_ALIGN = -3,        /* a pointer or leading dimension breaks the alignment */
+    NVFP4_ERR_WINDOW = -4,       /* lo/hi outside the supported sweep window            */
+    NVFP4_ERR_NONFINITE = -5,    /* written to a device status word: Inf/NaN in W       */
+    NVFP4_ERR_CUDA = -6,         /* a CUDA runtime call or kernel launch failed         */
+    NVFP4_ERR_WORKSPACE = -7     /* workspace NULL or smaller than the queried size     */
+} nvfp4_status;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int nvfp4_version(void);
+
+/* The cudaError_t behind the calling thread's most recent NVFP4_ERR_CUDA. */
+int nvfp4_last_cuda_error(void);
+
+/* ------------------------------------------------------------------------
+ * Step 1: diagonal Hessian proxy (H-Scale summary, sec. B: h = diag(X^T X);
+ * sec. 3 "Hessian-guided objective").
+ *
+ * h[j] = (accumulate ? h[j] : 0) + sum_{t < tokens} X[t * ldx + j]^2.
+ *   X          bf16 [tokens, ldx], 16-byte aligned; ldx % 8 == 0; ldx >= in.
+ *   tokens     >= 0 (0 leaves h unchanged with accumulate, else zeroes it).
+ *   in         > 0, in % 8 == 0.
+ *   h          float [in], 4-byte aligned.  Products are exact in FP32; sums are
+ *              FP32 in short runs, FP32 per thread, FP64 across threads, so the
+ *              result is within ~1e-6 relative of the exact sum for any input.
+ *   workspace  device scratch of at least nvfp4_diag_hessian_workspace_size()
+ *              bytes, 256-byte aligned; holds per-thread partial sums.  Its
+ *              contents need not be initialised and are garbage afterwards.
+ * Deterministic: the summation order depends only on (tokens, in) and the
+ * number of SMs of the current device.
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_diag_hessian_workspace_size(int64_t tokens, int64_t in);
+int nvfp4_diag_hessian(const void* X, int64_t tokens, int64_t in, int64_t ldx, float* h,
+                       int accumulate, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Step 2: FP32 global scale (ScaleSweep summary, sec. 2: S = max|x| / (Q*6)).
+ *
+ * amax = max |W|; S = fl32(amax / fl32(q_max * 6)), S = 0 when amax = 0.
+ *   W          bf16 [out, ldw], 16-byte aligned; ldw % 8 == 0; in % 8 == 0.
+ *   q_max      > 0 and finite (448: E4M3 max; 256: ScaleSweep's choice).
+ *   S          float, device scalar (written).
+ *   amax       float, device scalar, may be NULL.
+ *   status     int, device scalar, may be NULL: NVFP4_OK, or NVFP4_ERR_NONFINITE
+ *              when W holds an Inf or NaN (S and amax are then NaN).
+ *   workspace  at least nvfp4_global_scale_workspace_size() bytes, 256-byte
+ *              aligned; no initialisation needed.
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_global_scale_workspace_size(int64_t out, int64_t in);
+int nvfp4_global_scale(const void* W, int64_t out, int64_t in, int64_t ldw, float q_max,
+                       float* S, float* amax, int* status, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Steps 3-4: windowed scale sweep + quantize + pack (H-Scale summary, sec. 3
+ * "Group-wise scale selection", "Efficient scale search"; sec. B
+ * "HScaleGroupQuantize"; ScaleSweep summary, sec. 3).
+ *
+ *   W          bf16 [out, ldw], 16-byte aligned; ldw % 8 == 0; in % 16 == 0.
+ *   h          float [in], 16-byte aligned, non-negative; NULL = plain MSE
+ *              (h == 1).
+ *   S          float device scalar from nvfp4_global_scale (or the caller's).
+ *   lo, hi     offset window, -16 <= lo <= 0 <= hi <= 15, hi - lo <= 15.
+ *              H-Scale default [-9,+6]; ScaleSweep MSE [-3,+7], WMSE [-8,+7].
+ *   codes      uint8 [out, in/2], 8-byte aligned (written).
+ *   scales     uint8 [out, in/16] (written).
+ *   chosen_offset  int8 [out, in/16] or NULL: winning offset k (the lowest k
+ *              reaching the winning code; 0 for an all-zero group).
+ * The loss is evaluated in FP32; the decision of every element's E2M1 code and
+ * of the base code follows IEEE round-to-nearest-even as the definition does,
+ * so results agree with an exact evaluation except where two candidates' losses
+ * are within ~1e-7 relative of each other.
+ * ------------------------------------------------------------------------ */
+int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t ldw,
+                               const float* h, const float* S, int lo, int hi,
+                               uint8_t* codes, uint8_t* scales, int8_t* chosen_offset,
+                               void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dequantize (NVFP4 decode, H-Scale summary sec. 3: effective scale = global
+ * x local): W_out[r, j] = sign * fl32(g[k] * v(scale)) * S, float [out, in].
+ *   codes [out, in/2] 8-byte aligned; scales [out, in/16]; S device scalar;
+ *   W_out 16-byte aligned; in % 16 == 0.
+ * ------------------------------------------------------------------------ */
+int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S,
+                     int64_t out, int64_t in, float* W_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4HS_H */

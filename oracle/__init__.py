@@ -74,6 +74,8 @@ def lib():
             L.orc_sweep_group_list.restype = None
             L.orc_group_loss_list.argtypes = [u16p, f32p, i64, C.c_float, u8p, f64p]
             L.orc_group_loss_list.restype = None
+            L.orc_packed_loss_list.argtypes = [u16p, f32p, i64, C.c_float, u8p, u8p, f64p]
+            L.orc_packed_loss_list.restype = None
             L.orc_dequantize.argtypes = [u8p, u8p, C.c_float, i64, i64, f32p]
             L.orc_dequantize.restype = None
             _lib = L
@@ -194,6 +196,22 @@ def group_losses(w, h, S: float, codes) -> np.ndarray:
     out = np.zeros(n, np.float64)
     lib().orc_group_loss_list(_p(w, C.c_uint16), None if h is None else _p(h, C.c_float), n,
                               float(S), _p(c, C.c_uint8), _p(out, C.c_double))
+    return out
+
+
+def packed_losses(w, h, S: float, codes, scales) -> np.ndarray:
+    """Exact weighted loss of groups as packed by any quantizer: w[n,16] bf16
+    bits, h[n,16] or None, codes[n,8], scales[n]."""
+    w = _bf16_bits(w).reshape(-1, 16)
+    n = w.shape[0]
+    h = _h_arr(h)
+    if h is not None:
+        h = h.reshape(n, 16)
+    cd = np.ascontiguousarray(codes, dtype=np.uint8).reshape(n, 8)
+    sc = np.ascontiguousarray(scales, dtype=np.uint8).reshape(n)
+    out = np.zeros(n, np.float64)
+    lib().orc_packed_loss_list(_p(w, C.c_uint16), None if h is None else _p(h, C.c_float), n,
+                               float(S), _p(cd, C.c_uint8), _p(sc, C.c_uint8), _p(out, C.c_double))
     return out
 
 

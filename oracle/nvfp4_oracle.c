@@ -19,6 +19,7 @@
 #include "nvfp4_oracle.h"
 
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ---- number formats --------------------------------------------------- */
@@ -90,15 +91,23 @@ double orc_group_loss(const uint16_t* w, const float* h, float S, int code) {
 
 void orc_diag_hessian(const uint16_t* X, int64_t tokens, int64_t in, int64_t ldx,
                       float* h, int accumulate) {
+    /* acc_j = sum over t in increasing order of x_tj^2, in double.  The loops
+     * run row by row only so that memory is read in order; each column's sum
+     * still adds its terms in token order. */
+    double* acc = (double*)calloc((size_t)(in > 0 ? in : 1), sizeof(double));
+    if (!acc) return;
+    for (int64_t t = 0; t < tokens; ++t) {
+        const uint16_t* row = X + t * ldx;
+        for (int64_t j = 0; j < in; ++j) {
+            double x = bf16_to_double(row[j]);
+            acc[j] += x * x;                           /* x*x exact: 16 significant bits */
+        }
+    }
     for (int64_t j = 0; j < in; ++j) {
         double s = accumulate ? (double)h[j] : 0.0;
-        double acc = 0.0;
-        for (int64_t t = 0; t < tokens; ++t) {
-            double x = bf16_to_double(X[t * ldx + j]);
-            acc += x * x;                              /* x*x exact: 16 significant bits */
-        }
-        h[j] = (float)(s + acc);
+        h[j] = (float)(s + acc[j]);
     }
+    free(acc);
 }
 
 /* ---- global scale -------------------------------------------------------- */
@@ -194,6 +203,26 @@ void orc_group_loss_list(const uint16_t* w, const float* h, int64_t n, float S,
                          const uint8_t* code, double* losses) {
     for (int64_t i = 0; i < n; ++i)
         losses[i] = orc_group_loss(w + 16 * i, h ? h + 16 * i : NULL, S, code[i]);  /* code 0: all zero */
+}
+
+void orc_packed_loss_list(const uint16_t* w, const float* h, int64_t n, float S,
+                          const uint8_t* codes, const uint8_t* scale, double* losses) {
+    for (int64_t i = 0; i < n; ++i) {
+        double v = orc_e4m3_value(scale[i]);
+        if (v < 0.0) { losses[i] = NAN; continue; }
+        double vS = v * (double)S;
+        double L = 0.0;
+        for (int j = 0; j < 16; ++j) {
+            uint8_t byte = codes[8 * i + j / 2];
+            uint8_t nib = (j & 1) ? (byte >> 4) : (byte & 15);
+            double r = kGrid[nib & 7] * vS;                /* exact */
+            if (nib & 8) r = -r;
+            double d = bf16_to_double(w[16 * i + j]) - r;  /* exact */
+            double hj = h ? (double)h[16 * i + j] : 1.0;
+            L += hj * (d * d);
+        }
+        losses[i] = L;
+    }
 }
 
 /* ---- dequantize ----------------------------------------------------------- */

@@ -100,6 +100,13 @@ void orc_sweep_group_list(const uint16_t* w, const float* h, int64_t n, float S,
 void orc_group_loss_list(const uint16_t* w, const float* h, int64_t n, float S,
                          const uint8_t* code, double* losses);
 
+/* Loss of n groups as packed: w[n,16], h[n,16] or NULL, codes[n,8] (nibbles as
+ * in orc_sweep_group), scale[n] E4M3 codes.  The reconstruction of element j
+ * is decoded from its nibble (not re-derived), so this scores any packer's
+ * actual output: L = sum_j h_j (w_j - sign_j g[k_j] v S)^2. */
+void orc_packed_loss_list(const uint16_t* w, const float* h, int64_t n, float S,
+                          const uint8_t* codes, const uint8_t* scale, double* losses);
+
 /* W_out[r, j] = sign * fl32(g[k] * v(scale)) * S, float32 [out, in]. */
 void orc_dequantize(const uint8_t* codes, const uint8_t* scales, float S,
                     int64_t out, int64_t in, float* W_out);

@@ -1,0 +1,121 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/*.h declares, and rejects bad arguments on the host (before any CUDA
+call) with the documented status codes."""
+import ctypes as C
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session")
+def L():
+    from block_scale_search_b200 import _build, lib
+    _build.build()
+    return lib()
+
+
+def declared_functions():
+    names = []
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(hdr).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b(nvfp4_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert "nvfp4_scale_sweep_quantize" in names and len(names) >= 8
+    out = subprocess.run(["nm", "-D", "--defined-only", L._name], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (nvfp4_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(L, n)
+
+
+def test_version(L):
+    assert L.nvfp4_version() == 100
+
+
+P = 0x10000  # a 64 KiB-aligned fake device address: never dereferenced (checks fail first)
+
+
+def test_diag_hessian_validation(L):
+    f = L.nvfp4_diag_hessian
+    ws = P
+    assert f(None, 4, 16, 16, P, 0, ws, 1 << 20, None) == -1          # X NULL with tokens
+    assert f(P, 4, 16, 16, None, 0, ws, 1 << 20, None) == -1          # h NULL
+    assert f(P, -1, 16, 16, P, 0, ws, 1 << 20, None) == -1            # negative tokens
+    assert f(P, 4, 16, 16, P, 2, ws, 1 << 20, None) == -1             # accumulate flag
+    assert f(P, 4, 12, 16, P, 0, ws, 1 << 20, None) == -2             # in % 8
+    assert f(P, 4, 16, 8, P, 0, ws, 1 << 20, None) == -2              # ldx < in
+    assert f(P + 2, 4, 16, 16, P, 0, ws, 1 << 20, None) == -3         # X misaligned
+    assert f(P, 4, 16, 20, P, 0, ws, 1 << 20, None) == -3             # ldx % 8
+    assert f(P, 4, 16, 16, P + 2, 0, ws, 1 << 20, None) == -3         # h misaligned
+    assert f(P, 4, 16, 16, P, 0, None, 1 << 20, None) == -7           # no workspace
+    assert f(P, 4, 16, 16, P, 0, ws + 4, 1 << 20, None) == -3         # workspace misaligned
+
+
+def test_global_scale_validation(L):
+    f = L.nvfp4_global_scale
+    assert f(None, 4, 16, 16, 448.0, P, None, None, P, 1024, None) == -1
+    assert f(P, 4, 16, 16, 448.0, None, None, None, P, 1024, None) == -1   # S NULL
+    assert f(P, 4, 16, 16, 0.0, P, None, None, P, 1024, None) == -1       # q_max <= 0
+    assert f(P, 4, 16, 16, float("inf"), P, None, None, P, 1024, None) == -1
+    assert f(P, 4, 12, 16, 448.0, P, None, None, P, 1024, None) == -2      # in % 8
+    assert f(P, 4, 16, 8, 448.0, P, None, None, P, 1024, None) == -2       # ldw < in
+    assert f(P + 8, 4, 16, 16, 448.0, P, None, None, P, 1024, None) == -3  # W misaligned
+    assert f(P, 4, 16, 16, 448.0, P + 1, None, None, P, 1024, None) == -3  # S misaligned
+    assert f(P, 4, 16, 16, 448.0, P, None, None, None, 1024, None) == -7   # no workspace
+
+
+def test_sweep_validation(L):
+    f = L.nvfp4_scale_sweep_quantize
+    ok = (P, 4, 32, 32, None, P, -9, 6, P, P, None, None)
+
+    def call(**kw):
+        names = ["W", "out", "inp", "ldw", "h", "S", "lo", "hi", "codes", "scales", "offs", "st"]
+        a = dict(zip(names, ok))
+        a.update(kw)
+        return f(*[a[n] for n in names])
+
+    assert call(W=None) == -1
+    assert call(S=None) == -1
+    assert call(codes=None) == -1
+    assert call(scales=None) == -1
+    assert call(out=-1) == -1
+    assert call(inp=24, ldw=24) == -2                 # in % 16
+    assert call(ldw=16) == -2                         # ldw < in
+    assert call(W=P + 4) == -3
+    assert call(ldw=36) == -3                         # ldw % 8
+    assert call(h=P + 4) == -3                        # h must be 16-byte aligned
+    assert call(codes=P + 4) == -3
+    for lo, hi in ((1, 6), (-9, -1), (-17, 0), (0, 16), (-9, 7), (-16, 1)):
+        assert call(lo=lo, hi=hi) == -4, (lo, hi)
+    assert call(out=0) == 0                           # empty: nothing to do, no device needed
+    assert call(inp=0, ldw=0) == 0
+
+
+def test_dequantize_validation(L):
+    f = L.nvfp4_dequantize
+    assert f(P, P, P, -1, 16, P, None) == -1
+    assert f(P, P, P, 2, 24, P, None) == -2
+    assert f(None, P, P, 2, 16, P, None) == -1
+    assert f(P + 4, P, P, 2, 16, P, None) == -3
+    assert f(P, P, P, 2, 16, P + 8, None) == -3
+    assert f(P, P, P, 0, 16, P, None) == 0
+
+
+def test_binding_has_same_names_as_abi():
+    import block_scale_search_b200 as m
+    for n in declared_functions():
+        if n == "nvfp4_last_cuda_error":
+            continue
+        assert hasattr(m, n), n

@@ -356,3 +356,19 @@ def test_dequantize_round_trip_never_worse_than_base_rtn(orc):
         half = np.where(a < 2 * step, 0.25, np.where(a < 4 * step, 0.5, 1.0)) * step
         assert np.all(np.abs(Wf - Wq)[unsat] <= half[unsat] * (1 + 1e-6) + 1e-30)
     assert np.all(errs[0] <= errs[1] * (1 + 1e-5) + 1e-30)
+
+
+def test_packed_loss_equals_group_loss_on_oracle_output(orc):
+    """Scoring the oracle's own packed bytes reproduces the loss the sweep
+    reports (decoding nibbles must agree with the E2M1 decision and signs)."""
+    rng = np.random.default_rng(13)
+    w = _random_groups(3000, 14)
+    h = np.float32(np.exp(rng.normal(0, 1, w.shape)))
+    codes, scales, _, loss = orc.sweep_groups(w, h, 1.5e-3, -9, 6)
+    np.testing.assert_array_equal(orc.packed_losses(w, h, 1.5e-3, codes, scales), loss)
+    # flipping one nibble's sign changes the loss unless that element is zero
+    c2 = codes.copy()
+    c2[:, 0] ^= 0x08
+    l2 = orc.packed_losses(w, h, 1.5e-3, c2, scales)
+    changed = (codes[:, 0] & 0x07) != 0
+    assert np.all(l2[changed] > loss[changed])
