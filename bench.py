@@ -106,8 +106,7 @@ class ClockSampler:
 
 def build_layer(rank: int, device):
     import torch
-    import workloads
-    wl = workloads.llama33_70b_mlp(seed_offset=rank)
+    wl = rank_workload(rank)
     Ws = {m.name: m.make(device) for m in wl.matrices}
     Xs = {k: c.make(device) for k, c in wl.calibs.items()}
     torch.cuda.synchronize()
@@ -244,13 +243,21 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """Max of a per-rank timing over all ranks (the only collective: timing)."""
     import torch
     import torch.distributed as dist
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(rank: int):
+    """Weak scaling: rank r quantizes its own layer, drawn with seed offset r."""
+    import workloads
+    return workloads.llama33_70b_mlp(seed_offset=rank)
 
 
 def run_reference(args):

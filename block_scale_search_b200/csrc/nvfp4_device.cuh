@@ -64,6 +64,50 @@ __device__ __forceinline__ float e2m1_round(float x) {
   return fminf(q, 6.0f);
 }
 
+// Decode an E2M1 nibble pair with the sign dropped (bits 0..2 and 4..6 used).
+__device__ __forceinline__ float e2m1_nibble_value(uint32_t nib) {
+  const uint32_t hh = e2m1x2_to_f16x2(nib & 7u);
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(hh & 0xFFFFu)));
+}
+
+// ------------------------------------------------------------ packed FP32x2
+// sm_100 executes these as one instruction for two lanes of FP32 work.
+typedef unsigned long long f32x2_t;
+__device__ __forceinline__ f32x2_t f2_pack(float lo, float hi) {
+  f32x2_t r;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f32x2_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2_t f2_fma(f32x2_t a, f32x2_t b, f32x2_t c) {
+  f32x2_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f32x2_t f2_mul(f32x2_t a, f32x2_t b) {
+  f32x2_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Round two non-negative floats to E2M1 (RNE, saturating) and decode them
+// back to an f16x2 of grid values: low half <- lo, high half <- hi.
+__device__ __forceinline__ uint32_t e2m1x2_round_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.rn.f16x2.e2m1x2 %0, t; }"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// e = c - q * v with q, v half-precision (exact product) and one rounding.
+__device__ __forceinline__ float fma_f16_f32(uint16_t q, uint16_t nv, float c) {
+  float r;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(r) : "h"(q), "h"(nv), "f"(c));
+  return r;
+}
+
 // -------------------------------------------------------------------- bf16
 
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
