@@ -33,10 +33,10 @@ cudaError_t launch_global_scale(const uint16_t* W, int64_t out, int64_t ldw, flo
                                 float* S, float* amax, int* status, uint32_t* partial,
                                 const LanePlan& p, cudaStream_t stream);
 
-LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted, bool v8);
+LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted);
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi, uint8_t* codes,
-                               uint8_t* scales, int8_t* offs, bool v8, const LanePlan& p,
+                               uint8_t* scales, int8_t* offs, const LanePlan& p,
                                cudaStream_t stream);
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S,
