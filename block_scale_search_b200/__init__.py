@@ -20,6 +20,7 @@ from . import _build
 __all__ = [
     "NVFP4Error", "lib", "nvfp4_version", "nvfp4_diag_hessian_workspace_size",
     "nvfp4_diag_hessian", "nvfp4_global_scale_workspace_size", "nvfp4_global_scale",
+    "nvfp4_global_scale_noalloc",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize",
     "diag_hessian", "global_scale", "scale_sweep_quantize", "dequantize", "quantize_layer",
 ]
@@ -50,6 +51,7 @@ _SIGS = {
     "nvfp4_diag_hessian": ([_vp, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp], _int),
     "nvfp4_global_scale_workspace_size": ([_i64, _i64], _sz),
     "nvfp4_global_scale": ([_vp, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _vp, _sz, _vp], _int),
+    "nvfp4_global_scale_noalloc": ([_vp, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _vp], _int),
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
@@ -117,6 +119,14 @@ def nvfp4_global_scale(W, out, inp, ldw, q_max, S, amax, status, workspace, work
     _check("nvfp4_global_scale", lib().nvfp4_global_scale(
         _ptr(W), out, inp, ldw, float(q_max), _ptr(S), _ptr(amax), _ptr(status), _ptr(workspace),
         workspace_bytes, _stream(stream)))
+
+
+def nvfp4_global_scale_noalloc(W, out, inp, ldw, q_max, S, amax, status, stream=None):
+    """nvfp4_global_scale without a workspace, for callers that cannot
+    allocate: the library's built-in 64 KiB device array holds the partial
+    maxima.  Calls that overlap on the GPU share that array and race."""
+    _check("nvfp4_global_scale_noalloc", lib().nvfp4_global_scale_noalloc(
+        _ptr(W), out, inp, ldw, float(q_max), _ptr(S), _ptr(amax), _ptr(status), _stream(stream)))
 
 
 def nvfp4_scale_sweep_quantize(W, out, inp, ldw, h, S, lo, hi, codes, scales, chosen_offset,

@@ -103,6 +103,28 @@ int nvfp4_global_scale(const void* W, int64_t out, int64_t in, int64_t ldw, floa
                        size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Step 2 without caller-provided scratch.  (The method's pages have no
+ * counterpart: this is a deployment convenience.)
+ *
+ * Same arguments, result and status word as nvfp4_global_scale, minus the
+ * workspace.  For callers that cannot allocate device memory -- plugin hooks
+ * handed tensors but no allocator, or code under a hard memory cap or inside
+ * a pre-planned memory pool -- the per-CTA partial maxima go to a 64 KiB
+ * array compiled into the library, which every GPU that loads the library
+ * holds until the process exits.  Nothing is allocated.
+ *   - The first call on a device, made while that device is current, looks up
+ *     the array's device address (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU (different
+ *     streams without ordering between them) race and must not be issued.
+ *   - The array needs no initialisation; it is not cleared.
+ *   - A problem whose partials would not fit the array returns
+ *     NVFP4_ERR_WORKSPACE (never on current GPUs: one 4-byte partial per CTA).
+ * ------------------------------------------------------------------------ */
+int nvfp4_global_scale_noalloc(const void* W, int64_t out, int64_t in, int64_t ldw, float q_max,
+                               float* S, float* amax, int* status, void* stream);
+
+/* ------------------------------------------------------------------------
  * Steps 3-4: windowed scale sweep + quantize + pack (H-Scale summary, sec. 3
  * "Group-wise scale selection", "Efficient scale search"; sec. B
  * "HScaleGroupQuantize"; ScaleSweep summary, sec. 3).
