@@ -31,6 +31,11 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 LO, HI = -9, 6
 SWEEP_BYTES_PER_ELEM = 2 + 0.5 + 1 / 16   # read bf16 W; write 4-bit code + 1/16 E4M3 byte
+# The definition's work per weight element and candidate scale: the quotient
+# |w|/(vS), the E2M1 rounding, the reconstruction error |w| - q v S, the weight
+# h*e and the accumulation (h e) e -- five FP32 lane operations.
+SWEEP_OPS_PER_ELEM_CAND = 5
+SMS, LANES_PER_SM = 148, 128
 
 
 def measured_peaks():
@@ -45,22 +50,24 @@ def measured_peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 100 ms; only samples stamped inside the timed
+    region (mark_start .. mark_end) are summarised."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
-        self.lines: list[str] = []
+        self.lines: list[tuple[float, str]] = []
         self.t = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -70,7 +77,13 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
@@ -82,31 +95,34 @@ class ClockSampler:
             self.proc.kill()
         if self.t:
             self.t.join(timeout=2)
-        sm, mx, reasons = [], 0.0, set()
+        sm, mx, reasons, power = [], 0.0, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.lines:
+            if self.t0 is not None and not (self.t0 <= ts <= (self.t1 or ts) + 0.05):
+                continue
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
+                sm.append(float(f[2]))
+                mx = max(mx, float(f[3]))
+                power.append(float(f[4]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(names, f[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w_median": statistics.median(power) if power else None}
 
 
 # --------------------------------------------------------------- workload
 
-def build_layer(rank: int, device):
+def build_layer(rank: int, device, name: str = "llama33_70b_mlp"):
     import torch
-    wl = rank_workload(rank)
+    wl = rank_workload(rank, name)
     Ws = {m.name: m.make(device) for m in wl.matrices}
     Xs = {k: c.make(device) for k, c in wl.calibs.items()}
     torch.cuda.synchronize()
@@ -166,6 +182,24 @@ class Step:
                 self.codes[n], self.scales[n], None, stream))
 
 
+def profiled_traffic(kernel: str, units_per_launch: float):
+    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json),
+    scaled by the units one launch processes; None when the kernel's source has
+    changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha1(open(src, "rb").read()).hexdigest() != d["source_sha1"]:
+        return None
+    return d["dram_bytes_per_unit"] * units_per_launch
+
+
 def kernel_bytes(wl):
     wel = wl.weight_elems
     return {"diag_hessian": wl.calib_bytes + 4 * sum(c.inp for c in wl.calibs.values()),
@@ -175,44 +209,40 @@ def kernel_bytes(wl):
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_sample_rate(wl, Ws, Xs, threads=None, budget_rows=None):
-    """Time the CPU oracle on a bounded sample of this workload and extrapolate
-    to whole-job weight elements per second.  Returns (rate, info)."""
-    import numpy as np
+def oracle_sample_rate(wl, Ws, Xs, threads=None, row_frac=0.25, tokens=4096):
+    """Time the CPU oracle (as it stands) on a bounded sample of this workload --
+    the first `row_frac` of every weight's rows and the first `tokens` tokens of
+    every calibration matrix -- and extrapolate linearly to whole-job weight
+    elements per second.  Returns (rate, info)."""
     import torch
     import oracle
     threads = threads or oracle.default_threads()
-    rows = budget_rows or {"gate": 192, "up": 192, "down": 64}
     t_sweep = t_abs = t_h = 0.0
-    el_sweep = el_abs = 0
-    xel = 0
+    el_w = xel = 0
     hs = {}
     for k, X in Xs.items():
-        n_tok = 256
-        sub = X[:n_tok].cpu()
+        sub = X[:tokens].cpu()
         t0 = time.perf_counter()
         hs[k] = oracle.parallel_diag_hessian(sub, threads=threads)
         t_h += time.perf_counter() - t0
         xel += sub.numel()
     for m in wl.matrices:
-        W = Ws[m.name]
-        r = rows.get(m.name, 64)
-        sub = W[:r].cpu().view(torch.uint16).numpy()
+        r = max(1, int(m.out * row_frac))
+        sub = Ws[m.name][:r].cpu().view(torch.uint16).numpy()
         t0 = time.perf_counter()
         S, _, _ = oracle.global_scale(sub, wl.q_max)
         t_abs += time.perf_counter() - t0
-        el_abs += sub.size
-        h = hs[m.x_key]
         t0 = time.perf_counter()
-        oracle.parallel_sweep_quantize(sub, h, float(S) if S > 0 else 1e-3, LO, HI, threads=threads)
+        oracle.parallel_sweep_quantize(sub, hs[m.x_key], float(S) if S > 0 else 1e-3, LO, HI,
+                                       threads=threads)
         t_sweep += time.perf_counter() - t0
-        el_sweep += sub.size
+        el_w += sub.size
     wel = wl.weight_elems
     x_total = sum(c.tokens * c.inp for c in wl.calibs.values())
-    t_full = t_sweep * wel / el_sweep + t_abs * wel / el_abs + t_h * x_total / xel
-    info = {"sample": (f"oracle on {el_sweep} of {wel} weight elements "
-                       f"(rows {rows}) and 256 of {wl.calibs['gu'].tokens} tokens per X; "
-                       f"extrapolated linearly to the full layer"),
+    t_full = (t_sweep + t_abs) * wel / el_w + t_h * x_total / xel
+    info = {"sample": (f"oracle on the first {row_frac:.0%} of every weight's rows ({el_w} of {wel} "
+                       f"elements) and the first {tokens} tokens of every calibration matrix; "
+                       f"extrapolated linearly to the whole layer"),
             "cores": threads, "t_sample_s": round(t_sweep + t_abs + t_h, 3),
             "t_full_est_s": round(t_full, 2)}
     return wel / t_full, info
@@ -254,10 +284,19 @@ def max_over_ranks(x: float, ws: int) -> float:
     return float(t.item())
 
 
-def rank_workload(rank: int):
+WORKLOADS = {
+    "llama33_70b_mlp": ("llama33_70b_mlp: gate/up 28672x8192, down 8192x28672 bf16 N(0,0.015) "
+                        "0.1% x10 outliers; X 65536 tokens x {8192, 28672} bf16 lognormal(1.5) "
+                        "channel scales"),
+    "mlp_slice": ("mlp_slice (profiling size): W 8192x8192 bf16 N(0,0.015) 0.1% x10; X 16384 x "
+                  "8192 bf16 lognormal(1.5) channel scales"),
+}
+
+
+def rank_workload(rank: int, name: str = "llama33_70b_mlp"):
     """Weak scaling: rank r quantizes its own layer, drawn with seed offset r."""
     import workloads
-    return workloads.llama33_70b_mlp(seed_offset=rank)
+    return workloads.ALL[name](seed_offset=rank)
 
 
 def run_reference(args):
@@ -269,10 +308,10 @@ def run_reference(args):
     dev = "cuda:0" if torch.cuda.is_available() else "cpu"
     wl, Ws, Xs = build_layer(0, dev)
     for _ in range(args.warmup):
-        oracle_sample_rate(wl, Ws, Xs, budget_rows={"gate": 16, "up": 16, "down": 8})
+        oracle_sample_rate(wl, Ws, Xs, row_frac=1 / 256, tokens=256)
     rates, info = [], None
     for _ in range(args.steps):
-        r, info = oracle_sample_rate(wl, Ws, Xs, budget_rows={"gate": 64, "up": 64, "down": 16})
+        r, info = oracle_sample_rate(wl, Ws, Xs, row_frac=1 / 64, tokens=1024)
         rates.append(r)
     v = statistics.median(rates)
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "elem/s",
@@ -291,11 +330,12 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="llama33_70b_mlp", choices=WORKLOADS)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -309,7 +349,7 @@ def main():
     rank, local, ws = init_dist()
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
-    wl, Ws, Xs = build_layer(rank, dev)
+    wl, Ws, Xs = build_layer(rank, dev, args.workload)
     step = Step(nv, wl, Ws, Xs, dev)
 
     for _ in range(args.warmup):
@@ -325,11 +365,13 @@ def main():
     barrier(ws)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
     t0.record(stream)
     for _ in range(args.steps):
         step.run(ev)
     t1.record(stream)
     barrier(ws)
+    sampler.mark_end()
     clocks = sampler.stop()
     ms = t0.elapsed_time(t1) / args.steps
     ms_max = max_over_ranks(ms, ws)
@@ -388,13 +430,33 @@ def main():
 
     # ---- roofline of the dominant kernel
     dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
-    per_launch_ms = kern[dom]["ms_per_step"] / kern[dom]["launch_pairs_per_step"]
-    achieved = kb[dom] / kern[dom]["launch_pairs_per_step"] / (per_launch_ms * 1e-3) / 1e9
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS copy)", "unit": "GB/s",
-                "frac": round(achieved / peak, 4),
-                "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                "traffic": None}
+    launches = kern[dom]["launch_pairs_per_step"]
+    per_launch_s = kern[dom]["ms_per_step"] / launches * 1e-3
+    if dom == "scale_sweep":
+        # compute-bound: FP32 lane operations the definition needs, against
+        # 148 SMs x 128 FP32 lanes x the SM clock sampled during the run
+        ops = SWEEP_OPS_PER_ELEM_CAND * (HI - LO + 1) * wl.weight_elems / launches
+        clk = (clocks or {}).get("sm_mhz") or 1965.0
+        peak_top = SMS * LANES_PER_SM * clk * 1e6 / 1e12
+        achieved = ops / per_launch_s / 1e12
+        roofline = {"kernel": dom, "bound": "alu", "achieved": round(achieved, 2),
+                    "peak": round(peak_top, 2), "unit": "TOP/s",
+                    "peak_source": f"148 SMs x 128 FP32 lanes x {clk:.0f} MHz (sampled SM clock)",
+                    "frac": round(achieved / peak_top, 4),
+                    "ops_per_unit": f"{SWEEP_OPS_PER_ELEM_CAND} FP32 ops per weight element per candidate",
+                    "hbm_frac_of_measured": kern[dom][f"frac_of_{peak_kind}"],
+                    "traffic": profiled_traffic(dom, wl.weight_elems / launches),
+                    "traffic_note": "DRAM read+write bytes per launch, from the committed ncu "
+                                    "capture on the profiling-size layer, scaled by elements"}
+    else:
+        achieved = kb[dom] / launches / per_launch_s / 1e9
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                    "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS copy)", "unit": "GB/s",
+                    "frac": round(achieved / peak, 4),
+                    "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                    "traffic": profiled_traffic(dom, (wl.weight_elems if dom != "diag_hessian" else
+                                                      sum(c.tokens * c.inp for c in wl.calibs.values()))
+                                                / launches)}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -408,11 +470,10 @@ def main():
             "metric": METRIC, "value": value, "unit": "elem/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "llama33_70b_mlp: gate/up 28672x8192, down 8192x28672 bf16 "
-                                   "N(0,0.015) 0.1% x10 outliers; X 65536 tokens x {8192, 28672} "
-                                   "bf16 lognormal(1.5) channel scales",
+            "config": {"workload": WORKLOADS[args.workload],
                        "window": [LO, HI], "q_max": wl.q_max, "weighted": True,
-                       "l2": "inputs 6.2 GB per rank > 126 MB L2; no flush",
+                       "l2": f"inputs {(wl.calib_bytes + 2 * wl.weight_elems) / 1e9:.2f} GB per "
+                             f"rank > 126 MB L2; no flush",
                        "parallelism": f"weak: {ws} rank(s), one independent layer per rank"},
             "calib_gbs": round(xbytes / (kern["diag_hessian"]["ms_per_step"] * 1e-3) / 1e9, 1),
             "quantize_elems_per_s": wel / ((kern["global_scale"]["ms_per_step"] +

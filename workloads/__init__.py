@@ -197,6 +197,15 @@ def llama33_70b_mlp(seed_offset: int = 0) -> Workload:
     return Workload("llama33_70b_mlp", 448.0, mats, cal, [Run(-9, 6, True)])
 
 
+def mlp_slice(seed_offset: int = 0) -> Workload:
+    """One 70B-MLP-like layer at profiling size: W 8192x8192 N(0,0.015), 0.1% x10;
+    X 16384 x 8192, lognormal(1.5) channel scales (inputs larger than L2)."""
+    s = 700 + 97 * seed_offset
+    return Workload("mlp_slice_8192x8192", 448.0,
+                    [Matrix("w", 8192, 8192, "x", s + 1, 0.015, 0.001, 10.0)],
+                    {"x": Calib("x", 16384, 8192, 1.5, s + 41)}, [Run(-9, 6, True)])
+
+
 def moe_grouped(tokens: int = 262144, experts: int = 128, device="cpu") -> Workload:
     """128 experts x {gate, up 768x2048; down 2048x768}; 262144 tokens routed
     top-8 with Zipf(1.1) popularity; per-expert X slices and h."""
@@ -216,4 +225,4 @@ def moe_grouped(tokens: int = 262144, experts: int = 128, device="cpu") -> Workl
 
 
 ALL = {"single_layer": single_layer, "square_layer": square_layer, "llama3_8b": llama3_8b,
-       "llama33_70b_mlp": llama33_70b_mlp, "moe_grouped": moe_grouped}
+       "llama33_70b_mlp": llama33_70b_mlp, "mlp_slice": mlp_slice, "moe_grouped": moe_grouped}
