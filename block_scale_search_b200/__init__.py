@@ -20,7 +20,11 @@ from . import _build
 __all__ = [
     "NVFP4Error", "lib", "nvfp4_version", "nvfp4_diag_hessian_workspace_size",
     "nvfp4_diag_hessian", "nvfp4_global_scale_workspace_size", "nvfp4_global_scale",
-    "nvfp4_global_scale_noalloc",
+    "nvfp4_global_scale_noalloc", "nvfp4_diag_hessian_grouped_workspace_size",
+    "nvfp4_diag_hessian_grouped", "nvfp4_global_scale_batched_workspace_size",
+    "nvfp4_global_scale_batched", "nvfp4_scale_sweep_quantize_batched_workspace_size",
+    "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
+    "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize",
     "diag_hessian", "global_scale", "scale_sweep_quantize", "dequantize", "quantize_layer",
 ]
@@ -44,6 +48,19 @@ _lib = None
 LIB_PATH = _build.LIB
 
 _vp, _i64, _sz, _int, _f32 = C.c_void_p, C.c_int64, C.c_size_t, C.c_int, C.c_float
+
+
+class MatrixDesc(C.Structure):
+    """nvfp4_matrix_desc"""
+    _fields_ = [("W", _vp), ("out", _i64), ("inp", _i64), ("ldw", _i64)]
+
+
+class SweepDesc(C.Structure):
+    """nvfp4_sweep_desc"""
+    _fields_ = [("W", _vp), ("out", _i64), ("inp", _i64), ("ldw", _i64), ("h", _vp), ("S", _vp),
+                ("codes", _vp), ("scales", _vp), ("chosen_offset", _vp)]
+
+
 _SIGS = {
     "nvfp4_version": ([], _int),
     "nvfp4_last_cuda_error": ([], _int),
@@ -55,6 +72,15 @@ _SIGS = {
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
+    "nvfp4_diag_hessian_grouped_workspace_size": ([_i64, _i64, _i64], _sz),
+    "nvfp4_diag_hessian_grouped": ([_vp, _vp, _i64, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp],
+                                   _int),
+    "nvfp4_global_scale_batched_workspace_size": ([C.POINTER(MatrixDesc), _i64], _sz),
+    "nvfp4_global_scale_batched": ([C.POINTER(MatrixDesc), _i64, _f32, _vp, _vp, _vp, _vp, _sz,
+                                    _vp], _int),
+    "nvfp4_scale_sweep_quantize_batched_workspace_size": ([_i64], _sz),
+    "nvfp4_scale_sweep_quantize_batched": ([C.POINTER(SweepDesc), _i64, _int, _int, _vp, _sz, _vp],
+                                           _int),
 }
 
 
@@ -141,6 +167,47 @@ def nvfp4_dequantize(codes, scales, S, out, inp, W_out, stream=None):
         _ptr(codes), _ptr(scales), _ptr(S), out, inp, _ptr(W_out), _stream(stream)))
 
 
+def nvfp4_diag_hessian_grouped_workspace_size(total_tokens: int, experts: int, inp: int) -> int:
+    return lib().nvfp4_diag_hessian_grouped_workspace_size(total_tokens, experts, inp)
+
+
+def nvfp4_diag_hessian_grouped(X, row_offsets, experts, total_tokens, inp, ldx, h, accumulate,
+                               workspace, workspace_bytes, stream=None):
+    _check("nvfp4_diag_hessian_grouped", lib().nvfp4_diag_hessian_grouped(
+        _ptr(X), _ptr(row_offsets), experts, total_tokens, inp, ldx, _ptr(h), int(accumulate),
+        _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def _desc_array(cls, items):
+    arr = (cls * max(1, len(items)))()
+    for i, it in enumerate(items):
+        arr[i] = it
+    return arr
+
+
+def nvfp4_global_scale_batched_workspace_size(descs) -> int:
+    arr = _desc_array(MatrixDesc, descs)
+    return lib().nvfp4_global_scale_batched_workspace_size(arr, len(descs))
+
+
+def nvfp4_global_scale_batched(descs, q_max, S, amax, status, workspace, workspace_bytes,
+                               stream=None):
+    arr = _desc_array(MatrixDesc, descs)
+    _check("nvfp4_global_scale_batched", lib().nvfp4_global_scale_batched(
+        arr, len(descs), float(q_max), _ptr(S), _ptr(amax), _ptr(status), _ptr(workspace),
+        workspace_bytes, _stream(stream)))
+
+
+def nvfp4_scale_sweep_quantize_batched_workspace_size(n: int) -> int:
+    return lib().nvfp4_scale_sweep_quantize_batched_workspace_size(n)
+
+
+def nvfp4_scale_sweep_quantize_batched(descs, lo, hi, workspace, workspace_bytes, stream=None):
+    arr = _desc_array(SweepDesc, descs)
+    _check("nvfp4_scale_sweep_quantize_batched", lib().nvfp4_scale_sweep_quantize_batched(
+        arr, len(descs), int(lo), int(hi), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
 # -------------------------------------------------------- tensor conveniences
 
 def _bf16_2d(t: torch.Tensor, name: str) -> torch.Tensor:
@@ -218,3 +285,58 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor | None, q_max: float = 448.0
     S, _, _ = global_scale(W, q_max, stream=stream)
     codes, scales, _ = scale_sweep_quantize(W, h, S, lo, hi, stream=stream)
     return codes, scales, S, h
+
+
+def diag_hessian_grouped(X: torch.Tensor, row_offsets: torch.Tensor, h: torch.Tensor | None = None,
+                         accumulate: bool = False, stream=None) -> torch.Tensor:
+    """h[E, in]: per-expert sums of squares over expert-contiguous rows of X.
+    row_offsets: int64 CUDA tensor [E+1]."""
+    X = _bf16_2d(X, "X")
+    T, n = X.shape
+    E = row_offsets.numel() - 1
+    if h is None:
+        h = torch.empty(E, n, dtype=torch.float32, device=X.device)
+    nb = nvfp4_diag_hessian_grouped_workspace_size(T, E, n)
+    if nb == 0:
+        raise NVFP4Error("nvfp4_diag_hessian_grouped_workspace_size", -1)
+    ws = _workspace(nb, X.device)
+    nvfp4_diag_hessian_grouped(X, row_offsets, E, T, n, X.stride(0), h, accumulate, ws, ws.numel(),
+                               stream)
+    return h
+
+
+def global_scale_batched(Ws, q_max: float = 448.0, stream=None):
+    """S, amax, status (device [n]) of many bf16 matrices in one launch."""
+    descs = [MatrixDesc(_bf16_2d(W, "W").data_ptr(), W.shape[0], W.shape[1], W.stride(0)) for W in Ws]
+    dev = Ws[0].device
+    n = len(Ws)
+    S = torch.empty(n, dtype=torch.float32, device=dev)
+    amax = torch.empty(n, dtype=torch.float32, device=dev)
+    status = torch.empty(n, dtype=torch.int32, device=dev)
+    nb = nvfp4_global_scale_batched_workspace_size(descs)
+    if nb == 0:
+        raise NVFP4Error("nvfp4_global_scale_batched_workspace_size", -1)
+    ws = _workspace(nb, dev)
+    nvfp4_global_scale_batched(descs, q_max, S, amax, status, ws, ws.numel(), stream)
+    return S, amax, status
+
+
+def scale_sweep_quantize_batched(Ws, hs, Ss, lo: int = -9, hi: int = 6, want_offsets=False,
+                                 stream=None):
+    """Sweep many matrices in one launch.  hs: list of h (or None for all),
+    Ss: list of device scalars (e.g. views into global_scale_batched's S)."""
+    descs, outs = [], []
+    for i, W in enumerate(Ws):
+        W = _bf16_2d(W, "W")
+        o, n = W.shape
+        codes = torch.empty(o, n // 2, dtype=torch.uint8, device=W.device)
+        scales = torch.empty(o, n // 16, dtype=torch.uint8, device=W.device)
+        offs = torch.empty(o, n // 16, dtype=torch.int8, device=W.device) if want_offsets else None
+        h = None if hs is None else hs[i]
+        descs.append(SweepDesc(W.data_ptr(), o, n, W.stride(0), _ptr(h), Ss[i].data_ptr(),
+                               codes.data_ptr(), scales.data_ptr(), _ptr(offs)))
+        outs.append((codes, scales, offs))
+    nb = nvfp4_scale_sweep_quantize_batched_workspace_size(len(descs))
+    ws = _workspace(nb, Ws[0].device)
+    nvfp4_scale_sweep_quantize_batched(descs, lo, hi, ws, ws.numel(), stream)
+    return outs

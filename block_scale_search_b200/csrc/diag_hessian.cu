@@ -124,3 +124,151 @@ cudaError_t launch_diag_hessian(const uint16_t* X, int64_t T, int64_t in, int64_
 }
 
 }  // namespace nvfp4
+
+// ------------------------------------------------------------------------
+// Grouped diagonal Hessian: X holds the calibration rows of E experts one
+// after another (expert e owns rows row_offsets[e] .. row_offsets[e+1]) and
+// h[e, :] is each expert's own sum of squares -- one launch for all experts.
+// Rows are cut into chunks of kGroupedChunk rows that never straddle two
+// experts; a CTA sums one chunk for one strip of up to 256 16-byte column
+// vectors (a fixed-order reduction of its row lanes in shared memory) and
+// writes one partial row; the finalize kernel adds each expert's chunk rows in
+// chunk order in FP64 (deterministic) and rounds once.
+namespace nvfp4 {
+
+__global__ void grouped_chunk_starts_kernel(const int64_t* __restrict__ off, int64_t E,
+                                            int64_t total, int64_t cap,
+                                            int64_t* __restrict__ cstart) {
+  if (blockIdx.x != 0 || threadIdx.x != 0) return;
+  // cap = chunk rows the workspace holds; monotone offsets never reach it, and
+  // offsets that are not monotone cannot push a chunk past it
+  int64_t acc = 0;
+  for (int64_t e = 0; e < E; ++e) {
+    cstart[e] = acc < cap ? acc : cap;
+    int64_t a = off[e], b = off[e + 1];
+    a = a < 0 ? 0 : (a > total ? total : a);   // out-of-range offsets are clamped:
+    b = b < a ? a : (b > total ? total : b);   // no access can leave X
+    acc += (b - a + kGroupedChunk - 1) / kGroupedChunk;
+  }
+  cstart[E] = acc < cap ? acc : cap;
+}
+
+template <int U>
+__global__ void __launch_bounds__(256)
+diag_hessian_grouped_partial_kernel(const uint16_t* __restrict__ X, const int64_t* __restrict__ off,
+                                    const int64_t* __restrict__ cstart, int64_t E, int64_t total,
+                                    int64_t in, int64_t ldx, float* __restrict__ P) {
+  const int64_t q = blockIdx.x;            // chunk
+  const int64_t strip = blockIdx.y;        // 256 vectors per strip
+  if (q >= cstart[E]) return;
+  int64_t a = 0, z = E - 1;                // expert: last e with cstart[e] <= q
+  while (a < z) {
+    const int64_t mid = (a + z + 1) >> 1;
+    if (cstart[mid] <= q) a = mid; else z = mid - 1;
+  }
+  const int64_t e = a;
+  int64_t r_lo = off[e], r_hi = off[e + 1];
+  r_lo = r_lo < 0 ? 0 : (r_lo > total ? total : r_lo);
+  r_hi = r_hi < r_lo ? r_lo : (r_hi > total ? total : r_hi);
+  const int64_t rb = r_lo + (q - cstart[e]) * kGroupedChunk;
+  const int64_t re = (rb + kGroupedChunk < r_hi) ? rb + kGroupedChunk : r_hi;
+  const int64_t V = in / 8;
+  const int64_t v0 = strip * 256;
+  const int VLc = static_cast<int>((V - v0) < 256 ? (V - v0) : 256);
+  const int RL = 256 / VLc;
+  const int vl = threadIdx.x % VLc, rl = threadIdx.x / VLc;
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+  if (rl < RL) {
+    const uint16_t* col = X + (v0 + vl) * 8;
+    int64_t t = rb + rl;
+    for (; t + (U - 1) * RL < re; t += U * RL) {
+      uint4 qv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) qv[u] = ld_stream_v4(col + (t + u * RL) * ldx);
+      float s[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) s[c] = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float x0 = bf16_lo(w[k]), x1 = bf16_hi(w[k]);
+          s[2 * k] = fmaf(x0, x0, s[2 * k]);
+          s[2 * k + 1] = fmaf(x1, x1, s[2 * k + 1]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += s[c];
+    }
+    for (; t < re; t += RL) {
+      const uint4 qv = ld_stream_v4(col + t * ldx);
+      const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float x0 = bf16_lo(w[k]), x1 = bf16_hi(w[k]);
+        acc[2 * k] = fmaf(x0, x0, acc[2 * k]);
+        acc[2 * k + 1] = fmaf(x1, x1, acc[2 * k + 1]);
+      }
+    }
+  }
+  // fixed-order reduction over the row lanes of this CTA
+  __shared__ float red[256][9];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) red[threadIdx.x][c] = acc[c];
+  __syncthreads();
+  if (rl == 0) {
+    for (int r = 1; r < RL; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += red[r * VLc + vl][c];
+    float4* dst = reinterpret_cast<float4*>(P + q * in + (v0 + vl) * 8);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+__global__ void __launch_bounds__(256)
+diag_hessian_grouped_finalize_kernel(const float* __restrict__ P, const int64_t* __restrict__ cstart,
+                                     int64_t E, int64_t in, float* h, int accumulate) {
+  const int64_t e = blockIdx.y;
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= in || e >= E) return;
+  double s = accumulate ? static_cast<double>(h[e * in + j]) : 0.0;
+  double t = 0.0;
+  for (int64_t q = cstart[e]; q < cstart[e + 1]; ++q) t += P[q * in + j];
+  h[e * in + j] = static_cast<float>(s + t);
+}
+
+size_t diag_hessian_grouped_workspace_bytes(int64_t total, int64_t E, int64_t in) {
+  const int64_t chunks = (total + kGroupedChunk - 1) / kGroupedChunk + E;
+  const size_t head = ((static_cast<size_t>(E + 1) * sizeof(int64_t)) + 255) & ~size_t{255};
+  return head + static_cast<size_t>(chunks) * static_cast<size_t>(in) * sizeof(float);
+}
+
+cudaError_t launch_diag_hessian_grouped(const uint16_t* X, const int64_t* off, int64_t E,
+                                        int64_t total, int64_t in, int64_t ldx, float* h,
+                                        int accumulate, void* workspace, cudaStream_t stream) {
+  int64_t* cstart = static_cast<int64_t*>(workspace);
+  const size_t head = ((static_cast<size_t>(E + 1) * sizeof(int64_t)) + 255) & ~size_t{255};
+  float* P = reinterpret_cast<float*>(static_cast<char*>(workspace) + head);
+  const int64_t chunks = (total + kGroupedChunk - 1) / kGroupedChunk + E;
+  grouped_chunk_starts_kernel<<<1, 32, 0, stream>>>(off, E, total, chunks, cstart);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t strips = (in / 8 + 255) / 256;
+  if (total > 0) {
+    diag_hessian_grouped_partial_kernel<8><<<dim3(static_cast<unsigned>(chunks),
+                                                  static_cast<unsigned>(strips)),
+                                             256, 0, stream>>>(X, off, cstart, E, total, in, ldx, P);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  diag_hessian_grouped_finalize_kernel<<<dim3(static_cast<unsigned>((in + 255) / 256),
+                                              static_cast<unsigned>(E)),
+                                         256, 0, stream>>>(P, cstart, E, in, h, accumulate);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

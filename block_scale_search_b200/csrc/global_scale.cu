@@ -125,3 +125,105 @@ cudaError_t launch_global_scale(const uint16_t* W, int64_t out, int64_t ldw, flo
 }
 
 }  // namespace nvfp4
+
+// ------------------------------------------------------------------------
+// Batched global scale: one launch for many matrices.  CTA b works on the
+// matrix whose CTA range holds b, with that matrix's lane plan; per-CTA maxima
+// go to the workspace; one warp per matrix then reduces its CTAs' maxima and
+// writes S[m] (and amax[m], status[m]).
+namespace nvfp4 {
+
+__global__ void __launch_bounds__(256)
+absmax_batched_kernel(const MatDesc* __restrict__ d, int64_t n, uint32_t* __restrict__ partial) {
+  int64_t a = 0, z = n - 1;
+  while (a < z) {
+    const int64_t mid = (a + z + 1) >> 1;
+    if (d[mid].cta_begin <= static_cast<int64_t>(blockIdx.x)) a = mid; else z = mid - 1;
+  }
+  const MatDesc m = d[a];
+  const int64_t tid = (static_cast<int64_t>(blockIdx.x) - m.cta_begin) * blockDim.x + threadIdx.x;
+  uint32_t mx = 0;
+  if (tid < m.R * m.VL) {
+    const int64_t r = tid / m.VL;
+    const int64_t vl = tid - r * m.VL;
+    for (int64_t v = vl; v < m.V; v += m.VL) {
+      const uint16_t* col = m.W + v * 8;
+      int64_t t = r;
+      for (; t + 3 * m.R < m.out; t += 4 * m.R) {
+        uint4 q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = ld_stream_v4(col + (t + u * m.R) * m.ldw);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          mx = __vmaxu2(mx, q[u].x & 0x7FFF7FFFu);
+          mx = __vmaxu2(mx, q[u].y & 0x7FFF7FFFu);
+          mx = __vmaxu2(mx, q[u].z & 0x7FFF7FFFu);
+          mx = __vmaxu2(mx, q[u].w & 0x7FFF7FFFu);
+        }
+      }
+      for (; t < m.out; t += m.R) {
+        const uint4 q = ld_stream_v4(col + t * m.ldw);
+        mx = __vmaxu2(mx, q.x & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, q.y & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, q.z & 0x7FFF7FFFu);
+        mx = __vmaxu2(mx, q.w & 0x7FFF7FFFu);
+      }
+    }
+  }
+  mx = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  __shared__ uint32_t sm[8];
+  if ((threadIdx.x & 31) == 0) sm[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    mx = threadIdx.x < (blockDim.x >> 5) ? sm[threadIdx.x] : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (threadIdx.x == 0) partial[blockIdx.x] = mx;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+global_scale_batched_finalize_kernel(const MatDesc* __restrict__ d, int64_t n, int64_t total_ctas,
+                                     const uint32_t* __restrict__ partial, float q_max, float* S,
+                                     float* amax, int* status) {
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= n) return;
+  const int64_t c0 = d[m].cta_begin, c1 = (m + 1 < n) ? d[m + 1].cta_begin : total_ctas;
+  uint32_t mx = 0;
+  for (int64_t c = c0 + lane; c < c1; c += 32) mx = max(mx, partial[c]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  if (lane != 0) return;
+  if (mx >= 0x7F80u) {
+    S[m] = __uint_as_float(0x7FC00000u);
+    if (amax) amax[m] = __uint_as_float(0x7FC00000u);
+    if (status) status[m] = -5;  // NVFP4_ERR_NONFINITE
+    return;
+  }
+  const float a = __uint_as_float(mx << 16);
+  S[m] = (a == 0.0f) ? 0.0f : __fdiv_rn(a, __fmul_rn(q_max, 6.0f));
+  if (amax) amax[m] = a;
+  if (status) status[m] = 0;
+}
+
+int absmax_resident_ctas() {
+  static const int c = resident_ctas(reinterpret_cast<const void*>(&absmax_partial_kernel<4>), 256);
+  return c;
+}
+
+cudaError_t launch_global_scale_batched(const MatDesc* d_dev, int64_t n, int64_t total_ctas,
+                                        float q_max, float* S, float* amax, int* status,
+                                        uint32_t* partial, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  absmax_batched_kernel<<<static_cast<unsigned>(total_ctas), 256, 0, stream>>>(d_dev, n, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  global_scale_batched_finalize_kernel<<<static_cast<unsigned>((n + 7) / 8), 256, 0, stream>>>(
+      d_dev, n, total_ctas, partial, q_max, S, amax, status);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

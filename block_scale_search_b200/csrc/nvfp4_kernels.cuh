@@ -22,18 +22,52 @@ struct LanePlan {
 };
 
 LanePlan diag_hessian_plan(int64_t tokens, int64_t in, int num_sms);
+constexpr int64_t kGroupedChunk = 512;  // rows per chunk of the grouped diag-Hessian
+size_t diag_hessian_grouped_workspace_bytes(int64_t total, int64_t experts, int64_t in);
+cudaError_t launch_diag_hessian_grouped(const uint16_t* X, const int64_t* row_offsets, int64_t E,
+                                        int64_t total, int64_t in, int64_t ldx, float* h,
+                                        int accumulate, void* workspace, cudaStream_t stream);
 size_t diag_hessian_workspace_bytes(const LanePlan& p, int64_t in);
 cudaError_t launch_diag_hessian(const uint16_t* X, int64_t T, int64_t in, int64_t ldx, float* h,
                                 int accumulate, float* partials, const LanePlan& p,
                                 cudaStream_t stream);
 
 LanePlan global_scale_plan(int64_t out, int64_t in, int num_sms);
+int absmax_resident_ctas();
+
+// One matrix of a batched global scale, as the kernel reads it.
+struct MatDesc {
+  const uint16_t* W;
+  int64_t out, ldw;
+  int64_t V, VL, R;   // lane plan over 8-element vectors
+  int64_t cta_begin;  // first CTA of this matrix
+};
+cudaError_t launch_global_scale_batched(const MatDesc* d_dev, int64_t n, int64_t total_ctas,
+                                        float q_max, float* S, float* amax, int* status,
+                                        uint32_t* partial, cudaStream_t stream);
 size_t global_scale_workspace_bytes(const LanePlan& p);
 cudaError_t launch_global_scale(const uint16_t* W, int64_t out, int64_t ldw, float q_max,
                                 float* S, float* amax, int* status, uint32_t* partial,
                                 const LanePlan& p, cudaStream_t stream);
 
 LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted);
+LanePlan sweep_plan_threads(int64_t out, int64_t in, int64_t threads);
+int sweep_resident_ctas(bool weighted);
+constexpr int kSweepCta = 128;
+
+// One matrix of a batched sweep, as the kernel reads it from device memory.
+struct SweepDesc {
+  const uint16_t* W;
+  const float* h;
+  const float* S;
+  uint8_t* codes;
+  uint8_t* scales;
+  int8_t* offs;
+  int64_t out, G, ldw, GL, R;
+  int64_t cta_begin;  // first CTA of this matrix; CTAs up to the next matrix's
+};
+cudaError_t launch_scale_sweep_batched(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
+                                       bool weighted, int lo, int hi, cudaStream_t stream);
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi, uint8_t* codes,
                                uint8_t* scales, int8_t* offs, const LanePlan& p,

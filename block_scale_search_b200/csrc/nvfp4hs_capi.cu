@@ -9,6 +9,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <vector>
 
 #include "nvfp4_kernels.cuh"
 
@@ -165,6 +166,192 @@ int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S
   if (sms <= 0) return cuda_status(cudaErrorNoDevice);
   return cuda_status(nvfp4::launch_dequantize(codes, scales, S, out, in, W_out, sms,
                                               static_cast<cudaStream_t>(stream)));
+}
+
+
+// ------------------------------------------------------------- grouped / batched
+
+size_t nvfp4_diag_hessian_grouped_workspace_size(int64_t total_tokens, int64_t experts, int64_t in) {
+  if (total_tokens < 0 || experts <= 0 || experts > 65535 || in <= 0 || in % 8 != 0 ||
+      in > kMaxDim || total_tokens > kMaxDim)
+    return 0;
+  return nvfp4::diag_hessian_grouped_workspace_bytes(total_tokens, experts, in);
+}
+
+int nvfp4_diag_hessian_grouped(const void* X, const int64_t* row_offsets, int64_t experts,
+                               int64_t total_tokens, int64_t in, int64_t ldx, float* h,
+                               int accumulate, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  int st = check_diag_hessian(X, total_tokens, in, ldx, h, accumulate);
+  if (st != NVFP4_OK) return st;
+  if (row_offsets == nullptr || experts <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (experts > 65535) return NVFP4_ERR_SHAPE;
+  if (!aligned(row_offsets, 8)) return NVFP4_ERR_ALIGN;
+  if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  if (workspace_bytes < nvfp4::diag_hessian_grouped_workspace_bytes(total_tokens, experts, in))
+    return NVFP4_ERR_WORKSPACE;
+  return cuda_status(nvfp4::launch_diag_hessian_grouped(
+      static_cast<const uint16_t*>(X), row_offsets, experts, total_tokens, in, ldx, h, accumulate,
+      workspace, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+
+int check_batch(const nvfp4_matrix_desc* descs, int64_t n, int64_t in_multiple) {
+  if (n < 0 || (n > 0 && descs == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < n; ++i) {
+    const int st = check_matrix(descs[i].W, descs[i].out, descs[i].in, descs[i].ldw, in_multiple);
+    if (st != NVFP4_OK) return st;
+  }
+  return NVFP4_OK;
+}
+
+// CTAs per matrix: a one-wave budget shared in proportion to elements, >= 1 each.
+std::vector<int64_t> share_ctas(const std::vector<int64_t>& elems, int64_t budget) {
+  int64_t total = 0;
+  for (int64_t e : elems) total += e;
+  std::vector<int64_t> c(elems.size(), 1);
+  if (total > 0)
+    for (size_t i = 0; i < elems.size(); ++i) {
+      const double share = static_cast<double>(budget) * static_cast<double>(elems[i]) /
+                           static_cast<double>(total);
+      c[i] = share < 1.0 ? 1 : static_cast<int64_t>(share + 0.5);
+    }
+  return c;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t{255}; }
+
+struct GsBatchPlan {
+  std::vector<nvfp4::MatDesc> d;
+  int64_t total_ctas = 0;
+};
+
+GsBatchPlan plan_global_scale_batch(const nvfp4_matrix_desc* descs, int64_t n, int sms) {
+  GsBatchPlan p;
+  std::vector<int64_t> elems(n);
+  for (int64_t i = 0; i < n; ++i) elems[i] = descs[i].out * descs[i].in;
+  const std::vector<int64_t> ctas =
+      share_ctas(elems, static_cast<int64_t>(sms) * nvfp4::absmax_resident_ctas());
+  p.d.resize(n);
+  for (int64_t i = 0; i < n; ++i) {
+    nvfp4::MatDesc& m = p.d[i];
+    m.W = static_cast<const uint16_t*>(descs[i].W);
+    m.out = descs[i].out;
+    m.ldw = descs[i].ldw;
+    m.V = descs[i].in / 8;
+    const int64_t nt = ctas[i] * 256;
+    m.VL = m.V < nt ? (m.V > 0 ? m.V : 1) : nt;
+    int64_t R = nt / m.VL;
+    if (R > m.out) R = m.out;
+    if (R < 1) R = 1;
+    m.R = R;
+    m.cta_begin = p.total_ctas;
+    p.total_ctas += ctas[i];
+  }
+  return p;
+}
+
+}  // namespace
+
+size_t nvfp4_global_scale_batched_workspace_size(const nvfp4_matrix_desc* descs, int64_t n) {
+  if (check_batch(descs, n, 8) != NVFP4_OK) return 0;
+  const int sms = current_sm_count();
+  if (sms <= 0) return 0;
+  const GsBatchPlan p = plan_global_scale_batch(descs, n, sms);
+  return round256(static_cast<size_t>(n) * sizeof(nvfp4::MatDesc)) +
+         static_cast<size_t>(p.total_ctas) * sizeof(uint32_t) + 256;
+}
+
+int nvfp4_global_scale_batched(const nvfp4_matrix_desc* descs, int64_t n, float q_max, float* S,
+                               float* amax, int* status, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  int st = check_batch(descs, n, 8);
+  if (st != NVFP4_OK) return st;
+  if (n == 0) return NVFP4_OK;
+  if (S == nullptr || !std::isfinite(q_max) || !(q_max > 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(S, 4) || !aligned(amax, 4) || !aligned(status, 4)) return NVFP4_ERR_ALIGN;
+  if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  const GsBatchPlan p = plan_global_scale_batch(descs, n, sms);
+  const size_t head = round256(static_cast<size_t>(n) * sizeof(nvfp4::MatDesc));
+  if (workspace_bytes < head + static_cast<size_t>(p.total_ctas) * sizeof(uint32_t))
+    return NVFP4_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  nvfp4::MatDesc* d_dev = static_cast<nvfp4::MatDesc*>(workspace);
+  // the table is staged from host memory before this call returns
+  cudaError_t e = cudaMemcpyAsync(d_dev, p.d.data(), static_cast<size_t>(n) * sizeof(nvfp4::MatDesc),
+                                  cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  uint32_t* partial = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + head);
+  return cuda_status(nvfp4::launch_global_scale_batched(d_dev, n, p.total_ctas, q_max, S, amax,
+                                                        status, partial, s));
+}
+
+size_t nvfp4_scale_sweep_quantize_batched_workspace_size(int64_t n) {
+  if (n < 0) return 0;
+  return round256(static_cast<size_t>(n) * sizeof(nvfp4::SweepDesc)) + 256;
+}
+
+int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n, int lo, int hi,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (n < 0 || (n > 0 && descs == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  bool any_h = false, all_h = true;
+  std::vector<int64_t> groups(n);
+  for (int64_t i = 0; i < n; ++i) {
+    const nvfp4_sweep_desc& d = descs[i];
+    int st = check_matrix(d.W, d.out, d.in, d.ldw, 16);
+    if (st != NVFP4_OK) return st;
+    const bool empty = d.out == 0 || d.in == 0;
+    if (!empty && (d.S == nullptr || d.codes == nullptr || d.scales == nullptr))
+      return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(d.h, 16) || !aligned(d.S, 4) || !aligned(d.codes, 8)) return NVFP4_ERR_ALIGN;
+    any_h = any_h || d.h != nullptr;
+    all_h = all_h && d.h != nullptr;
+    groups[i] = empty ? 0 : d.out * (d.in / 16);
+  }
+  if (any_h && !all_h) return NVFP4_ERR_INVALID_ARG;  // one objective per batch
+  if (n == 0) return NVFP4_OK;
+  if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  if (workspace_bytes < round256(static_cast<size_t>(n) * sizeof(nvfp4::SweepDesc)))
+    return NVFP4_ERR_WORKSPACE;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  const bool weighted = any_h;
+  const std::vector<int64_t> ctas =
+      share_ctas(groups, static_cast<int64_t>(sms) * nvfp4::sweep_resident_ctas(weighted));
+  std::vector<nvfp4::SweepDesc> dv(n);
+  int64_t total_ctas = 0;
+  for (int64_t i = 0; i < n; ++i) {
+    const nvfp4_sweep_desc& d = descs[i];
+    nvfp4::SweepDesc& m = dv[i];
+    const int64_t c = groups[i] == 0 ? 1 : ctas[i];
+    const nvfp4::LanePlan p = nvfp4::sweep_plan_threads(d.out, d.in, c * nvfp4::kSweepCta);
+    m.W = static_cast<const uint16_t*>(d.W);
+    m.h = d.h;
+    m.S = d.S;
+    m.codes = d.codes;
+    m.scales = d.scales;
+    m.offs = d.chosen_offset;
+    m.out = groups[i] == 0 ? 0 : d.out;  // an empty matrix does no work
+    m.G = d.in / 16;
+    m.ldw = d.ldw;
+    m.GL = p.VL;
+    m.R = p.R;
+    m.cta_begin = total_ctas;
+    total_ctas += c;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  nvfp4::SweepDesc* d_dev = static_cast<nvfp4::SweepDesc*>(workspace);
+  cudaError_t e = cudaMemcpyAsync(d_dev, dv.data(), static_cast<size_t>(n) * sizeof(nvfp4::SweepDesc),
+                                  cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(nvfp4::launch_scale_sweep_batched(d_dev, n, total_ctas, weighted, lo, hi, s));
 }
 
 }  // extern "C"

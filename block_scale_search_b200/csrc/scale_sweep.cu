@@ -168,25 +168,38 @@ __device__ __forceinline__ uint32_t exact_e2m1_one(float xl, float a, float v, f
 
 // ------------------------------------------------------------------ kernel
 
-template <bool kWeighted>
-__global__ void __launch_bounds__(kCta, 5)
-scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64_t ldw,
-                   const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
-                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                   int8_t* __restrict__ offs, int64_t GL, int64_t R) {
-  __shared__ CandEntry tab[kTabSize];
-  __shared__ float Lsm[16][kCta];       // per-thread column of fast losses
-  __shared__ uint4 wbuf[2][2][kCta];    // staged groups: [buffer][half][thread]
-  __shared__ double tsm[kCta / 32][16]; // per-warp exchange of exact loss terms
+// Shared memory of one sweep CTA.
+struct SweepSmem {
+  CandEntry tab[kTabSize];
+  float Lsm[16][kCta];        // per-thread column of fast losses
+  uint4 wbuf[2][2][kCta];     // staged groups: [buffer][half][thread]
+  double tsm[kCta / 32][16];  // per-warp exchange of exact loss terms
+};
+
+__device__ __forceinline__ void fill_candidate_table(CandEntry* tab) {
   for (int i = threadIdx.x; i < kTabSize; i += blockDim.x) {
     const int c = clamp_code(i - kTabOffset);
     const float v = e4m3_value(c);
     const uint32_t nvh = __half_as_ushort(__float2half_rn(-v));
     tab[i] = CandEntry{v, __frcp_rn(v), nvh | (nvh << 16), static_cast<uint32_t>(c)};
   }
-  __syncthreads();
+}
 
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+// The sweep of one matrix by one thread lane: `tid` in [0, R*GL) is the
+// thread's position in the lane grid that covers this matrix.
+template <bool kWeighted>
+__device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __restrict__ W,
+                                             int64_t out, int64_t G, int64_t ldw,
+                                             const float* __restrict__ h,
+                                             const float* __restrict__ Sp, int lo, int hi,
+                                             uint8_t* __restrict__ codes,
+                                             uint8_t* __restrict__ scales,
+                                             int8_t* __restrict__ offs, int64_t GL, int64_t R,
+                                             int64_t tid) {
+  const CandEntry* tab = sm.tab;
+  auto& Lsm = sm.Lsm;
+  auto& wbuf = sm.wbuf;
+  auto& tsm = sm.tsm;
   if (tid >= R * GL) return;
   const int64_t r0 = tid / GL;
   const int64_t gl = tid - r0 * GL;
@@ -388,13 +401,64 @@ scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64
   cp_async_wait<0>();
 }
 
-LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted) {
+template <bool kWeighted>
+__global__ void __launch_bounds__(kCta, 5)
+scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64_t ldw,
+                   const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
+                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                   int8_t* __restrict__ offs, int64_t GL, int64_t R) {
+  __shared__ SweepSmem sm;
+  fill_candidate_table(sm.tab);
+  __syncthreads();
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  sweep_matrix<kWeighted>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, GL, R, tid);
+}
+
+// Batched sweep: CTA b belongs to the matrix whose [cta_begin, next cta_begin)
+// range holds b (binary search); within it, lanes follow that matrix's plan.
+template <bool kWeighted>
+__global__ void __launch_bounds__(kCta, 5)
+scale_sweep_batched_kernel(const SweepDesc* __restrict__ d, int64_t n, int lo, int hi) {
+  __shared__ SweepSmem sm;
+  fill_candidate_table(sm.tab);
+  __syncthreads();
+  int64_t a = 0, z = n - 1;  // last descriptor with cta_begin <= blockIdx.x
+  while (a < z) {
+    const int64_t mid = (a + z + 1) >> 1;
+    if (d[mid].cta_begin <= static_cast<int64_t>(blockIdx.x)) a = mid; else z = mid - 1;
+  }
+  const SweepDesc m = d[a];
+  const int64_t tid = (static_cast<int64_t>(blockIdx.x) - m.cta_begin) * kCta + threadIdx.x;
+  sweep_matrix<kWeighted>(sm, m.W, m.out, m.G, m.ldw, m.h, m.S, lo, hi, m.codes, m.scales,
+                          m.offs, m.GL, m.R, tid);
+}
+
+int sweep_resident_ctas(bool weighted) {
   static const int ctas[2] = {
       resident_ctas(reinterpret_cast<const void*>(&scale_sweep_kernel<false>), kCta),
       resident_ctas(reinterpret_cast<const void*>(&scale_sweep_kernel<true>), kCta)};
+  return ctas[weighted];
+}
+
+cudaError_t launch_scale_sweep_batched(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
+                                       bool weighted, int lo, int hi, cudaStream_t stream) {
+  if (n == 0 || total_ctas == 0) return cudaSuccess;
+  if (weighted)
+    scale_sweep_batched_kernel<true><<<static_cast<unsigned>(total_ctas), kCta, 0, stream>>>(
+        d_dev, n, lo, hi);
+  else
+    scale_sweep_batched_kernel<false><<<static_cast<unsigned>(total_ctas), kCta, 0, stream>>>(
+        d_dev, n, lo, hi);
+  return cudaGetLastError();
+}
+
+LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted) {
+  return sweep_plan_threads(out, in, static_cast<int64_t>(num_sms) * sweep_resident_ctas(weighted) * kCta);
+}
+
+LanePlan sweep_plan_threads(int64_t out, int64_t in, int64_t nt) {
   LanePlan p;
   p.V = in / 16;  // column groups per row
-  const int64_t nt = static_cast<int64_t>(num_sms) * ctas[weighted] * kCta;
   p.VL = p.V < nt ? (p.V > 0 ? p.V : 1) : nt;
   int64_t R = nt / p.VL;
   if (R > out) R = out;

@@ -150,6 +150,71 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
                                void* stream);
 
 /* ------------------------------------------------------------------------
+ * Grouped and batched forms: one launch for many matrices, as in a
+ * mixture-of-experts layer whose experts each see their own slice of the
+ * calibration tokens and get their own h and S.  Each computes exactly what
+ * the single-matrix call computes for every member (bit-identical outputs for
+ * the global scale and the sweep; h to the same tolerance, summed in a
+ * different fixed order).
+ * ------------------------------------------------------------------------ */
+
+/* Diagonal Hessian per expert (H-Scale summary, sec. B; one statistic per
+ * expert).  X holds the experts' calibration rows back to back:
+ *   expert e owns rows row_offsets[e] .. row_offsets[e+1]-1 of X[total_tokens, ldx].
+ *   row_offsets  DEVICE int64 [experts+1], non-decreasing, within [0, total_tokens]
+ *                (offsets outside that are clamped; a decreasing table gives
+ *                undefined h but never an out-of-bounds access), 8-byte aligned.
+ *   experts      1 .. 65535.
+ *   h            float [experts, in] (row e = expert e), accumulate as above.
+ *   workspace    at least nvfp4_diag_hessian_grouped_workspace_size() bytes,
+ *                256-byte aligned; contents need no initialisation.
+ * Other arguments as nvfp4_diag_hessian. */
+size_t nvfp4_diag_hessian_grouped_workspace_size(int64_t total_tokens, int64_t experts, int64_t in);
+int nvfp4_diag_hessian_grouped(const void* X, const int64_t* row_offsets, int64_t experts,
+                               int64_t total_tokens, int64_t in, int64_t ldx, float* h,
+                               int accumulate, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* One weight matrix of a batch: device pointer, shape, leading dimension. */
+typedef struct nvfp4_matrix_desc {
+    const void* W;
+    int64_t out, in, ldw;
+} nvfp4_matrix_desc;
+
+/* Global scale of n matrices (ScaleSweep summary, sec. 2), one per matrix.
+ *   descs        HOST array of n descriptors (read before the call returns).
+ *   S            DEVICE float [n]; amax, status: DEVICE [n] or NULL.
+ *   workspace    at least nvfp4_global_scale_batched_workspace_size(descs, n)
+ *                bytes, 256-byte aligned: a device copy of the table plus one
+ *                partial maximum per CTA.
+ * Each descriptor is checked as nvfp4_global_scale checks its arguments. */
+size_t nvfp4_global_scale_batched_workspace_size(const nvfp4_matrix_desc* descs, int64_t n);
+int nvfp4_global_scale_batched(const nvfp4_matrix_desc* descs, int64_t n, float q_max, float* S,
+                               float* amax, int* status, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* One matrix of a batched sweep: the arguments of nvfp4_scale_sweep_quantize. */
+typedef struct nvfp4_sweep_desc {
+    const void* W;
+    int64_t out, in, ldw;
+    const float* h;          /* NULL = plain MSE; all NULL or all non-NULL */
+    const float* S;          /* device scalar */
+    uint8_t* codes;
+    uint8_t* scales;
+    int8_t* chosen_offset;   /* may be NULL */
+} nvfp4_sweep_desc;
+
+/* Windowed sweep of n matrices with one window [lo, hi] (H-Scale summary,
+ * sec. 3 and B).
+ *   descs        HOST array of n descriptors (read before the call returns).
+ *   workspace    at least nvfp4_scale_sweep_quantize_batched_workspace_size(n)
+ *                bytes, 256-byte aligned (a device copy of the table).
+ * A batch mixing NULL and non-NULL h returns NVFP4_ERR_INVALID_ARG. */
+size_t nvfp4_scale_sweep_quantize_batched_workspace_size(int64_t n);
+int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n, int lo, int hi,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Dequantize (NVFP4 decode, H-Scale summary sec. 3: effective scale = global
  * x local): W_out[r, j] = sign * fl32(g[k] * v(scale)) * S, float [out, in].
  *   codes [out, in/2] 8-byte aligned; scales [out, in/16]; S device scalar;

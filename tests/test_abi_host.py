@@ -119,3 +119,43 @@ def test_binding_has_same_names_as_abi():
         if n == "nvfp4_last_cuda_error":
             continue
         assert hasattr(m, n), n
+
+
+def test_grouped_and_batched_validation(L):
+    import block_scale_search_b200 as nv
+    f = L.nvfp4_diag_hessian_grouped
+    f.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_int64, C.c_int64, C.c_int64, C.c_void_p,
+                  C.c_int, C.c_void_p, C.c_size_t, C.c_void_p]
+    ws = 0x100000
+    assert f(P, None, 4, 100, 64, 64, P, 0, ws, 1 << 30, None) == -1        # no offsets
+    assert f(P, P, 0, 100, 64, 64, P, 0, ws, 1 << 30, None) == -1           # no experts
+    assert f(P, P, 70000, 100, 64, 64, P, 0, ws, 1 << 30, None) == -2       # too many experts
+    assert f(P, P + 4, 4, 100, 64, 64, P, 0, ws, 1 << 30, None) == -3       # offsets misaligned
+    assert f(P, P, 4, 100, 64, 64, P, 0, ws + 16, 1 << 30, None) == -3      # workspace alignment
+    assert f(P, P, 4, 100, 64, 64, P, 0, ws, 16, None) == -7                # workspace too small
+    assert L.nvfp4_diag_hessian_grouped_workspace_size(100, 4, 64) >= 4 * 64 * 4
+
+    g = L.nvfp4_global_scale_batched
+    good = [nv.MatrixDesc(P, 4, 16, 16), nv.MatrixDesc(P, 2, 32, 40)]
+    arr = (nv.MatrixDesc * 2)(*good)
+    bad = (nv.MatrixDesc * 2)(nv.MatrixDesc(P, 4, 16, 16), nv.MatrixDesc(P + 2, 2, 32, 40))
+    assert g(bad, 2, 448.0, P, None, None, ws, 1 << 20, None) == -3
+    bad = (nv.MatrixDesc * 1)(nv.MatrixDesc(P, 4, 12, 16))
+    assert g(bad, 1, 448.0, P, None, None, ws, 1 << 20, None) == -2
+    assert g(None, 3, 448.0, P, None, None, ws, 1 << 20, None) == -1
+    assert g(arr, 2, 0.0, P, None, None, ws, 1 << 20, None) == -1
+    assert g(arr, 0, 448.0, P, None, None, None, 0, None) == 0             # empty batch
+
+    s = L.nvfp4_scale_sweep_quantize_batched
+    d = [nv.SweepDesc(P, 4, 32, 32, P, P, P, P, None), nv.SweepDesc(P, 4, 32, 32, None, P, P, P, None)]
+    arr = (nv.SweepDesc * 2)(*d)
+    assert s(arr, 2, -9, 6, ws, 1 << 20, None) == -1                        # mixed objectives
+    arr1 = (nv.SweepDesc * 1)(d[0])
+    assert s(arr1, 1, -9, 7, ws, 1 << 20, None) == -4                       # window too wide
+    arr1 = (nv.SweepDesc * 1)(nv.SweepDesc(P, 4, 24, 32, None, P, P, P, None))
+    assert s(arr1, 1, -9, 6, ws, 1 << 20, None) == -2                       # in % 16
+    arr1 = (nv.SweepDesc * 1)(nv.SweepDesc(P, 4, 32, 32, P + 4, P, P, P, None))
+    assert s(arr1, 1, -9, 6, ws, 1 << 20, None) == -3                       # h alignment
+    arr1 = (nv.SweepDesc * 1)(d[1])
+    assert s(arr1, 1, -9, 6, None, 0, None) == -7                           # no workspace
+    assert s(None, 0, -9, 6, None, 0, None) == 0                            # empty batch
