@@ -122,6 +122,13 @@ class ClockSampler:
 
 def build_layer(rank: int, device, name: str = "llama33_70b_mlp"):
     import torch
+    if name == "moe_grouped":
+        import workloads
+        wl = workloads.moe_grouped(device=device)
+        Ws = {m.name: m.make(device) for m in wl.matrices}
+        Xs = {k: c.make(device) for k, c in wl.calibs.items()}
+        torch.cuda.synchronize()
+        return wl, Ws, Xs
     wl = rank_workload(rank, name)
     Ws = {m.name: m.make(device) for m in wl.matrices}
     Xs = {k: c.make(device) for k, c in wl.calibs.items()}
@@ -180,6 +187,83 @@ class Step:
             rec("scale_sweep", lambda W=W, n=n: nv.nvfp4_scale_sweep_quantize(
                 W, W.shape[0], W.shape[1], W.stride(0), self.h[self.x_of[n]], self.S[n], LO, HI,
                 self.codes[n], self.scales[n], None, stream))
+
+
+class GroupedStep:
+    """Mixture-of-experts layer: one grouped diag-Hessian launch per
+    calibration tensor, one batched global scale and one batched sweep for all
+    matrices.  Descriptor tables are built once; run() calls the C ABI."""
+
+    def __init__(self, nv, wl, Ws, Xs, device):
+        import ctypes as C
+        import torch
+        self.nv, self.wl, self.Ws, self.Xs = nv, wl, Ws, Xs
+        L = nv.lib()
+        self.L = L
+        offs = wl.calibs[next(iter(wl.calibs))].row_offsets
+        self.E = len(offs) - 1
+        self.off = torch.tensor(offs, dtype=torch.int64, device=device)
+        self.h = {k: torch.empty(self.E, X.shape[1], dtype=torch.float32, device=device)
+                  for k, X in Xs.items()}
+        self.hws = {k: torch.empty(nv.nvfp4_diag_hessian_grouped_workspace_size(X.shape[0], self.E,
+                                                                                X.shape[1]),
+                                   dtype=torch.uint8, device=device) for k, X in Xs.items()}
+        mats = wl.matrices
+        n = len(mats)
+        self.n = n
+        self.mdesc = (nv.MatrixDesc * n)(*[nv.MatrixDesc(Ws[m.name].data_ptr(), m.out, m.inp, m.inp)
+                                          for m in mats])
+        self.S = torch.empty(n, dtype=torch.float32, device=device)
+        self.amax = torch.empty(n, dtype=torch.float32, device=device)
+        self.status = torch.empty(n, dtype=torch.int32, device=device)
+        self.gws = torch.empty(L.nvfp4_global_scale_batched_workspace_size(self.mdesc, n),
+                               dtype=torch.uint8, device=device)
+        self.codes = {m.name: torch.empty(m.out, m.inp // 2, dtype=torch.uint8, device=device)
+                      for m in mats}
+        self.scales = {m.name: torch.empty(m.out, m.inp // 16, dtype=torch.uint8, device=device)
+                       for m in mats}
+        sdesc = []
+        for i, m in enumerate(mats):
+            hrow = self.h[m.x_key][m.expert]
+            sdesc.append(nv.SweepDesc(Ws[m.name].data_ptr(), m.out, m.inp, m.inp, hrow.data_ptr(),
+                                      self.S.data_ptr() + 4 * i, self.codes[m.name].data_ptr(),
+                                      self.scales[m.name].data_ptr(), None))
+        self.sdesc = (nv.SweepDesc * n)(*sdesc)
+        self.sws = torch.empty(L.nvfp4_scale_sweep_quantize_batched_workspace_size(n),
+                               dtype=torch.uint8, device=device)
+        self.launches_per_step = 3 * len(Xs) + 2 + 1
+
+    def run(self, ev=None):
+        import torch
+        L = self.L
+        stream = torch.cuda.current_stream()
+        sp = stream.cuda_stream
+
+        def rec(kind, fn):
+            if ev is None:
+                fn()
+                return
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev.setdefault(kind, []).append((a, b))
+
+        def chk(st):
+            if st != 0:
+                raise RuntimeError(f"status {st}")
+
+        for k, X in self.Xs.items():
+            ws = self.hws[k]
+            rec("diag_hessian", lambda X=X, k=k, ws=ws: chk(L.nvfp4_diag_hessian_grouped(
+                X.data_ptr(), self.off.data_ptr(), self.E, X.shape[0], X.shape[1], X.stride(0),
+                self.h[k].data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)))
+        rec("global_scale", lambda: chk(L.nvfp4_global_scale_batched(
+            self.mdesc, self.n, float(self.wl.q_max), self.S.data_ptr(), self.amax.data_ptr(),
+            self.status.data_ptr(), self.gws.data_ptr(), self.gws.numel(), sp)))
+        rec("scale_sweep", lambda: chk(L.nvfp4_scale_sweep_quantize_batched(
+            self.sdesc, self.n, LO, HI, self.sws.data_ptr(), self.sws.numel(), sp)))
 
 
 def profiled_traffic(kernel: str, units_per_launch: float):
@@ -290,6 +374,9 @@ WORKLOADS = {
                         "channel scales"),
     "mlp_slice": ("mlp_slice (profiling size): W 8192x8192 bf16 N(0,0.015) 0.1% x10; X 16384 x "
                   "8192 bf16 lognormal(1.5) channel scales"),
+    "moe_grouped": ("moe_grouped: 128 experts x {gate, up 768x2048; down 2048x768} bf16 N(0,0.02) "
+                    "0.1% x10; 262144 tokens routed top-8 (Zipf 1.1), per-expert X slices and h; "
+                    "grouped diag-Hessian + batched global scale + batched sweep"),
 }
 
 
@@ -350,7 +437,7 @@ def main():
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     wl, Ws, Xs = build_layer(rank, dev, args.workload)
-    step = Step(nv, wl, Ws, Xs, dev)
+    step = (GroupedStep if args.workload == "moe_grouped" else Step)(nv, wl, Ws, Xs, dev)
 
     for _ in range(args.warmup):
         step.run()
@@ -390,12 +477,15 @@ def main():
     value = wel * ws / (ms_max * 1e-3)
 
     # ---- status of the quantized tensors (non-finite check) and sanity
-    for n in Ws:
-        assert int(step.status[n].item()) == 0, f"non-finite weights in {n}"
+    if isinstance(step.status, dict):
+        for n in Ws:
+            assert int(step.status[n].item()) == 0, f"non-finite weights in {n}"
+    else:
+        assert not step.status.any().item(), "non-finite weights"
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and args.workload != "moe_grouped":
         hostW = {n: W.cpu().pin_memory() for n, W in Ws.items()}
         hostX = {k: X.cpu().pin_memory() for k, X in Xs.items()}
         hostC = {n: torch.empty_like(c, device="cpu").pin_memory() for n, c in step.codes.items()}

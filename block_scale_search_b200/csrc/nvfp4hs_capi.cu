@@ -323,8 +323,11 @@ int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n,
   const int sms = current_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorNoDevice);
   const bool weighted = any_h;
+  // four waves' worth of CTAs shared by size: with many small matrices a
+  // one-wave share rounds to whole CTAs and can spill a few into a mostly
+  // empty second wave; at four waves that tail is a small fraction of a wave
   const std::vector<int64_t> ctas =
-      share_ctas(groups, static_cast<int64_t>(sms) * nvfp4::sweep_resident_ctas(weighted));
+      share_ctas(groups, 4 * static_cast<int64_t>(sms) * nvfp4::sweep_resident_ctas(weighted));
   std::vector<nvfp4::SweepDesc> dv(n);
   int64_t total_ctas = 0;
   for (int64_t i = 0; i < n; ++i) {
