@@ -51,10 +51,10 @@ namespace nvfp4 {
 // Per-code table in shared memory, indexed by code + 16 so that b + k for
 // k in [-16, 15] needs no clamping (entries beyond the ends repeat codes 1/126).
 struct CandEntry {
-  float v;        // E4M3 value of the (clamped) code
   float iv;       // 1 / v, correctly rounded
+  float iv2;      // the same again, so {iv, iv} loads as one f32x2 operand
   uint32_t nvh;   // -v as f16 bits (exact: E4M3 values are f16 values)
-  uint32_t code;  // the clamped code
+  float v;        // E4M3 value of the (clamped) code
 };
 constexpr int kTabOffset = 16;
 constexpr int kTabSize = 160;
@@ -131,11 +131,12 @@ __device__ __forceinline__ float weight_scale(float hmax) {
 
 // Fast FP32 loss of one candidate: E2M1 round of y/v by the hardware
 // conversion, decode, exact-product error, weighted square, two accumulators.
+template <bool kWeighted>
 __device__ __forceinline__ float fast_candidate_loss(const f32x2_t (&y2)[8], const f32x2_t (&h2)[8],
                                                      const CandEntry& t) {
-  const f32x2_t iv2 = f2_pack(t.iv, t.iv);
+  const f32x2_t iv2 = *reinterpret_cast<const f32x2_t*>(&t.iv);  // {iv, iv}
   const uint16_t nv = static_cast<uint16_t>(t.nvh);
-  f32x2_t acc0 = f2_pack(0.0f, 0.0f), acc1 = acc0;
+  f32x2_t acc0, acc1;
 #pragma unroll
   for (int pj = 0; pj < 8; ++pj) {
     float x0, x1, y0, y1;
@@ -145,13 +146,16 @@ __device__ __forceinline__ float fast_candidate_loss(const f32x2_t (&y2)[8], con
     const float e0 = fma_f16_f32(static_cast<uint16_t>(qh & 0xFFFFu), nv, y0);
     const float e1 = fma_f16_f32(static_cast<uint16_t>(qh >> 16), nv, y1);
     const f32x2_t e2 = f2_pack(e0, e1);
-    if (pj & 1) acc1 = f2_fma(f2_mul(h2[pj], e2), e2, acc1);
-    else acc0 = f2_fma(f2_mul(h2[pj], e2), e2, acc0);
+    // plain MSE (h == 1) needs no weighting multiply
+    const f32x2_t he2 = kWeighted ? f2_mul(h2[pj], e2) : e2;
+    if (pj == 0) acc0 = f2_mul(he2, e2);
+    else if (pj == 1) acc1 = f2_mul(he2, e2);
+    else if (pj & 1) acc1 = f2_fma(he2, e2, acc1);
+    else acc0 = f2_fma(he2, e2, acc0);
   }
-  float a0, a1, b0, b1;
-  f2_unpack(acc0, a0, a1);
-  f2_unpack(acc1, b0, b1);
-  return (a0 + a1) + (b0 + b1);
+  float a0, a1;
+  f2_unpack(f2_add(acc0, acc1), a0, a1);
+  return a0 + a1;
 }
 
 // ------------------------------------------------------- stage 2 (exact)
@@ -180,8 +184,9 @@ __device__ __forceinline__ void fill_candidate_table(CandEntry* tab) {
   for (int i = threadIdx.x; i < kTabSize; i += blockDim.x) {
     const int c = clamp_code(i - kTabOffset);
     const float v = e4m3_value(c);
+    const float iv = __frcp_rn(v);
     const uint32_t nvh = __half_as_ushort(__float2half_rn(-v));
-    tab[i] = CandEntry{v, __frcp_rn(v), nvh | (nvh << 16), static_cast<uint32_t>(c)};
+    tab[i] = CandEntry{iv, iv, nvh | (nvh << 16), v};
   }
 }
 
@@ -278,7 +283,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
       if (nonzero) {
         f32x2_t A2 = f2_pack(0.0f, 0.0f);  // sum h' y^2, for the error bound of stage 2
 #pragma unroll
-        for (int i = 0; i < 8; ++i) A2 = f2_fma(f2_mul(h2[i], y2[i]), y2[i], A2);
+        for (int i = 0; i < 8; ++i) A2 = f2_fma(kWeighted ? f2_mul(h2[i], y2[i]) : y2[i], y2[i], A2);
         float A0, A1;
         f2_unpack(A2, A0, A1);
         const float A = A0 + A1;
@@ -297,7 +302,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
         // ---- stage 1: fast FP32 losses of all candidates
         float best = __uint_as_float(0x7F800000u), second = best;
         for (int i = 0; i < K; ++i) {
-          const float Li = fast_candidate_loss(y2, h2, ce[i]);
+          const float Li = fast_candidate_loss<kWeighted>(y2, h2, ce[i]);
           Lsm[i][lane] = Li;
           if (Li < best) { second = best; best = Li; bi = i; }
           else if (Li < second) { second = Li; }
@@ -393,7 +398,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
         packed[pj >> 2] |= (nib | (sgn & nz)) << (8 * (pj & 3));
       }
       *reinterpret_cast<uint2*>(cdst) = make_uint2(packed[0], packed[1]);
-      scales[gi] = static_cast<uint8_t>(win.code);
+      scales[gi] = static_cast<uint8_t>(clamp_code(b + lo + bi));
       // ascending offsets + strict "<": lo + bi is the lowest offset reaching it
       if (offs) offs[gi] = static_cast<int8_t>(lo + bi);
     }
