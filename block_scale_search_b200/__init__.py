@@ -24,6 +24,7 @@ __all__ = [
     "nvfp4_diag_hessian_grouped", "nvfp4_global_scale_batched_workspace_size",
     "nvfp4_global_scale_batched", "nvfp4_scale_sweep_quantize_batched_workspace_size",
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
+    "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize",
     "diag_hessian", "global_scale", "scale_sweep_quantize", "dequantize", "quantize_layer",
@@ -72,6 +73,8 @@ _SIGS = {
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
+    "nvfp4_scale_sweep_quantize_full": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp],
+                                        _int),
     "nvfp4_diag_hessian_grouped_workspace_size": ([_i64, _i64, _i64], _sz),
     "nvfp4_diag_hessian_grouped": ([_vp, _vp, _i64, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp],
                                    _int),
@@ -160,6 +163,13 @@ def nvfp4_scale_sweep_quantize(W, out, inp, ldw, h, S, lo, hi, codes, scales, ch
     _check("nvfp4_scale_sweep_quantize", lib().nvfp4_scale_sweep_quantize(
         _ptr(W), out, inp, ldw, _ptr(h), _ptr(S), int(lo), int(hi), _ptr(codes), _ptr(scales),
         _ptr(chosen_offset), _stream(stream)))
+
+
+def nvfp4_scale_sweep_quantize_full(W, out, inp, ldw, h, S, codes, scales, chosen_offset,
+                                    stream=None):
+    _check("nvfp4_scale_sweep_quantize_full", lib().nvfp4_scale_sweep_quantize_full(
+        _ptr(W), out, inp, ldw, _ptr(h), _ptr(S), _ptr(codes), _ptr(scales), _ptr(chosen_offset),
+        _stream(stream)))
 
 
 def nvfp4_dequantize(codes, scales, S, out, inp, W_out, stream=None):
@@ -267,6 +277,18 @@ def scale_sweep_quantize(W: torch.Tensor, h: torch.Tensor | None, S: torch.Tenso
     else:
         codes, scales, offs = out
     nvfp4_scale_sweep_quantize(W, o, n, W.stride(0), h, S, lo, hi, codes, scales, offs, stream)
+    return codes, scales, offs
+
+
+def scale_sweep_quantize_full(W: torch.Tensor, h: torch.Tensor | None, S: torch.Tensor,
+                              want_offsets: bool = False, stream=None):
+    """Sweep over all 126 positive E4M3 codes: (codes, scales, offsets or None)."""
+    W = _bf16_2d(W, "W")
+    o, n = W.shape
+    codes = torch.empty(o, n // 2, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(o, n // 16, dtype=torch.uint8, device=W.device)
+    offs = torch.empty(o, n // 16, dtype=torch.int8, device=W.device) if want_offsets else None
+    nvfp4_scale_sweep_quantize_full(W, o, n, W.stride(0), h, S, codes, scales, offs, stream)
     return codes, scales, offs
 
 

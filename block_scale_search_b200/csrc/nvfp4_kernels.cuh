@@ -66,6 +66,10 @@ struct SweepDesc {
   int64_t out, G, ldw, GL, R;
   int64_t cta_begin;  // first CTA of this matrix; CTAs up to the next matrix's
 };
+cudaError_t launch_scale_sweep_full(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
+                                    const float* h, const float* S, uint8_t* codes,
+                                    uint8_t* scales, int8_t* offs, int num_sms,
+                                    cudaStream_t stream);
 cudaError_t launch_scale_sweep_batched(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
                                        bool weighted, int lo, int hi, cudaStream_t stream);
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,

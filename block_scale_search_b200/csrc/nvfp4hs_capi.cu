@@ -154,6 +154,23 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
                                                static_cast<cudaStream_t>(stream)));
 }
 
+int nvfp4_scale_sweep_quantize_full(const void* W, int64_t out, int64_t in, int64_t ldw,
+                                    const float* h, const float* S, uint8_t* codes,
+                                    uint8_t* scales, int8_t* chosen_offset, void* stream) {
+  int st = check_matrix(W, out, in, ldw, 16);
+  if (st != NVFP4_OK) return st;
+  const bool empty = out == 0 || in == 0;
+  if (!empty && (S == nullptr || codes == nullptr || scales == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(S, 4) || !aligned(codes, 8)) return NVFP4_ERR_ALIGN;
+  if (empty) return NVFP4_OK;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  return cuda_status(nvfp4::launch_scale_sweep_full(static_cast<const uint16_t*>(W), out, in, ldw,
+                                                    h, S, codes, scales, chosen_offset, sms,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S, int64_t out,
                      int64_t in, float* W_out, void* stream) {
   if (out < 0 || in < 0) return NVFP4_ERR_INVALID_ARG;

@@ -172,13 +172,16 @@ __device__ __forceinline__ uint32_t exact_e2m1_one(float xl, float a, float v, f
 
 // ------------------------------------------------------------------ kernel
 
-// Shared memory of one sweep CTA.
+// Shared memory of one sweep CTA; kMaxK candidates per group at most (16 for
+// windows, 126 for the full sweep over every positive E4M3 code).
+template <int kMaxK>
 struct SweepSmem {
   CandEntry tab[kTabSize];
-  float Lsm[16][kCta];        // per-thread column of fast losses
+  float Lsm[kMaxK][kCta];     // per-thread column of fast losses
   uint4 wbuf[2][2][kCta];     // staged groups: [buffer][half][thread]
   double tsm[kCta / 32][16];  // per-warp exchange of exact loss terms
 };
+constexpr int kFullK = 126;
 
 __device__ __forceinline__ void fill_candidate_table(CandEntry* tab) {
   for (int i = threadIdx.x; i < kTabSize; i += blockDim.x) {
@@ -191,9 +194,11 @@ __device__ __forceinline__ void fill_candidate_table(CandEntry* tab) {
 }
 
 // The sweep of one matrix by one thread lane: `tid` in [0, R*GL) is the
-// thread's position in the lane grid that covers this matrix.
-template <bool kWeighted>
-__device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __restrict__ W,
+// thread's position in the lane grid that covers this matrix.  kFull: the
+// candidates are all 126 positive codes in ascending order (lo, hi unused;
+// the reported offset is code - base code).
+template <bool kWeighted, bool kFull = false, int kMaxK = 16>
+__device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_t* __restrict__ W,
                                              int64_t out, int64_t G, int64_t ldw,
                                              const float* __restrict__ h,
                                              const float* __restrict__ Sp, int lo, int hi,
@@ -208,7 +213,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
   if (tid >= R * GL) return;
   const int64_t r0 = tid / GL;
   const int64_t gl = tid - r0 * GL;
-  const int K = hi - lo + 1;
+  const int K = kFull ? kFullK : hi - lo + 1;
   const int lane = threadIdx.x;
 
   const float S = *Sp;
@@ -297,7 +302,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
         const int bhi = e4m3_code_rne_sat(ua * (1.0f + 0x1p-20f));
         b = (blo == bhi && !exact_base) ? blo : e4m3_code_rne_sat(__fdiv_rn(__fdiv_rn(a, 6.0f), S));
         b = clamp_code(b);
-        const CandEntry* ce = tab + (b + lo + kTabOffset);
+        const CandEntry* ce = kFull ? tab + (1 + kTabOffset) : tab + (b + lo + kTabOffset);
 
         // ---- stage 1: fast FP32 losses of all candidates
         float best = __uint_as_float(0x7F800000u), second = best;
@@ -342,7 +347,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
           const int64_t g_f = __shfl_sync(amask, static_cast<long long>(g), f);
           const int cur_f = __shfl_sync(amask, cur, f);
           const float hs_f = __shfl_sync(amask, hs, f);
-          const CandEntry* ce_f = tab + (b_f + lo + kTabOffset);
+          const CandEntry* ce_f = kFull ? tab + (1 + kTabOffset) : tab + (b_f + lo + kTabOffset);
           const uint32_t* wf = reinterpret_cast<const uint32_t*>(&wbuf[cur_f][0][0]);
           double bestd = __longlong_as_double(0x7FF0000000000000ll);
           int bid = 0;
@@ -381,7 +386,8 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
         if (offs) offs[gi] = 0;
         continue;
       }
-      const CandEntry win = tab[b + lo + kTabOffset + bi];
+      const int wcode = kFull ? 1 + bi : clamp_code(b + lo + bi);
+      const CandEntry win = tab[wcode + kTabOffset];
 
       // ---- stage 3: quantize once with the winner, exact decisions, pack
       const f32x2_t ivlo = f2_pack(win.iv * (1.0f - 0x1p-20f), win.iv * (1.0f - 0x1p-20f));
@@ -398,9 +404,9 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem& sm, const uint16_t* __re
         packed[pj >> 2] |= (nib | (sgn & nz)) << (8 * (pj & 3));
       }
       *reinterpret_cast<uint2*>(cdst) = make_uint2(packed[0], packed[1]);
-      scales[gi] = static_cast<uint8_t>(clamp_code(b + lo + bi));
+      scales[gi] = static_cast<uint8_t>(wcode);
       // ascending offsets + strict "<": lo + bi is the lowest offset reaching it
-      if (offs) offs[gi] = static_cast<int8_t>(lo + bi);
+      if (offs) offs[gi] = static_cast<int8_t>(kFull ? wcode - b : lo + bi);
     }
   }
   cp_async_wait<0>();
@@ -412,11 +418,55 @@ scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64
                    const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                    int8_t* __restrict__ offs, int64_t GL, int64_t R) {
-  __shared__ SweepSmem sm;
+  __shared__ SweepSmem<16> sm;
   fill_candidate_table(sm.tab);
   __syncthreads();
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   sweep_matrix<kWeighted>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, GL, R, tid);
+}
+
+// Full sweep: every positive E4M3 code is a candidate.  The 126-entry loss
+// column needs dynamic shared memory (about 76 KB per CTA).
+template <bool kWeighted>
+__global__ void __launch_bounds__(kCta, 2)
+scale_sweep_full_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64_t ldw,
+                        const float* __restrict__ h, const float* __restrict__ Sp,
+                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                        int8_t* __restrict__ offs, int64_t GL, int64_t R) {
+  extern __shared__ __align__(16) unsigned char dsmem[];
+  auto& sm = *reinterpret_cast<SweepSmem<kFullK>*>(dsmem);
+  fill_candidate_table(sm.tab);
+  __syncthreads();
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  sweep_matrix<kWeighted, true, kFullK>(sm, W, out, G, ldw, h, Sp, 0, 0, codes, scales, offs, GL,
+                                        R, tid);
+}
+
+cudaError_t launch_scale_sweep_full(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
+                                    const float* h, const float* S, uint8_t* codes,
+                                    uint8_t* scales, int8_t* offs, int num_sms,
+                                    cudaStream_t stream) {
+  if (out == 0 || in == 0) return cudaSuccess;
+  const size_t smem = sizeof(SweepSmem<kFullK>);
+  const void* fn = h ? reinterpret_cast<const void*>(&scale_sweep_full_kernel<true>)
+                     : reinterpret_cast<const void*>(&scale_sweep_full_kernel<false>);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kCta, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const LanePlan p = sweep_plan_threads(out, in, static_cast<int64_t>(num_sms) * per_sm * kCta);
+  const unsigned blocks = static_cast<unsigned>((p.threads + kCta - 1) / kCta);
+  const int64_t G = in / 16;
+  if (h)
+    scale_sweep_full_kernel<true><<<blocks, kCta, smem, stream>>>(W, out, G, ldw, h, S, codes,
+                                                                  scales, offs, p.VL, p.R);
+  else
+    scale_sweep_full_kernel<false><<<blocks, kCta, smem, stream>>>(W, out, G, ldw, h, S, codes,
+                                                                   scales, offs, p.VL, p.R);
+  return cudaGetLastError();
 }
 
 // Batched sweep: CTA b belongs to the matrix whose [cta_begin, next cta_begin)
@@ -424,7 +474,7 @@ scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64
 template <bool kWeighted>
 __global__ void __launch_bounds__(kCta, 5)
 scale_sweep_batched_kernel(const SweepDesc* __restrict__ d, int64_t n, int lo, int hi) {
-  __shared__ SweepSmem sm;
+  __shared__ SweepSmem<16> sm;
   fill_candidate_table(sm.tab);
   __syncthreads();
   int64_t a = 0, z = n - 1;  // last descriptor with cta_begin <= blockIdx.x

@@ -150,6 +150,18 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
                                void* stream);
 
 /* ------------------------------------------------------------------------
+ * Full sweep: every one of the 126 positive E4M3 codes is a candidate --
+ * the exhaustive search that ScaleSweep summary sec. 2 calls too costly for
+ * routine use, here as the reference for window-recovery statistics (how much
+ * of the full search's gain a window keeps).  Arguments as
+ * nvfp4_scale_sweep_quantize without the window; ties go to the lowest code;
+ * chosen_offset (if not NULL) receives code - base code.
+ * ------------------------------------------------------------------------ */
+int nvfp4_scale_sweep_quantize_full(const void* W, int64_t out, int64_t in, int64_t ldw,
+                                    const float* h, const float* S, uint8_t* codes,
+                                    uint8_t* scales, int8_t* chosen_offset, void* stream);
+
+/* ------------------------------------------------------------------------
  * Grouped and batched forms: one launch for many matrices, as in a
  * mixture-of-experts layer whose experts each see their own slice of the
  * calibration tokens and get their own h and S.  Each computes exactly what

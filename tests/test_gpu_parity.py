@@ -304,3 +304,26 @@ def test_moe_grouped_sampled_experts(orc, nv):
             full_matrix_parity(orc, nv, W, X, wl.q_max, -9, 6, True, m.name)
     del Xs
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+def test_full_sweep_all_126_codes(orc, nv, weighted):
+    """The exhaustive sweep over every positive E4M3 code against the oracle's
+    sweep over offsets -125..+125 (which clamps to the same 126 codes)."""
+    import workloads
+    W = workloads.weight(96, 1024, 0.02, 0.01, 10.0, 123, DEV)
+    W[5, :48] *= 1e-3  # tiny groups: candidates far below the base code win
+    h = nv.diag_hessian(workloads.calib(300, 1024, 1.5, 124, DEV)) if weighted else None
+    S, _, _ = nv.global_scale(W)
+    codes, scales, offs = nv.scale_sweep_quantize_full(W, h, S, want_offsets=True)
+    bits = to_bits(W)
+    hn = None if h is None else h.cpu().numpy()
+    rc, rs, _ = orc.parallel_sweep_quantize(bits, hn, float(S.item()), -125, 125)
+    gc, gs = codes.cpu().numpy(), scales.cpu().numpy()
+    w, hh, _, _ = matrix_groups(bits, gc, gs, hn)
+    res = compare_groups(orc, w, hh, float(S.item()), gc, gs, rc, rs)
+    assert res["mismatch"] == 0, res
+    base = np.array([orc.base_code(bits.reshape(-1, 16)[i], float(S.item()))
+                     for i in range(bits.size // 16)]).reshape(gs.shape)
+    nz = base > 0
+    np.testing.assert_array_equal(offs.cpu().numpy()[nz], (gs.astype(int) - base)[nz])
