@@ -76,6 +76,9 @@ def lib():
             L.orc_group_loss_list.restype = None
             L.orc_packed_loss_list.argtypes = [u16p, f32p, i64, C.c_float, u8p, u8p, f64p]
             L.orc_packed_loss_list.restype = None
+            L.orc_quantize_activations.argtypes = [u16p, i64, i64, i64, C.c_float, C.c_int,
+                                                   C.c_int, f32p, u8p, u8p, i8p]
+            L.orc_quantize_activations.restype = C.c_int
             L.orc_dequantize.argtypes = [u8p, u8p, C.c_float, i64, i64, f32p]
             L.orc_dequantize.restype = None
             _lib = L
@@ -215,6 +218,22 @@ def packed_losses(w, h, S: float, codes, scales) -> np.ndarray:
     return out
 
 
+def quantize_activations(A, q_max: float = 256.0, lo: int = -3, hi: int = 7):
+    """Per-token online quantization of A[tokens, in] (bf16 bits or torch bf16).
+    Returns (S[tokens] float32, codes[tokens,in/2], scales[tokens,in/16],
+    offsets[tokens,in/16], status)."""
+    A = _bf16_bits(A)
+    t, n = A.shape
+    S = np.zeros(t, np.float32)
+    codes = np.zeros((t, n // 2), np.uint8)
+    scales = np.zeros((t, n // 16), np.uint8)
+    offs = np.zeros((t, n // 16), np.int8)
+    st = lib().orc_quantize_activations(_p(A, C.c_uint16), t, n, n, float(q_max), int(lo), int(hi),
+                                        _p(S, C.c_float), _p(codes, C.c_uint8),
+                                        _p(scales, C.c_uint8), _p(offs, C.c_int8))
+    return S, codes, scales, offs, st
+
+
 def dequantize(codes, scales, S: float) -> np.ndarray:
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
@@ -252,6 +271,31 @@ def parallel_sweep_quantize(W, h, S: float, lo: int, hi: int, threads: int | Non
     with ThreadPoolExecutor(threads) as ex:
         list(ex.map(lambda r: run(r, min(o, r + step)), range(0, o, step)))
     return codes, scales, offs
+
+
+def parallel_quantize_activations(A, q_max: float = 256.0, lo: int = -3, hi: int = 7,
+                                  threads: int | None = None):
+    """Token-chunked multi-threaded driver around orc_quantize_activations;
+    same returns as quantize_activations."""
+    A = _bf16_bits(A)
+    t, n = A.shape
+    S = np.zeros(t, np.float32)
+    codes = np.zeros((t, n // 2), np.uint8)
+    scales = np.zeros((t, n // 16), np.uint8)
+    offs = np.zeros((t, n // 16), np.int8)
+    threads = threads or default_threads()
+    L = lib()
+
+    def run(r0, r1):
+        return L.orc_quantize_activations(_p(A[r0:r1], C.c_uint16), r1 - r0, n, n, float(q_max),
+                                          int(lo), int(hi), _p(S[r0:r1], C.c_float),
+                                          _p(codes[r0:r1], C.c_uint8), _p(scales[r0:r1], C.c_uint8),
+                                          _p(offs[r0:r1], C.c_int8))
+
+    step = max(1, -(-t // (threads * 4)))
+    with ThreadPoolExecutor(threads) as ex:
+        rcs = list(ex.map(lambda r: run(r, min(t, r + step)), range(0, t, step)))
+    return S, codes, scales, offs, (min(rcs) if rcs else 0)
 
 
 def parallel_diag_hessian(X, threads: int | None = None) -> np.ndarray:

@@ -191,6 +191,34 @@ void orc_sweep_quantize(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                             offsets ? offsets + r * G + g : NULL, NULL);
 }
 
+/* ---- activations, quantized online ---------------------------------------
+ * [ScaleSweep] sec. 1-3 and "Experimental Results": in the W+A settings the
+ * activations are NVFP4 too, with the MSE objective (no Hessian) and the
+ * [-3, +7] window.  Reading taken where the page is silent: the global scale
+ * is dynamic, one per token (row), by the same formula as for a weight tensor,
+ * and each row is then swept as a one-row matrix. */
+int orc_quantize_activations(const uint16_t* A, int64_t tokens, int64_t in, int64_t lda,
+                             float q_max, int lo, int hi, float* S, uint8_t* codes,
+                             uint8_t* scales, int8_t* offsets) {
+    int64_t G = in / 16;
+    int rc = 0;
+    for (int64_t t = 0; t < tokens; ++t) {
+        const uint16_t* row = A + t * lda;
+        uint8_t* crow = codes + t * (in / 2);
+        uint8_t* srow = scales + t * G;
+        int8_t* orow = offsets ? offsets + t * G : NULL;
+        if (orc_global_scale(row, 1, in, lda, q_max, &S[t], NULL) != 0) {
+            rc = -5;                                   /* S[t] is NaN; outputs zero */
+            memset(crow, 0, (size_t)(in / 2));
+            memset(srow, 0, (size_t)G);
+            if (orow) memset(orow, 0, (size_t)G);
+            continue;
+        }
+        orc_sweep_quantize(row, 1, in, lda, NULL, S[t], lo, hi, crow, srow, orow);
+    }
+    return rc;
+}
+
 void orc_sweep_group_list(const uint16_t* w, const float* h, int64_t n, float S,
                           int lo, int hi, uint8_t* codes, uint8_t* scales,
                           int8_t* offsets, double* losses) {

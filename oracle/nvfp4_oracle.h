@@ -91,6 +91,17 @@ void orc_sweep_quantize(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                         const float* h, float S, int lo, int hi,
                         uint8_t* codes, uint8_t* scales, int8_t* offsets);
 
+/* Activations quantized online ([ScaleSweep] W+A settings: the MSE sweep
+ * applied to activations).  Per token t (row of A[tokens, in], row stride lda):
+ *   S[t] = fl32(amax_t / fl32(q_max * 6))   (0 for an all-zero row), then the
+ * row is swept as orc_sweep_quantize does with h == NULL and window [lo, hi].
+ * A row holding Inf or NaN gets S[t] = NaN and zero codes, scales and offsets;
+ * the return is -5 if any row did, else 0.  codes[tokens, in/2],
+ * scales[tokens, in/16], offsets[tokens, in/16] (NULL allowed). */
+int orc_quantize_activations(const uint16_t* A, int64_t tokens, int64_t in, int64_t lda,
+                             float q_max, int lo, int hi, float* S, uint8_t* codes,
+                             uint8_t* scales, int8_t* offsets);
+
 /* List form used for sampled checks: n groups, w[n,16], h[n,16] or NULL. */
 void orc_sweep_group_list(const uint16_t* w, const float* h, int64_t n, float S,
                           int lo, int hi, uint8_t* codes, uint8_t* scales,
