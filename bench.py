@@ -36,6 +36,11 @@ SWEEP_BYTES_PER_ELEM = 2 + 0.5 + 1 / 16   # read bf16 W; write 4-bit code + 1/16
 # h*e and the accumulation (h e) e -- five FP32 lane operations.
 SWEEP_OPS_PER_ELEM_CAND = 5
 SMS, LANES_PER_SM = 148, 128
+# Online activation quantization (W+A settings): plain MSE, so no weighting
+# multiply -- four FP32 lane operations per element and candidate.
+ACT_LO, ACT_HI, ACT_Q = -3, 7, 256.0
+ACT_OPS_PER_ELEM_CAND = 4
+ACT_BYTES_PER_ELEM = 2 + 0.5 + 1 / 16     # read bf16 A; write codes + scale bytes
 
 
 def measured_peaks():
@@ -278,8 +283,16 @@ def profiled_traffic(kernel: str, units_per_launch: float):
         d = json.load(f).get(kernel)
     if not d:
         return None
-    src = os.path.join(ROOT, d["source"])
-    if not os.path.exists(src) or hashlib.sha1(open(src, "rb").read()).hexdigest() != d["source_sha1"]:
+    # the capture is void once any file the kernel is compiled from has changed:
+    # sha1 over the listed sources' bytes, concatenated in order
+    srcs = [os.path.join(ROOT, x) for x in d.get("sources", [d.get("source", "")])]
+    if not all(os.path.exists(x) for x in srcs):
+        return None
+    h = hashlib.sha1()
+    for x in srcs:
+        with open(x, "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != d["source_sha1"]:
         return None
     return d["dram_bytes_per_unit"] * units_per_launch
 
@@ -330,6 +343,125 @@ def oracle_sample_rate(wl, Ws, Xs, threads=None, row_frac=0.25, tokens=4096):
             "cores": threads, "t_sample_s": round(t_sweep + t_abs + t_h, 3),
             "t_full_est_s": round(t_full, 2)}
     return wel / t_full, info
+
+
+# ------------------------------------------------- activation quantization
+
+ACT_WORKLOAD = ("act_llama33_70b: activations 65536 tokens x 8192 bf16 (the 70B-shaped MLP's "
+                "gate/up input), lognormal(1.5) channel scales; per-token S = amax/(256*6); MSE "
+                "sweep [-3,+7]")
+
+
+def oracle_act_rate(A, rows=1024, threads=None):
+    """The oracle as it stands on the first `rows` tokens, extrapolated to
+    elements per second."""
+    import torch
+    import oracle
+    threads = threads or oracle.default_threads()
+    sub = A[:rows].cpu().view(torch.uint16).numpy()
+    t0 = time.perf_counter()
+    oracle.parallel_quantize_activations(sub, ACT_Q, ACT_LO, ACT_HI, threads=threads)
+    dt = time.perf_counter() - t0
+    return sub.size / dt, {"cores": threads, "t_sample_s": round(dt, 3),
+                           "sample": f"oracle on the first {rows} of {A.shape[0]} tokens "
+                                     f"({sub.size} elements); rate extrapolated linearly"}
+
+
+def run_activations(args, nv, rank, local, ws, dev):
+    """One step = per-token NVFP4 quantization of one activation matrix in a
+    single fused launch (per-token S, then the MSE [-3,+7] sweep and pack)."""
+    import torch
+    import workloads
+    A = workloads.calib(65536, 8192, 1.5, 4 + 1000 * rank, dev)
+    t, n = A.shape
+    S = torch.empty(t, dtype=torch.float32, device=dev)
+    codes = torch.empty(t, n // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(t, n // 16, dtype=torch.uint8, device=dev)
+    status = torch.empty(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nv.nvfp4_quantize_activations(A, t, n, A.stride(0), ACT_Q, ACT_LO, ACT_HI, S, codes, scales,
+                                      None, status, stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(ws)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(ws)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    barrier(ws)
+    sampler.mark_end()
+    clocks = sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, ws)
+    assert int(status.item()) == 0, "non-finite activations"
+    el = t * n
+    value = el * ws / (ms * 1e-3)
+    K = ACT_HI - ACT_LO + 1
+    clk = (clocks or {}).get("sm_mhz") or 1965.0
+    peak_top = SMS * LANES_PER_SM * clk * 1e6 / 1e12
+    achieved = ACT_OPS_PER_ELEM_CAND * K * el / (ms * 1e-3) / 1e12
+    peak, peak_kind, _ = measured_peaks()
+    gbs = ACT_BYTES_PER_ELEM * el / (ms * 1e-3) / 1e9
+    roofline = {"kernel": "act_quant", "bound": "alu", "achieved": round(achieved, 2),
+                "peak": round(peak_top, 2), "unit": "TOP/s",
+                "peak_source": f"148 SMs x 128 FP32 lanes x {clk:.0f} MHz (sampled SM clock)",
+                "frac": round(achieved / peak_top, 4),
+                "ops_per_unit": f"{ACT_OPS_PER_ELEM_CAND} FP32 ops per element per candidate, "
+                                f"{K} candidates",
+                "hbm_gbs": round(gbs, 1), "hbm_frac_of_measured": round(gbs / peak, 4),
+                "traffic": profiled_traffic("act_quant", el)}
+    e2e = None
+    if args.e2e_steps > 0:
+        hA = A.cpu().pin_memory()
+        hS = torch.empty_like(S, device="cpu").pin_memory()
+        hC = torch.empty_like(codes, device="cpu").pin_memory()
+        hK = torch.empty_like(scales, device="cpu").pin_memory()
+
+        def e2e_step():
+            A.copy_(hA, non_blocking=True)
+            step()
+            hS.copy_(S, non_blocking=True)
+            hC.copy_(codes, non_blocking=True)
+            hK.copy_(scales, non_blocking=True)
+
+        e2e_step()
+        barrier(ws)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        barrier(ws)
+        e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, ws)
+        e2e = {"value": el * ws / (e_ms * 1e-3), "unit": "elem/s", "ms_per_step": round(e_ms, 3),
+               "h2d_bytes_per_step": int(hA.numel() * 2),
+               "d2h_bytes_per_step": int(hS.numel() * 4 + hC.numel() + hK.numel()),
+               "steps": args.e2e_steps}
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rate, info = oracle_act_rate(A)
+        cpu = {"value": rate, "unit": "elem/s", "kind": "oracle", **info}
+    if rank == 0:
+        out = {"metric": "NVFP4 activation elems/s quantized online (per-token S + MSE sweep)",
+               "value": value, "unit": "elem/s", "n_gpus": ws, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+               "config": {"workload": ACT_WORKLOAD, "window": [ACT_LO, ACT_HI], "q_max": ACT_Q,
+                          "l2": f"input {2 * el / 1e9:.2f} GB per rank > 126 MB L2; no flush",
+                          "parallelism": f"weak: {ws} rank(s), one activation matrix per rank"},
+               "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+               "cpu_baseline": cpu, "clocks": clocks}
+        print(json.dumps(out), flush=True)
 
 
 # ------------------------------------------------------------------ main
@@ -422,7 +554,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="llama33_70b_mlp", choices=WORKLOADS)
+    ap.add_argument("--workload", default="llama33_70b_mlp",
+                    choices=list(WORKLOADS) + ["act_llama33_70b"])
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -436,6 +569,13 @@ def main():
     rank, local, ws = init_dist()
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
+    if args.workload == "act_llama33_70b":
+        run_activations(args, nv, rank, local, ws, dev)
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     wl, Ws, Xs = build_layer(rank, dev, args.workload)
     step = (GroupedStep if args.workload == "moe_grouped" else Step)(nv, wl, Ws, Xs, dev)
 

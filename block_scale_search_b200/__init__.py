@@ -26,7 +26,8 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
-    "nvfp4_scale_sweep_quantize", "nvfp4_dequantize",
+    "nvfp4_scale_sweep_quantize", "nvfp4_dequantize", "nvfp4_quantize_activations",
+    "quantize_activations",
     "diag_hessian", "global_scale", "scale_sweep_quantize", "dequantize", "quantize_layer",
 ]
 
@@ -73,6 +74,8 @@ _SIGS = {
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
+    "nvfp4_quantize_activations": ([_vp, _i64, _i64, _i64, _f32, _int, _int, _vp, _vp, _vp, _vp,
+                                    _vp, _vp], _int),
     "nvfp4_scale_sweep_quantize_full": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp],
                                         _int),
     "nvfp4_diag_hessian_grouped_workspace_size": ([_i64, _i64, _i64], _sz),
@@ -170,6 +173,13 @@ def nvfp4_scale_sweep_quantize_full(W, out, inp, ldw, h, S, codes, scales, chose
     _check("nvfp4_scale_sweep_quantize_full", lib().nvfp4_scale_sweep_quantize_full(
         _ptr(W), out, inp, ldw, _ptr(h), _ptr(S), _ptr(codes), _ptr(scales), _ptr(chosen_offset),
         _stream(stream)))
+
+
+def nvfp4_quantize_activations(A, tokens, inp, lda, q_max, lo, hi, S, codes, scales,
+                               chosen_offset, status, stream=None):
+    _check("nvfp4_quantize_activations", lib().nvfp4_quantize_activations(
+        _ptr(A), tokens, inp, lda, float(q_max), int(lo), int(hi), _ptr(S), _ptr(codes),
+        _ptr(scales), _ptr(chosen_offset), _ptr(status), _stream(stream)))
 
 
 def nvfp4_dequantize(codes, scales, S, out, inp, W_out, stream=None):
@@ -297,6 +307,27 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, S: torch.Tensor, strea
     W = torch.empty(o, half * 2, dtype=torch.float32, device=codes.device)
     nvfp4_dequantize(codes, scales, S, o, half * 2, W, stream)
     return W
+
+
+def quantize_activations(A: torch.Tensor, q_max: float = 256.0, lo: int = -3, hi: int = 7,
+                         want_offsets: bool = False, out=None, stream=None):
+    """Per-token NVFP4 quantization of activations A[tokens, in] in one launch.
+    Returns (S[tokens] f32, codes[tokens, in/2] u8, scales[tokens, in/16] u8,
+    offsets or None, status[1] int32)."""
+    A = _bf16_2d(A, "A")
+    t, n = A.shape
+    dev = A.device
+    if out is None:
+        S = torch.empty(t, dtype=torch.float32, device=dev)
+        codes = torch.empty(t, n // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(t, n // 16, dtype=torch.uint8, device=dev)
+        offs = torch.empty(t, n // 16, dtype=torch.int8, device=dev) if want_offsets else None
+        status = torch.empty(1, dtype=torch.int32, device=dev)
+    else:
+        S, codes, scales, offs, status = out
+    nvfp4_quantize_activations(A, t, n, A.stride(0), q_max, lo, hi, S, codes, scales, offs, status,
+                               stream)
+    return S, codes, scales, offs, status
 
 
 def quantize_layer(W: torch.Tensor, X: torch.Tensor | None, q_max: float = 448.0, lo: int = -9,

@@ -1,0 +1,199 @@
+// act_quant.cu -- online NVFP4 quantization of activations: a dynamic global
+// scale per token and the plain-MSE scale sweep, fused in one kernel.
+//
+// ScaleSweep summary, sec. 1-3 and "Experimental Results" (the W+A settings):
+// activations are NVFP4 as well, quantized with the MSE objective and the
+// [-3, +7] window.  Where the page is silent the reading is: the FP32 global
+// scale is dynamic, one per token, S_t = fl32(amax_t / fl32(Q * 6)) by the
+// same formula as for a weight tensor, and each token row is then swept as a
+// one-row matrix (every group decided exactly as in scale_sweep.cu, h == 1).
+//
+// Work layout: a team of TW warps (TW = 1, 2 or 4 of the CTA's four) owns one
+// token row at a time; rows are dealt to teams in a stride over a one-wave
+// grid.
+//   Pass 1 reads the row with 16-byte loads and takes the max of the
+//   sign-cleared bf16 bit patterns: a warp reduction, then for TW > 1 an
+//   exchange through shared memory under a named barrier of the team.
+//   Pass 2 sweeps the row's groups.  Team lane l takes groups l, l + 32 TW, ...;
+//   the next group's 32 bytes are copied into shared memory with cp.async
+//   while the current one is scored.  The row was read a moment before, so
+//   those copies mostly hit L2.
+#include "nvfp4hs.h"
+#include "nvfp4_kernels.cuh"
+#include "sweep_core.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+// Named barrier of one team (ids 1 and 2 as immediates, so the kernel
+// reserves only the barriers it uses; id 0 is __syncthreads).
+template <int kThreads>
+__device__ __forceinline__ void team_barrier(int team) {
+  if (team == 0)
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+  else
+    asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+}
+
+template <int TW>
+__global__ void __launch_bounds__(kCta, 5)
+act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int64_t lda,
+                 float q_max, int lo, int hi, float* __restrict__ S_out,
+                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                 int8_t* __restrict__ offs, int* __restrict__ status) {
+  __shared__ SweepSmem<16> sm;
+  __shared__ uint32_t red[2][kCta / 32];  // per-warp row maxima, by row parity
+  fill_candidate_table(sm.tab);
+  __syncthreads();
+
+  constexpr int kTeams = (kCta / 32) / TW;
+  constexpr int kTeamThreads = 32 * TW;
+  const int lane = threadIdx.x;
+  const int warp = lane >> 5;
+  const int team = warp / TW;
+  const int tl = lane - team * kTeamThreads;  // position in the team
+  const int64_t nteams = static_cast<int64_t>(gridDim.x) * kTeams;
+  const int64_t nvec = G * 2;                  // 16-byte vectors per row
+  const int64_t half_in = G * 8;
+  const float q6 = __fmul_rn(q_max, 6.0f);
+  const int K = hi - lo + 1;
+  auto& wbuf = sm.wbuf;
+
+  f32x2_t ones[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ones[i] = f2_pack(1.0f, 1.0f);
+
+  int parity = 0, buf = 0;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kTeams + team; t < tokens;
+       t += nteams, parity ^= 1) {
+    const uint16_t* row = A + t * lda;
+
+    // ---- pass 1: the row's absmax as a bf16 bit pattern
+    uint32_t m2 = 0;
+    int64_t v = tl;
+    for (; v + 3 * kTeamThreads < nvec; v += 4 * kTeamThreads) {
+      uint4 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = ld_stream_v4(row + (v + u * kTeamThreads) * 8);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        m2 = __vmaxu2(__vmaxu2(m2, x[u].x & 0x7FFF7FFFu),
+                      __vmaxu2(__vmaxu2(x[u].y & 0x7FFF7FFFu, x[u].z & 0x7FFF7FFFu),
+                               x[u].w & 0x7FFF7FFFu));
+    }
+    for (; v < nvec; v += kTeamThreads) {
+      const uint4 x = ld_stream_v4(row + v * 8);
+      m2 = __vmaxu2(__vmaxu2(m2, x.x & 0x7FFF7FFFu),
+                    __vmaxu2(__vmaxu2(x.y & 0x7FFF7FFFu, x.z & 0x7FFF7FFFu), x.w & 0x7FFF7FFFu));
+    }
+    uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+    if constexpr (TW > 1) {
+      if ((lane & 31) == 0) red[parity][warp] = mb;
+      team_barrier<kTeamThreads>(team);
+#pragma unroll
+      for (int i = 0; i < TW; ++i) mb = max(mb, red[parity][team * TW + i]);
+    }
+
+    // S_t = fl32(amax / fl32(Q * 6)); Inf or NaN in the row (a pattern at or
+    // above 0x7F80) gives S_t = NaN, a zero row and the status word
+    const bool nonfinite = mb >= 0x7F80u;
+    const float S = nonfinite ? __uint_as_float(0x7FC00000u)
+                              : __fdiv_rn(__uint_as_float(mb << 16), q6);
+    if (tl == 0) {
+      S_out[t] = S;
+      if (nonfinite && status) *status = NVFP4_ERR_NONFINITE;
+    }
+    uint8_t* crow = codes + t * half_in;
+    uint8_t* srow = scales + t * G;
+    int8_t* orow = offs ? offs + t * G : nullptr;
+    if (nonfinite) {
+      for (int64_t g = tl; g < G; g += kTeamThreads) {
+        *reinterpret_cast<uint2*>(crow + g * 8) = make_uint2(0u, 0u);
+        srow[g] = 0;
+        if (orow) orow[g] = 0;
+      }
+      continue;
+    }
+
+    // ---- pass 2: sweep the row's groups with this row's S
+    const ScaleConsts sc = scale_consts(S);
+    auto issue = [&](int64_t gg, int b) {
+      const uint16_t* src = row + gg * 16;
+      cp_async16(&wbuf[b][0][lane], src);
+      cp_async16(&wbuf[b][1][lane], src + 8);
+    };
+    if (tl < G) issue(tl, buf);
+    cp_async_commit();
+    for (int64_t g = tl; g < G; g += kTeamThreads) {
+      const unsigned amask = __activemask();
+      if (g + kTeamThreads < G) issue(g + kTeamThreads, buf ^ 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+      const int cur = buf;
+      buf ^= 1;
+      sweep_group<false, false, 16>(sm, amask, cur, ones, 1.0f, nullptr, g, sc, lo, K,
+                                    [&](uint2 c, uint8_t s, int8_t o) {
+                                      *reinterpret_cast<uint2*>(crow + g * 8) = c;
+                                      srow[g] = s;
+                                      if (orow) orow[g] = o;
+                                    });
+    }
+    cp_async_wait<0>();
+  }
+}
+
+template <int TW>
+const void* act_kernel_ptr() {
+  return reinterpret_cast<const void*>(&act_quant_kernel<TW>);
+}
+
+}  // namespace
+
+int act_quant_resident_ctas() {
+  static const int n = resident_ctas(act_kernel_ptr<1>(), kCta);
+  return n;
+}
+
+int act_quant_team_warps(int64_t tokens, int64_t in, int num_sms) {
+  // cost of a team size: rounds of rows per team x groups per lane per row;
+  // the smallest wins, ties to fewer warps per team (no barrier)
+  const int64_t wave_warps = static_cast<int64_t>(num_sms) * act_quant_resident_ctas() * (kCta / 32);
+  const int64_t G = in / 16;
+  int best_tw = 1;
+  int64_t best = -1;
+  for (int tw = 1; tw <= 4; tw *= 2) {
+    const int64_t teams = wave_warps / tw;
+    const int64_t rounds = (tokens + teams - 1) / teams;
+    const int64_t per_row = (G + 32 * tw - 1) / (32 * tw);
+    const int64_t cost = rounds * (per_row > 0 ? per_row : 1);
+    if (best < 0 || cost < best) { best = cost; best_tw = tw; }
+  }
+  return best_tw;
+}
+
+cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64_t in,
+                                        int64_t lda, float q_max, int lo, int hi, float* S,
+                                        uint8_t* codes, uint8_t* scales, int8_t* offs,
+                                        int* status, int num_sms, cudaStream_t stream) {
+  if (tokens == 0) return cudaSuccess;
+  const int tw = act_quant_team_warps(tokens, in, num_sms);
+  const int64_t teams_per_cta = (kCta / 32) / tw;
+  int64_t blocks = (tokens + teams_per_cta - 1) / teams_per_cta;
+  const int64_t wave = static_cast<int64_t>(num_sms) * act_quant_resident_ctas();
+  if (blocks > wave) blocks = wave;
+  const int64_t G = in / 16;
+  const unsigned nb = static_cast<unsigned>(blocks);
+  if (tw == 1)
+    act_quant_kernel<1><<<nb, kCta, 0, stream>>>(A, tokens, G, lda, q_max, lo, hi, S, codes,
+                                                 scales, offs, status);
+  else if (tw == 2)
+    act_quant_kernel<2><<<nb, kCta, 0, stream>>>(A, tokens, G, lda, q_max, lo, hi, S, codes,
+                                                 scales, offs, status);
+  else
+    act_quant_kernel<4><<<nb, kCta, 0, stream>>>(A, tokens, G, lda, q_max, lo, hi, S, codes,
+                                                 scales, offs, status);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -77,6 +77,14 @@ cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64
                                uint8_t* scales, int8_t* offs, const LanePlan& p,
                                cudaStream_t stream);
 
+// Online activation quantization: per-token S and the MSE sweep in one launch.
+// A team of 1, 2 or 4 warps owns a row at a time (chosen from the shape).
+int act_quant_team_warps(int64_t tokens, int64_t in, int num_sms);
+cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64_t in,
+                                        int64_t lda, float q_max, int lo, int hi, float* S,
+                                        uint8_t* codes, uint8_t* scales, int8_t* offs,
+                                        int* status, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S,
                               int64_t out, int64_t in, float* W_out, int num_sms,
                               cudaStream_t stream);

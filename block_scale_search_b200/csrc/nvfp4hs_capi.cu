@@ -171,6 +171,31 @@ int nvfp4_scale_sweep_quantize_full(const void* W, int64_t out, int64_t in, int6
                                                     static_cast<cudaStream_t>(stream)));
 }
 
+int nvfp4_quantize_activations(const void* A, int64_t tokens, int64_t in, int64_t lda,
+                               float q_max, int lo, int hi, float* S, uint8_t* codes,
+                               uint8_t* scales, int8_t* chosen_offset, int* status,
+                               void* stream) {
+  int st = check_matrix(A, tokens, in, lda, 16);
+  if (st != NVFP4_OK) return st;
+  if (!std::isfinite(q_max) || !(q_max > 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  if (tokens > 0 && S == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (tokens > 0 && in > 0 && (codes == nullptr || scales == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  if (!aligned(S, 4) || !aligned(codes, 8) || !aligned(status, 4)) return NVFP4_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (status != nullptr) {
+    const cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  if (tokens == 0) return NVFP4_OK;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  return cuda_status(nvfp4::launch_quantize_activations(static_cast<const uint16_t*>(A), tokens,
+                                                        in, lda, q_max, lo, hi, S, codes, scales,
+                                                        chosen_offset, status, sms, s));
+}
+
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S, int64_t out,
                      int64_t in, float* W_out, void* stream) {
   if (out < 0 || in < 0) return NVFP4_ERR_INVALID_ARG;

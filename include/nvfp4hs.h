@@ -227,6 +227,34 @@ int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n,
                                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Online activation quantization (ScaleSweep summary, sec. 1-3 and
+ * "Experimental Results": in the W+A settings the activations are NVFP4 too,
+ * their scales chosen with the MSE objective and the [-3, +7] window).  One
+ * launch does, for every token row t of A:
+ *   S[t] = fl32(amax_t / fl32(q_max * 6))   (0 for an all-zero row), then
+ *   the windowed sweep of nvfp4_scale_sweep_quantize on that row alone, with
+ *   h == 1 and the scale S[t].
+ * The page does not say how the activations' FP32 scale is set; the reading
+ * taken is a dynamic scale per token by the weight-tensor formula, so a row's
+ * results do not depend on the other rows.
+ *   A          bf16 [tokens, lda], 16-byte aligned; lda % 8 == 0; in % 16 == 0.
+ *   q_max      > 0 and finite (ScaleSweep uses 256).
+ *   lo, hi     as nvfp4_scale_sweep_quantize; [-3, +7] on the page.
+ *   S          float [tokens] (written).
+ *   codes      uint8 [tokens, in/2], 8-byte aligned; scales uint8 [tokens, in/16];
+ *   chosen_offset  int8 [tokens, in/16] or NULL.
+ *   status     int, device scalar, may be NULL: the call first sets it to
+ *              NVFP4_OK (an asynchronous memset on `stream`); a row holding Inf
+ *              or NaN sets it to NVFP4_ERR_NONFINITE and gets S[t] = NaN and
+ *              zero codes, scales and offsets.
+ * Layout of codes and scales as for a weight matrix [tokens, in].
+ * ------------------------------------------------------------------------ */
+int nvfp4_quantize_activations(const void* A, int64_t tokens, int64_t in, int64_t lda,
+                               float q_max, int lo, int hi, float* S, uint8_t* codes,
+                               uint8_t* scales, int8_t* chosen_offset, int* status,
+                               void* stream);
+
+/* ------------------------------------------------------------------------
  * Dequantize (NVFP4 decode, H-Scale summary sec. 3: effective scale = global
  * x local): W_out[r, j] = sign * fl32(g[k] * v(scale)) * S, float [out, in].
  *   codes [out, in/2] 8-byte aligned; scales [out, in/16]; S device scalar;

@@ -159,3 +159,33 @@ def test_grouped_and_batched_validation(L):
     arr1 = (nv.SweepDesc * 1)(d[1])
     assert s(arr1, 1, -9, 6, None, 0, None) == -7                           # no workspace
     assert s(None, 0, -9, 6, None, 0, None) == 0                            # empty batch
+
+
+def test_activation_validation(L):
+    f = L.nvfp4_quantize_activations
+    names = ["A", "tokens", "inp", "lda", "q", "lo", "hi", "S", "codes", "scales", "offs", "st",
+             "stream"]
+    ok = (P, 4, 32, 32, 256.0, -3, 7, P, P, P, None, None, None)
+
+    def call(**kw):
+        a = dict(zip(names, ok))
+        a.update(kw)
+        return f(*[a[n] for n in names])
+
+    assert call(A=None) == -1
+    assert call(S=None) == -1
+    assert call(codes=None) == -1
+    assert call(scales=None) == -1
+    assert call(tokens=-1) == -1
+    assert call(q=0.0) == -1
+    assert call(q=float("nan")) == -1
+    assert call(inp=24, lda=24) == -2                 # in % 16
+    assert call(lda=16) == -2                         # lda < in
+    assert call(A=P + 8) == -3
+    assert call(lda=36) == -3                         # lda % 8
+    assert call(S=P + 2) == -3
+    assert call(codes=P + 4) == -3
+    assert call(st=P + 2) == -3
+    for lo, hi in ((1, 6), (-3, -1), (-17, 0), (0, 16), (-9, 7)):
+        assert call(lo=lo, hi=hi) == -4, (lo, hi)
+    assert call(tokens=0, S=None, codes=None, scales=None) == 0   # empty, no status: no device
