@@ -27,7 +27,8 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize", "nvfp4_quantize_activations",
-    "quantize_activations",
+    "quantize_activations", "nvfp4_blocked_scales_size", "nvfp4_scales_to_blocked",
+    "scales_to_blocked",
     "diag_hessian", "global_scale", "scale_sweep_quantize", "dequantize", "quantize_layer",
 ]
 
@@ -74,6 +75,8 @@ _SIGS = {
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
+    "nvfp4_blocked_scales_size": ([_i64, _i64], _sz),
+    "nvfp4_scales_to_blocked": ([_vp, _i64, _i64, _i64, _vp, _vp], _int),
     "nvfp4_quantize_activations": ([_vp, _i64, _i64, _i64, _f32, _int, _int, _vp, _vp, _vp, _vp,
                                     _vp, _vp], _int),
     "nvfp4_scale_sweep_quantize_full": ([_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp],
@@ -180,6 +183,15 @@ def nvfp4_quantize_activations(A, tokens, inp, lda, q_max, lo, hi, S, codes, sca
     _check("nvfp4_quantize_activations", lib().nvfp4_quantize_activations(
         _ptr(A), tokens, inp, lda, float(q_max), int(lo), int(hi), _ptr(S), _ptr(codes),
         _ptr(scales), _ptr(chosen_offset), _ptr(status), _stream(stream)))
+
+
+def nvfp4_blocked_scales_size(rows: int, cols: int) -> int:
+    return lib().nvfp4_blocked_scales_size(rows, cols)
+
+
+def nvfp4_scales_to_blocked(scales, rows, cols, ld, out, stream=None):
+    _check("nvfp4_scales_to_blocked", lib().nvfp4_scales_to_blocked(
+        _ptr(scales), rows, cols, ld, _ptr(out), _stream(stream)))
 
 
 def nvfp4_dequantize(codes, scales, S, out, inp, W_out, stream=None):
@@ -328,6 +340,16 @@ def quantize_activations(A: torch.Tensor, q_max: float = 256.0, lo: int = -3, hi
     nvfp4_quantize_activations(A, t, n, A.stride(0), q_max, lo, hi, S, codes, scales, offs, status,
                                stream)
     return S, codes, scales, offs, status
+
+
+def scales_to_blocked(scales: torch.Tensor, stream=None) -> torch.Tensor:
+    """Row-major scale bytes [rows, in/16] -> the tensor-core tiled layout
+    (flat uint8, rows padded to 128 and columns to 4)."""
+    rows, cols = scales.shape
+    out = torch.empty(max(16, nvfp4_blocked_scales_size(rows, cols)), dtype=torch.uint8,
+                      device=scales.device)
+    nvfp4_scales_to_blocked(scales, rows, cols, scales.stride(0), out, stream)
+    return out[:nvfp4_blocked_scales_size(rows, cols)]
 
 
 def quantize_layer(W: torch.Tensor, X: torch.Tensor | None, q_max: float = 448.0, lo: int = -9,

@@ -85,6 +85,11 @@ cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64
                                         uint8_t* codes, uint8_t* scales, int8_t* offs,
                                         int* status, int num_sms, cudaStream_t stream);
 
+// Row-major scale bytes -> the tensor-core MMA's tiled 128 x 4 scale layout.
+size_t blocked_scales_bytes(int64_t rows, int64_t cols);
+cudaError_t launch_scales_to_blocked(const uint8_t* sf, int64_t rows, int64_t cols, int64_t ld,
+                                     uint8_t* out, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S,
                               int64_t out, int64_t in, float* W_out, int num_sms,
                               cudaStream_t stream);

@@ -196,6 +196,24 @@ int nvfp4_quantize_activations(const void* A, int64_t tokens, int64_t in, int64_
                                                         chosen_offset, status, sms, s));
 }
 
+size_t nvfp4_blocked_scales_size(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0 || rows > kMaxDim || cols > kMaxDim) return 0;
+  return nvfp4::blocked_scales_bytes(rows, cols);
+}
+
+int nvfp4_scales_to_blocked(const uint8_t* scales, int64_t rows, int64_t cols, int64_t ld,
+                            uint8_t* out, void* stream) {
+  if (rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
+  if (ld < cols || rows > kMaxDim || cols > kMaxDim || ld > kMaxDim) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (scales == nullptr || out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return NVFP4_ERR_ALIGN;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  return cuda_status(nvfp4::launch_scales_to_blocked(scales, rows, cols, ld, out, sms,
+                                                     static_cast<cudaStream_t>(stream)));
+}
+
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S, int64_t out,
                      int64_t in, float* W_out, void* stream) {
   if (out < 0 || in < 0) return NVFP4_ERR_INVALID_ARG;

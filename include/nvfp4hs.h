@@ -255,6 +255,23 @@ int nvfp4_quantize_activations(const void* A, int64_t tokens, int64_t in, int64_
                                void* stream);
 
 /* ------------------------------------------------------------------------
+ * Scale bytes in the tensor-core layout.  The pages return groups "in native
+ * NVFP4 representation" (H-Scale summary, sec. 3); a Blackwell block-scaled
+ * NVFP4 GEMM reads the codes as they are (two E2M1 values per byte, element
+ * 2k in the low nibble) but wants the E4M3 scales tiled:
+ *   rows padded to a multiple of 128 and columns to a multiple of 4 (padding
+ *   bytes 0); 128 x 4 blocks of 512 bytes stored block-row by block-row;
+ *   inside a block, scale (r, c) at byte (r % 32) * 16 + (r / 32) * 4 + c.
+ * This is the 16-element E4M3 scale-vector layout of cuBLASLt's NVFP4 GEMM.
+ *   scales     uint8 [rows, ld] (row-major as written by the sweep), cols <= ld.
+ *   cols       in / 16 (scales per row).
+ *   out        uint8 [nvfp4_blocked_scales_size(rows, cols)], 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_blocked_scales_size(int64_t rows, int64_t cols);
+int nvfp4_scales_to_blocked(const uint8_t* scales, int64_t rows, int64_t cols, int64_t ld,
+                            uint8_t* out, void* stream);
+
+/* ------------------------------------------------------------------------
  * Dequantize (NVFP4 decode, H-Scale summary sec. 3: effective scale = global
  * x local): W_out[r, j] = sign * fl32(g[k] * v(scale)) * S, float [out, in].
  *   codes [out, in/2] 8-byte aligned; scales [out, in/16]; S device scalar;

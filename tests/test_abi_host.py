@@ -189,3 +189,16 @@ def test_activation_validation(L):
     for lo, hi in ((1, 6), (-3, -1), (-17, 0), (0, 16), (-9, 7)):
         assert call(lo=lo, hi=hi) == -4, (lo, hi)
     assert call(tokens=0, S=None, codes=None, scales=None) == 0   # empty, no status: no device
+
+
+def test_blocked_scales_validation(L):
+    f = L.nvfp4_scales_to_blocked
+    assert L.nvfp4_blocked_scales_size(300, 130) == 384 * 132
+    assert L.nvfp4_blocked_scales_size(128, 4) == 512
+    assert L.nvfp4_blocked_scales_size(-1, 4) == 0
+    assert f(P, -1, 4, 4, P, None) == -1
+    assert f(P, 4, 8, 4, P, None) == -2              # ld < cols
+    assert f(None, 4, 4, 4, P, None) == -1
+    assert f(P, 4, 4, 4, None, None) == -1
+    assert f(P, 4, 4, 4, P + 8, None) == -3          # out must be 16-byte aligned
+    assert f(P, 0, 4, 4, None, None) == 0            # empty
