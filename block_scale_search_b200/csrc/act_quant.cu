@@ -18,6 +18,8 @@
 //   the next group's 32 bytes are copied into shared memory with cp.async
 //   while the current one is scored.  The row was read a moment before, so
 //   those copies mostly hit L2.
+#include <type_traits>
+
 #include "nvfp4hs.h"
 #include "nvfp4_kernels.cuh"
 #include "sweep_core.cuh"
@@ -36,7 +38,7 @@ __device__ __forceinline__ void team_barrier(int team) {
     asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
 }
 
-template <int TW>
+template <int TW, int kK>
 __global__ void __launch_bounds__(kCta, 5)
 act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int64_t lda,
                  float q_max, int lo, int hi, float* __restrict__ S_out,
@@ -132,7 +134,7 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
       cp_async_wait<1>();
       const int cur = buf;
       buf ^= 1;
-      sweep_group<false, false, 16>(sm, amask, cur, ones, 1.0f, nullptr, g, sc, lo, K,
+      sweep_group<false, false, 16, kK>(sm, amask, cur, ones, 1.0f, nullptr, g, sc, lo, K,
                                     [&](uint2 c, uint8_t s, int8_t o) {
                                       *reinterpret_cast<uint2*>(crow + g * 8) = c;
                                       srow[g] = s;
@@ -145,7 +147,7 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
 
 template <int TW>
 const void* act_kernel_ptr() {
-  return reinterpret_cast<const void*>(&act_quant_kernel<TW>);
+  return reinterpret_cast<const void*>(&act_quant_kernel<TW, 0>);
 }
 
 }  // namespace
@@ -184,15 +186,21 @@ cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64
   if (blocks > wave) blocks = wave;
   const int64_t G = in / 16;
   const unsigned nb = static_cast<unsigned>(blocks);
-  if (tw == 1)
-    act_quant_kernel<1><<<nb, kCta, 0, stream>>>(A, tokens, G, lda, q_max, lo, hi, S, codes,
-                                                 scales, offs, status);
-  else if (tw == 2)
-    act_quant_kernel<2><<<nb, kCta, 0, stream>>>(A, tokens, G, lda, q_max, lo, hi, S, codes,
-                                                 scales, offs, status);
-  else
-    act_quant_kernel<4><<<nb, kCta, 0, stream>>>(A, tokens, G, lda, q_max, lo, hi, S, codes,
-                                                 scales, offs, status);
+  // the page's [-3, +7] window (11 candidates) gets a compile-time count
+  const bool k11 = hi - lo + 1 == 11;
+  auto launch = [&](auto tw_c, auto kk) {
+    act_quant_kernel<decltype(tw_c)::value, decltype(kk)::value><<<nb, kCta, 0, stream>>>(
+        A, tokens, G, lda, q_max, lo, hi, S, codes, scales, offs, status);
+  };
+  using T11 = std::integral_constant<int, 11>;
+  using T0 = std::integral_constant<int, 0>;
+  if (tw == 1) {
+    if (k11) launch(std::integral_constant<int, 1>{}, T11{}); else launch(std::integral_constant<int, 1>{}, T0{});
+  } else if (tw == 2) {
+    if (k11) launch(std::integral_constant<int, 2>{}, T11{}); else launch(std::integral_constant<int, 2>{}, T0{});
+  } else {
+    if (k11) launch(std::integral_constant<int, 4>{}, T11{}); else launch(std::integral_constant<int, 4>{}, T0{});
+  }
   return cudaGetLastError();
 }
 

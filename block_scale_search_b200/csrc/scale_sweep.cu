@@ -22,6 +22,8 @@
 // exact FP64 re-scoring of near-ties, exact-decision pack); they live in
 // sweep_core.cuh, shared with the online activation quantizer.
 
+#include <type_traits>
+
 #include "nvfp4_kernels.cuh"
 #include "sweep_core.cuh"
 
@@ -30,7 +32,7 @@ namespace nvfp4 {
 // thread's position in the lane grid that covers this matrix.  kFull: the
 // candidates are all 126 positive codes in ascending order (lo, hi unused;
 // the reported offset is code - base code).
-template <bool kWeighted, bool kFull = false, int kMaxK = 16>
+template <bool kWeighted, bool kFull = false, int kMaxK = 16, int kK = 0>
 __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_t* __restrict__ W,
                                              int64_t out, int64_t G, int64_t ldw,
                                              const float* __restrict__ h,
@@ -91,7 +93,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
       }
       const int cur = buf;
       buf ^= 1;
-      sweep_group<kWeighted, kFull, kMaxK>(
+      sweep_group<kWeighted, kFull, kMaxK, kK>(
           sm, amask, cur, h2, hs, h, g, sc, lo, K, [&](uint2 c, uint8_t s, int8_t o) {
             const int64_t gi = r * G + g;
             *reinterpret_cast<uint2*>(codes + r * half_in + g * 8) = c;
@@ -103,7 +105,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
   cp_async_wait<0>();
 }
 
-template <bool kWeighted>
+template <bool kWeighted, int kK>
 __global__ void __launch_bounds__(kCta, 5)
 scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64_t ldw,
                    const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
@@ -113,7 +115,8 @@ scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64
   fill_candidate_table(sm.tab);
   __syncthreads();
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  sweep_matrix<kWeighted>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, GL, R, tid);
+  sweep_matrix<kWeighted, false, 16, kK>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, GL,
+                                         R, tid);
 }
 
 // Full sweep: every positive E4M3 code is a candidate.  The 126-entry loss
@@ -162,7 +165,7 @@ cudaError_t launch_scale_sweep_full(const uint16_t* W, int64_t out, int64_t in, 
 
 // Batched sweep: CTA b belongs to the matrix whose [cta_begin, next cta_begin)
 // range holds b (binary search); within it, lanes follow that matrix's plan.
-template <bool kWeighted>
+template <bool kWeighted, int kK>
 __global__ void __launch_bounds__(kCta, 5)
 scale_sweep_batched_kernel(const SweepDesc* __restrict__ d, int64_t n, int lo, int hi) {
   __shared__ SweepSmem<16> sm;
@@ -175,26 +178,29 @@ scale_sweep_batched_kernel(const SweepDesc* __restrict__ d, int64_t n, int lo, i
   }
   const SweepDesc m = d[a];
   const int64_t tid = (static_cast<int64_t>(blockIdx.x) - m.cta_begin) * kCta + threadIdx.x;
-  sweep_matrix<kWeighted>(sm, m.W, m.out, m.G, m.ldw, m.h, m.S, lo, hi, m.codes, m.scales,
-                          m.offs, m.GL, m.R, tid);
+  sweep_matrix<kWeighted, false, 16, kK>(sm, m.W, m.out, m.G, m.ldw, m.h, m.S, lo, hi, m.codes,
+                                         m.scales, m.offs, m.GL, m.R, tid);
 }
 
 int sweep_resident_ctas(bool weighted) {
   static const int ctas[2] = {
-      resident_ctas(reinterpret_cast<const void*>(&scale_sweep_kernel<false>), kCta),
-      resident_ctas(reinterpret_cast<const void*>(&scale_sweep_kernel<true>), kCta)};
+      resident_ctas(reinterpret_cast<const void*>(&scale_sweep_kernel<false, 0>), kCta),
+      resident_ctas(reinterpret_cast<const void*>(&scale_sweep_kernel<true, 0>), kCta)};
   return ctas[weighted];
 }
 
 cudaError_t launch_scale_sweep_batched(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
                                        bool weighted, int lo, int hi, cudaStream_t stream) {
   if (n == 0 || total_ctas == 0) return cudaSuccess;
-  if (weighted)
-    scale_sweep_batched_kernel<true><<<static_cast<unsigned>(total_ctas), kCta, 0, stream>>>(
-        d_dev, n, lo, hi);
-  else
-    scale_sweep_batched_kernel<false><<<static_cast<unsigned>(total_ctas), kCta, 0, stream>>>(
-        d_dev, n, lo, hi);
+  const unsigned blocks = static_cast<unsigned>(total_ctas);
+  const int K = hi - lo + 1;
+  if (weighted) {
+    if (K == 16) scale_sweep_batched_kernel<true, 16><<<blocks, kCta, 0, stream>>>(d_dev, n, lo, hi);
+    else scale_sweep_batched_kernel<true, 0><<<blocks, kCta, 0, stream>>>(d_dev, n, lo, hi);
+  } else {
+    if (K == 16) scale_sweep_batched_kernel<false, 16><<<blocks, kCta, 0, stream>>>(d_dev, n, lo, hi);
+    else scale_sweep_batched_kernel<false, 0><<<blocks, kCta, 0, stream>>>(d_dev, n, lo, hi);
+  }
   return cudaGetLastError();
 }
 
@@ -221,12 +227,24 @@ cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64
   if (out == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((p.threads + kCta - 1) / kCta);
   const int64_t G = in / 16;
-  if (h)
-    scale_sweep_kernel<true><<<blocks, kCta, 0, stream>>>(W, out, G, ldw, h, S, lo, hi, codes,
-                                                          scales, offs, p.VL, p.R);
-  else
-    scale_sweep_kernel<false><<<blocks, kCta, 0, stream>>>(W, out, G, ldw, h, S, lo, hi, codes,
-                                                           scales, offs, p.VL, p.R);
+  // the two window sizes the pages use get a compile-time candidate count
+  const int K = hi - lo + 1;
+  auto launch = [&](auto weighted, auto kk) {
+    scale_sweep_kernel<decltype(weighted)::value, decltype(kk)::value>
+        <<<blocks, kCta, 0, stream>>>(W, out, G, ldw, h, S, lo, hi, codes, scales, offs, p.VL, p.R);
+  };
+  using T16 = std::integral_constant<int, 16>;
+  using T11 = std::integral_constant<int, 11>;
+  using T0 = std::integral_constant<int, 0>;
+  if (h) {
+    if (K == 16) launch(std::true_type{}, T16{});
+    else if (K == 11) launch(std::true_type{}, T11{});
+    else launch(std::true_type{}, T0{});
+  } else {
+    if (K == 16) launch(std::false_type{}, T16{});
+    else if (K == 11) launch(std::false_type{}, T11{});
+    else launch(std::false_type{}, T0{});
+  }
   return cudaGetLastError();
 }
 

@@ -212,12 +212,13 @@ __device__ __forceinline__ ScaleConsts scale_consts(float S) {
 //   amask      the warp's lanes taking part; all of them use the same S.
 //   h2, hs     the group's weights scaled by the power of two hs (ones for MSE);
 //   h, g       the unscaled weights and the column group, for exact re-scoring.
-//   K          candidates: hi - lo + 1, or 126 for the full sweep (kFull).
+//   K          candidates: hi - lo + 1, or 126 for the full sweep (kFull);
+//              kK > 0 fixes it at compile time (the candidate loop unrolls).
 //   store      called once as store(uint2 codes, uint8_t scale, int8_t offset):
 //              the 8 packed code bytes, the scale byte and the winning offset
 //              (addresses are formed there, after the candidate loop, so they
 //              hold no registers during it).
-template <bool kWeighted, bool kFull, int kMaxK, typename Store>
+template <bool kWeighted, bool kFull, int kMaxK, int kK, typename Store>
 __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK>& sm, unsigned amask, int cur,
                                             const f32x2_t (&h2)[8], float hs,
                                             const float* __restrict__ h, int64_t g,
@@ -264,13 +265,42 @@ __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK>& sm, unsigned amask
     b = clamp_code(b);
     const CandEntry* ce = kFull ? tab + (1 + kTabOffset) : tab + (b + lo + kTabOffset);
 
-    // ---- stage 1: fast FP32 losses of all candidates
-    float best = __uint_as_float(0x7F800000u), second = best;
-    for (int i = 0; i < K; ++i) {
-      const float Li = fast_candidate_loss<kWeighted>(y2, h2, ce[i]);
-      Lsm[i][lane] = Li;
-      if (Li < best) { second = best; best = Li; bi = i; }
-      else if (Li < second) { second = Li; }
+    // ---- stage 1: fast FP32 losses of all candidates.  With at most 16
+    // candidates the minimum and second minimum are kept as keys: a loss's
+    // bit pattern (which orders like the non-negative value) with its low 4
+    // mantissa bits replaced by the candidate index, so three integer min/max
+    // per candidate track both and equal keys go to the lowest offset.  The
+    // truncation moves a loss by less than 2^-19 of itself: two candidates it
+    // could reorder both lie below the near-tie threshold T and are re-scored
+    // exactly, and T is formed from the truncated minimum raised by 2^-18.
+    float best, second;
+    if constexpr (kMaxK <= 16) {
+      uint32_t kbest = 0xFFFFFFFFu, ksec = 0xFFFFFFFFu;
+      auto cand = [&](int i) {
+        const float Li = fast_candidate_loss<kWeighted>(y2, h2, ce[i]);
+        Lsm[i][lane] = Li;
+        const uint32_t key = (__float_as_uint(Li) & ~0xFu) | static_cast<uint32_t>(i);
+        ksec = min(ksec, max(kbest, key));
+        kbest = min(kbest, key);
+      };
+      if constexpr (kK > 0) {
+#pragma unroll
+        for (int i = 0; i < kK; ++i) cand(i);
+      } else {
+        for (int i = 0; i < K; ++i) cand(i);
+      }
+      bi = static_cast<int>(kbest & 0xFu);
+      best = __uint_as_float(kbest & ~0xFu) * (1.0f + 0x1p-18f);
+      second = __uint_as_float(ksec & ~0xFu);
+    } else {
+      best = __uint_as_float(0x7F800000u);
+      second = best;
+      for (int i = 0; i < K; ++i) {
+        const float Li = fast_candidate_loss<kWeighted>(y2, h2, ce[i]);
+        Lsm[i][lane] = Li;
+        if (Li < best) { second = best; best = Li; bi = i; }
+        else if (Li < second) { second = Li; }
+      }
     }
 
     // ---- stage 2 guard.  L is flagged when L - best <= c1 sqrt(A L) + c2 L;
