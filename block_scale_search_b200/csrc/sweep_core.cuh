@@ -107,6 +107,33 @@ __device__ __forceinline__ f32x2_t scaled_pair(uint32_t w, float p, float inv_sp
   return f2_mul(a2, f2_pack(inv_sp, inv_sp));
 }
 
+// The same with the signs kept: w / S.  E2M1 round-to-nearest-even and its
+// saturation are symmetric, so a signed quotient rounds to the negated code of
+// its magnitude and the error y - q v is the exact negation -- every fast loss
+// is bit-identical to the magnitude form -- while the conversion in stage 3
+// yields the sign bits of the packed nibbles directly.
+__device__ __forceinline__ f32x2_t scaled_pair_signed(uint32_t w, float p, float inv_sp,
+                                                      bool tiny_s) {
+  f32x2_t a2 = f2_pack(bf16_lo(w), bf16_hi(w));
+  if (tiny_s) a2 = f2_mul(a2, f2_pack(p, p));
+  return f2_mul(a2, f2_pack(inv_sp, inv_sp));
+}
+
+// Eight floats to four E2M1 bytes (RNE, saturating) in one word: byte k holds
+// v[2k] in its low nibble and v[2k+1] in its high nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const float* v) {
+  uint32_t r;
+  asm("{ .reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3}; }"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
 // Group weights h' = h * hs, hs the power of two that puts max h' in [0.5, 1)
 // (exact; the argmin is invariant and neither overflow nor underflow can
 // distort the sums).
@@ -208,6 +235,32 @@ __device__ __forceinline__ ScaleConsts scale_consts(float S) {
   return c;
 }
 
+// Final codes of eight elements (bf16 bits w8[0..7]) from the E2M1 words
+// of the two ends of their quotients' brackets: where the ends differ a
+// midpoint m lies inside, and the sign of fma(m v, S, -|w|) -- one rounding of
+// the exact m v S - |w| -- decides, zero being a tie to the even code.  Then
+// +0 for a zero magnitude: the sign of every nibble whose magnitude is 0 is
+// cleared (adding 7 to a 3-bit magnitude sets bit 3 iff it is nonzero).
+__device__ __forceinline__ uint32_t settle_word(uint32_t lo, uint32_t hi,
+                                                const uint16_t* __restrict__ w8, float v,
+                                                float S) {
+  uint32_t diff = (lo ^ hi) & 0x77777777u;
+  while (diff) {  // rare
+    const int n = (__ffs(diff) - 1) >> 2;
+    diff &= ~(0xFu << (4 * n));
+    const uint32_t kl = (lo >> (4 * n)) & 7u, kh = (hi >> (4 * n)) & 7u;
+    // |w| of the element, from the group's bytes staged in shared memory (a
+    // run-time index into the register copy would move it to local memory)
+    const float a = __uint_as_float(static_cast<uint32_t>(w8[n] & 0x7FFFu) << 16);
+    const float m = 0.5f * (e2m1_nibble_value(kl) + e2m1_nibble_value(kh));  // exact
+    const float rr = fmaf(m * v, S, -a);
+    const uint32_t k = (rr < 0.0f) ? kh : (rr > 0.0f ? kl : ((kl & 1u) ? kh : kl));
+    lo = (lo & ~(7u << (4 * n))) | (k << (4 * n));
+  }
+  const uint32_t mag = lo & 0x77777777u;
+  return lo & (0x77777777u | ((mag + 0x77777777u) & 0x88888888u));
+}
+
 // Stages 1-3 for the group this thread holds in sm.wbuf[cur][*][threadIdx.x].
 //   amask      the warp's lanes taking part; all of them use the same S.
 //   h2, hs     the group's weights scaled by the power of two hs (ones for MSE);
@@ -241,7 +294,7 @@ __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK>& sm, unsigned amask
 
   f32x2_t y2[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) y2[i] = scaled_pair(wr[i], sc.p, sc.inv_sp, sc.tiny_s);
+  for (int i = 0; i < 8; ++i) y2[i] = scaled_pair_signed(wr[i], sc.p, sc.inv_sp, sc.tiny_s);
   int b = 1, bi = 0;
   float T = 0.0f;
   bool flagged = false;
@@ -375,20 +428,23 @@ __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK>& sm, unsigned amask
   const int wcode = kFull ? 1 + bi : clamp_code(b + lo + bi);
   const CandEntry win = tab[wcode + kTabOffset];
 
-  // ---- stage 3: quantize once with the winner, exact decisions, pack
+  // ---- stage 3: quantize once with the winner, exact decisions, pack.  The
+  // signed quotient is converted at both ends of its bracket, four pairs to
+  // a word; the words differ only where an E2M1 midpoint lies inside.
+  float xl[16], xh[16];
   const f32x2_t ivlo = f2_pack(win.iv * (1.0f - 0x1p-20f), win.iv * (1.0f - 0x1p-20f));
-  uint32_t packed[2] = {0u, 0u};
+  const f32x2_t up = f2_pack(1.0f + 0x1p-19f, 1.0f + 0x1p-19f);
 #pragma unroll
   for (int pj = 0; pj < 8; ++pj) {
-    float xl0, xl1;
-    f2_unpack(f2_mul(y2[pj], ivlo), xl0, xl1);
-    const uint32_t nib = exact_e2m1_pair(xl0, xl1, fabsf(bf16_lo(wr[pj])),
-                                         fabsf(bf16_hi(wr[pj])), win.v, S);
-    // signs: bf16 bit 15 (low element) and bit 31 (high element); +0 for zero
-    const uint32_t sgn = ((wr[pj] >> 15) & 1u) << 3 | ((wr[pj] >> 31) & 1u) << 7;
-    const uint32_t nz = ((nib & 7u) ? 0x8u : 0u) | ((nib & 0x70u) ? 0x80u : 0u);
-    packed[pj >> 2] |= (nib | (sgn & nz)) << (8 * (pj & 3));
+    const f32x2_t x2 = f2_mul(y2[pj], ivlo);
+    f2_unpack(x2, xl[2 * pj], xl[2 * pj + 1]);
+    f2_unpack(f2_mul(x2, up), xh[2 * pj], xh[2 * pj + 1]);
   }
+  uint32_t packed[2] = {e2m1x8(xl), e2m1x8(xl + 8)};
+  packed[0] = settle_word(packed[0], e2m1x8(xh),
+                          reinterpret_cast<const uint16_t*>(&wbuf[cur][0][lane]), win.v, S);
+  packed[1] = settle_word(packed[1], e2m1x8(xh + 8),
+                          reinterpret_cast<const uint16_t*>(&wbuf[cur][1][lane]), win.v, S);
   // ascending offsets + strict "<": lo + bi is the lowest offset reaching it
   store(make_uint2(packed[0], packed[1]), static_cast<uint8_t>(wcode),
         static_cast<int8_t>(kFull ? wcode - b : lo + bi));
