@@ -55,20 +55,47 @@ def measured_peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi samples every 100 ms; only samples stamped inside the timed
-    region (mark_start .. mark_end) are summarised."""
+    """SM clock, power and clock-event reasons sampled during the timed region:
+    through NVML every 10 ms (read-only queries), else nvidia-smi every 100 ms.
+    Only samples stamped inside mark_start .. mark_end are summarised."""
     Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    # NVML clock-event reason bits for the four names above
+    BITS = [0x8, 0x40, 0x20, 0x4]
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
+        self.nvml = None
+        self.stop_flag = False
+        self.samples: list[tuple[float, float, float, float, set]] = []   # t, sm, max, W, reasons
         self.lines: list[tuple[float, str]] = []
         self.t = None
         self.t0 = self.t1 = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.idx)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def start(self):
+        try:
+            self.nvml = self._nvml_handle()
+            self.source = "nvml 10 ms"
+            self.t = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
@@ -77,12 +104,35 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
             return
+        self.source = "nvidia-smi 100 ms"
         self.t = threading.Thread(target=self._read, daemon=True)
         self.t.start()
 
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                w = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                rs = {n for n, b in zip(self.NAMES, self.BITS) if bits & b}
+                self.samples.append((time.time(), float(sm), float(mx), w, rs))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            ts = time.time()
+            f = [x.strip() for x in line.strip().split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                rs = {n for n, v in zip(self.NAMES, f[6:10]) if v.lower() == "active"}
+                self.samples.append((ts, float(f[2]), float(f[3]), float(f[4]), rs))
+            except ValueError:
+                continue
 
     def mark_start(self):
         self.t0 = time.time()
@@ -91,36 +141,28 @@ class ClockSampler:
         self.t1 = time.time()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        self.stop_flag = True
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
         if self.t:
             self.t.join(timeout=2)
         sm, mx, reasons, power = [], 0.0, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ts, ln in self.lines:
-            if self.t0 is not None and not (self.t0 <= ts <= (self.t1 or ts) + 0.05):
+        for ts, c, m, w, rs in self.samples:
+            if self.t0 is not None and not (self.t0 <= ts <= (self.t1 or ts) + 0.01):
                 continue
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 10:
-                continue
-            try:
-                sm.append(float(f[2]))
-                mx = max(mx, float(f[3]))
-                power.append(float(f[4]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[6:10]):
-                if v.lower() == "active":
-                    reasons.add(n)
+            sm.append(c)
+            mx = max(mx, m)
+            power.append(w)
+            reasons |= rs
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_median": statistics.median(power) if power else None}
+                "samples": len(sm), "power_w_median": statistics.median(power) if power else None,
+                "source": self.source}
 
 
 # --------------------------------------------------------------- workload
