@@ -186,7 +186,7 @@ def build_layer(rank: int, device, name: str = "llama33_70b_mlp"):
 class Step:
     """Preallocated buffers + one pass of the hot path through the C ABI."""
 
-    def __init__(self, nv, wl, Ws, Xs, device):
+    def __init__(self, nv, wl, Ws, Xs, device, serial=False):
         import torch
         self.nv, self.wl, self.Ws, self.Xs = nv, wl, Ws, Xs
         self.h = {k: torch.empty(X.shape[1], dtype=torch.float32, device=device) for k, X in Xs.items()}
@@ -203,45 +203,92 @@ class Step:
                        for n, W in Ws.items()}
         self.x_of = {m.name: m.x_key for m in wl.matrices}
         self.launches_per_step = 2 * len(Xs) + 2 * len(Ws) + len(Ws)
+        self.serial = serial
+        self.aux = torch.cuda.Stream(device=device)
 
     def run(self, ev=None):
-        """ev: optional dict kind -> list of (start, end) event pairs to record."""
+        """One layer.  ev: optional dict kind -> list of (start, end) event pairs
+        recorded on the stream each call is launched on.
+
+        Overlapped order (default): the first weight's h and S, then its sweep on
+        the main stream; the other weights' S and any further h go to a second
+        stream, launched after that sweep so the sweep's CTAs are dispatched
+        first, and each later sweep waits only for its own inputs.  The
+        HBM-bound calls thereby fill the sweeps' tails and gaps.  With
+        serial=True every call runs on the main stream in the order h, S, sweep."""
         import torch
         nv = self.nv
-        stream = torch.cuda.current_stream()
+        main = torch.cuda.current_stream()
 
-        def rec(kind, fn):
+        def rec(kind, s, fn):
             if ev is None:
                 fn()
                 return
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
+            a.record(s)
             fn()
-            b.record(stream)
+            b.record(s)
             ev.setdefault(kind, []).append((a, b))
 
-        for k, X in self.Xs.items():
-            ws = self.hws[k]
-            rec("diag_hessian", lambda X=X, k=k, ws=ws: nv.nvfp4_diag_hessian(
-                X, X.shape[0], X.shape[1], X.stride(0), self.h[k], 0, ws, ws.numel(), stream))
-        for n, W in self.Ws.items():
-            ws = self.gws[n]
-            rec("global_scale", lambda W=W, n=n, ws=ws: nv.nvfp4_global_scale(
+        def dh(k, s):
+            X, ws = self.Xs[k], self.hws[k]
+            rec("diag_hessian", s, lambda: nv.nvfp4_diag_hessian(
+                X, X.shape[0], X.shape[1], X.stride(0), self.h[k], 0, ws, ws.numel(), s))
+
+        def gs(n, s):
+            W, ws = self.Ws[n], self.gws[n]
+            rec("global_scale", s, lambda: nv.nvfp4_global_scale(
                 W, W.shape[0], W.shape[1], W.stride(0), self.wl.q_max, self.S[n], self.amax[n],
-                self.status[n], ws, ws.numel(), stream))
-        for n, W in self.Ws.items():
-            rec("scale_sweep", lambda W=W, n=n: nv.nvfp4_scale_sweep_quantize(
+                self.status[n], ws, ws.numel(), s))
+
+        def sw(n, s):
+            W = self.Ws[n]
+            rec("scale_sweep", s, lambda: nv.nvfp4_scale_sweep_quantize(
                 W, W.shape[0], W.shape[1], W.stride(0), self.h[self.x_of[n]], self.S[n], LO, HI,
-                self.codes[n], self.scales[n], None, stream))
+                self.codes[n], self.scales[n], None, s))
+
+        if self.serial:
+            for k in self.Xs:
+                dh(k, main)
+            for n in self.Ws:
+                gs(n, main)
+            for n in self.Ws:
+                sw(n, main)
+            return
+        mats = [m.name for m in self.wl.matrices]
+        first = mats[0]
+        done = {self.x_of[first]}
+        dh(self.x_of[first], main)
+        gs(first, main)
+        start = torch.cuda.Event()
+        start.record(main)
+        sw(first, main)
+        aux = self.aux
+        aux.wait_event(start)
+        ready = {}
+        for n in mats[1:]:
+            k = self.x_of[n]
+            if k not in done:
+                dh(k, aux)
+                done.add(k)
+            gs(n, aux)
+            ready[n] = torch.cuda.Event()
+            ready[n].record(aux)
+        for n in mats[1:]:
+            main.wait_event(ready[n])
+            sw(n, main)
 
 
 class GroupedStep:
     """Mixture-of-experts layer: one grouped diag-Hessian launch per
-    calibration tensor, one batched global scale and one batched sweep for all
-    matrices.  Descriptor tables are built once; run() calls the C ABI."""
+    calibration tensor, one batched global scale for all matrices, and the
+    batched sweep -- one launch for all matrices (serial), or one per
+    calibration input with the later inputs' h on a second stream beside the
+    first batch (overlapped, the default).  Descriptor tables are built once;
+    run() calls the C ABI."""
 
-    def __init__(self, nv, wl, Ws, Xs, device):
+    def __init__(self, nv, wl, Ws, Xs, device, serial=False):
         import ctypes as C
         import torch
         self.nv, self.wl, self.Ws, self.Xs = nv, wl, Ws, Xs
@@ -278,7 +325,22 @@ class GroupedStep:
         self.sdesc = (nv.SweepDesc * n)(*sdesc)
         self.sws = torch.empty(L.nvfp4_scale_sweep_quantize_batched_workspace_size(n),
                                dtype=torch.uint8, device=device)
-        self.launches_per_step = 3 * len(Xs) + 2 + 1
+        # overlapped order: the sweep batch is split by calibration input, so the
+        # first input's sweeps run while the other inputs' h are computed
+        self.serial = serial
+        self.keys = list(Xs)
+        self.part = {}
+        for k in self.keys:
+            sel = [d for d, m in zip(sdesc, mats) if m.x_key == k]
+            self.part[k] = ((nv.SweepDesc * len(sel))(*sel), len(sel),
+                            torch.empty(L.nvfp4_scale_sweep_quantize_batched_workspace_size(len(sel)),
+                                        dtype=torch.uint8, device=device))
+        self.aux = torch.cuda.Stream(device=device)
+
+    @property
+    def launches_per_step(self):
+        # grouped diag-Hessian 3 per input, batched global scale 2, sweeps 1 or 1 per input
+        return 3 * len(self.Xs) + 2 + (1 if self.serial else len(self.keys))
 
     def run(self, ev=None):
         import torch
@@ -286,31 +348,56 @@ class GroupedStep:
         stream = torch.cuda.current_stream()
         sp = stream.cuda_stream
 
-        def rec(kind, fn):
+        def rec(kind, s, fn):
             if ev is None:
                 fn()
                 return
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
+            a.record(s)
             fn()
-            b.record(stream)
+            b.record(s)
             ev.setdefault(kind, []).append((a, b))
 
         def chk(st):
             if st != 0:
                 raise RuntimeError(f"status {st}")
 
-        for k, X in self.Xs.items():
-            ws = self.hws[k]
-            rec("diag_hessian", lambda X=X, k=k, ws=ws: chk(L.nvfp4_diag_hessian_grouped(
+        def dh(k, s):
+            X, ws = self.Xs[k], self.hws[k]
+            rec("diag_hessian", s, lambda: chk(L.nvfp4_diag_hessian_grouped(
                 X.data_ptr(), self.off.data_ptr(), self.E, X.shape[0], X.shape[1], X.stride(0),
-                self.h[k].data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)))
-        rec("global_scale", lambda: chk(L.nvfp4_global_scale_batched(
-            self.mdesc, self.n, float(self.wl.q_max), self.S.data_ptr(), self.amax.data_ptr(),
-            self.status.data_ptr(), self.gws.data_ptr(), self.gws.numel(), sp)))
-        rec("scale_sweep", lambda: chk(L.nvfp4_scale_sweep_quantize_batched(
-            self.sdesc, self.n, LO, HI, self.sws.data_ptr(), self.sws.numel(), sp)))
+                self.h[k].data_ptr(), 0, ws.data_ptr(), ws.numel(), s.cuda_stream)))
+
+        def gs(s):
+            rec("global_scale", s, lambda: chk(L.nvfp4_global_scale_batched(
+                self.mdesc, self.n, float(self.wl.q_max), self.S.data_ptr(), self.amax.data_ptr(),
+                self.status.data_ptr(), self.gws.data_ptr(), self.gws.numel(), s.cuda_stream)))
+
+        def sw(table, n, ws, s):
+            rec("scale_sweep", s, lambda: chk(L.nvfp4_scale_sweep_quantize_batched(
+                table, n, LO, HI, ws.data_ptr(), ws.numel(), s.cuda_stream)))
+
+        if self.serial:
+            for k in self.keys:
+                dh(k, stream)
+            gs(stream)
+            sw(self.sdesc, self.n, self.sws, stream)
+            return
+        first = self.keys[0]
+        dh(first, stream)
+        gs(stream)
+        start = torch.cuda.Event()
+        start.record(stream)
+        sw(*self.part[first], stream)
+        self.aux.wait_event(start)
+        for k in self.keys[1:]:
+            dh(k, self.aux)
+        done = torch.cuda.Event()
+        done.record(self.aux)
+        stream.wait_event(done)
+        for k in self.keys[1:]:
+            sw(*self.part[k], stream)
 
 
 def profiled_traffic(kernel: str, units_per_launch: float):
@@ -588,6 +675,55 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def kernel_table(ev, steps, wl):
+    """Per kind: ms per step (sum of its launches' CUDA-event durations on the
+    stream each ran on), launches per step and algorithmic GB/s."""
+    kb = kernel_bytes(wl)
+    peak, peak_kind, _ = measured_peaks()
+    kern = {}
+    for kind, pairs in ev.items():
+        tot = sum(a.elapsed_time(b) for a, b in pairs) / steps   # ms per step
+        gbs = kb[kind] / (tot * 1e-3) / 1e9
+        kern[kind] = {"ms_per_step": round(tot, 4), "launch_pairs_per_step": len(pairs) // steps,
+                      "algorithmic_bytes_per_step": int(kb[kind]), "gbs": round(gbs, 1),
+                      f"frac_of_{peak_kind}": round(gbs / peak, 4),
+                      "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)}
+    return kern
+
+
+def dominant_roofline(kern, wl, clocks):
+    """Roofline object of the kernel with the most time per step."""
+    kb = kernel_bytes(wl)
+    peak, peak_kind, _ = measured_peaks()
+    dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
+    launches = kern[dom]["launch_pairs_per_step"]
+    per_launch_s = kern[dom]["ms_per_step"] / launches * 1e-3
+    if dom == "scale_sweep":
+        # compute-bound: FP32 lane operations the definition needs, against
+        # 148 SMs x 128 FP32 lanes x the SM clock sampled during the run
+        ops = SWEEP_OPS_PER_ELEM_CAND * (HI - LO + 1) * wl.weight_elems / launches
+        clk = (clocks or {}).get("sm_mhz") or 1965.0
+        peak_top = SMS * LANES_PER_SM * clk * 1e6 / 1e12
+        achieved = ops / per_launch_s / 1e12
+        return {"kernel": dom, "bound": "alu", "achieved": round(achieved, 2),
+                "peak": round(peak_top, 2), "unit": "TOP/s",
+                "peak_source": f"148 SMs x 128 FP32 lanes x {clk:.0f} MHz (sampled SM clock)",
+                "frac": round(achieved / peak_top, 4),
+                "ops_per_unit": f"{SWEEP_OPS_PER_ELEM_CAND} FP32 ops per weight element per candidate",
+                "hbm_frac_of_measured": kern[dom][f"frac_of_{peak_kind}"],
+                "traffic": profiled_traffic(dom, wl.weight_elems / launches),
+                "traffic_note": "DRAM read+write bytes per launch, from the committed ncu "
+                                "capture on the profiling-size layer, scaled by elements"}
+    achieved = kb[dom] / launches / per_launch_s / 1e9
+    units = wl.weight_elems if dom != "diag_hessian" else sum(c.tokens * c.inp
+                                                                for c in wl.calibs.values())
+    return {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS copy)", "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+            "traffic": profiled_traffic(dom, units / launches)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -596,6 +732,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serial", action="store_true",
+                    help="one stream, calls in the order h, S, sweep (no overlap)")
     ap.add_argument("--workload", default="llama33_70b_mlp",
                     choices=list(WORKLOADS) + ["act_llama33_70b"])
     args = ap.parse_args()
@@ -619,7 +757,10 @@ def main():
             dist.destroy_process_group()
         return
     wl, Ws, Xs = build_layer(rank, dev, args.workload)
-    step = (GroupedStep if args.workload == "moe_grouped" else Step)(nv, wl, Ws, Xs, dev)
+    if args.workload == "moe_grouped":
+        step = GroupedStep(nv, wl, Ws, Xs, dev, serial=args.serial)
+    else:
+        step = Step(nv, wl, Ws, Xs, dev, serial=args.serial)
 
     for _ in range(args.warmup):
         step.run()
@@ -645,16 +786,8 @@ def main():
     ms = t0.elapsed_time(t1) / args.steps
     ms_max = max_over_ranks(ms, ws)
 
-    kern = {}
-    kb = kernel_bytes(wl)
+    kern = kernel_table(ev, args.steps, wl)
     peak, peak_kind, peaks = measured_peaks()
-    for kind, pairs in ev.items():
-        tot = sum(a.elapsed_time(b) for a, b in pairs) / args.steps   # ms per step
-        gbs = kb[kind] / (tot * 1e-3) / 1e9
-        kern[kind] = {"ms_per_step": round(tot, 4), "launch_pairs_per_step": len(pairs) // args.steps,
-                      "algorithmic_bytes_per_step": int(kb[kind]), "gbs": round(gbs, 1),
-                      f"frac_of_{peak_kind}": round(gbs / peak, 4),
-                      "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)}
     wel = wl.weight_elems
     value = wel * ws / (ms_max * 1e-3)
 
@@ -700,35 +833,26 @@ def main():
                "steps": args.e2e_steps}
         del hostW, hostX
 
-    # ---- roofline of the dominant kernel
-    dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
-    launches = kern[dom]["launch_pairs_per_step"]
-    per_launch_s = kern[dom]["ms_per_step"] / launches * 1e-3
-    if dom == "scale_sweep":
-        # compute-bound: FP32 lane operations the definition needs, against
-        # 148 SMs x 128 FP32 lanes x the SM clock sampled during the run
-        ops = SWEEP_OPS_PER_ELEM_CAND * (HI - LO + 1) * wl.weight_elems / launches
-        clk = (clocks or {}).get("sm_mhz") or 1965.0
-        peak_top = SMS * LANES_PER_SM * clk * 1e6 / 1e12
-        achieved = ops / per_launch_s / 1e12
-        roofline = {"kernel": dom, "bound": "alu", "achieved": round(achieved, 2),
-                    "peak": round(peak_top, 2), "unit": "TOP/s",
-                    "peak_source": f"148 SMs x 128 FP32 lanes x {clk:.0f} MHz (sampled SM clock)",
-                    "frac": round(achieved / peak_top, 4),
-                    "ops_per_unit": f"{SWEEP_OPS_PER_ELEM_CAND} FP32 ops per weight element per candidate",
-                    "hbm_frac_of_measured": kern[dom][f"frac_of_{peak_kind}"],
-                    "traffic": profiled_traffic(dom, wl.weight_elems / launches),
-                    "traffic_note": "DRAM read+write bytes per launch, from the committed ncu "
-                                    "capture on the profiling-size layer, scaled by elements"}
-    else:
-        achieved = kb[dom] / launches / per_launch_s / 1e9
-        roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                    "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS copy)", "unit": "GB/s",
-                    "frac": round(achieved / peak, 4),
-                    "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                    "traffic": profiled_traffic(dom, (wl.weight_elems if dom != "diag_hessian" else
-                                                      sum(c.tokens * c.inp for c in wl.calibs.values()))
-                                                / launches)}
+    # ---- roofline of the dominant kernel, as timed in the region above
+    roofline = dominant_roofline(kern, wl, clocks)
+
+    # ---- the same kernels in isolation: a short serial pass (one stream,
+    # nothing beside each kernel), for the per-kernel rooflines without the
+    # contention and queueing that the overlapped schedule puts in the events
+    kern_iso = roof_iso = None
+    if not step.serial:
+        step.serial = True
+        for _ in range(3):
+            step.run()
+        barrier(ws)
+        ev_iso = {}
+        n_iso = min(args.steps, 20)
+        for _ in range(n_iso):
+            step.run(ev_iso)
+        barrier(ws)
+        step.serial = False
+        kern_iso = kernel_table(ev_iso, n_iso, wl)
+        roof_iso = dominant_roofline(kern_iso, wl, clocks)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -746,11 +870,16 @@ def main():
                        "window": [LO, HI], "q_max": wl.q_max, "weighted": True,
                        "l2": f"inputs {(wl.calib_bytes + 2 * wl.weight_elems) / 1e9:.2f} GB per "
                              f"rank > 126 MB L2; no flush",
-                       "parallelism": f"weak: {ws} rank(s), one independent layer per rank"},
+                       "parallelism": f"weak: {ws} rank(s), one independent layer per rank",
+                       "schedule": ("serial: one stream, h then S then sweeps"
+                                    if getattr(step, "serial", True) else
+                                    "overlapped: later weights' S and h on a second stream "
+                                    "beside the sweeps, each sweep waiting for its own inputs")},
             "calib_gbs": round(xbytes / (kern["diag_hessian"]["ms_per_step"] * 1e-3) / 1e9, 1),
             "quantize_elems_per_s": wel / ((kern["global_scale"]["ms_per_step"] +
                                             kern["scale_sweep"]["ms_per_step"]) * 1e-3),
-            "kernels": kern, "roofline": roofline, "e2e": e2e,
+            "kernels": kern, "roofline": roofline,
+            "kernels_isolated": kern_iso, "roofline_isolated": roof_iso, "e2e": e2e,
             "gpu_launches": step.launches_per_step * args.steps,
             "cpu_baseline": cpu, "clocks": clocks,
         }
