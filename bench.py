@@ -732,8 +732,11 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--serial", action="store_true",
-                    help="one stream, calls in the order h, S, sweep (no overlap)")
+    ap.add_argument("--schedule", default="auto", choices=["auto", "serial", "overlapped"],
+                    help="serial: one stream, calls in the order h, S, sweep; overlapped: later "
+                         "weights' S and h on a second stream beside the sweeps; auto: "
+                         "overlapped for a dense layer, serial for the MoE layer (whose split "
+                         "sweep costs more than the overlap hides)")
     ap.add_argument("--workload", default="llama33_70b_mlp",
                     choices=list(WORKLOADS) + ["act_llama33_70b"])
     args = ap.parse_args()
@@ -758,9 +761,9 @@ def main():
         return
     wl, Ws, Xs = build_layer(rank, dev, args.workload)
     if args.workload == "moe_grouped":
-        step = GroupedStep(nv, wl, Ws, Xs, dev, serial=args.serial)
+        step = GroupedStep(nv, wl, Ws, Xs, dev, serial=args.schedule != "overlapped")
     else:
-        step = Step(nv, wl, Ws, Xs, dev, serial=args.serial)
+        step = Step(nv, wl, Ws, Xs, dev, serial=args.schedule == "serial")
 
     for _ in range(args.warmup):
         step.run()

@@ -129,28 +129,43 @@ cudaError_t launch_diag_hessian(const uint16_t* X, int64_t T, int64_t in, int64_
 // Grouped diagonal Hessian: X holds the calibration rows of E experts one
 // after another (expert e owns rows row_offsets[e] .. row_offsets[e+1]) and
 // h[e, :] is each expert's own sum of squares -- one launch for all experts.
-// Rows are cut into chunks of kGroupedChunk rows that never straddle two
-// experts; a CTA sums one chunk for one strip of up to 256 16-byte column
-// vectors (a fixed-order reduction of its row lanes in shared memory) and
-// writes one partial row; the finalize kernel adds each expert's chunk rows in
-// chunk order in FP64 (deterministic) and rounds once.
+// Rows are cut into slices of about equal length that never straddle two
+// experts, about one wave of them (the plain kernel's shape: each CTA streams
+// one long contiguous run of rows).  A CTA sums one slice for one strip of up
+// to 256 16-byte column vectors (a fixed-order reduction of its row lanes in
+// shared memory) and writes one partial row; the finalize kernel adds each
+// expert's partial rows in slice order in FP64 (deterministic) and rounds once.
 namespace nvfp4 {
 
-__global__ void grouped_chunk_starts_kernel(const int64_t* __restrict__ off, int64_t E,
-                                            int64_t total, int64_t cap,
-                                            int64_t* __restrict__ cstart) {
+// Plan, on the device since the row offsets live there: slices of about
+// `target` rows (total rows / nt), cut at expert boundaries, so that the
+// partial kernel's grid is one wave with long contiguous slices per CTA.
+// cstart[e] is the first slice of expert e; cstart[E] the number of slices
+// (at most nt + E = cap); cstart[E + 1] holds the target.
+__global__ void grouped_plan_kernel(const int64_t* __restrict__ off, int64_t E, int64_t total,
+                                    int64_t nt, int64_t cap, int64_t* __restrict__ cstart) {
   if (blockIdx.x != 0 || threadIdx.x != 0) return;
-  // cap = chunk rows the workspace holds; monotone offsets never reach it, and
-  // offsets that are not monotone cannot push a chunk past it
+  int64_t rows = 0;
+  for (int64_t e = 0; e < E; ++e) {
+    int64_t a = off[e], b = off[e + 1];
+    a = a < 0 ? 0 : (a > total ? total : a);   // out-of-range offsets are clamped:
+    b = b < a ? a : (b > total ? total : b);   // no access can leave X
+    rows += b - a;
+  }
+  int64_t target = (rows + nt - 1) / nt;
+  if (target < 1) target = 1;
+  // cap bounds the slices the workspace holds; monotone offsets stay within it
+  // (sum of ceil(rows_e / target) <= nt + E), others cannot push past it
   int64_t acc = 0;
   for (int64_t e = 0; e < E; ++e) {
     cstart[e] = acc < cap ? acc : cap;
     int64_t a = off[e], b = off[e + 1];
-    a = a < 0 ? 0 : (a > total ? total : a);   // out-of-range offsets are clamped:
-    b = b < a ? a : (b > total ? total : b);   // no access can leave X
-    acc += (b - a + kGroupedChunk - 1) / kGroupedChunk;
+    a = a < 0 ? 0 : (a > total ? total : a);
+    b = b < a ? a : (b > total ? total : b);
+    acc += (b - a + target - 1) / target;
   }
   cstart[E] = acc < cap ? acc : cap;
+  cstart[E + 1] = target;
 }
 
 template <int U>
@@ -158,9 +173,10 @@ __global__ void __launch_bounds__(256)
 diag_hessian_grouped_partial_kernel(const uint16_t* __restrict__ X, const int64_t* __restrict__ off,
                                     const int64_t* __restrict__ cstart, int64_t E, int64_t total,
                                     int64_t in, int64_t ldx, float* __restrict__ P) {
-  const int64_t q = blockIdx.x;            // chunk
+  const int64_t q = blockIdx.x;            // slice
   const int64_t strip = blockIdx.y;        // 256 vectors per strip
   if (q >= cstart[E]) return;
+  const int64_t target = cstart[E + 1];
   int64_t a = 0, z = E - 1;                // expert: last e with cstart[e] <= q
   while (a < z) {
     const int64_t mid = (a + z + 1) >> 1;
@@ -170,12 +186,12 @@ diag_hessian_grouped_partial_kernel(const uint16_t* __restrict__ X, const int64_
   int64_t r_lo = off[e], r_hi = off[e + 1];
   r_lo = r_lo < 0 ? 0 : (r_lo > total ? total : r_lo);
   r_hi = r_hi < r_lo ? r_lo : (r_hi > total ? total : r_hi);
-  const int64_t rb = r_lo + (q - cstart[e]) * kGroupedChunk;
-  const int64_t re = (rb + kGroupedChunk < r_hi) ? rb + kGroupedChunk : r_hi;
+  const int64_t rb = r_lo + (q - cstart[e]) * target;
+  const int64_t re = (rb + target < r_hi) ? rb + target : r_hi;
   const int64_t V = in / 8;
   const int64_t v0 = strip * 256;
   const int VLc = static_cast<int>((V - v0) < 256 ? (V - v0) : 256);
-  const int RL = 256 / VLc;
+  const int RL = static_cast<int>(blockDim.x) / VLc;   // the block is a multiple of the widest strip
   const int vl = threadIdx.x % VLc, rl = threadIdx.x / VLc;
   float acc[8];
 #pragma unroll
@@ -241,27 +257,53 @@ diag_hessian_grouped_finalize_kernel(const float* __restrict__ P, const int64_t*
   h[e * in + j] = static_cast<float>(s + t);
 }
 
-size_t diag_hessian_grouped_workspace_bytes(int64_t total, int64_t E, int64_t in) {
-  const int64_t chunks = (total + kGroupedChunk - 1) / kGroupedChunk + E;
-  const size_t head = ((static_cast<size_t>(E + 1) * sizeof(int64_t)) + 255) & ~size_t{255};
-  return head + static_cast<size_t>(chunks) * static_cast<size_t>(in) * sizeof(float);
+namespace {
+// slices of the partial kernel: about one wave of it, less one per expert
+// (the rounding at expert boundaries adds at most one slice per expert)
+struct GroupedPlan {
+  int64_t strips, nt, cap;
+  int block;
+};
+GroupedPlan grouped_plan(int64_t E, int64_t in, int num_sms) {
+  GroupedPlan p;
+  p.strips = (in / 8 + 255) / 256;
+  // threads: row lanes x the widest strip's vectors, so no thread of a
+  // narrow row (e.g. 96 vectors for in = 768) idles
+  const int64_t v0 = in / 8 < 256 ? in / 8 : 256;
+  p.block = static_cast<int>(v0 > 0 ? v0 * (256 / v0) : 256);
+  const int ctas = resident_ctas(
+      reinterpret_cast<const void*>(&diag_hessian_grouped_partial_kernel<8>), p.block);
+  const int64_t per_strip = static_cast<int64_t>(num_sms) * ctas / p.strips;
+  p.nt = per_strip - E > 1 ? per_strip - E : 1;
+  p.cap = p.nt + E;
+  return p;
+}
+size_t grouped_head_bytes(int64_t E) {
+  return ((static_cast<size_t>(E + 2) * sizeof(int64_t)) + 255) & ~size_t{255};
+}
+}  // namespace
+
+size_t diag_hessian_grouped_workspace_bytes(int64_t total, int64_t E, int64_t in, int num_sms) {
+  (void)total;
+  const GroupedPlan p = grouped_plan(E, in, num_sms);
+  return grouped_head_bytes(E) + static_cast<size_t>(p.cap) * static_cast<size_t>(in) * sizeof(float);
 }
 
 cudaError_t launch_diag_hessian_grouped(const uint16_t* X, const int64_t* off, int64_t E,
                                         int64_t total, int64_t in, int64_t ldx, float* h,
-                                        int accumulate, void* workspace, cudaStream_t stream) {
+                                        int accumulate, void* workspace, int num_sms,
+                                        cudaStream_t stream) {
+  const GroupedPlan p = grouped_plan(E, in, num_sms);
   int64_t* cstart = static_cast<int64_t*>(workspace);
-  const size_t head = ((static_cast<size_t>(E + 1) * sizeof(int64_t)) + 255) & ~size_t{255};
-  float* P = reinterpret_cast<float*>(static_cast<char*>(workspace) + head);
-  const int64_t chunks = (total + kGroupedChunk - 1) / kGroupedChunk + E;
-  grouped_chunk_starts_kernel<<<1, 32, 0, stream>>>(off, E, total, chunks, cstart);
+  float* P = reinterpret_cast<float*>(static_cast<char*>(workspace) + grouped_head_bytes(E));
+  grouped_plan_kernel<<<1, 32, 0, stream>>>(off, E, total, p.nt, p.cap, cstart);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const int64_t strips = (in / 8 + 255) / 256;
   if (total > 0) {
-    diag_hessian_grouped_partial_kernel<8><<<dim3(static_cast<unsigned>(chunks),
-                                                  static_cast<unsigned>(strips)),
-                                             256, 0, stream>>>(X, off, cstart, E, total, in, ldx, P);
+    diag_hessian_grouped_partial_kernel<8><<<dim3(static_cast<unsigned>(p.cap),
+                                                  static_cast<unsigned>(p.strips)),
+                                             p.block, 0, stream>>>(X, off, cstart, E, total, in,
+                                                                   ldx, P);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }

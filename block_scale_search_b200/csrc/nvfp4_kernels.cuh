@@ -22,11 +22,12 @@ struct LanePlan {
 };
 
 LanePlan diag_hessian_plan(int64_t tokens, int64_t in, int num_sms);
-constexpr int64_t kGroupedChunk = 512;  // rows per chunk of the grouped diag-Hessian
-size_t diag_hessian_grouped_workspace_bytes(int64_t total, int64_t experts, int64_t in);
+size_t diag_hessian_grouped_workspace_bytes(int64_t total, int64_t experts, int64_t in,
+                                            int num_sms);
 cudaError_t launch_diag_hessian_grouped(const uint16_t* X, const int64_t* row_offsets, int64_t E,
                                         int64_t total, int64_t in, int64_t ldx, float* h,
-                                        int accumulate, void* workspace, cudaStream_t stream);
+                                        int accumulate, void* workspace, int num_sms,
+                                        cudaStream_t stream);
 size_t diag_hessian_workspace_bytes(const LanePlan& p, int64_t in);
 cudaError_t launch_diag_hessian(const uint16_t* X, int64_t T, int64_t in, int64_t ldx, float* h,
                                 int accumulate, float* partials, const LanePlan& p,

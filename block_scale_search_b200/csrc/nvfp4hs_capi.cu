@@ -235,7 +235,9 @@ size_t nvfp4_diag_hessian_grouped_workspace_size(int64_t total_tokens, int64_t e
   if (total_tokens < 0 || experts <= 0 || experts > 65535 || in <= 0 || in % 8 != 0 ||
       in > kMaxDim || total_tokens > kMaxDim)
     return 0;
-  return nvfp4::diag_hessian_grouped_workspace_bytes(total_tokens, experts, in);
+  const int sms = current_sm_count();
+  if (sms <= 0) return 0;
+  return nvfp4::diag_hessian_grouped_workspace_bytes(total_tokens, experts, in, sms);
 }
 
 int nvfp4_diag_hessian_grouped(const void* X, const int64_t* row_offsets, int64_t experts,
@@ -249,11 +251,16 @@ int nvfp4_diag_hessian_grouped(const void* X, const int64_t* row_offsets, int64_
   if (!aligned(row_offsets, 8)) return NVFP4_ERR_ALIGN;
   if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
-  if (workspace_bytes < nvfp4::diag_hessian_grouped_workspace_bytes(total_tokens, experts, in))
+  // at least one partial row per expert plus one, whatever the device
+  if (workspace_bytes < static_cast<size_t>(experts + 1) * static_cast<size_t>(in) * sizeof(float))
+    return NVFP4_ERR_WORKSPACE;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  if (workspace_bytes < nvfp4::diag_hessian_grouped_workspace_bytes(total_tokens, experts, in, sms))
     return NVFP4_ERR_WORKSPACE;
   return cuda_status(nvfp4::launch_diag_hessian_grouped(
       static_cast<const uint16_t*>(X), row_offsets, experts, total_tokens, in, ldx, h, accumulate,
-      workspace, static_cast<cudaStream_t>(stream)));
+      workspace, sms, static_cast<cudaStream_t>(stream)));
 }
 
 namespace {

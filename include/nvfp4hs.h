@@ -171,7 +171,10 @@ int nvfp4_scale_sweep_quantize_full(const void* W, int64_t out, int64_t in, int6
  * ------------------------------------------------------------------------ */
 
 /* Diagonal Hessian per expert (H-Scale summary, sec. B; one statistic per
- * expert).  X holds the experts' calibration rows back to back:
+ * expert).  The rows are cut into about one wave of equal slices that never
+ * straddle two experts; each slice's sums land in the workspace and are added
+ * per expert in a fixed order.  X holds the experts' calibration rows back to
+ * back:
  *   expert e owns rows row_offsets[e] .. row_offsets[e+1]-1 of X[total_tokens, ldx].
  *   row_offsets  DEVICE int64 [experts+1], non-decreasing, within [0, total_tokens]
  *                (offsets outside that are clamped; a decreasing table gives
@@ -179,7 +182,8 @@ int nvfp4_scale_sweep_quantize_full(const void* W, int64_t out, int64_t in, int6
  *   experts      1 .. 65535.
  *   h            float [experts, in] (row e = expert e), accumulate as above.
  *   workspace    at least nvfp4_diag_hessian_grouped_workspace_size() bytes,
- *                256-byte aligned; contents need no initialisation.
+ *                256-byte aligned; contents need no initialisation.  The size
+ *                depends on the current device's SM count (0 without a device).
  * Other arguments as nvfp4_diag_hessian. */
 size_t nvfp4_diag_hessian_grouped_workspace_size(int64_t total_tokens, int64_t experts, int64_t in);
 int nvfp4_diag_hessian_grouped(const void* X, const int64_t* row_offsets, int64_t experts,
