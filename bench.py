@@ -435,7 +435,8 @@ def kernel_bytes(wl):
 
 # ------------------------------------------------------------ CPU oracle
 
-def oracle_sample_rate(wl, Ws, Xs, threads=None, row_frac=0.25, tokens=4096):
+def oracle_sample_rate(wl, Ws, Xs, threads=None, row_frac=0.25, tokens=4096,
+                       single_thread=False):
     """Time the CPU oracle (as it stands) on a bounded sample of this workload --
     the first `row_frac` of every weight's rows and the first `tokens` tokens of
     every calibration matrix -- and extrapolate linearly to whole-job weight
@@ -470,8 +471,48 @@ def oracle_sample_rate(wl, Ws, Xs, threads=None, row_frac=0.25, tokens=4096):
                        f"elements) and the first {tokens} tokens of every calibration matrix; "
                        f"extrapolated linearly to the whole layer"),
             "cores": threads, "t_sample_s": round(t_sweep + t_abs + t_h, 3),
-            "t_full_est_s": round(t_full, 2)}
+            "t_full_est_s": round(t_full, 2), "cpu_model": cpu_model()}
+    if single_thread:
+        info["single_thread"] = oracle_single_thread_rate(wl, Ws, Xs, hs)
     return wel / t_full, info
+
+
+def cpu_model() -> str | None:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def oracle_single_thread_rate(wl, Ws, Xs, hs):
+    """The oracle on one thread, on 1/64 of the first weight's rows (global
+    scale and sweep) and 1/64 of its calibration tokens (diag-Hessian);
+    extrapolated linearly to the whole layer and labelled so."""
+    import torch
+    import oracle
+    m = wl.matrices[0]
+    r = max(1, m.out // 64)
+    sub = Ws[m.name][:r].cpu().view(torch.uint16).numpy()
+    X = Xs[m.x_key]
+    xs = X[:max(1, X.shape[0] // 64)].cpu()
+    t0 = time.perf_counter()
+    oracle.parallel_diag_hessian(xs, threads=1)
+    t_h = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    S, _, _ = oracle.global_scale(sub, wl.q_max)
+    oracle.parallel_sweep_quantize(sub, hs[m.x_key], float(S) if S > 0 else 1e-3, LO, HI, threads=1)
+    t_w = time.perf_counter() - t0
+    x_total = sum(c.tokens * c.inp for c in wl.calibs.values())
+    t_full = t_w * wl.weight_elems / sub.size + t_h * x_total / xs.numel()
+    return {"value": wl.weight_elems / t_full, "unit": "elem/s", "threads": 1,
+            "sample": (f"1/64 of {m.name}'s rows ({sub.size} elements) and 1/64 of its "
+                       f"calibration tokens ({xs.numel()} elements), one thread; "
+                       f"extrapolated linearly to the whole layer"),
+            "t_sample_s": round(t_w + t_h, 3)}
 
 
 # ------------------------------------------------- activation quantization
@@ -491,7 +532,7 @@ def oracle_act_rate(A, rows=1024, threads=None):
     t0 = time.perf_counter()
     oracle.parallel_quantize_activations(sub, ACT_Q, ACT_LO, ACT_HI, threads=threads)
     dt = time.perf_counter() - t0
-    return sub.size / dt, {"cores": threads, "t_sample_s": round(dt, 3),
+    return sub.size / dt, {"cores": threads, "t_sample_s": round(dt, 3), "cpu_model": cpu_model(),
                            "sample": f"oracle on the first {rows} of {A.shape[0]} tokens "
                                      f"({sub.size} elements); rate extrapolated linearly"}
 
@@ -670,7 +711,7 @@ def run_reference(args):
                                   "X 65536 tokens; window [-9,+6]; Q=448",
                       "impl": "CPU oracle (plain C, fp64), sampled and extrapolated"},
            "cpu_baseline": {"value": v, "unit": "elem/s", "cores": info["cores"], "kind": "oracle",
-                            "sample": info["sample"]},
+                            "sample": info["sample"], "cpu_model": info["cpu_model"]},
            "e2e": {"value": v, "unit": "elem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
@@ -859,9 +900,10 @@ def main():
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        rate, info = oracle_sample_rate(wl, Ws, Xs)
+        rate, info = oracle_sample_rate(wl, Ws, Xs, single_thread=True)
         cpu = {"value": rate, "unit": "elem/s", "cores": info["cores"], "kind": "oracle",
-               "sample": info["sample"], "t_full_est_s": info["t_full_est_s"]}
+               "sample": info["sample"], "t_full_est_s": info["t_full_est_s"],
+               "cpu_model": info["cpu_model"], "single_thread": info.get("single_thread")}
 
     if rank == 0:
         xbytes = wl.calib_bytes
