@@ -923,6 +923,12 @@ def main():
             "calib_gbs": round(xbytes / (kern["diag_hessian"]["ms_per_step"] * 1e-3) / 1e9, 1),
             "quantize_elems_per_s": wel / ((kern["global_scale"]["ms_per_step"] +
                                             kern["scale_sweep"]["ms_per_step"]) * 1e-3),
+            # the same two rates from the serial pass (no kernel running beside another)
+            "calib_gbs_isolated": (round(xbytes / (kern_iso["diag_hessian"]["ms_per_step"] * 1e-3)
+                                         / 1e9, 1) if kern_iso else None),
+            "quantize_elems_per_s_isolated": (wel / ((kern_iso["global_scale"]["ms_per_step"] +
+                                                      kern_iso["scale_sweep"]["ms_per_step"]) * 1e-3)
+                                              if kern_iso else None),
             "kernels": kern, "roofline": roofline,
             "kernels_isolated": kern_iso, "roofline_isolated": roof_iso, "e2e": e2e,
             "gpu_launches": step.launches_per_step * args.steps,
