@@ -9,7 +9,11 @@ layer-output error ||X (W - W_hat)^T||^2 against
   * plain-MSE ScaleSweep ([-3, +7], h = 1),
 while MSE ScaleSweep should lower the plain weight error against Min-Max.
 W_hat is decoded by this library's dequantize; the matmul that measures the
-output error is only the yardstick."""
+output error is only the yardstick.
+
+Also here: the chosen scale is never worse than the max-abs base scale under
+the exact evaluator (offset 0 lies in every window)."""
+import numpy as np
 import pytest
 import torch
 
@@ -53,3 +57,32 @@ def test_hessian_weighted_scales_lower_the_output_error(nv, sigma):
     assert res["mse"]["w"] < res["minmax"]["w"]
     # the weighted objective it minimises is lower than both others'
     assert res["hscale"]["hw"] < min(res["mse"]["hw"], res["minmax"]["hw"])
+
+
+@pytest.mark.parametrize("lo,hi,weighted", [(-9, 6, True), (-3, 7, False), (-8, 7, True)])
+def test_never_worse_than_the_base_scale(orc, nv, lo, hi, weighted):
+    """Offset 0 is in every window, so the chosen scale's exact loss never
+    exceeds the max-abs base scale's (ScaleSweep summary, retaining the
+    status quo).  Checked on every group of a 70B-MLP-shaped slice: the base
+    code comes from the GPU's own [0, 0] sweep, the losses from the oracle's
+    exact evaluator -- the window's on the GPU's packed bytes, the base's by
+    the definition."""
+    import workloads
+    W = workloads.weight(2048, 8192, 0.015, 0.001, 10.0, 81, DEV)
+    X = workloads.calib(8192, 8192, 1.5, 82, DEV)
+    h = nv.diag_hessian(X) if weighted else None
+    S, _, _ = nv.global_scale(W)
+    codes, scales, _ = nv.scale_sweep_quantize(W, h, S, lo, hi)
+    _, base, _ = nv.scale_sweep_quantize(W, h, S, 0, 0)
+    torch.cuda.synchronize()
+    bits = W.cpu().view(torch.uint16).numpy().reshape(-1, 16)
+    n = bits.shape[0]
+    hh = None
+    if weighted:
+        hh = np.broadcast_to(h.cpu().numpy().reshape(1, -1, 16), (2048, 512, 16)).reshape(n, 16)
+    Sf = float(S.item())
+    won = orc.packed_losses(bits, hh, Sf, codes.cpu().numpy().reshape(n, 8),
+                            scales.cpu().numpy().reshape(n))
+    at_base = orc.group_losses(bits, hh, Sf, base.cpu().numpy().reshape(n))
+    assert np.all(won <= at_base), int(np.sum(won > at_base))
+    assert np.mean(won < at_base) > 0.3      # and the search does move most groups
