@@ -44,7 +44,7 @@ namespace nvfp4 {
 
 // Per-code table in shared memory, indexed by code + 16 so that b + k for
 // k in [-16, 15] needs no clamping (entries beyond the ends repeat codes 1/126).
-struct CandEntry {
+struct alignas(16) CandEntry {
   float iv;       // 1 / v, correctly rounded
   float iv2;      // the same again, so {iv, iv} loads as one f32x2 operand
   uint32_t nvh;   // -v as f16 bits (exact: E4M3 values are f16 values)
@@ -155,8 +155,9 @@ __device__ __forceinline__ float weight_scale(float hmax) {
 template <bool kWeighted>
 __device__ __forceinline__ float fast_candidate_loss(const f32x2_t (&y2)[8], const f32x2_t (&h2)[8],
                                                      const CandEntry& t) {
-  const f32x2_t iv2 = *reinterpret_cast<const f32x2_t*>(&t.iv);  // {iv, iv}
-  const uint16_t nv = static_cast<uint16_t>(t.nvh);
+  const uint4 ent = *reinterpret_cast<const uint4*>(&t);          // one 16-byte load
+  const f32x2_t iv2 = f2_pack(__uint_as_float(ent.x), __uint_as_float(ent.y));  // {iv, iv}
+  const uint16_t nv = static_cast<uint16_t>(ent.z);
   f32x2_t acc0, acc1;
 #pragma unroll
   for (int pj = 0; pj < 8; ++pj) {
