@@ -39,6 +39,10 @@ __device__ __forceinline__ void team_barrier(int team) {
     asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
 }
 
+// CTAs per SM the compile-time 11-candidate form is built for (it needs the
+// fewest registers; more resident warps hide more latency).
+constexpr int kActCtas11 = 7;
+
 // L2 eviction priorities for the row's two reads.  Pass 1 marks the row
 // evict-last so that it is still in L2 when pass 2 reads it back; pass 2
 // marks it evict-first once used.  Without them about 60% of the rows were
@@ -65,7 +69,7 @@ __device__ __forceinline__ void cp_async16_policy(void* smem, const void* gmem, 
 }
 
 template <int TW, int kK>
-__global__ void __launch_bounds__(kCta, 5)
+__global__ void __launch_bounds__(kCta, kK == 11 ? kActCtas11 : 5)
 act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int64_t lda,
                  float q_max, int lo, int hi, float* __restrict__ S_out,
                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -172,30 +176,34 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
   }
 }
 
-template <int TW>
-const void* act_kernel_ptr() {
-  return reinterpret_cast<const void*>(&act_quant_kernel<TW, 0>);
-}
-
 }  // namespace
 
-int act_quant_resident_ctas() {
-  static const int n = resident_ctas(act_kernel_ptr<1>(), kCta);
-  return n;
+// Resident CTAs per SM of the instantiation launched for a team size and
+// window (the 11-candidate form holds more CTAs than the general one).
+int act_quant_resident_ctas(int tw, bool k11) {
+  static const int n[3][2] = {
+      {resident_ctas(reinterpret_cast<const void*>(&act_quant_kernel<1, 0>), kCta),
+       resident_ctas(reinterpret_cast<const void*>(&act_quant_kernel<1, 11>), kCta)},
+      {resident_ctas(reinterpret_cast<const void*>(&act_quant_kernel<2, 0>), kCta),
+       resident_ctas(reinterpret_cast<const void*>(&act_quant_kernel<2, 11>), kCta)},
+      {resident_ctas(reinterpret_cast<const void*>(&act_quant_kernel<4, 0>), kCta),
+       resident_ctas(reinterpret_cast<const void*>(&act_quant_kernel<4, 11>), kCta)}};
+  return n[tw == 1 ? 0 : (tw == 2 ? 1 : 2)][k11 ? 1 : 0];
 }
 
-int act_quant_team_warps(int64_t tokens, int64_t in, int num_sms) {
+int act_quant_team_warps(int64_t tokens, int64_t in, int num_sms, bool k11) {
   // cost of a team size: rounds of rows per team x groups per lane per row,
   // times the team's own overhead (the exchange and barrier of each row, and
   // fewer rows in flight per SM), measured on B200 as about 5% for two warps
   // and 15% for four at equal parallelism.  The smallest cost wins: a large
   // batch gets one warp per row, a small one spreads each row over four.
-  const int64_t wave_warps = static_cast<int64_t>(num_sms) * act_quant_resident_ctas() * (kCta / 32);
   const int64_t G = in / 16;
   const double overhead[3] = {1.0, 1.05, 1.15};
   int best_tw = 1;
   double best = -1.0;
   for (int i = 0, tw = 1; tw <= 4; ++i, tw *= 2) {
+    const int64_t wave_warps =
+        static_cast<int64_t>(num_sms) * act_quant_resident_ctas(tw, k11) * (kCta / 32);
     const int64_t teams = wave_warps / tw;
     const int64_t rounds = (tokens + teams - 1) / teams;
     const int64_t per_row = (G + 32 * tw - 1) / (32 * tw);
@@ -210,15 +218,15 @@ cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64
                                         uint8_t* codes, uint8_t* scales, int8_t* offs,
                                         int* status, int num_sms, cudaStream_t stream) {
   if (tokens == 0) return cudaSuccess;
-  const int tw = act_quant_team_warps(tokens, in, num_sms);
+  const bool k11 = hi - lo + 1 == 11;
+  const int tw = act_quant_team_warps(tokens, in, num_sms, k11);
   const int64_t teams_per_cta = (kCta / 32) / tw;
   int64_t blocks = (tokens + teams_per_cta - 1) / teams_per_cta;
-  const int64_t wave = static_cast<int64_t>(num_sms) * act_quant_resident_ctas();
+  const int64_t wave = static_cast<int64_t>(num_sms) * act_quant_resident_ctas(tw, k11);
   if (blocks > wave) blocks = wave;
   const int64_t G = in / 16;
   const unsigned nb = static_cast<unsigned>(blocks);
   // the page's [-3, +7] window (11 candidates) gets a compile-time count
-  const bool k11 = hi - lo + 1 == 11;
   auto launch = [&](auto tw_c, auto kk) {
     act_quant_kernel<decltype(tw_c)::value, decltype(kk)::value><<<nb, kCta, 0, stream>>>(
         A, tokens, G, lda, q_max, lo, hi, S, codes, scales, offs, status);

@@ -51,9 +51,10 @@ cudaError_t launch_global_scale(const uint16_t* W, int64_t out, int64_t ldw, flo
                                 float* S, float* amax, int* status, uint32_t* partial,
                                 const LanePlan& p, cudaStream_t stream);
 
-LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted);
+LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted, int K);
 LanePlan sweep_plan_threads(int64_t out, int64_t in, int64_t threads);
 int sweep_resident_ctas(bool weighted);
+int sweep_resident_ctas(bool weighted, int K);
 constexpr int kSweepCta = 128;
 
 // One matrix of a batched sweep, as the kernel reads it from device memory.
@@ -80,7 +81,7 @@ cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64
 
 // Online activation quantization: per-token S and the MSE sweep in one launch.
 // A team of 1, 2 or 4 warps owns a row at a time (chosen from the shape).
-int act_quant_team_warps(int64_t tokens, int64_t in, int num_sms);
+int act_quant_team_warps(int64_t tokens, int64_t in, int num_sms, bool k11);
 cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64_t in,
                                         int64_t lda, float q_max, int lo, int hi, float* S,
                                         uint8_t* codes, uint8_t* scales, int8_t* offs,

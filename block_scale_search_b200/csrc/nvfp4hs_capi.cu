@@ -148,7 +148,7 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
   if (empty) return NVFP4_OK;
   const int sms = current_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorNoDevice);
-  const nvfp4::LanePlan p = nvfp4::sweep_plan(out, in, sms, h != nullptr);
+  const nvfp4::LanePlan p = nvfp4::sweep_plan(out, in, sms, h != nullptr, hi - lo + 1);
   return cuda_status(nvfp4::launch_scale_sweep(static_cast<const uint16_t*>(W), out, in, ldw, h,
                                                S, lo, hi, codes, scales, chosen_offset, p,
                                                static_cast<cudaStream_t>(stream)));
