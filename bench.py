@@ -206,9 +206,15 @@ class Step:
         self.serial = serial
         self.aux = torch.cuda.Stream(device=device)
 
-    def run(self, ev=None):
+    def run(self, ev=None, io=None):
         """One layer.  ev: optional dict kind -> list of (start, end) event pairs
         recorded on the stream each call is launched on.
+
+        io (optional, for a pipelined end-to-end step): dict with "ready"
+        {"X:<input>" or "W:<weight>": event} the call using that X or W waits
+        for, "free" {weight: event} its sweep waits for before overwriting codes
+        and scales; run() fills "consumed" (same keys as "ready") after each
+        input's last reader and "produced" {weight: event} after each sweep.
 
         Overlapped order (default): the first weight's h and S, then its sweep on
         the main stream; the other weights' S and any further h go to a second
@@ -231,22 +237,39 @@ class Step:
             b.record(s)
             ev.setdefault(kind, []).append((a, b))
 
+        def wait(s, kind, name):
+            if io is not None and name in io.get(kind, {}):
+                s.wait_event(io[kind][name])
+
+        def signal(s, kind, name):
+            if io is not None:
+                e = torch.cuda.Event()
+                e.record(s)
+                io.setdefault(kind, {})[name] = e
+
         def dh(k, s):
             X, ws = self.Xs[k], self.hws[k]
+            wait(s, "ready", "X:" + k)
             rec("diag_hessian", s, lambda: nv.nvfp4_diag_hessian(
                 X, X.shape[0], X.shape[1], X.stride(0), self.h[k], 0, ws, ws.numel(), s))
+            signal(s, "consumed", "X:" + k)
 
         def gs(n, s):
             W, ws = self.Ws[n], self.gws[n]
+            wait(s, "ready", "W:" + n)
             rec("global_scale", s, lambda: nv.nvfp4_global_scale(
                 W, W.shape[0], W.shape[1], W.stride(0), self.wl.q_max, self.S[n], self.amax[n],
                 self.status[n], ws, ws.numel(), s))
 
         def sw(n, s):
             W = self.Ws[n]
+            wait(s, "ready", "W:" + n)
+            wait(s, "free", n)
             rec("scale_sweep", s, lambda: nv.nvfp4_scale_sweep_quantize(
                 W, W.shape[0], W.shape[1], W.stride(0), self.h[self.x_of[n]], self.S[n], LO, HI,
                 self.codes[n], self.scales[n], None, s))
+            signal(s, "produced", n)
+            signal(s, "consumed", "W:" + n)
 
         if self.serial:
             for k in self.Xs:
@@ -850,25 +873,59 @@ def main():
         hostC = {n: torch.empty_like(c, device="cpu").pin_memory() for n, c in step.codes.items()}
         hostS = {n: torch.empty_like(s, device="cpu").pin_memory() for n, s in step.scales.items()}
 
-        def e2e_step():
-            for k in Xs:
-                Xs[k].copy_(hostX[k], non_blocking=True)
-            for n in Ws:
-                Ws[n].copy_(hostW[n], non_blocking=True)
-            step.run()
-            for n in Ws:
-                hostC[n].copy_(step.codes[n], non_blocking=True)
-                hostS[n].copy_(step.scales[n], non_blocking=True)
+        # pipelined: inputs go in on one copy stream in the order the layer needs
+        # them, each call waits only for its own inputs, and each weight's codes
+        # and scales come back on another copy stream as soon as its sweep ends;
+        # a buffer is refilled only after its last reader (or, for outputs, the
+        # previous copy back) has finished
+        copy_in = torch.cuda.Stream(device=dev)
+        copy_out = torch.cuda.Stream(device=dev)
+        first = wl.matrices[0]
+        order = ["X:" + first.x_key, "W:" + first.name] + ["W:" + m.name for m in wl.matrices[1:]]
+        order += ["X:" + k for k in Xs if "X:" + k not in order]
+        host = {**{"X:" + k: t for k, t in hostX.items()}, **{"W:" + n: t for n, t in hostW.items()}}
+        devb = {**{"X:" + k: t for k, t in Xs.items()}, **{"W:" + n: t for n, t in Ws.items()}}
+        assert len(order) == len(host) == len(Xs) + len(Ws)
+        state = {"consumed": {}, "d2h": {}}
+
+        def e2e_step(start=None):
+            if start is not None:
+                copy_in.wait_event(start)
+            io = {"ready": {}, "free": state["d2h"]}
+            with torch.cuda.stream(copy_in):
+                for name in order:
+                    if name in state["consumed"]:
+                        copy_in.wait_event(state["consumed"][name])
+                    devb[name].copy_(host[name], non_blocking=True)
+                    e = torch.cuda.Event()
+                    e.record(copy_in)
+                    io["ready"][name] = e
+            step.run(io=io)
+            d2h = {}
+            with torch.cuda.stream(copy_out):
+                for m in wl.matrices:
+                    copy_out.wait_event(io["produced"][m.name])
+                    hostC[m.name].copy_(step.codes[m.name], non_blocking=True)
+                    hostS[m.name].copy_(step.scales[m.name], non_blocking=True)
+                    e = torch.cuda.Event()
+                    e.record(copy_out)
+                    d2h[m.name] = e
+            state["consumed"], state["d2h"] = io["consumed"], d2h
 
         e2e_step()
         barrier(ws)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        for i in range(args.e2e_steps):
+            e2e_step(a if i == 0 else None)
+        for e in state["d2h"].values():
+            stream.wait_event(e)
         b.record(stream)
         barrier(ws)
+        for n in Ws:   # what came back is what the device holds
+            assert torch.equal(hostC[n], step.codes[n].cpu()) and \
+                torch.equal(hostS[n], step.scales[n].cpu()), f"e2e copy of {n}"
         e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, ws)
         h2d = sum(t.numel() * t.element_size() for t in list(hostW.values()) + list(hostX.values()))
         d2h = sum(t.numel() for t in list(hostC.values()) + list(hostS.values()))
