@@ -24,7 +24,7 @@ __all__ = [
     "nvfp4_diag_hessian_grouped", "nvfp4_global_scale_batched_workspace_size",
     "nvfp4_global_scale_batched", "nvfp4_scale_sweep_quantize_batched_workspace_size",
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
-    "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full",
+    "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize", "nvfp4_quantize_activations",
     "quantize_activations", "nvfp4_blocked_scales_size", "nvfp4_scales_to_blocked",
@@ -74,6 +74,7 @@ _SIGS = {
     "nvfp4_global_scale_noalloc": ([_vp, _i64, _i64, _i64, _f32, _vp, _vp, _vp, _vp], _int),
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
+    "nvfp4_debug_row_counters": ([C.POINTER(_vp), C.POINTER(_sz)], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
     "nvfp4_blocked_scales_size": ([_i64, _i64], _sz),
     "nvfp4_scales_to_blocked": ([_vp, _i64, _i64, _i64, _vp, _vp], _int),
@@ -169,6 +170,14 @@ def nvfp4_scale_sweep_quantize(W, out, inp, ldw, h, S, lo, hi, codes, scales, ch
     _check("nvfp4_scale_sweep_quantize", lib().nvfp4_scale_sweep_quantize(
         _ptr(W), out, inp, ldw, _ptr(h), _ptr(S), int(lo), int(hi), _ptr(codes), _ptr(scales),
         _ptr(chosen_offset), _stream(stream)))
+
+
+def nvfp4_debug_row_counters():
+    """(device address, bytes) of the sweep's run-time row counters on the
+    current device; for tests only."""
+    p, n = _vp(), _sz()
+    _check("nvfp4_debug_row_counters", lib().nvfp4_debug_row_counters(C.byref(p), C.byref(n)))
+    return p.value, n.value
 
 
 def nvfp4_scale_sweep_quantize_full(W, out, inp, ldw, h, S, codes, scales, chosen_offset,

@@ -154,6 +154,11 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
                                                static_cast<cudaStream_t>(stream)));
 }
 
+int nvfp4_debug_row_counters(void** ptr, size_t* bytes) {
+  if (ptr == nullptr || bytes == nullptr) return NVFP4_ERR_INVALID_ARG;
+  return cuda_status(nvfp4::row_counters_symbol(ptr, bytes));
+}
+
 int nvfp4_scale_sweep_quantize_full(const void* W, int64_t out, int64_t in, int64_t ldw,
                                     const float* h, const float* S, uint8_t* codes,
                                     uint8_t* scales, int8_t* chosen_offset, void* stream) {

@@ -18,10 +18,24 @@
 // being scored (two buffers per thread), which hides the load latency without
 // spending registers.
 //
+// Where a row's column groups fill whole warps (G a multiple of 32), rows are
+// handed out at run time instead: the warps of one 32-group column strip take
+// chunks of two rows from that strip's counter as they finish, so that warps
+// the schedulers favour do more rows and every warp of the grid ends at about
+// the same time (with a fixed share per thread, the favoured warps finish
+// early and leave their SMs short of warps; the run-time hand-out is 6-8%
+// faster).  The counters live in a small pool of slots in device memory; the
+// host leases a slot to one launch at a time (an event recorded after the
+// launch tells when it is free again), the launch's last CTA zeroes it, and a
+// launch that finds no free slot, or is being captured into a graph, keeps
+// the fixed stride.
+//
 // Each group is decided in three stages (fast FP32 pass over all candidates,
 // exact FP64 re-scoring of near-ties, exact-decision pack); they live in
 // sweep_core.cuh, shared with the online activation quantizer.
 
+#include <algorithm>
+#include <mutex>
 #include <type_traits>
 
 #include "nvfp4_kernels.cuh"
@@ -105,6 +119,96 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
   cp_async_wait<0>();
 }
 
+// ------------------------------------------------- run-time row hand-out
+
+constexpr int kRowChunk = 2;           // rows per hand-out
+constexpr int kCounterSlots = 64;      // launches in flight that can lease a slot
+constexpr int kMaxStrips = 256;        // 32-group strips per row (in <= 131072)
+constexpr int kSlotWords = kMaxStrips + 2;  // strip counters, CTAs done, launches served
+
+// Zero at module load; every launch that leases a slot leaves it zeroed again
+// (apart from its count of launches served, kept for tests).
+__device__ unsigned int g_row_counters[kCounterSlots][kSlotWords];
+
+// The sweep of one matrix with rows handed out at run time.  G % 32 == 0 and
+// every lane of the grid's R * G covers one column group of every row chunk
+// it takes: chunk r0 first (rows 2 r0, 2 r0 + 1), then chunks R + t for the
+// t its strip's counter returns, until they pass the last row.  `slot` is a
+// leased slot of g_row_counters, zero at launch.
+template <bool kWeighted, int kK>
+__device__ __forceinline__ void sweep_rows_dynamic(SweepSmem<16>& sm, const uint16_t* __restrict__ W,
+                                                   int64_t out, int64_t G, int64_t ldw,
+                                                   const float* __restrict__ h,
+                                                   const float* __restrict__ Sp, int lo, int hi,
+                                                   uint8_t* __restrict__ codes,
+                                                   uint8_t* __restrict__ scales,
+                                                   int8_t* __restrict__ offs, int64_t R,
+                                                   unsigned int* __restrict__ slot, int64_t tid) {
+  auto& wbuf = sm.wbuf;
+  const int64_t r0 = tid / G;
+  const int64_t g = tid - r0 * G;
+  const int K = hi - lo + 1;
+  const int lane = threadIdx.x;
+  const ScaleConsts sc = scale_consts(*Sp);
+  const int64_t half_in = G * 8;
+  auto issue = [&](int64_t rr, int b) {
+    const uint16_t* src = W + rr * ldw + g * 16;
+    cp_async16(&wbuf[b][0][lane], src);
+    cp_async16(&wbuf[b][1][lane], src + 8);
+  };
+  f32x2_t h2[8];
+  float hs = 1.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) h2[i] = f2_pack(1.0f, 1.0f);
+  if constexpr (kWeighted) {
+    const float4* hp = reinterpret_cast<const float4*>(h + g * 16);
+    float4 hv[4];
+    float hmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      hv[i] = hp[i];
+      hmax = fmaxf(fmaxf(fmaxf(hmax, hv[i].x), fmaxf(hv[i].y, hv[i].z)), hv[i].w);
+    }
+    hs = weight_scale(hmax);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      h2[2 * i] = f2_pack(hv[i].x * hs, hv[i].y * hs);
+      h2[2 * i + 1] = f2_pack(hv[i].z * hs, hv[i].w * hs);
+    }
+  }
+  // rows fit in 32 bits here (out <= 2^23), which keeps the loop's state small
+  int r = static_cast<int>(r0) * kRowChunk;
+  int end = r + kRowChunk;
+  const int rows = static_cast<int>(out), Ri = static_cast<int>(R);
+  int buf = 0;
+  if (r < rows) issue(r, 0);
+  cp_async_commit();
+  while (r < rows) {
+    int nr = r + 1;
+    if (nr >= end) {  // warp-uniform: every lane has the same rows
+      unsigned int t = 0;
+      if ((lane & 31) == 0) t = atomicAdd(slot + (g >> 5), 1u);
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+      nr = (Ri + static_cast<int>(t)) * kRowChunk;
+      end = nr + kRowChunk;
+    }
+    if (nr < rows) issue(nr, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    const int cur = buf;
+    buf ^= 1;
+    sweep_group<kWeighted, false, 16, kK>(
+        sm, 0xFFFFFFFFu, cur, h2, hs, h, g, sc, lo, K, [&](uint2 cw, uint8_t sb, int8_t o) {
+          const int64_t gi = static_cast<int64_t>(r) * G + g;
+          *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * half_in + g * 8) = cw;
+          scales[gi] = sb;
+          if (offs) offs[gi] = o;
+        });
+    r = nr;
+  }
+  cp_async_wait<0>();
+}
+
 // Plain MSE over 11 candidates needs the fewest registers; bounded for 7
 // CTAs per SM it runs about 3% faster, while the other forms lose to spills.
 template <bool kWeighted, int kK>
@@ -119,6 +223,34 @@ scale_sweep_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   sweep_matrix<kWeighted, false, 16, kK>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, GL,
                                          R, tid);
+}
+
+// The same with rows handed out at run time (G % 32 == 0); same resources as
+// scale_sweep_kernel, so the same number of CTAs fit on an SM.  The last CTA
+// to finish zeroes the slot's counters for its next lease.
+template <bool kWeighted, int kK>
+__global__ void __launch_bounds__(kCta, (!kWeighted && kK == 11) ? 7 : 5)
+scale_sweep_rows_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64_t ldw,
+                        const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
+                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                        int8_t* __restrict__ offs, int64_t R, unsigned int* slot) {
+  __shared__ SweepSmem<16> sm;
+  fill_candidate_table(sm.tab);
+  __syncthreads();
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (tid < R * G)
+    sweep_rows_dynamic<kWeighted, kK>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, R,
+                                      slot, tid);
+  __syncthreads();  // every hand-out of this CTA is done
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(slot + kMaxStrips, 1u) == gridDim.x - 1) {
+      for (int64_t i = 0; i < (G >> 5); ++i) slot[i] = 0u;
+      slot[kMaxStrips] = 0u;
+      slot[kMaxStrips + 1] += 1u;
+      __threadfence();
+    }
+  }
 }
 
 // Full sweep: every positive E4M3 code is a candidate.  The 126-entry loss
@@ -237,18 +369,128 @@ LanePlan sweep_plan_threads(int64_t out, int64_t in, int64_t nt) {
   return p;
 }
 
+namespace {
+
+// cuEventQuery, reached through the runtime so that the library needs no
+// link to the driver library; unlike the runtime's query it leaves the
+// runtime's last-error state alone when the event is still pending.
+using EventQueryFn = int (*)(cudaEvent_t);
+EventQueryFn event_query() {
+  static const EventQueryFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuEventQuery", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return static_cast<EventQueryFn>(nullptr);
+    }
+    return reinterpret_cast<EventQueryFn>(p);
+  }();
+  return fn;
+}
+
+// The counter slots of one device: a slot is leased to one launch at a time
+// and is free again once the event recorded after that launch has completed.
+struct SlotPool {
+  std::mutex mu;
+  unsigned int* base = nullptr;  // device address of g_row_counters
+  cudaEvent_t ev[kCounterSlots] = {};
+  bool leased[kCounterSlots] = {};
+  bool retired[kCounterSlots] = {};
+  int next = 0;
+
+  // A free slot (its event created), or -1.  Called with mu held.
+  int acquire() {
+    if (base == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_row_counters) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+      }
+      base = static_cast<unsigned int*>(p);
+    }
+    const EventQueryFn query = event_query();
+    if (query == nullptr) return -1;
+    for (int k = 0; k < kCounterSlots; ++k) {
+      const int i = (next + k) % kCounterSlots;
+      if (ev[i] == nullptr) {
+        if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
+          cudaGetLastError();
+          ev[i] = nullptr;
+          return -1;
+        }
+        leased[i] = false;
+      }
+      if (retired[i] || (leased[i] && query(ev[i]) != 0)) continue;  // pending or failed
+      next = (i + 1) % kCounterSlots;
+      return i;
+    }
+    return -1;
+  }
+};
+
+SlotPool* slot_pool() {
+  static SlotPool pools[128];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return &pools[dev];
+}
+
+// A launch recorded into a graph may be replayed any number of times, also
+// concurrently, so captured launches keep the fixed row stride.
+bool capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return true;
+  }
+  return cs != cudaStreamCaptureStatusNone;
+}
+
+}  // namespace
+
+cudaError_t row_counters_symbol(void** ptr, size_t* bytes) {
+  *bytes = sizeof(g_row_counters);
+  return cudaGetSymbolAddress(ptr, g_row_counters);
+}
+
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi, uint8_t* codes,
                                uint8_t* scales, int8_t* offs, const LanePlan& p,
                                cudaStream_t stream) {
   if (out == 0) return cudaSuccess;
-  const unsigned blocks = static_cast<unsigned>((p.threads + kCta - 1) / kCta);
   const int64_t G = in / 16;
   // the two window sizes the pages use get a compile-time candidate count
   const int K = hi - lo + 1;
+  // run-time row hand-out where whole warps fit a row's groups and every row
+  // lane would otherwise take at least four rows
+  SlotPool* pool = nullptr;
+  if (G % 32 == 0 && p.VL == G && G / 32 <= kMaxStrips && out <= (int64_t{1} << 23) &&
+      out >= 4 * p.R && !capturing(stream))
+    pool = slot_pool();
+  std::unique_lock<std::mutex> lk;
+  int slot = -1;
+  if (pool != nullptr) {
+    lk = std::unique_lock<std::mutex>(pool->mu);
+    slot = pool->acquire();
+  }
+  const int64_t Rd = std::min<int64_t>(p.R, (out + kRowChunk - 1) / kRowChunk);
   auto launch = [&](auto weighted, auto kk) {
-    scale_sweep_kernel<decltype(weighted)::value, decltype(kk)::value>
-        <<<blocks, kCta, 0, stream>>>(W, out, G, ldw, h, S, lo, hi, codes, scales, offs, p.VL, p.R);
+    constexpr bool kW = decltype(weighted)::value;
+    constexpr int kKK = decltype(kk)::value;
+    if (slot >= 0) {
+      const unsigned blocks = static_cast<unsigned>((Rd * G + kCta - 1) / kCta);
+      scale_sweep_rows_kernel<kW, kKK><<<blocks, kCta, 0, stream>>>(
+          W, out, G, ldw, h, S, lo, hi, codes, scales, offs, Rd,
+          pool->base + static_cast<int64_t>(slot) * kSlotWords);
+    } else {
+      const unsigned blocks = static_cast<unsigned>((p.threads + kCta - 1) / kCta);
+      scale_sweep_kernel<kW, kKK><<<blocks, kCta, 0, stream>>>(W, out, G, ldw, h, S, lo, hi, codes,
+                                                             scales, offs, p.VL, p.R);
+    }
   };
   using T16 = std::integral_constant<int, 16>;
   using T11 = std::integral_constant<int, 11>;
@@ -262,7 +504,18 @@ cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64
     else if (K == 11) launch(std::false_type{}, T11{});
     else launch(std::false_type{}, T0{});
   }
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (slot >= 0 && e == cudaSuccess) {
+    // the slot is free again once this event completes; if it cannot be
+    // recorded, nothing would tell, and the slot is retired
+    if (cudaEventRecord(pool->ev[slot], stream) == cudaSuccess) {
+      pool->leased[slot] = true;
+    } else {
+      pool->retired[slot] = true;
+      return cudaGetLastError();
+    }
+  }
+  return e;
 }
 
 }  // namespace nvfp4

@@ -194,14 +194,15 @@ __device__ __forceinline__ uint32_t exact_e2m1_one(float xl, float a, float v, f
 
 // ------------------------------------------------------------------ kernel
 
-// Shared memory of one sweep CTA; kMaxK candidates per group at most (16 for
-// windows, 126 for the full sweep over every positive E4M3 code).
-template <int kMaxK>
+// Shared memory of one sweep CTA of kThreads threads; kMaxK candidates per
+// group at most (16 for windows, 126 for the full sweep over every positive
+// E4M3 code).
+template <int kMaxK, int kThreads = kCta>
 struct SweepSmem {
   CandEntry tab[kTabSize];
-  float Lsm[kMaxK][kCta];     // per-thread column of fast losses
-  uint4 wbuf[2][2][kCta];     // staged groups: [buffer][half][thread]
-  double tsm[kCta / 32][16];  // per-warp exchange of exact loss terms
+  float Lsm[kMaxK][kThreads];     // per-thread column of fast losses
+  uint4 wbuf[2][2][kThreads];     // staged groups: [buffer][half][thread]
+  double tsm[kThreads / 32][16];  // per-warp exchange of exact loss terms
 };
 constexpr int kFullK = 126;
 
@@ -272,8 +273,8 @@ __device__ __forceinline__ uint32_t settle_word(uint32_t lo, uint32_t hi,
 //              the 8 packed code bytes, the scale byte and the winning offset
 //              (addresses are formed there, after the candidate loop, so they
 //              hold no registers during it).
-template <bool kWeighted, bool kFull, int kMaxK, int kK, typename Store>
-__device__ __forceinline__ void sweep_group(SweepSmem<kMaxK>& sm, unsigned amask, int cur,
+template <bool kWeighted, bool kFull, int kMaxK, int kK, int kThreads, typename Store>
+__device__ __forceinline__ void sweep_group(SweepSmem<kMaxK, kThreads>& sm, unsigned amask, int cur,
                                             const f32x2_t (&h2)[8], float hs,
                                             const float* __restrict__ h, int64_t g,
                                             const ScaleConsts& sc, int lo, int K, Store&& store) {
@@ -402,7 +403,7 @@ __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK>& sm, unsigned amask
         const double vS = __dmul_rn(static_cast<double>(t.v), static_cast<double>(S));
         for (int j = rank; j < 16; j += nact) {
           // element j of group f: bf16 word (j >> 1) of its two staged halves
-          const uint32_t word = wf[((j >> 3) * kCta + tx) * 4 + ((j >> 1) & 3)];
+          const uint32_t word = wf[((j >> 3) * kThreads + tx) * 4 + ((j >> 1) & 3)];
           const float aj = fabsf((j & 1) ? bf16_hi(word) : bf16_lo(word));
           const float yj = (sc.tiny_s ? aj * sc.p : aj) * sc.inv_sp;
           const float hj = kWeighted ? h[g_f * 16 + j] * hs_f : 1.0f;

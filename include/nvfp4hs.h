@@ -143,11 +143,27 @@ int nvfp4_global_scale_noalloc(const void* W, int64_t out, int64_t in, int64_t l
  * of the base code follows IEEE round-to-nearest-even as the definition does,
  * so results agree with an exact evaluation except where two candidates' losses
  * are within ~1e-7 relative of each other.
+ * Scheduling: where in/16 is a multiple of 32 and every row lane of the grid
+ * would take four rows or more, rows are handed out at run time from counters
+ * the library keeps in device memory (one per 32-group column strip).  The
+ * counters form 64 slots, each leased to one launch at a time: the library
+ * records an event after the launch on `stream` and reuses the slot once it
+ * has completed; the launch zeroes the slot before it ends.  A launch that
+ * finds no free slot, or is being captured into a CUDA graph, uses a fixed
+ * row stride.  The bytes written do not depend on the order rows are taken
+ * in.  The library serialises its own slot bookkeeping (a mutex per device).
  * ------------------------------------------------------------------------ */
 int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi,
                                uint8_t* codes, uint8_t* scales, int8_t* chosen_offset,
                                void* stream);
+
+/* Test support: device address and size in bytes of the run-time row
+ * counters of nvfp4_scale_sweep_quantize on the current device, read-only for
+ * the caller: 64 slots of 258 uint32 words (256 strip counters, a count of
+ * finished CTAs, a count of launches the slot has served).  Returns NVFP4_OK,
+ * NVFP4_ERR_INVALID_ARG for NULL outputs, NVFP4_ERR_CUDA without a device. */
+int nvfp4_debug_row_counters(void** ptr, size_t* bytes);
 
 /* ------------------------------------------------------------------------
  * Full sweep: every one of the 126 positive E4M3 codes is a candidate --

@@ -203,3 +203,9 @@ def test_blocked_scales_validation(L):
     assert f(P, 4, 4, 4, None, None) == -1
     assert f(P, 4, 4, 4, P + 8, None) == -3          # out must be 16-byte aligned
     assert f(P, 0, 4, 4, None, None) == 0            # empty
+
+
+def test_debug_row_counters_validation(L):
+    p, n = C.c_void_p(), C.c_size_t()
+    assert L.nvfp4_debug_row_counters(None, C.byref(n)) == -1
+    assert L.nvfp4_debug_row_counters(C.byref(p), None) == -1
