@@ -9,8 +9,10 @@
 // one-row matrix (every group decided exactly as in scale_sweep.cu, h == 1).
 //
 // Work layout: a team of TW warps (TW = 1, 2 or 4 of the CTA's four) owns one
-// token row at a time; rows are dealt to teams in a stride over a one-wave
-// grid.
+// token row at a time over a one-wave grid.  Each team starts with the row of
+// its own index; with at least four rows per team it takes every further row
+// from a leased counter (row_counters.cuh) as it finishes one, otherwise it
+// strides by the number of teams.
 //   Pass 1 reads the row with 16-byte loads and takes the max of the
 //   sign-cleared bf16 bit patterns: a warp reduction, then for TW > 1 an
 //   exchange through shared memory under a named barrier of the team.
@@ -23,6 +25,7 @@
 
 #include "nvfp4hs.h"
 #include "nvfp4_kernels.cuh"
+#include "row_counters.cuh"
 #include "sweep_core.cuh"
 
 namespace nvfp4 {
@@ -73,9 +76,11 @@ __global__ void __launch_bounds__(kCta, kK == 11 ? kActCtas11 : 5)
 act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int64_t lda,
                  float q_max, int lo, int hi, float* __restrict__ S_out,
                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                 int8_t* __restrict__ offs, int* __restrict__ status) {
+                 int8_t* __restrict__ offs, int* __restrict__ status,
+                 unsigned int* __restrict__ slot) {
   __shared__ SweepSmem<16> sm;
   __shared__ uint32_t red[2][kCta / 32];  // per-warp row maxima, by row parity
+  __shared__ uint32_t nxt[2][kCta / 32];  // next row of each team, by row parity
   fill_candidate_table(sm.tab);
   __syncthreads();
 
@@ -98,9 +103,12 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
 
   const uint64_t keep = l2_policy(true), drop = l2_policy(false);
   int parity = 0, buf = 0;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kTeams + team; t < tokens;
-       t += nteams, parity ^= 1) {
+  int64_t t = static_cast<int64_t>(blockIdx.x) * kTeams + team;
+  while (t < tokens) {
     const uint16_t* row = A + t * lda;
+    // the next row, taken now and used once this one is done
+    uint32_t grab = 0;
+    if (slot != nullptr && tl == 0) grab = atomicAdd(slot, 1u);
 
     // ---- pass 1: the row's absmax as a bf16 bit pattern
     uint32_t m2 = 0;
@@ -121,11 +129,17 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
                     __vmaxu2(__vmaxu2(x.y & 0x7FFF7FFFu, x.z & 0x7FFF7FFFu), x.w & 0x7FFF7FFFu));
     }
     uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+    // the next row's index waits in shared memory (read once this row is
+    // done; the slot of this parity is not written again before the team
+    // has passed the next row's barrier)
+    if (tl == 0) nxt[parity][team] = grab;
     if constexpr (TW > 1) {
       if ((lane & 31) == 0) red[parity][warp] = mb;
       team_barrier<kTeamThreads>(team);
 #pragma unroll
       for (int i = 0; i < TW; ++i) mb = max(mb, red[parity][team * TW + i]);
+    } else {
+      __syncwarp();
     }
 
     // S_t = fl32(amax / fl32(Q * 6)); Inf or NaN in the row (a pattern at or
@@ -146,6 +160,8 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
         srow[g] = 0;
         if (orow) orow[g] = 0;
       }
+      t = slot != nullptr ? nteams + nxt[parity][team] : t + nteams;
+      parity ^= 1;
       continue;
     }
 
@@ -173,7 +189,10 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
                                     });
     }
     cp_async_wait<0>();
+    t = slot != nullptr ? nteams + nxt[parity][team] : t + nteams;
+    parity ^= 1;
   }
+  if (slot != nullptr) finish_slot(slot, 1);
 }
 
 }  // namespace
@@ -226,10 +245,13 @@ cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64
   if (blocks > wave) blocks = wave;
   const int64_t G = in / 16;
   const unsigned nb = static_cast<unsigned>(blocks);
+  // rows from a counter once every team would take four rows or more
+  CounterLease lease(stream, tokens >= 4 * blocks * teams_per_cta && tokens < (int64_t{1} << 31));
+  unsigned int* slot = lease.slot();
   // the page's [-3, +7] window (11 candidates) gets a compile-time count
   auto launch = [&](auto tw_c, auto kk) {
     act_quant_kernel<decltype(tw_c)::value, decltype(kk)::value><<<nb, kCta, 0, stream>>>(
-        A, tokens, G, lda, q_max, lo, hi, S, codes, scales, offs, status);
+        A, tokens, G, lda, q_max, lo, hi, S, codes, scales, offs, status, slot);
   };
   using T11 = std::integral_constant<int, 11>;
   using T0 = std::integral_constant<int, 0>;
@@ -240,7 +262,7 @@ cudaError_t launch_quantize_activations(const uint16_t* A, int64_t tokens, int64
   } else {
     if (k11) launch(std::integral_constant<int, 4>{}, T11{}); else launch(std::integral_constant<int, 4>{}, T0{});
   }
-  return cudaGetLastError();
+  return lease.commit(cudaGetLastError());
 }
 
 }  // namespace nvfp4

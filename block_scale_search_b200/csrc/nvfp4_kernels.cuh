@@ -74,8 +74,6 @@ cudaError_t launch_scale_sweep_full(const uint16_t* W, int64_t out, int64_t in, 
                                     cudaStream_t stream);
 cudaError_t launch_scale_sweep_batched(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
                                        bool weighted, int lo, int hi, cudaStream_t stream);
-// Address and size of the run-time row counters on the current device.
-cudaError_t row_counters_symbol(void** ptr, size_t* bytes);
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi, uint8_t* codes,
                                uint8_t* scales, int8_t* offs, const LanePlan& p,

@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "nvfp4_kernels.cuh"
+#include "row_counters.cuh"
 
 namespace {
 

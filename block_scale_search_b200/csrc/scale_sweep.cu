@@ -35,10 +35,10 @@
 // sweep_core.cuh, shared with the online activation quantizer.
 
 #include <algorithm>
-#include <mutex>
 #include <type_traits>
 
 #include "nvfp4_kernels.cuh"
+#include "row_counters.cuh"
 #include "sweep_core.cuh"
 
 namespace nvfp4 {
@@ -121,20 +121,14 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
 
 // ------------------------------------------------- run-time row hand-out
 
-constexpr int kRowChunk = 2;           // rows per hand-out
-constexpr int kCounterSlots = 64;      // launches in flight that can lease a slot
-constexpr int kMaxStrips = 256;        // 32-group strips per row (in <= 131072)
-constexpr int kSlotWords = kMaxStrips + 2;  // strip counters, CTAs done, launches served
-
-// Zero at module load; every launch that leases a slot leaves it zeroed again
-// (apart from its count of launches served, kept for tests).
-__device__ unsigned int g_row_counters[kCounterSlots][kSlotWords];
+constexpr int kRowChunk = 2;  // rows per hand-out
 
 // The sweep of one matrix with rows handed out at run time.  G % 32 == 0 and
 // every lane of the grid's R * G covers one column group of every row chunk
 // it takes: chunk r0 first (rows 2 r0, 2 r0 + 1), then chunks R + t for the
 // t its strip's counter returns, until they pass the last row.  `slot` is a
-// leased slot of g_row_counters, zero at launch.
+// leased counter slot (row_counters.cuh), zero at launch: counter s serves
+// strip s.
 template <bool kWeighted, int kK>
 __device__ __forceinline__ void sweep_rows_dynamic(SweepSmem<16>& sm, const uint16_t* __restrict__ W,
                                                    int64_t out, int64_t G, int64_t ldw,
@@ -241,16 +235,7 @@ scale_sweep_rows_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, 
   if (tid < R * G)
     sweep_rows_dynamic<kWeighted, kK>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, R,
                                       slot, tid);
-  __syncthreads();  // every hand-out of this CTA is done
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(slot + kMaxStrips, 1u) == gridDim.x - 1) {
-      for (int64_t i = 0; i < (G >> 5); ++i) slot[i] = 0u;
-      slot[kMaxStrips] = 0u;
-      slot[kMaxStrips + 1] += 1u;
-      __threadfence();
-    }
-  }
+  finish_slot(slot, static_cast<int>(G >> 5));
 }
 
 // Full sweep: every positive E4M3 code is a candidate.  The 126-entry loss
@@ -369,94 +354,6 @@ LanePlan sweep_plan_threads(int64_t out, int64_t in, int64_t nt) {
   return p;
 }
 
-namespace {
-
-// cuEventQuery, reached through the runtime so that the library needs no
-// link to the driver library; unlike the runtime's query it leaves the
-// runtime's last-error state alone when the event is still pending.
-using EventQueryFn = int (*)(cudaEvent_t);
-EventQueryFn event_query() {
-  static const EventQueryFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuEventQuery", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      cudaGetLastError();
-      return static_cast<EventQueryFn>(nullptr);
-    }
-    return reinterpret_cast<EventQueryFn>(p);
-  }();
-  return fn;
-}
-
-// The counter slots of one device: a slot is leased to one launch at a time
-// and is free again once the event recorded after that launch has completed.
-struct SlotPool {
-  std::mutex mu;
-  unsigned int* base = nullptr;  // device address of g_row_counters
-  cudaEvent_t ev[kCounterSlots] = {};
-  bool leased[kCounterSlots] = {};
-  bool retired[kCounterSlots] = {};
-  int next = 0;
-
-  // A free slot (its event created), or -1.  Called with mu held.
-  int acquire() {
-    if (base == nullptr) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_row_counters) != cudaSuccess) {
-        cudaGetLastError();
-        return -1;
-      }
-      base = static_cast<unsigned int*>(p);
-    }
-    const EventQueryFn query = event_query();
-    if (query == nullptr) return -1;
-    for (int k = 0; k < kCounterSlots; ++k) {
-      const int i = (next + k) % kCounterSlots;
-      if (ev[i] == nullptr) {
-        if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
-          cudaGetLastError();
-          ev[i] = nullptr;
-          return -1;
-        }
-        leased[i] = false;
-      }
-      if (retired[i] || (leased[i] && query(ev[i]) != 0)) continue;  // pending or failed
-      next = (i + 1) % kCounterSlots;
-      return i;
-    }
-    return -1;
-  }
-};
-
-SlotPool* slot_pool() {
-  static SlotPool pools[128];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  return &pools[dev];
-}
-
-// A launch recorded into a graph may be replayed any number of times, also
-// concurrently, so captured launches keep the fixed row stride.
-bool capturing(cudaStream_t s) {
-  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
-    cudaGetLastError();
-    return true;
-  }
-  return cs != cudaStreamCaptureStatusNone;
-}
-
-}  // namespace
-
-cudaError_t row_counters_symbol(void** ptr, size_t* bytes) {
-  *bytes = sizeof(g_row_counters);
-  return cudaGetSymbolAddress(ptr, g_row_counters);
-}
-
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi, uint8_t* codes,
                                uint8_t* scales, int8_t* offs, const LanePlan& p,
@@ -467,25 +364,18 @@ cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64
   const int K = hi - lo + 1;
   // run-time row hand-out where whole warps fit a row's groups and every row
   // lane would otherwise take at least four rows
-  SlotPool* pool = nullptr;
-  if (G % 32 == 0 && p.VL == G && G / 32 <= kMaxStrips && out <= (int64_t{1} << 23) &&
-      out >= 4 * p.R && !capturing(stream))
-    pool = slot_pool();
-  std::unique_lock<std::mutex> lk;
-  int slot = -1;
-  if (pool != nullptr) {
-    lk = std::unique_lock<std::mutex>(pool->mu);
-    slot = pool->acquire();
-  }
+  const bool handout = G % 32 == 0 && p.VL == G && G / 32 <= kSlotCounters &&
+                       out <= (int64_t{1} << 23) && out >= 4 * p.R;
+  CounterLease lease(stream, handout);
+  unsigned int* slot = lease.slot();
   const int64_t Rd = std::min<int64_t>(p.R, (out + kRowChunk - 1) / kRowChunk);
   auto launch = [&](auto weighted, auto kk) {
     constexpr bool kW = decltype(weighted)::value;
     constexpr int kKK = decltype(kk)::value;
-    if (slot >= 0) {
+    if (slot != nullptr) {
       const unsigned blocks = static_cast<unsigned>((Rd * G + kCta - 1) / kCta);
       scale_sweep_rows_kernel<kW, kKK><<<blocks, kCta, 0, stream>>>(
-          W, out, G, ldw, h, S, lo, hi, codes, scales, offs, Rd,
-          pool->base + static_cast<int64_t>(slot) * kSlotWords);
+          W, out, G, ldw, h, S, lo, hi, codes, scales, offs, Rd, slot);
     } else {
       const unsigned blocks = static_cast<unsigned>((p.threads + kCta - 1) / kCta);
       scale_sweep_kernel<kW, kKK><<<blocks, kCta, 0, stream>>>(W, out, G, ldw, h, S, lo, hi, codes,
@@ -504,18 +394,7 @@ cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64
     else if (K == 11) launch(std::false_type{}, T11{});
     else launch(std::false_type{}, T0{});
   }
-  const cudaError_t e = cudaGetLastError();
-  if (slot >= 0 && e == cudaSuccess) {
-    // the slot is free again once this event completes; if it cannot be
-    // recorded, nothing would tell, and the slot is retired
-    if (cudaEventRecord(pool->ev[slot], stream) == cudaSuccess) {
-      pool->leased[slot] = true;
-    } else {
-      pool->retired[slot] = true;
-      return cudaGetLastError();
-    }
-  }
-  return e;
+  return lease.commit(cudaGetLastError());
 }
 
 }  // namespace nvfp4

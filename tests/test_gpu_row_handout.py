@@ -1,9 +1,10 @@
-"""The sweep's run-time row hand-out writes the same bytes as the fixed row
-stride.  A sweep recorded into a CUDA graph keeps the fixed stride, so a graph
-replay gives the reference bytes; direct launches of the same shapes lease a
-counter slot and take rows from it (checked by reading the slots).  Also:
-more launches in flight at once than there are slots, where the launches
-that find none keep the fixed stride.  Needs a B200."""
+"""The run-time row hand-out (weight sweep and activation quantizer) writes
+the same bytes as the fixed row stride.  A launch recorded into a CUDA graph
+keeps the fixed stride, so a graph replay gives the reference bytes; direct
+launches of the same shapes lease a counter slot and take rows from it
+(checked by reading the slots).  Also: more launches in flight at once than
+there are slots, where the launches that find none keep the fixed stride.
+Needs a B200."""
 import pytest
 import torch
 
@@ -115,22 +116,58 @@ def test_more_launches_in_flight_than_slots(nv):
     n0 = _served(nv)
     n = SLOTS + 16
     streams = [torch.cuda.Stream() for _ in range(n)]
+    outs = [_alloc(*mats[i % len(mats)][0].shape) for i in range(n)]
+    torch.cuda.synchronize()
     gate = torch.cuda.Event()
-    torch.cuda._sleep(200_000_000)  # about 0.1 s: every launch below is queued behind it
+    torch.cuda._sleep(1_000_000_000)  # about 0.5 s: every launch below is queued behind it
     gate.record()
     runs = []
     for i in range(n):
         W, h, S, lo, hi, ref = mats[i % len(mats)]
         out, inp = W.shape
-        bufs = _alloc(out, inp)
         s = streams[i]
         s.wait_event(gate)
-        nv.nvfp4_scale_sweep_quantize(W, out, inp, inp, h, S, lo, hi, *bufs, stream=s)
-        runs.append((bufs, ref))
+        nv.nvfp4_scale_sweep_quantize(W, out, inp, inp, h, S, lo, hi, *outs[i], stream=s)
+        runs.append((outs[i], ref))
     torch.cuda.synchronize()
     for bufs, ref in runs:
         for a, b in zip(bufs, ref):
             assert torch.equal(a, b)
     # the first 64 leased a slot each; the 16 that found none kept the stride
     assert _served(nv) - n0 == SLOTS
+    assert torch.all(_slots(nv)[:, :STRIPS + 1] == 0)
+
+
+@pytest.mark.parametrize("tokens,inp,lo,hi", [(20011, 2048, -3, 7), (70000, 256, -9, 6)])
+def test_activation_rows_from_the_counter(nv, tokens, inp, lo, hi):
+    """The activation quantizer takes rows from a leased counter once every
+    team would have four rows or more; a graph replay keeps the stride."""
+    import workloads
+    A = workloads.calib(tokens, inp, 1.5, 41 + tokens % 7, DEV)
+
+    def bufs():
+        return (torch.empty(tokens, dtype=torch.float32, device=DEV),
+                torch.empty(tokens, inp // 2, dtype=torch.uint8, device=DEV),
+                torch.empty(tokens, inp // 16, dtype=torch.uint8, device=DEV),
+                torch.empty(tokens, inp // 16, dtype=torch.int8, device=DEV),
+                torch.empty(1, dtype=torch.int32, device=DEV))
+
+    ref = bufs()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    n0 = _served(nv)
+    with torch.cuda.graph(g, stream=s):
+        nv.nvfp4_quantize_activations(A, tokens, inp, inp, 256.0, lo, hi, *ref, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    del g
+    n1 = _served(nv)
+    got = bufs()
+    nv.nvfp4_quantize_activations(A, tokens, inp, inp, 256.0, lo, hi, *got)
+    torch.cuda.synchronize()
+    assert n1 == n0 and _served(nv) == n1 + 1
+    assert int(got[4].item()) == 0 and int(ref[4].item()) == 0
+    for a, b in zip(got[:4], ref[:4]):
+        assert torch.equal(a, b)
     assert torch.all(_slots(nv)[:, :STRIPS + 1] == 0)
