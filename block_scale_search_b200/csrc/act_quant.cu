@@ -181,7 +181,7 @@ act_quant_kernel(const uint16_t* __restrict__ A, int64_t tokens, int64_t G, int6
       cp_async_wait<1>();
       const int cur = buf;
       buf ^= 1;
-      sweep_group<false, false, 16, kK>(sm, amask, cur, ones, 1.0f, nullptr, g, sc, lo, K,
+      sweep_group<false, false, 16, kK>(sm, amask, cur, ones, 1.0f, 16.0f, nullptr, g, sc, lo, K,
                                     [&](uint2 c, uint8_t s, int8_t o) {
                                       *reinterpret_cast<uint2*>(crow + g * 8) = c;
                                       srow[g] = s;

@@ -75,25 +75,10 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
 
   for (int64_t g = gl; g < G; g += GL) {
     f32x2_t h2[8];
-    float hs = 1.0f;
+    float hs = 1.0f, hsum = 16.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) h2[i] = f2_pack(1.0f, 1.0f);
-    if constexpr (kWeighted) {
-      const float4* hp = reinterpret_cast<const float4*>(h + g * 16);
-      float4 hv[4];
-      float hmax = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        hv[i] = hp[i];
-        hmax = fmaxf(fmaxf(fmaxf(hmax, hv[i].x), fmaxf(hv[i].y, hv[i].z)), hv[i].w);
-      }
-      hs = weight_scale(hmax);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        h2[2 * i] = f2_pack(hv[i].x * hs, hv[i].y * hs);
-        h2[2 * i + 1] = f2_pack(hv[i].z * hs, hv[i].w * hs);
-      }
-    }
+    if constexpr (kWeighted) group_weights(h, g, h2, hs, hsum);
 
     for (int64_t r = r0; r < out; r += R) {
       const unsigned amask = __activemask();
@@ -108,7 +93,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
       const int cur = buf;
       buf ^= 1;
       sweep_group<kWeighted, kFull, kMaxK, kK>(
-          sm, amask, cur, h2, hs, h, g, sc, lo, K, [&](uint2 c, uint8_t s, int8_t o) {
+          sm, amask, cur, h2, hs, hsum, h, g, sc, lo, K, [&](uint2 c, uint8_t s, int8_t o) {
             const int64_t gi = r * G + g;
             *reinterpret_cast<uint2*>(codes + r * half_in + g * 8) = c;
             scales[gi] = s;
@@ -151,25 +136,10 @@ __device__ __forceinline__ void sweep_rows_dynamic(SweepSmem<16>& sm, const uint
     cp_async16(&wbuf[b][1][lane], src + 8);
   };
   f32x2_t h2[8];
-  float hs = 1.0f;
+  float hs = 1.0f, hsum = 16.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) h2[i] = f2_pack(1.0f, 1.0f);
-  if constexpr (kWeighted) {
-    const float4* hp = reinterpret_cast<const float4*>(h + g * 16);
-    float4 hv[4];
-    float hmax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      hv[i] = hp[i];
-      hmax = fmaxf(fmaxf(fmaxf(hmax, hv[i].x), fmaxf(hv[i].y, hv[i].z)), hv[i].w);
-    }
-    hs = weight_scale(hmax);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      h2[2 * i] = f2_pack(hv[i].x * hs, hv[i].y * hs);
-      h2[2 * i + 1] = f2_pack(hv[i].z * hs, hv[i].w * hs);
-    }
-  }
+  if constexpr (kWeighted) group_weights(h, g, h2, hs, hsum);
   // rows fit in 32 bits here (out <= 2^23), which keeps the loop's state small
   int r = static_cast<int>(r0) * kRowChunk;
   int end = r + kRowChunk;
@@ -192,7 +162,7 @@ __device__ __forceinline__ void sweep_rows_dynamic(SweepSmem<16>& sm, const uint
     const int cur = buf;
     buf ^= 1;
     sweep_group<kWeighted, false, 16, kK>(
-        sm, 0xFFFFFFFFu, cur, h2, hs, h, g, sc, lo, K, [&](uint2 cw, uint8_t sb, int8_t o) {
+        sm, 0xFFFFFFFFu, cur, h2, hs, hsum, h, g, sc, lo, K, [&](uint2 cw, uint8_t sb, int8_t o) {
           const int64_t gi = static_cast<int64_t>(r) * G + g;
           *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * half_in + g * 8) = cw;
           scales[gi] = sb;

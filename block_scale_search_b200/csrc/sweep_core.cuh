@@ -148,6 +148,31 @@ __device__ __forceinline__ float weight_scale(float hmax) {
   return hs;
 }
 
+// The group's weights h' = h * hs as eight pairs, hs from weight_scale, and
+// their sum (which bounds sum h' y^2 by sum h' * max y^2 for the guard).
+__device__ __forceinline__ void group_weights(const float* __restrict__ h, int64_t g,
+                                              f32x2_t (&h2)[8], float& hs, float& hsum) {
+  const float4* hp = reinterpret_cast<const float4*>(h + g * 16);
+  float4 hv[4];
+  float hmax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hv[i] = hp[i];
+    hmax = fmaxf(fmaxf(fmaxf(hmax, hv[i].x), fmaxf(hv[i].y, hv[i].z)), hv[i].w);
+  }
+  hs = weight_scale(hmax);
+  f32x2_t s2 = f2_pack(0.0f, 0.0f);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    h2[2 * i] = f2_pack(hv[i].x * hs, hv[i].y * hs);
+    h2[2 * i + 1] = f2_pack(hv[i].z * hs, hv[i].w * hs);
+    s2 = f2_add(s2, f2_add(h2[2 * i], h2[2 * i + 1]));
+  }
+  float s0, s1;
+  f2_unpack(s2, s0, s1);
+  hsum = s0 + s1;
+}
+
 // -------------------------------------------------------- stage 1 (fast)
 
 // Fast FP32 loss of one candidate: E2M1 round of y/v by the hardware
@@ -266,6 +291,7 @@ __device__ __forceinline__ uint32_t settle_word(uint32_t lo, uint32_t hi,
 // Stages 1-3 for the group this thread holds in sm.wbuf[cur][*][threadIdx.x].
 //   amask      the warp's lanes taking part; all of them use the same S.
 //   h2, hs     the group's weights scaled by the power of two hs (ones for MSE);
+//   hsum       the sum of the scaled weights (16 for MSE);
 //   h, g       the unscaled weights and the column group, for exact re-scoring.
 //   K          candidates: hi - lo + 1, or 126 for the full sweep (kFull);
 //              kK > 0 fixes it at compile time (the candidate loop unrolls).
@@ -275,7 +301,7 @@ __device__ __forceinline__ uint32_t settle_word(uint32_t lo, uint32_t hi,
 //              hold no registers during it).
 template <bool kWeighted, bool kFull, int kMaxK, int kK, int kThreads, typename Store>
 __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK, kThreads>& sm, unsigned amask, int cur,
-                                            const f32x2_t (&h2)[8], float hs,
+                                            const f32x2_t (&h2)[8], float hs, float hsum,
                                             const float* __restrict__ h, int64_t g,
                                             const ScaleConsts& sc, int lo, int K, Store&& store) {
   const CandEntry* tab = sm.tab;
@@ -301,13 +327,6 @@ __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK, kThreads>& sm, unsi
   float T = 0.0f;
   bool flagged = false;
   if (nonzero) {
-    f32x2_t A2 = f2_pack(0.0f, 0.0f);  // sum h' y^2, for the error bound of stage 2
-#pragma unroll
-    for (int i = 0; i < 8; ++i) A2 = f2_fma(kWeighted ? f2_mul(h2[i], y2[i]) : y2[i], y2[i], A2);
-    float A0, A1;
-    f2_unpack(A2, A0, A1);
-    const float A = A0 + A1;
-
     // base code: E4M3_RNE_sat(fl32(fl32(a / 6) / S)), clamped to [1, 126].
     // An FP32 approximation within 2^-21 decides unless an E4M3 rounding
     // boundary lies within 2^-20 of it; then the two IEEE divisions do.
@@ -365,10 +384,27 @@ __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK, kThreads>& sm, unsi
     // other candidate is flagged iff the second-smallest loss is.
     constexpr float c1 = 0x1p-19f, c2 = 0x1p-15f;
     constexpr float k2 = 1.0f / (2.0f * (1.0f - c2));
-    const float ca = c1 * sqrt_approx(A);
-    const float sr = (ca + sqrt_approx(fmaf(ca, ca, 4.0f * (1.0f - c2) * best))) * k2;
-    T = sr * sr * (1.0f + 0x1p-16f);
+    auto threshold = [&](float A) {
+      const float ca = c1 * sqrt_approx(A);
+      const float sr = (ca + sqrt_approx(fmaf(ca, ca, 4.0f * (1.0f - c2) * best))) * k2;
+      return sr * sr * (1.0f + 0x1p-16f);
+    };
+    // A = sum h' y^2.  T grows with A, so the bound sum h' * max y^2 (max |y|
+    // is |w|max taken through the same operations as every y) leaves
+    // unflagged every group that A itself would; only where it flags is A
+    // summed and the test repeated.
+    const float ymax = (sc.tiny_s ? a * sc.p : a) * sc.inv_sp;
+    T = threshold(hsum * ymax * ymax);
     flagged = second <= T;
+    if (flagged) {
+      f32x2_t A2 = f2_pack(0.0f, 0.0f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) A2 = f2_fma(kWeighted ? f2_mul(h2[i], y2[i]) : y2[i], y2[i], A2);
+      float A0, A1;
+      f2_unpack(A2, A0, A1);
+      T = threshold(A0 + A1);
+      flagged = second <= T;
+    }
   }
 
   // ---- stage 2, rare: the warp resolves its flagged groups together.  For
