@@ -209,3 +209,6 @@ def test_debug_row_counters_validation(L):
     p, n = C.c_void_p(), C.c_size_t()
     assert L.nvfp4_debug_row_counters(None, C.byref(n)) == -1
     assert L.nvfp4_debug_row_counters(C.byref(p), None) == -1
+    import torch
+    if not torch.cuda.is_available():   # no device: a CUDA error, not a crash
+        assert L.nvfp4_debug_row_counters(C.byref(p), C.byref(n)) == -6
