@@ -186,7 +186,7 @@ def build_layer(rank: int, device, name: str = "llama33_70b_mlp"):
 class Step:
     """Preallocated buffers + one pass of the hot path through the C ABI."""
 
-    def __init__(self, nv, wl, Ws, Xs, device, serial=False):
+    def __init__(self, nv, wl, Ws, Xs, device, serial=False, layer=False):
         import torch
         self.nv, self.wl, self.Ws, self.Xs = nv, wl, Ws, Xs
         self.h = {k: torch.empty(X.shape[1], dtype=torch.float32, device=device) for k, X in Xs.items()}
@@ -204,7 +204,22 @@ class Step:
         self.x_of = {m.name: m.x_key for m in wl.matrices}
         self.launches_per_step = 2 * len(Xs) + 2 * len(Ws) + len(Ws)
         self.serial = serial
+        self.layer = layer
         self.aux = torch.cuda.Stream(device=device)
+        # the one-call form: descriptors for nvfp4_quantize_layer over the same buffers
+        keys = list(Xs)
+        self.mats = [m.name for m in wl.matrices]
+        self.layer_w = [nv.LayerWeight(Ws[n].data_ptr(), Ws[n].shape[0], Ws[n].shape[1],
+                                       Ws[n].stride(0), keys.index(self.x_of[n]),
+                                       self.S[n].data_ptr(), self.amax[n].data_ptr(),
+                                       self.status[n].data_ptr(), self.codes[n].data_ptr(),
+                                       self.scales[n].data_ptr(), None) for n in self.mats]
+        self.layer_x = [nv.LayerInput(Xs[k].data_ptr(), Xs[k].shape[0], Xs[k].shape[1],
+                                      Xs[k].stride(0), self.h[k].data_ptr()) for k in keys]
+        self.layer_arrays = nv._layer_arrays(self.layer_w, self.layer_x)
+        nb = nv.nvfp4_quantize_layer_workspace_size(self.layer_w, self.layer_x)
+        self.layer_ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+        self.layer_nb = nb
 
     def run(self, ev=None, io=None):
         """One layer.  ev: optional dict kind -> list of (start, end) event pairs
@@ -225,6 +240,38 @@ class Step:
         import torch
         nv = self.nv
         main = torch.cuda.current_stream()
+
+        if self.layer and not self.serial:
+            # one call: the library streams the HBM-bound reductions beside the
+            # FP32-bound sweeps; events around each sweep launch time the
+            # sweeps (with what they carry), one pair around the call the rest
+            if io is not None:
+                for e in io.get("ready", {}).values():
+                    main.wait_event(e)
+                for e in io.get("free", {}).values():
+                    main.wait_event(e)
+            sev = None
+            if ev is not None:
+                sev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(self.mats))]
+                for e in sev:   # torch creates the CUDA event at its first record
+                    e.record(main)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(main)
+            wa, xa = self.layer_arrays
+            nv.nvfp4_quantize_layer(wa, xa, self.wl.q_max, LO, HI, self.layer_ws, self.layer_nb,
+                                    sweep_events=sev, stream=main)
+            if ev is not None:
+                b.record(main)
+                ev.setdefault("layer_call", []).append((a, b))
+                for j in range(len(self.mats)):
+                    ev.setdefault("scale_sweep", []).append((sev[2 * j], sev[2 * j + 1]))
+            if io is not None:
+                e = torch.cuda.Event()
+                e.record(main)
+                io["consumed"] = {**{"X:" + k: e for k in self.Xs}, **{"W:" + n: e for n in self.Ws}}
+                io["produced"] = {n: e for n in self.Ws}
+            return
 
         def rec(kind, s, fn):
             if ev is None:
@@ -626,6 +673,10 @@ def run_activations(args, nv, rank, local, ws, dev):
             hC.copy_(codes, non_blocking=True)
             hK.copy_(scales, non_blocking=True)
 
+        # the per-step calls pipeline with the copies (each waits for its own
+        # inputs); the one-call form would wait for all of them
+        layer_mode = getattr(step, "layer", False)
+        step.layer = False
         e2e_step()
         barrier(ws)
         a = torch.cuda.Event(enable_timing=True)
@@ -635,6 +686,7 @@ def run_activations(args, nv, rank, local, ws, dev):
             e2e_step()
         b.record(stream)
         barrier(ws)
+        step.layer = layer_mode
         e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, ws)
         e2e = {"value": el * ws / (e_ms * 1e-3), "unit": "elem/s", "ms_per_step": round(e_ms, 3),
                "h2d_bytes_per_step": int(hA.numel() * 2),
@@ -746,6 +798,8 @@ def kernel_table(ev, steps, wl):
     peak, peak_kind, _ = measured_peaks()
     kern = {}
     for kind, pairs in ev.items():
+        if kind not in kb:
+            continue
         tot = sum(a.elapsed_time(b) for a, b in pairs) / steps   # ms per step
         gbs = kb[kind] / (tot * 1e-3) / 1e9
         kern[kind] = {"ms_per_step": round(tot, 4), "launch_pairs_per_step": len(pairs) // steps,
@@ -755,8 +809,9 @@ def kernel_table(ev, steps, wl):
     return kern
 
 
-def dominant_roofline(kern, wl, clocks):
-    """Roofline object of the kernel with the most time per step."""
+def dominant_roofline(kern, wl, clocks, traffic_key=None):
+    """Roofline object of the kernel with the most time per step.  traffic_key:
+    the traffic record to report (default: the kernel's own kind)."""
     kb = kernel_bytes(wl)
     peak, peak_kind, _ = measured_peaks()
     dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
@@ -775,7 +830,7 @@ def dominant_roofline(kern, wl, clocks):
                 "frac": round(achieved / peak_top, 4),
                 "ops_per_unit": f"{SWEEP_OPS_PER_ELEM_CAND} FP32 ops per weight element per candidate",
                 "hbm_frac_of_measured": kern[dom][f"frac_of_{peak_kind}"],
-                "traffic": profiled_traffic(dom, wl.weight_elems / launches),
+                "traffic": profiled_traffic(traffic_key or dom, wl.weight_elems / launches),
                 "traffic_note": "DRAM read+write bytes per launch, from the committed ncu "
                                 "capture on the profiling-size layer, scaled by elements"}
     achieved = kb[dom] / launches / per_launch_s / 1e9
@@ -796,11 +851,13 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--schedule", default="auto", choices=["auto", "serial", "overlapped"],
-                    help="serial: one stream, calls in the order h, S, sweep; overlapped: later "
-                         "weights' S and h on a second stream beside the sweeps; auto: "
-                         "overlapped for a dense layer, serial for the MoE layer (whose split "
-                         "sweep costs more than the overlap hides)")
+    ap.add_argument("--schedule", default="auto",
+                    choices=["auto", "layer", "serial", "overlapped"],
+                    help="layer: one nvfp4_quantize_layer call per step, which streams the "
+                         "HBM-bound reductions beside the FP32-bound sweeps; serial: the per-step "
+                         "calls on one stream in the order h, S, sweep; overlapped: the per-step "
+                         "calls with later weights' S and h on a second stream; auto: layer for "
+                         "a dense layer, serial for the MoE layer (grouped calls)")
     ap.add_argument("--workload", default="llama33_70b_mlp",
                     choices=list(WORKLOADS) + ["act_llama33_70b"])
     args = ap.parse_args()
@@ -827,7 +884,12 @@ def main():
     if args.workload == "moe_grouped":
         step = GroupedStep(nv, wl, Ws, Xs, dev, serial=args.schedule != "overlapped")
     else:
-        step = Step(nv, wl, Ws, Xs, dev, serial=args.schedule == "serial")
+        step = Step(nv, wl, Ws, Xs, dev, serial=args.schedule == "serial",
+                    layer=args.schedule in ("auto", "layer"))
+        if step.layer:
+            # prologue (2 reductions x partial + finalize), the sweeps, and one
+            # finalize per reduction carried by a sweep
+            step.launches_per_step = 2 * 2 + len(Ws) + (len(Ws) - 1) + (len(Xs) - 1)
 
     for _ in range(args.warmup):
         step.run()
@@ -935,13 +997,39 @@ def main():
         del hostW, hostX
 
     # ---- roofline of the dominant kernel, as timed in the region above
-    roofline = dominant_roofline(kern, wl, clocks)
+    in_layer = getattr(step, "layer", False) and not getattr(step, "serial", True)
+    roofline = dominant_roofline(kern, wl, clocks,
+                                 traffic_key="scale_sweep_layer" if in_layer else None)
+    layer_info = None
+    if in_layer:
+        # the sweeps carry every reduction but the first weight's S and its
+        # input's h: their bytes ride in the sweep launches timed above
+        call_ms = sum(a.elapsed_time(b) for a, b in ev["layer_call"]) / args.steps
+        sweep_ms = kern["scale_sweep"]["ms_per_step"]
+        first = wl.matrices[0]
+        side = (wl.calib_bytes - 2 * wl.calibs[first.x_key].tokens * wl.calibs[first.x_key].inp
+                + 2 * (wl.weight_elems - first.out * first.inp))
+        sweep_launches = kern["scale_sweep"]["launch_pairs_per_step"]
+        carry = [m for m in wl.matrices[:-1]]
+        carry_ms = sum(a.elapsed_time(b) for i, (a, b) in enumerate(ev["scale_sweep"])
+                       if i % sweep_launches < len(carry)) / args.steps
+        layer_info = {
+            "call_ms_per_step": round(call_ms, 4), "sweeps_ms_per_step": round(sweep_ms, 4),
+            "rest_ms_per_step": round(call_ms - sweep_ms, 4),
+            "side_bytes_per_step": int(side),
+            "carrying_sweeps_ms_per_step": round(carry_ms, 4),
+            "carrying_sweeps_hbm_gbs": (round((side + SWEEP_BYTES_PER_ELEM * sum(
+                m.out * m.inp for m in carry)) / (carry_ms * 1e-3) / 1e9, 1)
+                if carry_ms > 0 else None),
+            "note": "the first weight's S and its input's h run first on their own (rest); "
+                    "the other weights' S and the other inputs' h are streamed by a fifth warp "
+                    "in each CTA of the earlier sweeps (carrying sweeps)"}
 
     # ---- the same kernels in isolation: a short serial pass (one stream,
     # nothing beside each kernel), for the per-kernel rooflines without the
     # contention and queueing that the overlapped schedule puts in the events
     kern_iso = roof_iso = None
-    if not step.serial:
+    if not getattr(step, "serial", True):
         step.serial = True
         for _ in range(3):
             step.run()
@@ -973,13 +1061,19 @@ def main():
                        "l2": f"inputs {(wl.calib_bytes + 2 * wl.weight_elems) / 1e9:.2f} GB per "
                              f"rank > 126 MB L2; no flush",
                        "parallelism": f"weak: {ws} rank(s), one independent layer per rank",
-                       "schedule": ("serial: one stream, h then S then sweeps"
+                       "schedule": ("layer: one nvfp4_quantize_layer call per step; the "
+                                    "HBM-bound reductions ride in the FP32-bound sweeps"
+                                    if in_layer else
+                                    "serial: one stream, h then S then sweeps"
                                     if getattr(step, "serial", True) else
                                     "overlapped: later weights' S and h on a second stream "
                                     "beside the sweeps, each sweep waiting for its own inputs")},
-            "calib_gbs": round(xbytes / (kern["diag_hessian"]["ms_per_step"] * 1e-3) / 1e9, 1),
-            "quantize_elems_per_s": wel / ((kern["global_scale"]["ms_per_step"] +
-                                            kern["scale_sweep"]["ms_per_step"]) * 1e-3),
+            "calib_gbs": (round(xbytes / (kern["diag_hessian"]["ms_per_step"] * 1e-3) / 1e9, 1)
+                          if "diag_hessian" in kern else None),
+            "quantize_elems_per_s": (wel / ((kern["global_scale"]["ms_per_step"] +
+                                             kern["scale_sweep"]["ms_per_step"]) * 1e-3)
+                                     if "global_scale" in kern else None),
+            "layer": layer_info,
             # the same two rates from the serial pass (no kernel running beside another)
             "calib_gbs_isolated": (round(xbytes / (kern_iso["diag_hessian"]["ms_per_step"] * 1e-3)
                                          / 1e9, 1) if kern_iso else None),

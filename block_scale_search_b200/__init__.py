@@ -25,6 +25,8 @@ __all__ = [
     "nvfp4_global_scale_batched", "nvfp4_scale_sweep_quantize_batched_workspace_size",
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
+    "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "quantize_layer_many",
+    "LayerWeight", "LayerInput",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize", "nvfp4_quantize_activations",
     "quantize_activations", "nvfp4_blocked_scales_size", "nvfp4_scales_to_blocked",
@@ -64,6 +66,18 @@ class SweepDesc(C.Structure):
                 ("codes", _vp), ("scales", _vp), ("chosen_offset", _vp)]
 
 
+class LayerWeight(C.Structure):
+    """nvfp4_layer_weight"""
+    _fields_ = [("W", _vp), ("out", _i64), ("inp", _i64), ("ldw", _i64), ("input", _int),
+                ("S", _vp), ("amax", _vp), ("status", _vp), ("codes", _vp), ("scales", _vp),
+                ("chosen_offset", _vp)]
+
+
+class LayerInput(C.Structure):
+    """nvfp4_layer_input"""
+    _fields_ = [("X", _vp), ("tokens", _i64), ("inp", _i64), ("ldx", _i64), ("h", _vp)]
+
+
 _SIGS = {
     "nvfp4_version": ([], _int),
     "nvfp4_last_cuda_error": ([], _int),
@@ -75,6 +89,10 @@ _SIGS = {
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
     "nvfp4_debug_row_counters": ([C.POINTER(_vp), C.POINTER(_sz)], _int),
+    "nvfp4_quantize_layer_workspace_size": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput),
+                                             _int], _sz),
+    "nvfp4_quantize_layer": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput), _int, _f32, _int,
+                              _int, _vp, _sz, C.POINTER(_vp), _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
     "nvfp4_blocked_scales_size": ([_i64, _i64], _sz),
     "nvfp4_scales_to_blocked": ([_vp, _i64, _i64, _i64, _vp, _vp], _int),
@@ -170,6 +188,36 @@ def nvfp4_scale_sweep_quantize(W, out, inp, ldw, h, S, lo, hi, codes, scales, ch
     _check("nvfp4_scale_sweep_quantize", lib().nvfp4_scale_sweep_quantize(
         _ptr(W), out, inp, ldw, _ptr(h), _ptr(S), int(lo), int(hi), _ptr(codes), _ptr(scales),
         _ptr(chosen_offset), _stream(stream)))
+
+
+def _layer_arrays(weights, inputs):
+    wa = (LayerWeight * max(1, len(weights)))(*weights)
+    xa = (LayerInput * max(1, len(inputs)))(*inputs)
+    return wa, xa
+
+
+def nvfp4_quantize_layer_workspace_size(weights, inputs) -> int:
+    """weights: list of LayerWeight, inputs: list of LayerInput."""
+    wa, xa = _layer_arrays(weights, inputs)
+    return lib().nvfp4_quantize_layer_workspace_size(wa, len(weights), xa, len(inputs))
+
+
+def nvfp4_quantize_layer(weights, inputs, q_max, lo, hi, workspace, workspace_bytes,
+                         sweep_events=None, stream=None):
+    """weights/inputs: lists of LayerWeight/LayerInput (or ready ctypes arrays);
+    sweep_events: None or 2 * len(weights) torch.cuda.Event, recorded around
+    each weight's sweep launch (torch creates a CUDA event at its first
+    record, so record each once before passing it)."""
+    if isinstance(weights, list):
+        wa, xa = _layer_arrays(weights, inputs)
+    else:
+        wa, xa = weights, inputs
+    ev = None
+    if sweep_events is not None:
+        ev = (_vp * len(sweep_events))(*[e.cuda_event for e in sweep_events])
+    _check("nvfp4_quantize_layer", lib().nvfp4_quantize_layer(
+        wa, len(weights), xa, len(inputs), float(q_max), int(lo), int(hi), _ptr(workspace),
+        workspace_bytes, ev, _stream(stream)))
 
 
 def nvfp4_debug_row_counters():
@@ -369,6 +417,39 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor | None, q_max: float = 448.0
     S, _, _ = global_scale(W, q_max, stream=stream)
     codes, scales, _ = scale_sweep_quantize(W, h, S, lo, hi, stream=stream)
     return codes, scales, S, h
+
+
+def quantize_layer_many(Ws, Xs, inputs, q_max: float = 448.0, lo: int = -9, hi: int = 6,
+                        want_offsets: bool = False, stream=None):
+    """Several projections of one layer in one call (nvfp4_quantize_layer).
+    Ws: bf16 weights; Xs: bf16 calibration inputs; inputs[j]: index into Xs of
+    W_j's input, or -1 for plain MSE.  Returns (list of (codes, scales, S,
+    offsets or None, status) per weight, list of h per input)."""
+    Ws = [_bf16_2d(W, "W") for W in Ws]
+    Xs = [_bf16_2d(X, "X") for X in Xs]
+    dev = (Ws or Xs)[0].device
+    hs = [torch.empty(X.shape[1], dtype=torch.float32, device=dev) for X in Xs]
+    outs, wd = [], []
+    for W, k in zip(Ws, inputs):
+        o, n = W.shape
+        codes = torch.empty(o, n // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(o, n // 16, dtype=torch.uint8, device=dev)
+        S = torch.empty(1, dtype=torch.float32, device=dev)
+        status = torch.empty(1, dtype=torch.int32, device=dev)
+        offs = torch.empty(o, n // 16, dtype=torch.int8, device=dev) if want_offsets else None
+        wd.append(LayerWeight(W.data_ptr(), o, n, W.stride(0), int(k), S.data_ptr(), None,
+                              status.data_ptr(), codes.data_ptr(), scales.data_ptr(), _ptr(offs)))
+        outs.append((codes, scales, S, offs, status))
+    xd = [LayerInput(X.data_ptr(), X.shape[0], X.shape[1], X.stride(0), h.data_ptr())
+          for X, h in zip(Xs, hs)]
+    nb = nvfp4_quantize_layer_workspace_size(wd, xd)
+    if nb == 0:
+        raise NVFP4Error("nvfp4_quantize_layer_workspace_size", -1)
+    ws = torch.empty(nb + 256, dtype=torch.uint8, device=dev)
+    base = (-ws.data_ptr()) % 256
+    wsv = ws[base:base + nb]
+    nvfp4_quantize_layer(wd, xd, q_max, lo, hi, wsv, nb, stream)
+    return outs, hs
 
 
 def diag_hessian_grouped(X: torch.Tensor, row_offsets: torch.Tensor, h: torch.Tensor | None = None,

@@ -69,22 +69,34 @@ diag_hessian_partial_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t i
   }
 }
 
+// Second pass: 8 threads per column, thread g adding partial rows g, g + 8,
+// ... in FP64 in order; the eight sums are combined in a fixed tree, and the
+// result is rounded once to FP32 (deterministic for a given R).  Block:
+// 32 columns x 8 row groups.
 __global__ void __launch_bounds__(256)
 diag_hessian_finalize_kernel(const float* __restrict__ P, int64_t R, int64_t in, float* h,
                              int accumulate) {
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= in) return;
-  double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-  int64_t r = 0;
-  for (; r + 3 < R; r += 4) {
-    s0 += P[(r + 0) * in + j];
-    s1 += P[(r + 1) * in + j];
-    s2 += P[(r + 2) * in + j];
-    s3 += P[(r + 3) * in + j];
+  __shared__ double part[8][33];
+  const int c = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + c;
+  double s = 0.0;
+  if (j < in)
+    for (int64_t r = g; r < R; r += 8) s += P[r * in + j];
+  part[g][c] = s;
+  __syncthreads();
+  if (g == 0 && j < in) {
+    const double t = ((part[0][c] + part[1][c]) + (part[2][c] + part[3][c])) +
+                     ((part[4][c] + part[5][c]) + (part[6][c] + part[7][c]));
+    const double base = accumulate ? static_cast<double>(h[j]) : 0.0;
+    h[j] = static_cast<float>(base + t);
   }
-  for (; r < R; ++r) s0 += P[r * in + j];
-  const double base = accumulate ? static_cast<double>(h[j]) : 0.0;
-  h[j] = static_cast<float>(base + ((s0 + s1) + (s2 + s3)));
+}
+
+cudaError_t launch_diag_hessian_finalize(const float* partials, int64_t rows, int64_t in, float* h,
+                                         int accumulate, cudaStream_t stream) {
+  diag_hessian_finalize_kernel<<<static_cast<unsigned>((in + 31) / 32), 256, 0, stream>>>(
+      partials, rows, in, h, accumulate);
+  return cudaGetLastError();
 }
 
 // Lane plan shared by the host-side workspace query and the launch.
@@ -118,9 +130,7 @@ cudaError_t launch_diag_hessian(const uint16_t* X, int64_t T, int64_t in, int64_
     if (e != cudaSuccess) return e;
   }
   const int64_t rows = T > 0 ? p.R : 0;  // no tokens: finalize adds nothing
-  diag_hessian_finalize_kernel<<<static_cast<unsigned>((in + 255) / 256), 256, 0, stream>>>(
-      partials, rows, in, h, accumulate);
-  return cudaGetLastError();
+  return launch_diag_hessian_finalize(partials, rows, in, h, accumulate, stream);
 }
 
 }  // namespace nvfp4

@@ -111,6 +111,12 @@ size_t global_scale_workspace_bytes(const LanePlan& p) {
   return static_cast<size_t>(blocks) * sizeof(uint32_t);
 }
 
+cudaError_t launch_global_scale_finalize(const uint32_t* partial, int n, float q_max, float* S,
+                                         float* amax, int* status, cudaStream_t stream) {
+  global_scale_finalize_kernel<<<1, 256, 0, stream>>>(partial, n, q_max, S, amax, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_global_scale(const uint16_t* W, int64_t out, int64_t ldw, float q_max,
                                 float* S, float* amax, int* status, uint32_t* partial,
                                 const LanePlan& p, cudaStream_t stream) {

@@ -32,6 +32,9 @@ size_t diag_hessian_workspace_bytes(const LanePlan& p, int64_t in);
 cudaError_t launch_diag_hessian(const uint16_t* X, int64_t T, int64_t in, int64_t ldx, float* h,
                                 int accumulate, float* partials, const LanePlan& p,
                                 cudaStream_t stream);
+// The second pass alone: h[j] (+)= sum over the `rows` partial rows, in order.
+cudaError_t launch_diag_hessian_finalize(const float* partials, int64_t rows, int64_t in, float* h,
+                                         int accumulate, cudaStream_t stream);
 
 LanePlan global_scale_plan(int64_t out, int64_t in, int num_sms);
 int absmax_resident_ctas();
@@ -50,6 +53,9 @@ size_t global_scale_workspace_bytes(const LanePlan& p);
 cudaError_t launch_global_scale(const uint16_t* W, int64_t out, int64_t ldw, float q_max,
                                 float* S, float* amax, int* status, uint32_t* partial,
                                 const LanePlan& p, cudaStream_t stream);
+// S (and amax, status) from n partial maxima of sign-cleared bf16 patterns.
+cudaError_t launch_global_scale_finalize(const uint32_t* partial, int n, float q_max, float* S,
+                                         float* amax, int* status, cudaStream_t stream);
 
 LanePlan sweep_plan(int64_t out, int64_t in, int num_sms, bool weighted, int K);
 LanePlan sweep_plan_threads(int64_t out, int64_t in, int64_t threads);
@@ -74,10 +80,44 @@ cudaError_t launch_scale_sweep_full(const uint16_t* W, int64_t out, int64_t in, 
                                     cudaStream_t stream);
 cudaError_t launch_scale_sweep_batched(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
                                        bool weighted, int lo, int hi, cudaStream_t stream);
+// A sweep that streams side reductions (side_reduce.cuh) with a fifth warp
+// per CTA.  Only shapes that hand rows out at run time qualify
+// (sweep_can_carry); *carried says whether it was launched that way -- if
+// not, nothing was launched and the caller sweeps and reduces by itself.
+struct SideWork;
+bool sweep_can_carry(int64_t out, int64_t in, int num_sms);
+cudaError_t launch_scale_sweep_side(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
+                                    const float* h, const float* S, int lo, int hi,
+                                    uint8_t* codes, uint8_t* scales, int8_t* offs,
+                                    const SideWork& side, int num_sms, bool* carried,
+                                    cudaStream_t stream);
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi, uint8_t* codes,
                                uint8_t* scales, int8_t* offs, const LanePlan& p,
                                cudaStream_t stream);
+
+// A layer's projections in one call (layer.cu).  input: index of the
+// calibration input whose h weights the matrix, -1 for plain MSE.
+struct LayerWeight {
+  const uint16_t* W;
+  int64_t out, in, ldw;
+  int input;
+  float* S;
+  float* amax;
+  int* status;
+  uint8_t* codes;
+  uint8_t* scales;
+  int8_t* offs;
+};
+struct LayerInput {
+  const uint16_t* X;
+  int64_t tokens, in, ldx;
+  float* h;
+};
+size_t layer_workspace_bytes(const LayerWeight* w, int nw, const LayerInput* x, int nx, int sms);
+cudaError_t quantize_layer(const LayerWeight* w, int nw, const LayerInput* x, int nx, float q_max,
+                           int lo, int hi, void* workspace, int sms, const cudaEvent_t* events,
+                           cudaStream_t stream);
 
 // Online activation quantization: per-token S and the MSE sweep in one launch.
 // A team of 1, 2 or 4 warps owns a row at a time (chosen from the shape).

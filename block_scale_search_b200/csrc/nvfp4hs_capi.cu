@@ -67,6 +67,37 @@ int check_matrix(const void* W, int64_t out, int64_t in, int64_t ldw, int64_t in
   return NVFP4_OK;
 }
 
+// Arguments of nvfp4_quantize_layer, converted for the planner; NVFP4_OK or
+// the first failing status.
+int check_layer(const nvfp4_layer_weight* w, int nw, const nvfp4_layer_input* x, int nx,
+                std::vector<nvfp4::LayerWeight>* wv, std::vector<nvfp4::LayerInput>* xv) {
+  if (nw < 0 || nx < 0 || (nw > 0 && w == nullptr) || (nx > 0 && x == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  for (int k = 0; k < nx; ++k) {
+    const nvfp4_layer_input& in = x[k];
+    int st = check_diag_hessian(in.X, in.tokens, in.in, in.ldx, in.h, 0);
+    if (st != NVFP4_OK) return st;
+    if (!aligned(in.h, 16)) return NVFP4_ERR_ALIGN;  // the sweep reads h in 16-byte vectors
+    if (xv) xv->push_back(nvfp4::LayerInput{static_cast<const uint16_t*>(in.X), in.tokens, in.in,
+                                            in.ldx, in.h});
+  }
+  for (int j = 0; j < nw; ++j) {
+    const nvfp4_layer_weight& m = w[j];
+    int st = check_matrix(m.W, m.out, m.in, m.ldw, 16);
+    if (st != NVFP4_OK) return st;
+    if (m.out == 0 || m.in == 0) return NVFP4_ERR_SHAPE;
+    if (m.S == nullptr || m.codes == nullptr || m.scales == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (m.input < -1 || m.input >= nx) return NVFP4_ERR_INVALID_ARG;
+    if (m.input >= 0 && x[m.input].in != m.in) return NVFP4_ERR_SHAPE;
+    if (!aligned(m.S, 4) || !aligned(m.amax, 4) || !aligned(m.status, 4) || !aligned(m.codes, 8))
+      return NVFP4_ERR_ALIGN;
+    if (wv) wv->push_back(nvfp4::LayerWeight{static_cast<const uint16_t*>(m.W), m.out, m.in, m.ldw,
+                                             m.input, m.S, m.amax, m.status, m.codes, m.scales,
+                                             m.chosen_offset});
+  }
+  return NVFP4_OK;
+}
+
 }  // namespace
 
 namespace nvfp4 {
@@ -153,6 +184,41 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
   return cuda_status(nvfp4::launch_scale_sweep(static_cast<const uint16_t*>(W), out, in, ldw, h,
                                                S, lo, hi, codes, scales, chosen_offset, p,
                                                static_cast<cudaStream_t>(stream)));
+}
+
+size_t nvfp4_quantize_layer_workspace_size(const nvfp4_layer_weight* weights, int n_weights,
+                                           const nvfp4_layer_input* inputs, int n_inputs) {
+  std::vector<nvfp4::LayerWeight> wv;
+  std::vector<nvfp4::LayerInput> xv;
+  if (check_layer(weights, n_weights, inputs, n_inputs, &wv, &xv) != NVFP4_OK) return 0;
+  const int sms = current_sm_count();
+  if (sms <= 0) return 0;
+  return nvfp4::layer_workspace_bytes(wv.data(), n_weights, xv.data(), n_inputs, sms);
+}
+
+int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
+                         const nvfp4_layer_input* inputs, int n_inputs, float q_max, int lo,
+                         int hi, void* workspace, size_t workspace_bytes,
+                         void* const* sweep_events, void* stream) {
+  std::vector<nvfp4::LayerWeight> wv;
+  std::vector<nvfp4::LayerInput> xv;
+  int st = check_layer(weights, n_weights, inputs, n_inputs, &wv, &xv);
+  if (st != NVFP4_OK) return st;
+  if (!std::isfinite(q_max) || !(q_max > 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  if (n_weights == 0 && n_inputs == 0) return NVFP4_OK;
+  if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  if (workspace_bytes < nvfp4::layer_workspace_bytes(wv.data(), n_weights, xv.data(), n_inputs, sms))
+    return NVFP4_ERR_WORKSPACE;
+  if (sweep_events != nullptr)
+    for (int j = 0; j < 2 * n_weights; ++j)
+      if (sweep_events[j] == nullptr) return NVFP4_ERR_INVALID_ARG;
+  return cuda_status(nvfp4::quantize_layer(
+      wv.data(), n_weights, xv.data(), n_inputs, q_max, lo, hi, workspace, sms,
+      reinterpret_cast<cudaEvent_t const*>(sweep_events), static_cast<cudaStream_t>(stream)));
 }
 
 int nvfp4_debug_row_counters(void** ptr, size_t* bytes) {

@@ -3,29 +3,11 @@
 
 namespace nvfp4 {
 
-// Zero at module load; every launch that leases a slot leaves it zeroed again
+// Zero at module load; every launch that takes a slot leaves it zeroed again
 // (apart from its count of launches served, kept for tests).
 __device__ unsigned int g_row_counters[kCounterSlots][kSlotWords];
 
 namespace {
-
-// cuEventQuery, reached through the runtime so that the library needs no
-// link to the driver library; unlike the runtime's query it leaves the
-// runtime's last-error state alone while the event is pending.
-using EventQueryFn = int (*)(cudaEvent_t);
-EventQueryFn event_query() {
-  static const EventQueryFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuEventQuery", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      cudaGetLastError();
-      return static_cast<EventQueryFn>(nullptr);
-    }
-    return reinterpret_cast<EventQueryFn>(p);
-  }();
-  return fn;
-}
 
 // A launch recorded into a graph may be replayed any number of times, also
 // concurrently, so captured launches keep the fixed share.
@@ -40,17 +22,20 @@ bool capturing(cudaStream_t s) {
 
 }  // namespace
 
-// The slots of one device: a slot is leased to one launch at a time and is
-// free again once the event recorded after that launch has completed.
+// The slots of one device, handed out in turn.  A launch that takes a slot
+// first makes its stream wait for the event recorded after the slot's
+// previous launch: on the same stream that costs nothing (stream order), on
+// another it orders the two launches, so two launches never share a slot at
+// the same time and no launch is ever refused one.
 struct CounterLease::Pool {
   std::mutex mu;
   unsigned int* base = nullptr;  // device address of g_row_counters
   cudaEvent_t ev[kCounterSlots] = {};
-  bool leased[kCounterSlots] = {};
+  bool used[kCounterSlots] = {};
   bool retired[kCounterSlots] = {};
   int next = 0;
 
-  // A free slot (its event created), or -1.  Called with mu held.
+  // The next usable slot (its event created), or -1.  Called with mu held.
   int acquire() {
     if (base == nullptr) {
       void* p = nullptr;
@@ -60,19 +45,15 @@ struct CounterLease::Pool {
       }
       base = static_cast<unsigned int*>(p);
     }
-    const EventQueryFn query = event_query();
-    if (query == nullptr) return -1;
     for (int k = 0; k < kCounterSlots; ++k) {
       const int i = (next + k) % kCounterSlots;
-      if (ev[i] == nullptr) {
-        if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
-          cudaGetLastError();
-          ev[i] = nullptr;
-          return -1;
-        }
-        leased[i] = false;
+      if (retired[i]) continue;
+      if (ev[i] == nullptr &&
+          cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        ev[i] = nullptr;
+        return -1;
       }
-      if (retired[i] || (leased[i] && query(ev[i]) != 0)) continue;  // pending or failed
       next = (i + 1) % kCounterSlots;
       return i;
     }
@@ -91,18 +72,24 @@ CounterLease::CounterLease(cudaStream_t stream, bool want) : stream_(stream) {
   pool_ = &pools[dev];
   lock_ = std::unique_lock<std::mutex>(pool_->mu);
   index_ = pool_->acquire();
-  if (index_ >= 0) slot_ = pool_->base + static_cast<size_t>(index_) * kSlotWords;
+  if (index_ < 0) return;
+  if (pool_->used[index_] && cudaStreamWaitEvent(stream, pool_->ev[index_], 0) != cudaSuccess) {
+    cudaGetLastError();
+    index_ = -1;
+    return;
+  }
+  slot_ = pool_->base + static_cast<size_t>(index_) * kSlotWords;
 }
 
 cudaError_t CounterLease::commit(cudaError_t launch_status) {
   if (slot_ == nullptr || launch_status != cudaSuccess) return launch_status;
-  // if the event cannot be recorded nothing would tell when the slot is
-  // free again, so it is retired
+  // if the event cannot be recorded, the slot's next user could not wait for
+  // this launch, so the slot is retired
   if (cudaEventRecord(pool_->ev[index_], stream_) != cudaSuccess) {
     pool_->retired[index_] = true;
     return cudaGetLastError();
   }
-  pool_->leased[index_] = true;
+  pool_->used[index_] = true;
   return cudaSuccess;
 }
 

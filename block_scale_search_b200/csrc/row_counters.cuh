@@ -5,8 +5,9 @@
 // and leave their SMs short of warps for the rest of the launch.  Instead,
 // warps take their next rows from a counter in device memory as they finish,
 // so that every warp of the grid ends at about the same time.  The counters
-// form a small pool of slots; the host leases a slot to one launch at a time
-// (CounterLease), and the launch's last CTA zeroes it (finish_slot).
+// form a small pool of slots that launches take in turn (CounterLease): a
+// launch's stream first waits for the slot's previous launch, and the
+// launch's last CTA zeroes the slot for the next (finish_slot).
 #pragma once
 
 #include <mutex>
@@ -15,7 +16,7 @@
 
 namespace nvfp4 {
 
-constexpr int kCounterSlots = 64;           // launches in flight that can hold a slot
+constexpr int kCounterSlots = 64;           // slots, taken in turn
 constexpr int kSlotCounters = 256;          // counters a launch may use
 constexpr int kSlotWords = kSlotCounters + 2;  // counters, CTAs done, launches served
 
@@ -37,9 +38,9 @@ __device__ __forceinline__ void finish_slot(unsigned int* slot, int used) {
 
 // One launch's lease of a counter slot on the current device.  Construct it
 // right before the launch (want = false: no lease), pass slot() (null: no
-// slot; keep the fixed share) to the kernel, and call commit() with the
-// launch's status right after.  The pool's mutex is held from construction
-// to destruction.
+// slot -- stream capture or a CUDA error; keep the fixed share) to the
+// kernel, and call commit() with the launch's status right after.  The pool's
+// mutex is held from construction to destruction.
 class CounterLease {
  public:
   CounterLease(cudaStream_t stream, bool want);

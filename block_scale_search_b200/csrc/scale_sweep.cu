@@ -24,11 +24,10 @@
 // the schedulers favour do more rows and every warp of the grid ends at about
 // the same time (with a fixed share per thread, the favoured warps finish
 // early and leave their SMs short of warps; the run-time hand-out is 6-8%
-// faster).  The counters live in a small pool of slots in device memory; the
-// host leases a slot to one launch at a time (an event recorded after the
-// launch tells when it is free again), the launch's last CTA zeroes it, and a
-// launch that finds no free slot, or is being captured into a graph, keeps
-// the fixed stride.
+// faster).  The counters live in a small pool of slots in device memory
+// that launches take in turn (row_counters.cuh); a launch's stream waits for
+// the slot's previous launch, the launch's last CTA zeroes the slot, and a
+// launch being captured into a graph keeps the fixed stride.
 //
 // Each group is decided in three stages (fast FP32 pass over all candidates,
 // exact FP64 re-scoring of near-ties, exact-decision pack); they live in
@@ -39,6 +38,7 @@
 
 #include "nvfp4_kernels.cuh"
 #include "row_counters.cuh"
+#include "side_reduce.cuh"
 #include "sweep_core.cuh"
 
 namespace nvfp4 {
@@ -208,6 +208,31 @@ scale_sweep_rows_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, 
   finish_slot(slot, static_cast<int>(G >> 5));
 }
 
+// The run-time-row sweep with a fifth warp per CTA streaming side reductions
+// (side_reduce.cuh).  Four CTAs of 160 threads fit an SM at 96 registers;
+// the sweep's four warps per CTA work exactly as in scale_sweep_rows_kernel.
+template <bool kWeighted, int kK>
+__global__ void __launch_bounds__(kCta + 32, 4)
+scale_sweep_side_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t G, int64_t ldw,
+                        const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
+                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                        int8_t* __restrict__ offs, int64_t R, unsigned int* slot,
+                        const __grid_constant__ SideWork side) {
+  __shared__ SweepSmem<16> sm;
+  __shared__ SideRing ring;
+  fill_candidate_table(sm.tab);
+  __syncthreads();
+  if (threadIdx.x < kCta) {
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * kCta + threadIdx.x;
+    if (tid < R * G)
+      sweep_rows_dynamic<kWeighted, kK>(sm, W, out, G, ldw, h, Sp, lo, hi, codes, scales, offs, R,
+                                        slot, tid);
+  } else {
+    run_side_work(side, ring, static_cast<int>(threadIdx.x - kCta), blockIdx.x, gridDim.x);
+  }
+  finish_slot(slot, static_cast<int>(G >> 5));
+}
+
 // Full sweep: every positive E4M3 code is a candidate.  The 126-entry loss
 // column needs dynamic shared memory (about 76 KB per CTA).
 template <bool kWeighted>
@@ -322,6 +347,50 @@ LanePlan sweep_plan_threads(int64_t out, int64_t in, int64_t nt) {
   p.R = R;
   p.threads = p.R * p.VL;
   return p;
+}
+
+bool sweep_can_carry(int64_t out, int64_t in, int num_sms) {
+  const int64_t G = in / 16;
+  if (G == 0 || G % 32 != 0 || G / 32 > kSlotCounters || out > (int64_t{1} << 23)) return false;
+  const int64_t nt = static_cast<int64_t>(num_sms) * 4 * kCta;
+  return G <= nt && out >= 4 * (nt / G);
+}
+
+cudaError_t launch_scale_sweep_side(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
+                                    const float* h, const float* S, int lo, int hi,
+                                    uint8_t* codes, uint8_t* scales, int8_t* offs,
+                                    const SideWork& side, int num_sms, bool* carried,
+                                    cudaStream_t stream) {
+  *carried = false;
+  if (!sweep_can_carry(out, in, num_sms)) return cudaSuccess;
+  CounterLease lease(stream, true);
+  unsigned int* slot = lease.slot();
+  if (slot == nullptr) return cudaSuccess;
+  const int64_t G = in / 16;
+  const int64_t R = std::min<int64_t>(static_cast<int64_t>(num_sms) * 4 * kCta / G,
+                                      (out + kRowChunk - 1) / kRowChunk);
+  const unsigned blocks = static_cast<unsigned>((R * G + kCta - 1) / kCta);
+  const int K = hi - lo + 1;
+  auto launch = [&](auto weighted, auto kk) {
+    scale_sweep_side_kernel<decltype(weighted)::value, decltype(kk)::value>
+        <<<blocks, kCta + 32, 0, stream>>>(W, out, G, ldw, h, S, lo, hi, codes, scales, offs, R,
+                                           slot, side);
+  };
+  using T16 = std::integral_constant<int, 16>;
+  using T11 = std::integral_constant<int, 11>;
+  using T0 = std::integral_constant<int, 0>;
+  if (h) {
+    if (K == 16) launch(std::true_type{}, T16{});
+    else if (K == 11) launch(std::true_type{}, T11{});
+    else launch(std::true_type{}, T0{});
+  } else {
+    if (K == 16) launch(std::false_type{}, T16{});
+    else if (K == 11) launch(std::false_type{}, T11{});
+    else launch(std::false_type{}, T0{});
+  }
+  const cudaError_t e = lease.commit(cudaGetLastError());
+  *carried = e == cudaSuccess;
+  return e;
 }
 
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,

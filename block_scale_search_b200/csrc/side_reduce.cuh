@@ -1,0 +1,158 @@
+// side_reduce.cuh -- reductions a sweep launch streams beside its own work.
+//
+// The sweep is bound by FP32 arithmetic and leaves HBM nearly idle, while the
+// diagonal Hessian and the absmax of a global scale are bound by HBM.  A sweep
+// CTA can therefore carry one extra warp that streams other inputs' reductions
+// for weights swept later.  The warp's lanes each own one task of the
+// standalone kernels' lane grid -- R row lanes x V 16-byte column vectors; task
+// (r, v) covers rows r, r + R, ... of vector v -- so a diagonal-Hessian task
+// writes exactly the partial row the standalone kernel writes (same order of
+// operations, bit for bit), and the standalone finalize applies.  An absmax
+// task folds its maximum into one word with atomicMax (exact in any order).
+//
+// Loads go through a per-lane ring in shared memory with cp.async (four
+// batches of eight rows in flight), so no registers wait on memory; squares
+// are summed with the mixed-precision bf16 FMA, whose exact product and single
+// rounding equal fmaf on the widened values.
+#pragma once
+
+#include "nvfp4_device.cuh"
+#include "sweep_core.cuh"
+
+namespace nvfp4 {
+
+constexpr int kSideRows = 8;     // rows per batch (the standalone kernel's run length)
+constexpr int kSideBatches = 4;  // batches in flight per lane
+constexpr int kMaxSideJobs = 8;
+
+// One reduction's share of tasks [t0, t1) of its R x V task grid.
+struct SideJob {
+  const uint16_t* A;   // bf16 [rows, ld]
+  int64_t rows, ld;
+  int64_t cols;        // elements per row (a multiple of 8)
+  int64_t R;           // row lanes of the task grid
+  int64_t t0, t1;      // task range
+  float* P;            // kind 0: partials [R, cols]
+  uint32_t* amax;      // kind 1: the max word (bf16 bit pattern of |a|)
+  int kind;            // 0: diagonal Hessian, 1: absmax
+};
+
+struct SideWork {
+  SideJob job[kMaxSideJobs];
+  int n;
+  int64_t tasks;       // sum of t1 - t0
+};
+
+// Ring of the side warp: [batch slot * rows][lane].
+struct SideRing {
+  uint4 v[kSideBatches * kSideRows][32];
+};
+
+// x^2 + s for the two bf16 halves of w, each with one rounding.
+__device__ __forceinline__ void sq_acc_bf16x2(uint32_t w, float& s0, float& s1) {
+  asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, l, l, %0;\n\t"
+      "fma.rn.f32.bf16 %1, h, h, %1; }"
+      : "+f"(s0), "+f"(s1) : "r"(w));
+}
+
+// Task (r, v) of a job: runs of kSideRows rows through the ring, then the
+// remaining rows one by one, as the standalone kernels order them.
+__device__ __forceinline__ void side_task(const SideJob& j, int64_t r, int64_t v, SideRing& ring,
+                                          int lane) {
+  const uint16_t* col = j.A + v * 8;
+  const int64_t R = j.R;
+  const int64_t n = (j.rows - r + R - 1) / R;  // rows of this task (r < R <= rows)
+  const int64_t runs = n / kSideRows;
+  auto issue = [&](int64_t k) {
+    const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
+#pragma unroll
+    for (int u = 0; u < kSideRows; ++u)
+      cp_async16(&ring.v[slot + u][lane], col + (r + (k * kSideRows + u) * R) * j.ld);
+  };
+#pragma unroll
+  for (int k = 0; k < kSideBatches; ++k) {
+    if (k < runs) issue(k);
+    cp_async_commit();
+  }
+  if (j.kind == 0) {
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+    for (int64_t k = 0; k < runs; ++k) {
+      cp_async_wait<kSideBatches - 1>();
+      const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
+      float s[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) s[c] = 0.0f;
+#pragma unroll
+      for (int u = 0; u < kSideRows; ++u) {
+        const uint4 q = ring.v[slot + u][lane];
+        sq_acc_bf16x2(q.x, s[0], s[1]);
+        sq_acc_bf16x2(q.y, s[2], s[3]);
+        sq_acc_bf16x2(q.z, s[4], s[5]);
+        sq_acc_bf16x2(q.w, s[6], s[7]);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] += s[c];
+      if (k + kSideBatches < runs) issue(k + kSideBatches);
+      cp_async_commit();
+    }
+    cp_async_wait<0>();
+    for (int64_t t = r + runs * kSideRows * R; t < j.rows; t += R) {
+      const uint4 q = ld_stream_v4(col + t * j.ld);
+      sq_acc_bf16x2(q.x, acc[0], acc[1]);
+      sq_acc_bf16x2(q.y, acc[2], acc[3]);
+      sq_acc_bf16x2(q.z, acc[4], acc[5]);
+      sq_acc_bf16x2(q.w, acc[6], acc[7]);
+    }
+    float4* dst = reinterpret_cast<float4*>(j.P + r * j.cols + v * 8);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  } else {
+    uint32_t m = 0;
+    for (int64_t k = 0; k < runs; ++k) {
+      cp_async_wait<kSideBatches - 1>();
+      const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
+#pragma unroll
+      for (int u = 0; u < kSideRows; ++u) {
+        const uint4 q = ring.v[slot + u][lane];
+        m = __vmaxu2(__vmaxu2(m, q.x & 0x7FFF7FFFu),
+                     __vmaxu2(__vmaxu2(q.y & 0x7FFF7FFFu, q.z & 0x7FFF7FFFu), q.w & 0x7FFF7FFFu));
+      }
+      if (k + kSideBatches < runs) issue(k + kSideBatches);
+      cp_async_commit();
+    }
+    cp_async_wait<0>();
+    for (int64_t t = r + runs * kSideRows * R; t < j.rows; t += R) {
+      const uint4 q = ld_stream_v4(col + t * j.ld);
+      m = __vmaxu2(__vmaxu2(m, q.x & 0x7FFF7FFFu),
+                   __vmaxu2(__vmaxu2(q.y & 0x7FFF7FFFu, q.z & 0x7FFF7FFFu), q.w & 0x7FFF7FFFu));
+    }
+    m = max(m & 0xFFFFu, m >> 16);
+    if (m != 0u) atomicMax(j.amax, m);
+  }
+}
+
+// The side warp of CTA `cta` of `ctas`: lane l takes tasks cta*32 + l,
+// cta*32 + l + 32*ctas, ... of the jobs' concatenated ranges (adjacent lanes
+// take adjacent column vectors of one row lane: coalesced loads).
+__device__ __forceinline__ void run_side_work(const SideWork& w, SideRing& ring, int lane,
+                                              int64_t cta, int64_t ctas) {
+  int jb = 0;
+  int64_t base = 0;  // tasks of the jobs before jb
+  for (int64_t k = cta * 32 + lane; k < w.tasks; k += ctas * 32) {
+    while (jb < w.n && k - base >= w.job[jb].t1 - w.job[jb].t0) {
+      base += w.job[jb].t1 - w.job[jb].t0;
+      ++jb;
+    }
+    if (jb >= w.n) break;
+    const SideJob& j = w.job[jb];
+    const int64_t t = j.t0 + (k - base);
+    const int64_t V = j.cols / 8;
+    const int64_t r = t / V;
+    side_task(j, r, t - r * V, ring, lane);
+  }
+}
+
+}  // namespace nvfp4

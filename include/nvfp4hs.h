@@ -146,12 +146,13 @@ int nvfp4_global_scale_noalloc(const void* W, int64_t out, int64_t in, int64_t l
  * Scheduling: where in/16 is a multiple of 32 and every row lane of the grid
  * would take four rows or more, rows are handed out at run time from counters
  * the library keeps in device memory (one per 32-group column strip).  The
- * counters form 64 slots, each leased to one launch at a time: the library
- * records an event after the launch on `stream` and reuses the slot once it
- * has completed; the launch zeroes the slot before it ends.  A launch that
- * finds no free slot, or is being captured into a CUDA graph, uses a fixed
- * row stride.  The bytes written do not depend on the order rows are taken
- * in.  The library serialises its own slot bookkeeping (a mutex per device).
+ * counters form 64 slots that launches take in turn; before a launch, its
+ * stream waits for an event the library recorded after the slot's previous
+ * launch (free on the same stream), so launches sharing a slot never
+ * overlap, and each launch zeroes its slot before it ends.  A launch being
+ * captured into a CUDA graph uses a fixed row stride.  The bytes written do
+ * not depend on the order rows are taken in.  The library serialises its own
+ * slot bookkeeping (a mutex per device).
  * ------------------------------------------------------------------------ */
 int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi,
@@ -245,6 +246,70 @@ typedef struct nvfp4_sweep_desc {
 size_t nvfp4_scale_sweep_quantize_batched_workspace_size(int64_t n);
 int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n, int lo, int hi,
                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * A layer in one call: steps 1-4 for several projections that share
+ * calibration inputs (for example an MLP's gate and up projections reading
+ * one input, its down projection another).  For every input k,
+ * h_k = diag(X_k^T X_k) as nvfp4_diag_hessian writes it (not accumulated);
+ * for every weight j, S_j as nvfp4_global_scale writes it, then the windowed
+ * sweep of nvfp4_scale_sweep_quantize with the h of its input (input = -1:
+ * plain MSE).  The bytes written equal those of the per-step calls.
+ *
+ * The library orders the work itself: weight 0's S and its input's h first;
+ * the other reductions, which are bound by HBM bandwidth, are streamed by an
+ * extra warp in each CTA of earlier sweeps, which are bound by FP32
+ * arithmetic (H-Scale summary, sec. 4 "Efficiency and Hardware Deployment":
+ * the added cost is the offline search and one activation pass).  Weights are swept in the order
+ * given; a reduction that no earlier sweep can carry (the sweep's row length
+ * is not a multiple of 512 elements, or it is short) runs on its own before
+ * it is needed.
+ *
+ *   weights    n_weights descriptors: W bf16 [out, ldw] (16-byte aligned,
+ *              ldw % 8 == 0, in % 16 == 0, out and in > 0); input in
+ *              [-1, n_inputs) with inputs[input].in == in; S device scalar
+ *              (written); amax, status nullable device scalars (status: 0, or
+ *              NVFP4_ERR_NONFINITE when W holds Inf/NaN, as
+ *              nvfp4_global_scale); codes [out, in/2] 8-byte aligned; scales
+ *              [out, in/16]; chosen_offset [out, in/16] or NULL.
+ *   inputs     n_inputs descriptors: X bf16 [tokens, ldx] (16-byte aligned,
+ *              in % 8 == 0, tokens >= 0); h float [in], 16-byte aligned
+ *              (written).
+ *   q_max      448 or 256 as for nvfp4_global_scale; lo, hi as for the sweep.
+ *   workspace  device, 256-byte aligned, at least
+ *              nvfp4_quantize_layer_workspace_size(...) bytes (which depends
+ *              on the device; 0 for invalid descriptors or no device).
+ *   sweep_events  NULL, or 2 * n_weights cudaEvent_t (as void*) created by
+ *              the caller on this device: events[2j] and events[2j+1] are
+ *              recorded on `stream` right before and after weight j's sweep
+ *              launch (with the reductions it carries), for timing.
+ * Descriptors are read on the host during the call.  Asynchronous on
+ * `stream`.  Returns NVFP4_OK or the status of the first failing check.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* W;
+  int64_t out, in, ldw;
+  int input;
+  float* S;
+  float* amax;
+  int* status;
+  uint8_t* codes;
+  uint8_t* scales;
+  int8_t* chosen_offset;
+} nvfp4_layer_weight;
+
+typedef struct {
+  const void* X;
+  int64_t tokens, in, ldx;
+  float* h;
+} nvfp4_layer_input;
+
+size_t nvfp4_quantize_layer_workspace_size(const nvfp4_layer_weight* weights, int n_weights,
+                                           const nvfp4_layer_input* inputs, int n_inputs);
+int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
+                         const nvfp4_layer_input* inputs, int n_inputs, float q_max, int lo,
+                         int hi, void* workspace, size_t workspace_bytes,
+                         void* const* sweep_events, void* stream);
 
 /* ------------------------------------------------------------------------
  * Online activation quantization (ScaleSweep summary, sec. 1-3 and

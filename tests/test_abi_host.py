@@ -212,3 +212,36 @@ def test_debug_row_counters_validation(L):
     import torch
     if not torch.cuda.is_available():   # no device: a CUDA error, not a crash
         assert L.nvfp4_debug_row_counters(C.byref(p), C.byref(n)) == -6
+
+
+def test_quantize_layer_validation(L):
+    import block_scale_search_b200 as nv
+    W = lambda **k: nv.LayerWeight(**{**dict(W=P, out=64, inp=256, ldw=256, input=0, S=P, amax=None,
+                                            status=None, codes=P, scales=P, chosen_offset=None), **k})
+    X = lambda **k: nv.LayerInput(**{**dict(X=P, tokens=32, inp=256, ldx=256, h=P), **k})
+    ws = P
+
+    def call(ws_list, xs_list, q=448.0, lo=-9, hi=6, nb=1 << 30):
+        wa = (nv.LayerWeight * max(1, len(ws_list)))(*ws_list)
+        xa = (nv.LayerInput * max(1, len(xs_list)))(*xs_list)
+        return L.nvfp4_quantize_layer(wa, len(ws_list), xa, len(xs_list), q, lo, hi, ws, nb, None, None)
+
+    assert call([W(input=1)], [X()]) == -1                 # input index out of range
+    assert call([W(input=-2)], [X()]) == -1
+    assert call([W(S=None)], [X()]) == -1                  # S missing
+    assert call([W(inp=128, ldw=128)], [X()]) == -2        # in differs from the input's
+    assert call([W(out=0)], [X()]) == -2                   # empty weight
+    assert call([W(inp=72, ldw=72)], [X(inp=72, ldx=72)]) == -2   # in % 16
+    assert call([W(W=P + 8)], [X()]) == -3                 # W misaligned
+    assert call([W()], [X(h=P + 4)]) == -3                 # h not 16-byte aligned
+    assert call([W()], [X(tokens=-1)]) == -1
+    assert call([W()], [X()], q=float("nan")) == -1
+    assert call([W()], [X()], lo=-10, hi=6) == -4          # window over 16
+    assert L.nvfp4_quantize_layer(None, 1, None, 0, 448.0, -9, 6, ws, 1 << 30, None, None) == -1
+    # no device here: the workspace query returns 0 and a valid call a CUDA error
+    import torch
+    if not torch.cuda.is_available():
+        wa = (nv.LayerWeight * 1)(W())
+        xa = (nv.LayerInput * 1)(X())
+        assert L.nvfp4_quantize_layer_workspace_size(wa, 1, xa, 1) == 0
+        assert call([W()], [X()]) == -6

@@ -1,0 +1,93 @@
+"""nvfp4_quantize_layer writes exactly what the per-step calls write: h of
+every input, S (and status) of every weight, codes, scales and offsets of
+every sweep -- whether the reductions ride along earlier sweeps (shapes whose
+rows hold a multiple of 512 elements, long enough to hand rows out at run
+time) or run on their own.  Needs a B200."""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import block_scale_search_b200 as nv
+    nv.lib()
+    return nv
+
+
+def _per_step(nv, Ws, Xs, inputs, q_max, lo, hi):
+    hs = [nv.diag_hessian(X) for X in Xs]
+    res = []
+    for W, k in zip(Ws, inputs):
+        S, _, st = nv.global_scale(W, q_max)
+        h = hs[k] if k >= 0 else None
+        codes, scales, offs = nv.scale_sweep_quantize(W, h, S, lo, hi, want_offsets=True)
+        res.append((codes, scales, S, offs, st))
+    torch.cuda.synchronize()
+    return res, hs
+
+
+def _check_same(nv, Ws, Xs, inputs, q_max=448.0, lo=-9, hi=6):
+    ref, href = _per_step(nv, Ws, Xs, inputs, q_max, lo, hi)
+    got, hgot = nv.quantize_layer_many(Ws, Xs, inputs, q_max, lo, hi, want_offsets=True)
+    torch.cuda.synchronize()
+    for a, b in zip(hgot, href):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    for (c, s, S, o, st), (rc, rs, rS, ro, rst) in zip(got, ref):
+        assert torch.equal(S.view(torch.int32), rS.view(torch.int32))
+        assert int(st.item()) == int(rst.item())
+        assert torch.equal(c, rc) and torch.equal(s, rs) and torch.equal(o, ro)
+
+
+def _mlp(gu_out, gu_in, down_out, tokens, seed):
+    import workloads
+    Ws = [workloads.weight(gu_out, gu_in, 0.015, 0.001, 10.0, seed, DEV),
+          workloads.weight(gu_out, gu_in, 0.015, 0.001, 10.0, seed + 1, DEV),
+          workloads.weight(down_out, gu_out, 0.015, 0.001, 10.0, seed + 2, DEV)]
+    Xs = [workloads.calib(tokens, gu_in, 1.5, seed + 3, DEV),
+          workloads.calib(tokens, gu_out, 1.5, seed + 4, DEV)]
+    return Ws, Xs, [0, 0, 1]
+
+
+def test_mlp_with_reductions_carried(nv):
+    # gate/up 3072x2048 and down 2048x3072: both gate and up carry side work
+    Ws, Xs, inputs = _mlp(3072, 2048, 2048, 4096, 11)
+    _check_same(nv, Ws, Xs, inputs)
+
+
+def test_mlp_at_the_benchmarked_size(nv):
+    # the 70B-shaped MLP the bench times: gate/up 28672x8192, down 8192x28672,
+    # 65536 calibration tokens per input
+    Ws, Xs, inputs = _mlp(28672, 8192, 8192, 65536, 4)
+    _check_same(nv, Ws, Xs, inputs)
+
+
+def test_small_or_ragged_shapes_run_on_their_own(nv):
+    # rows too short or not a multiple of 512 elements: nothing rides along
+    Ws, Xs, inputs = _mlp(256, 768, 96, 300, 21)
+    _check_same(nv, Ws, Xs, inputs)
+
+
+def test_mse_weights_shared_and_unused_inputs(nv):
+    import workloads
+    Ws = [workloads.weight(3000, 4096, 0.02, 0.001, 8.0, 31, DEV),   # MSE, first
+          workloads.weight(4096, 4096, 0.02, 0.001, 8.0, 32, DEV),   # input 1
+          workloads.weight(2500, 4096, 0.02, 0.001, 8.0, 33, DEV),   # input 1 again
+          workloads.weight(4096, 2048, 0.02, 0.001, 8.0, 34, DEV)]   # input 2
+    Xs = [workloads.calib(512, 1024, 1.0, 35, DEV),                   # used by no weight
+          workloads.calib(2048, 4096, 1.0, 36, DEV),
+          workloads.calib(3000, 2048, 1.0, 37, DEV)]
+    _check_same(nv, Ws, Xs, [-1, 1, 1, 2], q_max=256.0, lo=-3, hi=7)
+    _check_same(nv, Ws, Xs, [-1, 1, 1, 2], q_max=448.0, lo=-8, hi=7)
+
+
+def test_nonfinite_weight_reports_its_own_status(nv):
+    Ws, Xs, inputs = _mlp(3072, 2048, 2048, 2048, 41)
+    Ws[1][5, 7] = float("inf")   # up: its S is carried by the gate sweep
+    Ws[2][9, 3] = float("nan")   # down
+    got, _ = nv.quantize_layer_many(Ws, Xs, inputs)
+    torch.cuda.synchronize()
+    assert [int(g[4].item()) for g in got] == [0, -5, -5]
+    assert torch.isnan(got[1][2]).all() and torch.isnan(got[2][2]).all()

@@ -2,9 +2,9 @@
 the same bytes as the fixed row stride.  A launch recorded into a CUDA graph
 keeps the fixed stride, so a graph replay gives the reference bytes; direct
 launches of the same shapes lease a counter slot and take rows from it
-(checked by reading the slots).  Also: more launches in flight at once than
-there are slots, where the launches that find none keep the fixed stride.
-Needs a B200."""
+(checked by reading the slots).  Also: more launches in flight at once, on
+as many streams, than there are slots, where a launch waits for its slot's
+previous user.  Needs a B200."""
 import pytest
 import torch
 
@@ -133,8 +133,9 @@ def test_more_launches_in_flight_than_slots(nv):
     for bufs, ref in runs:
         for a, b in zip(bufs, ref):
             assert torch.equal(a, b)
-    # the first 64 leased a slot each; the 16 that found none kept the stride
-    assert _served(nv) - n0 == SLOTS
+    # every launch took a slot: the last 16 waited, on their own streams, for
+    # the launches that had their slots before them
+    assert _served(nv) - n0 == n
     assert torch.all(_slots(nv)[:, :STRIPS + 1] == 0)
 
 
