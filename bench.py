@@ -751,6 +751,9 @@ WORKLOADS = {
                         "channel scales"),
     "mlp_slice": ("mlp_slice (profiling size): W 8192x8192 bf16 N(0,0.015) 0.1% x10; X 16384 x "
                   "8192 bf16 lognormal(1.5) channel scales"),
+    "mlp_layer_slice": ("mlp_layer_slice (profiling size): gate/up 8192x4096, down 4096x8192 "
+                        "bf16 N(0,0.015) 0.1% x10; X 16384 tokens x {4096, 8192} bf16 "
+                        "lognormal(1.5) channel scales"),
     "moe_grouped": ("moe_grouped: 128 experts x {gate, up 768x2048; down 2048x768} bf16 N(0,0.02) "
                     "0.1% x10; 262144 tokens routed top-8 (Zipf 1.1), per-expert X slices and h; "
                     "grouped diag-Hessian + batched global scale + batched sweep"),
@@ -998,8 +1001,7 @@ def main():
 
     # ---- roofline of the dominant kernel, as timed in the region above
     in_layer = getattr(step, "layer", False) and not getattr(step, "serial", True)
-    roofline = dominant_roofline(kern, wl, clocks,
-                                 traffic_key="scale_sweep_layer" if in_layer else None)
+    roofline = dominant_roofline(kern, wl, clocks)
     layer_info = None
     if in_layer:
         # the sweeps carry every reduction but the first weight's S and its
@@ -1024,6 +1026,20 @@ def main():
             "note": "the first weight's S and its input's h run first on their own (rest); "
                     "the other weights' S and the other inputs' h are streamed by a fifth warp "
                     "in each CTA of the earlier sweeps (carrying sweeps)"}
+        # DRAM bytes of the step's sweep launches, per launch: the carrying
+        # sweeps' from their capture (per algorithmic byte, side bytes
+        # included), the last sweep's from the plain sweep's capture
+        plain = wl.weight_elems - sum(m.out * m.inp for m in carry)
+        t_side = profiled_traffic("scale_sweep_layer",
+                                  SWEEP_BYTES_PER_ELEM * sum(m.out * m.inp for m in carry) + side)
+        t_plain = profiled_traffic("scale_sweep", plain)
+        roofline["traffic"] = (None if t_side is None or t_plain is None
+                               else (t_side + t_plain) / sweep_launches)
+        roofline["traffic_note"] = ("DRAM read+write bytes per sweep launch, averaged over the "
+                                    "layer call's sweeps, including the reductions the carrying "
+                                    "sweeps stream; from the committed captures on the "
+                                    "profiling-size layer, scaled by bytes")
+        roofline["side_bytes_per_launch"] = int(side / sweep_launches)
 
     # ---- the same kernels in isolation: a short serial pass (one stream,
     # nothing beside each kernel), for the per-kernel rooflines without the

@@ -197,6 +197,19 @@ def llama33_70b_mlp(seed_offset: int = 0) -> Workload:
     return Workload("llama33_70b_mlp", 448.0, mats, cal, [Run(-9, 6, True)])
 
 
+def mlp_layer_slice(seed_offset: int = 0) -> Workload:
+    """A whole 70B-MLP-like layer at profiling size: gate/up 8192x4096, down
+    4096x8192, N(0,0.015), 0.1% x10; X 16384 tokens x {4096, 8192},
+    lognormal(1.5) channel scales (inputs larger than L2)."""
+    s = 800 + 97 * seed_offset
+    mats = [Matrix("gate", 8192, 4096, "gu", s + 1, 0.015, 0.001, 10.0),
+            Matrix("up", 8192, 4096, "gu", s + 2, 0.015, 0.001, 10.0),
+            Matrix("down", 4096, 8192, "down", s + 3, 0.015, 0.001, 10.0)]
+    cal = {"gu": Calib("gu", 16384, 4096, 1.5, s + 41),
+           "down": Calib("down", 16384, 8192, 1.5, s + 42)}
+    return Workload("mlp_layer_slice", 448.0, mats, cal, [Run(-9, 6, True)])
+
+
 def mlp_slice(seed_offset: int = 0) -> Workload:
     """One 70B-MLP-like layer at profiling size: W 8192x8192 N(0,0.015), 0.1% x10;
     X 16384 x 8192, lognormal(1.5) channel scales (inputs larger than L2)."""
@@ -225,4 +238,5 @@ def moe_grouped(tokens: int = 262144, experts: int = 128, device="cpu") -> Workl
 
 
 ALL = {"single_layer": single_layer, "square_layer": square_layer, "llama3_8b": llama3_8b,
-       "llama33_70b_mlp": llama33_70b_mlp, "mlp_slice": mlp_slice, "moe_grouped": moe_grouped}
+       "llama33_70b_mlp": llama33_70b_mlp, "mlp_slice": mlp_slice, "moe_grouped": moe_grouped,
+       "mlp_layer_slice": mlp_layer_slice}
