@@ -1040,6 +1040,11 @@ def main():
                                     "sweeps stream; from the committed captures on the "
                                     "profiling-size layer, scaled by bytes")
         roofline["side_bytes_per_launch"] = int(side / sweep_launches)
+        per_launch_s = kern["scale_sweep"]["ms_per_step"] / sweep_launches * 1e-3
+        hbm = (SWEEP_BYTES_PER_ELEM * wl.weight_elems + side) / sweep_launches / per_launch_s / 1e9
+        peak, peak_kind, _ = measured_peaks()
+        roofline["hbm_gbs_with_side"] = round(hbm, 1)
+        roofline["hbm_frac_with_side_of_measured"] = round(hbm / peak, 4)
 
     # ---- the same kernels in isolation: a short serial pass (one stream,
     # nothing beside each kernel), for the per-kernel rooflines without the
