@@ -91,3 +91,56 @@ def test_nonfinite_weight_reports_its_own_status(nv):
     torch.cuda.synchronize()
     assert [int(g[4].item()) for g in got] == [0, -5, -5]
     assert torch.isnan(got[1][2]).all() and torch.isnan(got[2][2]).all()
+
+
+def test_layer_call_captured_in_a_graph(nv):
+    """Under stream capture no sweep can take a counter slot: every sweep
+    keeps the fixed stride and every reduction runs on its own; a replay
+    writes the same bytes as the per-step calls."""
+    Ws, Xs, inputs = _mlp(3072, 2048, 2048, 4096, 51)
+    ref, href = _per_step(nv, Ws, Xs, inputs, 448.0, -9, 6)
+    got = []
+    hs = [torch.empty(X.shape[1], dtype=torch.float32, device=DEV) for X in Xs]
+    wd = []
+    for W, k in zip(Ws, inputs):
+        o, n = W.shape
+        t = (torch.empty(o, n // 2, dtype=torch.uint8, device=DEV),
+             torch.empty(o, n // 16, dtype=torch.uint8, device=DEV),
+             torch.empty(1, dtype=torch.float32, device=DEV),
+             torch.empty(o, n // 16, dtype=torch.int8, device=DEV),
+             torch.empty(1, dtype=torch.int32, device=DEV))
+        got.append(t)
+        wd.append(nv.LayerWeight(W.data_ptr(), o, n, W.stride(0), k, t[2].data_ptr(), None,
+                                 t[4].data_ptr(), t[0].data_ptr(), t[1].data_ptr(), t[3].data_ptr()))
+    xd = [nv.LayerInput(X.data_ptr(), X.shape[0], X.shape[1], X.stride(0), h.data_ptr())
+          for X, h in zip(Xs, hs)]
+    nb = nv.nvfp4_quantize_layer_workspace_size(wd, xd)
+    ws = torch.empty(nb, dtype=torch.uint8, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        nv.nvfp4_quantize_layer(wd, xd, 448.0, -9, 6, ws, nb, stream=s)
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    del g
+    for a, b in zip(hs, href):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+    for (c, sc, S, o, st), (rc, rs, rS, ro, rst) in zip(got, ref):
+        assert torch.equal(S.view(torch.int32), rS.view(torch.int32)) and int(st.item()) == 0
+        assert torch.equal(c, rc) and torch.equal(sc, rs) and torch.equal(o, ro)
+
+
+def test_many_projections_fill_the_side_job_slots(nv):
+    """Twelve weights over four inputs: later sweeps have up to eleven earlier
+    carriers and a sweep can carry at most eight reductions at once, so the
+    planner both spreads and caps; the bytes are still the per-step calls'."""
+    import workloads
+    shapes = [(4096, 2048, 0), (3072, 2048, 0), (2048, 4096, 1), (4096, 4096, 1),
+              (2560, 2048, 2), (3000, 4096, 1), (2048, 2048, 3), (4096, 2048, 0),
+              (2048, 4096, -1), (3072, 2048, 2), (2048, 2048, 3), (2600, 4096, 1)]
+    Ws = [workloads.weight(o, i, 0.02, 0.001, 10.0, 600 + k, DEV) for k, (o, i, _) in enumerate(shapes)]
+    Xs = [workloads.calib(2048, 2048, 1.0, 650, DEV), workloads.calib(1536, 4096, 1.0, 651, DEV),
+          workloads.calib(3000, 2048, 1.0, 652, DEV), workloads.calib(1024, 2048, 1.0, 653, DEV)]
+    _check_same(nv, Ws, Xs, [k for _, _, k in shapes])
