@@ -19,8 +19,8 @@
 //     proportion to their size (earliest deadlines first), and finalized right
 //     after the last sweep carrying part of it;
 //   * a reduction with no carrier before its deadline, or whose carrier could
-//     not lease a counter slot, runs as the standalone kernels instead (for a
-//     failed carrier, right after that sweep).
+//     not launch as one (stream capture: no counter slot), runs as the
+//     standalone kernels instead (for such a carrier, right after its sweep).
 #include <algorithm>
 #include <vector>
 
