@@ -217,6 +217,18 @@ class Step:
         self.layer_x = [nv.LayerInput(Xs[k].data_ptr(), Xs[k].shape[0], Xs[k].shape[1],
                                       Xs[k].stride(0), self.h[k].data_ptr()) for k in keys]
         self.layer_arrays = nv._layer_arrays(self.layer_w, self.layer_x)
+        # what the layer call's sweeps carry here: every reduction but the
+        # first weight's S and its input's h, in the sweeps before the last
+        first = wl.matrices[0]
+        fx = wl.calibs[first.x_key]
+        self.side_bytes = (wl.calib_bytes - 2 * fx.tokens * fx.inp
+                           + 2 * (wl.weight_elems - first.out * first.inp))
+        self.carry_launches = len(wl.matrices) - 1
+        self.carry_elems = sum(m.out * m.inp for m in wl.matrices[:-1])
+        self.traffic_key = "scale_sweep_layer"
+        self.layer_note = ("the first weight's S and its input's h run first on their own (rest); "
+                           "the other weights' S and the other inputs' h are streamed by a fifth "
+                           "warp in each CTA of the earlier sweeps (carrying sweeps)")
         nb = nv.nvfp4_quantize_layer_workspace_size(self.layer_w, self.layer_x)
         self.layer_ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
         self.layer_nb = nb
@@ -358,10 +370,11 @@ class GroupedStep:
     first batch (overlapped, the default).  Descriptor tables are built once;
     run() calls the C ABI."""
 
-    def __init__(self, nv, wl, Ws, Xs, device, serial=False):
+    def __init__(self, nv, wl, Ws, Xs, device, serial=False, layer=False):
         import ctypes as C
         import torch
         self.nv, self.wl, self.Ws, self.Xs = nv, wl, Ws, Xs
+        self.layer = layer
         L = nv.lib()
         self.L = L
         offs = wl.calibs[next(iter(wl.calibs))].row_offsets
@@ -406,9 +419,43 @@ class GroupedStep:
                             torch.empty(L.nvfp4_scale_sweep_quantize_batched_workspace_size(len(sel)),
                                         dtype=torch.uint8, device=device))
         self.aux = torch.cuda.Stream(device=device)
+        # the one-call form (nvfp4_quantize_grouped_layer): the first input's
+        # matrices, then the second's, with S laid out in that order
+        assert len(self.keys) == 2
+        k1, k2 = self.keys
+        first = [m for m in mats if m.x_key == k1]
+        second = [m for m in mats if m.x_key == k2]
+        self.lS = torch.empty(n, dtype=torch.float32, device=device)
+        self.lamax = torch.empty(n, dtype=torch.float32, device=device)
+        self.lstatus = torch.empty(n, dtype=torch.int32, device=device)
+        ld = []
+        for i, m in enumerate(first + second):
+            hrow = self.h[m.x_key][m.expert]
+            ld.append(nv.SweepDesc(Ws[m.name].data_ptr(), m.out, m.inp, m.inp, hrow.data_ptr(),
+                                   self.lS.data_ptr() + 4 * i, self.codes[m.name].data_ptr(),
+                                   self.scales[m.name].data_ptr(), None))
+        self.lfirst = (nv.SweepDesc * len(first))(*ld[:len(first)])
+        self.lsecond = (nv.SweepDesc * len(second))(*ld[len(first):])
+        self.lx = [nv.GroupedInput(Xs[k].data_ptr(), self.off.data_ptr(), Xs[k].shape[0],
+                                   Xs[k].shape[1], Xs[k].stride(0), self.h[k].data_ptr())
+                   for k in (k1, k2)]
+        nb = nv.nvfp4_quantize_grouped_layer_workspace_size(self.lfirst, self.lsecond, self.lx[0],
+                                                            self.lx[1], self.E, self.lS)
+        self.lws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
+        self.lnb = nb
+        self.side_bytes = Xs[k2].numel() * 2       # streamed beside the first batch's sweep
+        self.carry_launches = 1
+        self.carry_elems = sum(m.out * m.inp for m in first)
+        self.traffic_key = "scale_sweep_grouped_layer"   # no capture recorded: traffic null
+        self.layer_note = ("the first input's h and every matrix's S run first (rest); the second "
+                           "input's h is streamed by a fifth warp in each CTA of the first batch's "
+                           "sweep (carrying sweep)")
 
     @property
     def launches_per_step(self):
+        if self.layer and not self.serial:
+            # grouped diag 3 + plan 1 + finalize 1, batched S 2, two sweeps
+            return 3 + 1 + 1 + 2 + 2
         # grouped diag-Hessian 3 per input, batched global scale 2, sweeps 1 or 1 per input
         return 3 * len(self.Xs) + 2 + (1 if self.serial else len(self.keys))
 
@@ -432,6 +479,26 @@ class GroupedStep:
         def chk(st):
             if st != 0:
                 raise RuntimeError(f"status {st}")
+
+        if self.layer and not self.serial:
+            sev = None
+            if ev is not None:
+                sev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                for e in sev:   # torch creates the CUDA event at its first record
+                    e.record(stream)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+            self.nv.nvfp4_quantize_grouped_layer(
+                self.lfirst, self.lsecond, self.lx[0], self.lx[1], self.E, float(self.wl.q_max),
+                LO, HI, self.lS, self.lamax, self.lstatus, self.lws, self.lnb, sweep_events=sev,
+                stream=stream)
+            if ev is not None:
+                b.record(stream)
+                ev.setdefault("layer_call", []).append((a, b))
+                ev.setdefault("scale_sweep", []).append((sev[0], sev[1]))
+                ev.setdefault("scale_sweep", []).append((sev[2], sev[3]))
+            return
 
         def dh(k, s):
             X, ws = self.Xs[k], self.hws[k]
@@ -885,7 +952,8 @@ def main():
         return
     wl, Ws, Xs = build_layer(rank, dev, args.workload)
     if args.workload == "moe_grouped":
-        step = GroupedStep(nv, wl, Ws, Xs, dev, serial=args.schedule != "overlapped")
+        step = GroupedStep(nv, wl, Ws, Xs, dev, serial=args.schedule == "serial",
+                           layer=args.schedule in ("auto", "layer"))
     else:
         step = Step(nv, wl, Ws, Xs, dev, serial=args.schedule == "serial",
                     layer=args.schedule in ("auto", "layer"))
@@ -928,7 +996,8 @@ def main():
         for n in Ws:
             assert int(step.status[n].item()) == 0, f"non-finite weights in {n}"
     else:
-        assert not step.status.any().item(), "non-finite weights"
+        st = step.lstatus if getattr(step, "layer", False) and not step.serial else step.status
+        assert not st.any().item(), "non-finite weights"
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -1004,35 +1073,29 @@ def main():
     roofline = dominant_roofline(kern, wl, clocks)
     layer_info = None
     if in_layer:
-        # the sweeps carry every reduction but the first weight's S and its
-        # input's h: their bytes ride in the sweep launches timed above
+        # the carrying sweeps stream every reduction but the first ones: their
+        # bytes ride in the sweep launches timed above
         call_ms = sum(a.elapsed_time(b) for a, b in ev["layer_call"]) / args.steps
         sweep_ms = kern["scale_sweep"]["ms_per_step"]
-        first = wl.matrices[0]
-        side = (wl.calib_bytes - 2 * wl.calibs[first.x_key].tokens * wl.calibs[first.x_key].inp
-                + 2 * (wl.weight_elems - first.out * first.inp))
+        side = step.side_bytes
         sweep_launches = kern["scale_sweep"]["launch_pairs_per_step"]
-        carry = [m for m in wl.matrices[:-1]]
+        nc = step.carry_launches
         carry_ms = sum(a.elapsed_time(b) for i, (a, b) in enumerate(ev["scale_sweep"])
-                       if i % sweep_launches < len(carry)) / args.steps
+                       if i % sweep_launches < nc) / args.steps
         layer_info = {
             "call_ms_per_step": round(call_ms, 4), "sweeps_ms_per_step": round(sweep_ms, 4),
             "rest_ms_per_step": round(call_ms - sweep_ms, 4),
             "side_bytes_per_step": int(side),
             "carrying_sweeps_ms_per_step": round(carry_ms, 4),
-            "carrying_sweeps_hbm_gbs": (round((side + SWEEP_BYTES_PER_ELEM * sum(
-                m.out * m.inp for m in carry)) / (carry_ms * 1e-3) / 1e9, 1)
-                if carry_ms > 0 else None),
-            "note": "the first weight's S and its input's h run first on their own (rest); "
-                    "the other weights' S and the other inputs' h are streamed by a fifth warp "
-                    "in each CTA of the earlier sweeps (carrying sweeps)"}
+            "carrying_sweeps_hbm_gbs": (round((side + SWEEP_BYTES_PER_ELEM * step.carry_elems)
+                                              / (carry_ms * 1e-3) / 1e9, 1)
+                                        if carry_ms > 0 else None),
+            "note": step.layer_note}
         # DRAM bytes of the step's sweep launches, per launch: the carrying
         # sweeps' from their capture (per algorithmic byte, side bytes
         # included), the last sweep's from the plain sweep's capture
-        plain = wl.weight_elems - sum(m.out * m.inp for m in carry)
-        t_side = profiled_traffic("scale_sweep_layer",
-                                  SWEEP_BYTES_PER_ELEM * sum(m.out * m.inp for m in carry) + side)
-        t_plain = profiled_traffic("scale_sweep", plain)
+        t_side = profiled_traffic(step.traffic_key, SWEEP_BYTES_PER_ELEM * step.carry_elems + side)
+        t_plain = profiled_traffic("scale_sweep", wl.weight_elems - step.carry_elems)
         roofline["traffic"] = (None if t_side is None or t_plain is None
                                else (t_side + t_plain) / sweep_launches)
         roofline["traffic_note"] = ("DRAM read+write bytes per sweep launch, averaged over the "
@@ -1082,9 +1145,9 @@ def main():
                        "l2": f"inputs {(wl.calib_bytes + 2 * wl.weight_elems) / 1e9:.2f} GB per "
                              f"rank > 126 MB L2; no flush",
                        "parallelism": f"weak: {ws} rank(s), one independent layer per rank",
-                       "schedule": ("layer: one nvfp4_quantize_layer call per step; the "
-                                    "HBM-bound reductions ride in the FP32-bound sweeps"
-                                    if in_layer else
+                       "schedule": ("layer: one nvfp4_quantize_layer (or _grouped_layer) call "
+                                    "per step; the HBM-bound reductions ride in the FP32-bound "
+                                    "sweeps" if in_layer else
                                     "serial: one stream, h then S then sweeps"
                                     if getattr(step, "serial", True) else
                                     "overlapped: later weights' S and h on a second stream "

@@ -26,7 +26,8 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
     "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "quantize_layer_many",
-    "LayerWeight", "LayerInput",
+    "LayerWeight", "LayerInput", "GroupedInput", "nvfp4_quantize_grouped_layer_workspace_size",
+    "nvfp4_quantize_grouped_layer",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize", "nvfp4_quantize_activations",
     "quantize_activations", "nvfp4_blocked_scales_size", "nvfp4_scales_to_blocked",
@@ -78,6 +79,12 @@ class LayerInput(C.Structure):
     _fields_ = [("X", _vp), ("tokens", _i64), ("inp", _i64), ("ldx", _i64), ("h", _vp)]
 
 
+class GroupedInput(C.Structure):
+    """nvfp4_grouped_input"""
+    _fields_ = [("X", _vp), ("row_offsets", _vp), ("total_tokens", _i64), ("inp", _i64),
+                ("ldx", _i64), ("h", _vp)]
+
+
 _SIGS = {
     "nvfp4_version": ([], _int),
     "nvfp4_last_cuda_error": ([], _int),
@@ -89,6 +96,13 @@ _SIGS = {
     "nvfp4_scale_sweep_quantize": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp,
                                     _vp], _int),
     "nvfp4_debug_row_counters": ([C.POINTER(_vp), C.POINTER(_sz)], _int),
+    "nvfp4_quantize_grouped_layer_workspace_size": ([C.POINTER(SweepDesc), _i64, C.POINTER(SweepDesc),
+                                                     _i64, C.POINTER(GroupedInput),
+                                                     C.POINTER(GroupedInput), _i64, _vp], _sz),
+    "nvfp4_quantize_grouped_layer": ([C.POINTER(SweepDesc), _i64, C.POINTER(SweepDesc), _i64,
+                                      C.POINTER(GroupedInput), C.POINTER(GroupedInput), _i64, _f32,
+                                      _int, _int, _vp, _vp, _vp, _vp, _sz, C.POINTER(_vp), _vp],
+                                     _int),
     "nvfp4_quantize_layer_workspace_size": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput),
                                              _int], _sz),
     "nvfp4_quantize_layer": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput), _int, _f32, _int,
@@ -217,6 +231,34 @@ def nvfp4_quantize_layer(weights, inputs, q_max, lo, hi, workspace, workspace_by
         ev = (_vp * len(sweep_events))(*[e.cuda_event for e in sweep_events])
     _check("nvfp4_quantize_layer", lib().nvfp4_quantize_layer(
         wa, len(weights), xa, len(inputs), float(q_max), int(lo), int(hi), _ptr(workspace),
+        workspace_bytes, ev, _stream(stream)))
+
+
+def _sweep_array(descs):
+    return descs if not isinstance(descs, list) else (SweepDesc * max(1, len(descs)))(*descs)
+
+
+def nvfp4_quantize_grouped_layer_workspace_size(first, second, first_input, second_input,
+                                                experts, S) -> int:
+    fa, sa = _sweep_array(first), _sweep_array(second)
+    return lib().nvfp4_quantize_grouped_layer_workspace_size(
+        fa, len(first), sa, len(second), C.byref(first_input), C.byref(second_input), experts,
+        _ptr(S))
+
+
+def nvfp4_quantize_grouped_layer(first, second, first_input, second_input, experts, q_max, lo, hi,
+                                 S, amax, status, workspace, workspace_bytes, sweep_events=None,
+                                 stream=None):
+    """first/second: lists (or ready ctypes arrays) of SweepDesc; first_input,
+    second_input: GroupedInput; sweep_events: None or 4 recorded-once
+    torch.cuda.Event around the two batches' sweep launches."""
+    fa, sa = _sweep_array(first), _sweep_array(second)
+    ev = None
+    if sweep_events is not None:
+        ev = (_vp * 4)(*[e.cuda_event for e in sweep_events])
+    _check("nvfp4_quantize_grouped_layer", lib().nvfp4_quantize_grouped_layer(
+        fa, len(first), sa, len(second), C.byref(first_input), C.byref(second_input), experts,
+        float(q_max), int(lo), int(hi), _ptr(S), _ptr(amax), _ptr(status), _ptr(workspace),
         workspace_bytes, ev, _stream(stream)))
 
 

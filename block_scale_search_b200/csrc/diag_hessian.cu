@@ -299,6 +299,34 @@ size_t diag_hessian_grouped_workspace_bytes(int64_t total, int64_t E, int64_t in
   return grouped_head_bytes(E) + static_cast<size_t>(p.cap) * static_cast<size_t>(in) * sizeof(float);
 }
 
+// The grouped kernel's plan and partials, for a caller that streams the
+// partial pass elsewhere (side_reduce.cuh, kind 2): launch the plan, let the
+// tasks (slice q < cap, vector v) write the partials, then the finalize.
+GroupedSide grouped_diag_side(int64_t E, int64_t in, void* workspace, int num_sms) {
+  const GroupedPlan p = grouped_plan(E, in, num_sms);
+  GroupedSide g;
+  g.cstart = static_cast<int64_t*>(workspace);
+  g.P = reinterpret_cast<float*>(static_cast<char*>(workspace) + grouped_head_bytes(E));
+  g.cap = p.cap;
+  g.block = p.block;
+  g.nt = p.nt;
+  return g;
+}
+
+cudaError_t launch_grouped_diag_plan(const int64_t* off, int64_t E, int64_t total,
+                                     const GroupedSide& g, cudaStream_t stream) {
+  grouped_plan_kernel<<<1, 32, 0, stream>>>(off, E, total, g.nt, g.cap, g.cstart);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_grouped_diag_finalize(int64_t E, int64_t in, float* h, int accumulate,
+                                         const GroupedSide& g, cudaStream_t stream) {
+  diag_hessian_grouped_finalize_kernel<<<dim3(static_cast<unsigned>((in + 255) / 256),
+                                              static_cast<unsigned>(E)),
+                                         256, 0, stream>>>(g.P, g.cstart, E, in, h, accumulate);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_diag_hessian_grouped(const uint16_t* X, const int64_t* off, int64_t E,
                                         int64_t total, int64_t in, int64_t ldx, float* h,
                                         int accumulate, void* workspace, int num_sms,

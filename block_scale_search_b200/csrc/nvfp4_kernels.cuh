@@ -28,6 +28,20 @@ cudaError_t launch_diag_hessian_grouped(const uint16_t* X, const int64_t* row_of
                                         int64_t total, int64_t in, int64_t ldx, float* h,
                                         int accumulate, void* workspace, int num_sms,
                                         cudaStream_t stream);
+// The grouped kernel's plan (slices of expert-contiguous rows, planned on
+// the device) and partials in its workspace, for streaming its partial pass
+// from another launch (side_reduce.cuh, kind 2).
+struct GroupedSide {
+  int64_t* cstart;  // [E + 2]: first slice of each expert, slices, rows per slice
+  float* P;         // [cap, in] partials
+  int64_t cap, nt;  // slices at most; the plan's target slice count
+  int block;        // the partial kernel's CTA size (row lanes x vectors)
+};
+GroupedSide grouped_diag_side(int64_t E, int64_t in, void* workspace, int num_sms);
+cudaError_t launch_grouped_diag_plan(const int64_t* off, int64_t E, int64_t total,
+                                     const GroupedSide& g, cudaStream_t stream);
+cudaError_t launch_grouped_diag_finalize(int64_t E, int64_t in, float* h, int accumulate,
+                                         const GroupedSide& g, cudaStream_t stream);
 size_t diag_hessian_workspace_bytes(const LanePlan& p, int64_t in);
 cudaError_t launch_diag_hessian(const uint16_t* X, int64_t T, int64_t in, int64_t ldx, float* h,
                                 int accumulate, float* partials, const LanePlan& p,
@@ -91,6 +105,10 @@ cudaError_t launch_scale_sweep_side(const uint16_t* W, int64_t out, int64_t in, 
                                     uint8_t* codes, uint8_t* scales, int8_t* offs,
                                     const SideWork& side, int num_sms, bool* carried,
                                     cudaStream_t stream);
+// The batched sweep with a streaming fifth warp per CTA (4 CTAs per SM).
+cudaError_t launch_scale_sweep_batched_side(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
+                                            bool weighted, int lo, int hi, const SideWork& side,
+                                            cudaStream_t stream);
 cudaError_t launch_scale_sweep(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                const float* h, const float* S, int lo, int hi, uint8_t* codes,
                                uint8_t* scales, int8_t* offs, const LanePlan& p,

@@ -13,6 +13,7 @@
 
 #include "nvfp4_kernels.cuh"
 #include "row_counters.cuh"
+#include "side_reduce.cuh"
 
 namespace {
 
@@ -362,6 +363,41 @@ std::vector<int64_t> share_ctas(const std::vector<int64_t>& elems, int64_t budge
 
 size_t round256(size_t x) { return (x + 255) & ~size_t{255}; }
 
+// The batched sweep's device descriptors: `budget` CTAs shared by the
+// matrices' group counts (eight waves' worth for the plain batched sweep:
+// with many small matrices a one-wave share rounds to whole CTAs and can
+// spill a few into a mostly empty second wave, and every CTA ends with its
+// slowest warp; the more, shorter CTAs the hardware deals out as others
+// finish, the smaller both tails -- measured on the 128-expert layer: 2, 4,
+// 8, 16 waves take 2.33, 2.12, 2.07, 2.08 ms).  Returns the CTAs in all.
+int64_t plan_sweep_batch(const nvfp4_sweep_desc* descs, int64_t n,
+                         const std::vector<int64_t>& groups, int64_t budget,
+                         std::vector<nvfp4::SweepDesc>* dv) {
+  const std::vector<int64_t> ctas = share_ctas(groups, budget);
+  dv->assign(n, nvfp4::SweepDesc{});
+  int64_t total_ctas = 0;
+  for (int64_t i = 0; i < n; ++i) {
+    const nvfp4_sweep_desc& d = descs[i];
+    nvfp4::SweepDesc& m = (*dv)[i];
+    const int64_t c = groups[i] == 0 ? 1 : ctas[i];
+    const nvfp4::LanePlan p = nvfp4::sweep_plan_threads(d.out, d.in, c * nvfp4::kSweepCta);
+    m.W = static_cast<const uint16_t*>(d.W);
+    m.h = d.h;
+    m.S = d.S;
+    m.codes = d.codes;
+    m.scales = d.scales;
+    m.offs = d.chosen_offset;
+    m.out = groups[i] == 0 ? 0 : d.out;  // an empty matrix does no work
+    m.G = d.in / 16;
+    m.ldw = d.ldw;
+    m.GL = p.VL;
+    m.R = p.R;
+    m.cta_begin = total_ctas;
+    total_ctas += c;
+  }
+  return total_ctas;
+}
+
 struct GsBatchPlan {
   std::vector<nvfp4::MatDesc> d;
   int64_t total_ctas = 0;
@@ -433,6 +469,83 @@ int nvfp4_global_scale_batched(const nvfp4_matrix_desc* descs, int64_t n, float 
                                                         status, partial, s));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Validation of nvfp4_quantize_grouped_layer's arguments (NVFP4_OK or the
+// first failing status); the matrices' descriptors for the batched S.
+int check_grouped_layer(const nvfp4_sweep_desc* first, int64_t nf, const nvfp4_sweep_desc* second,
+                        int64_t ns, const nvfp4_grouped_input* x1, const nvfp4_grouped_input* x2,
+                        int64_t experts, float* S, std::vector<nvfp4_matrix_desc>* md,
+                        bool* weighted1, bool* weighted2) {
+  if (nf < 0 || ns < 0 || (nf > 0 && first == nullptr) || (ns > 0 && second == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (x1 == nullptr || x2 == nullptr || S == nullptr || experts <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (experts > 65535) return NVFP4_ERR_SHAPE;
+  for (const nvfp4_grouped_input* x : {x1, x2}) {
+    int st = check_diag_hessian(x->X, x->total_tokens, x->in, x->ldx, x->h, 0);
+    if (st != NVFP4_OK) return st;
+    if (x->row_offsets == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(x->row_offsets, 8) || !aligned(x->h, 16)) return NVFP4_ERR_ALIGN;
+  }
+  if (!aligned(S, 4)) return NVFP4_ERR_ALIGN;
+  md->clear();
+  for (int b = 0; b < 2; ++b) {
+    const nvfp4_sweep_desc* d = b == 0 ? first : second;
+    const int64_t n = b == 0 ? nf : ns;
+    bool any_h = false, all_h = true;
+    for (int64_t i = 0; i < n; ++i) {
+      const nvfp4_sweep_desc& m = d[i];
+      int st = check_matrix(m.W, m.out, m.in, m.ldw, 16);
+      if (st != NVFP4_OK) return st;
+      if (m.out == 0 || m.in == 0) return NVFP4_ERR_SHAPE;
+      if (m.codes == nullptr || m.scales == nullptr) return NVFP4_ERR_INVALID_ARG;
+      // each matrix's S is its place in the one S array the call writes
+      if (m.S != S + (b == 0 ? i : nf + i)) return NVFP4_ERR_INVALID_ARG;
+      if (!aligned(m.h, 16) || !aligned(m.codes, 8)) return NVFP4_ERR_ALIGN;
+      any_h = any_h || m.h != nullptr;
+      all_h = all_h && m.h != nullptr;
+      md->push_back(nvfp4_matrix_desc{m.W, m.out, m.in, m.ldw});
+    }
+    if (any_h && !all_h) return NVFP4_ERR_INVALID_ARG;  // one objective per batch
+    *(b == 0 ? weighted1 : weighted2) = any_h;
+  }
+  return NVFP4_OK;
+}
+
+struct GroupedLayerLayout {
+  size_t gd1 = 0, gd2 = 0, gs = 0, sw1 = 0, sw2 = 0, bytes = 0;
+  GsBatchPlan gsp;
+};
+
+GroupedLayerLayout grouped_layer_layout(int64_t nf, int64_t ns, const nvfp4_grouped_input* x1,
+                                        const nvfp4_grouped_input* x2, int64_t experts,
+                                        const std::vector<nvfp4_matrix_desc>& md, int sms) {
+  GroupedLayerLayout L;
+  size_t off = 0;
+  L.gd1 = off;
+  off = round256(off + nvfp4::diag_hessian_grouped_workspace_bytes(x1->total_tokens, experts,
+                                                                   x1->in, sms));
+  L.gd2 = off;
+  off = round256(off + nvfp4::diag_hessian_grouped_workspace_bytes(x2->total_tokens, experts,
+                                                                   x2->in, sms));
+  L.gsp = plan_global_scale_batch(md.data(), static_cast<int64_t>(md.size()), sms);
+  L.gs = off;
+  off = round256(off + round256(md.size() * sizeof(nvfp4::MatDesc)) +
+                 static_cast<size_t>(L.gsp.total_ctas) * sizeof(uint32_t));
+  L.sw1 = off;
+  off = round256(off + static_cast<size_t>(nf) * sizeof(nvfp4::SweepDesc));
+  L.sw2 = off;
+  off = round256(off + static_cast<size_t>(ns) * sizeof(nvfp4::SweepDesc));
+  L.bytes = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t nvfp4_scale_sweep_quantize_batched_workspace_size(int64_t n) {
   if (n < 0) return 0;
   return round256(static_cast<size_t>(n) * sizeof(nvfp4::SweepDesc)) + 256;
@@ -465,41 +578,142 @@ int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n,
   const int sms = current_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorNoDevice);
   const bool weighted = any_h;
-  // eight waves' worth of CTAs shared by size: with many small matrices a
-  // one-wave share rounds to whole CTAs and can spill a few into a mostly
-  // empty second wave, and every CTA ends with its slowest warp; the more,
-  // shorter CTAs the hardware deals out as others finish, the smaller both
-  // tails (measured on the 128-expert layer: 2, 4, 8, 16 waves take 2.33,
-  // 2.12, 2.07, 2.08 ms)
-  const std::vector<int64_t> ctas =
-      share_ctas(groups, 8 * static_cast<int64_t>(sms) * nvfp4::sweep_resident_ctas(weighted));
-  std::vector<nvfp4::SweepDesc> dv(n);
-  int64_t total_ctas = 0;
-  for (int64_t i = 0; i < n; ++i) {
-    const nvfp4_sweep_desc& d = descs[i];
-    nvfp4::SweepDesc& m = dv[i];
-    const int64_t c = groups[i] == 0 ? 1 : ctas[i];
-    const nvfp4::LanePlan p = nvfp4::sweep_plan_threads(d.out, d.in, c * nvfp4::kSweepCta);
-    m.W = static_cast<const uint16_t*>(d.W);
-    m.h = d.h;
-    m.S = d.S;
-    m.codes = d.codes;
-    m.scales = d.scales;
-    m.offs = d.chosen_offset;
-    m.out = groups[i] == 0 ? 0 : d.out;  // an empty matrix does no work
-    m.G = d.in / 16;
-    m.ldw = d.ldw;
-    m.GL = p.VL;
-    m.R = p.R;
-    m.cta_begin = total_ctas;
-    total_ctas += c;
-  }
+  std::vector<nvfp4::SweepDesc> dv;
+  const int64_t total_ctas = plan_sweep_batch(
+      descs, n, groups, 8 * static_cast<int64_t>(sms) * nvfp4::sweep_resident_ctas(weighted), &dv);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   nvfp4::SweepDesc* d_dev = static_cast<nvfp4::SweepDesc*>(workspace);
   cudaError_t e = cudaMemcpyAsync(d_dev, dv.data(), static_cast<size_t>(n) * sizeof(nvfp4::SweepDesc),
                                   cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(nvfp4::launch_scale_sweep_batched(d_dev, n, total_ctas, weighted, lo, hi, s));
+}
+
+size_t nvfp4_quantize_grouped_layer_workspace_size(const nvfp4_sweep_desc* first, int64_t n_first,
+                                                   const nvfp4_sweep_desc* second, int64_t n_second,
+                                                   const nvfp4_grouped_input* first_input,
+                                                   const nvfp4_grouped_input* second_input,
+                                                   int64_t experts, float* S) {
+  std::vector<nvfp4_matrix_desc> md;
+  bool w1 = false, w2 = false;
+  if (check_grouped_layer(first, n_first, second, n_second, first_input, second_input, experts, S,
+                          &md, &w1, &w2) != NVFP4_OK)
+    return 0;
+  const int sms = current_sm_count();
+  if (sms <= 0) return 0;
+  return grouped_layer_layout(n_first, n_second, first_input, second_input, experts, md, sms).bytes;
+}
+
+int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
+                                 const nvfp4_sweep_desc* second, int64_t n_second,
+                                 const nvfp4_grouped_input* first_input,
+                                 const nvfp4_grouped_input* second_input, int64_t experts,
+                                 float q_max, int lo, int hi, float* S, float* amax, int* status,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* const* sweep_events, void* stream) {
+  std::vector<nvfp4_matrix_desc> md;
+  bool w1 = false, w2 = false;
+  int st = check_grouped_layer(first, n_first, second, n_second, first_input, second_input,
+                               experts, S, &md, &w1, &w2);
+  if (st != NVFP4_OK) return st;
+  if (!std::isfinite(q_max) || !(q_max > 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  if (!aligned(amax, 4) || !aligned(status, 4)) return NVFP4_ERR_ALIGN;
+  if (sweep_events != nullptr)
+    for (int k = 0; k < 4; ++k)
+      if (sweep_events[k] == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  const GroupedLayerLayout L =
+      grouped_layer_layout(n_first, n_second, first_input, second_input, experts, md, sms);
+  if (workspace_bytes < L.bytes) return NVFP4_ERR_WORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const nvfp4_grouped_input& x1 = *first_input;
+  const nvfp4_grouped_input& x2 = *second_input;
+  auto fail = [](cudaError_t e) { return e != cudaSuccess; };
+  cudaError_t e;
+  // 1. h of the first input (the first batch needs it), the second input's
+  //    slice plan, and every matrix's S
+  if (fail(e = nvfp4::launch_diag_hessian_grouped(static_cast<const uint16_t*>(x1.X),
+                                                  x1.row_offsets, experts, x1.total_tokens, x1.in,
+                                                  x1.ldx, x1.h, 0, ws + L.gd1, sms, s)))
+    return cuda_status(e);
+  const nvfp4::GroupedSide g2 = nvfp4::grouped_diag_side(experts, x2.in, ws + L.gd2, sms);
+  if (fail(e = nvfp4::launch_grouped_diag_plan(x2.row_offsets, experts, x2.total_tokens, g2, s)))
+    return cuda_status(e);
+  const int64_t nm = static_cast<int64_t>(md.size());
+  if (nm > 0) {
+    nvfp4::MatDesc* gd = reinterpret_cast<nvfp4::MatDesc*>(ws + L.gs);
+    if (fail(e = cudaMemcpyAsync(gd, L.gsp.d.data(), static_cast<size_t>(nm) * sizeof(nvfp4::MatDesc),
+                                 cudaMemcpyHostToDevice, s)))
+      return cuda_status(e);
+    uint32_t* partial = reinterpret_cast<uint32_t*>(
+        ws + L.gs + round256(static_cast<size_t>(nm) * sizeof(nvfp4::MatDesc)));
+    if (fail(e = nvfp4::launch_global_scale_batched(gd, nm, L.gsp.total_ctas, q_max, S, amax,
+                                                    status, partial, s)))
+      return cuda_status(e);
+  }
+  // 2. the first batch's sweep, its CTAs' fifth warp streaming the second
+  //    input's partials (the grouped kernel's tasks: slice x vector)
+  nvfp4::SideWork side{};
+  side.n = 0;
+  side.tasks = 0;
+  if (x2.total_tokens > 0) {
+    nvfp4::SideJob& j = side.job[side.n++];
+    j.A = static_cast<const uint16_t*>(x2.X);
+    j.rows = x2.total_tokens;
+    j.ld = x2.ldx;
+    j.cols = x2.in;
+    j.P = g2.P;
+    j.off = x2.row_offsets;
+    j.cstart = g2.cstart;
+    j.E = experts;
+    j.block = g2.block;
+    j.kind = 2;
+    j.t0 = 0;
+    j.t1 = g2.cap * (x2.in / 8);
+    side.tasks = j.t1;
+  }
+  auto record = [&](int k) -> cudaError_t {
+    return sweep_events != nullptr ? cudaEventRecord(static_cast<cudaEvent_t>(sweep_events[k]), s)
+                                   : cudaSuccess;
+  };
+  auto sweep_batch = [&](const nvfp4_sweep_desc* d, int64_t n, bool weighted, size_t off,
+                         bool carry) -> cudaError_t {
+    if (n == 0) return cudaSuccess;
+    std::vector<int64_t> groups(n);
+    for (int64_t i = 0; i < n; ++i) groups[i] = d[i].out * (d[i].in / 16);
+    std::vector<nvfp4::SweepDesc> dv;
+    const int64_t per_sm = carry ? 4 : nvfp4::sweep_resident_ctas(weighted);
+    const int64_t total = plan_sweep_batch(d, n, groups, 8 * static_cast<int64_t>(sms) * per_sm, &dv);
+    nvfp4::SweepDesc* dd = reinterpret_cast<nvfp4::SweepDesc*>(ws + off);
+    cudaError_t c = cudaMemcpyAsync(dd, dv.data(), static_cast<size_t>(n) * sizeof(nvfp4::SweepDesc),
+                                    cudaMemcpyHostToDevice, s);
+    if (c != cudaSuccess) return c;
+    return carry ? nvfp4::launch_scale_sweep_batched_side(dd, n, total, weighted, lo, hi, side, s)
+                 : nvfp4::launch_scale_sweep_batched(dd, n, total, weighted, lo, hi, s);
+  };
+  const bool carry = n_first > 0 && side.tasks > 0;
+  if (fail(e = record(0)) || fail(e = sweep_batch(first, n_first, w1, L.sw1, carry)) ||
+      fail(e = record(1)))
+    return cuda_status(e);
+  if (!carry && x2.total_tokens > 0) {
+    // nothing to carry it: the grouped partial pass on its own
+    if (fail(e = nvfp4::launch_diag_hessian_grouped(static_cast<const uint16_t*>(x2.X),
+                                                    x2.row_offsets, experts, x2.total_tokens,
+                                                    x2.in, x2.ldx, x2.h, 0, ws + L.gd2, sms, s)))
+      return cuda_status(e);
+  } else if (fail(e = nvfp4::launch_grouped_diag_finalize(experts, x2.in, x2.h, 0, g2, s))) {
+    return cuda_status(e);
+  }
+  // 3. the second batch's sweep
+  if (fail(e = record(2)) || fail(e = sweep_batch(second, n_second, w2, L.sw2, false)) ||
+      fail(e = record(3)))
+    return cuda_status(e);
+  return NVFP4_OK;
 }
 
 }  // extern "C"

@@ -296,6 +296,52 @@ scale_sweep_batched_kernel(const SweepDesc* __restrict__ d, int64_t n, int lo, i
                                          m.scales, m.offs, m.GL, m.R, tid);
 }
 
+// The batched sweep with a fifth warp per CTA streaming side reductions
+// (side_reduce.cuh): four CTAs of 160 threads per SM; the side tasks are
+// dealt to all CTAs of the launch, which the hardware runs in waves.
+template <bool kWeighted, int kK>
+__global__ void __launch_bounds__(kCta + 32, 4)
+scale_sweep_batched_side_kernel(const SweepDesc* __restrict__ d, int64_t n, int lo, int hi,
+                                const __grid_constant__ SideWork side) {
+  __shared__ SweepSmem<16> sm;
+  __shared__ SideRing ring;
+  fill_candidate_table(sm.tab);
+  __syncthreads();
+  if (threadIdx.x < kCta) {
+    int64_t a = 0, z = n - 1;  // last descriptor with cta_begin <= blockIdx.x
+    while (a < z) {
+      const int64_t mid = (a + z + 1) >> 1;
+      if (d[mid].cta_begin <= static_cast<int64_t>(blockIdx.x)) a = mid; else z = mid - 1;
+    }
+    const SweepDesc m = d[a];
+    const int64_t tid = (static_cast<int64_t>(blockIdx.x) - m.cta_begin) * kCta + threadIdx.x;
+    sweep_matrix<kWeighted, false, 16, kK>(sm, m.W, m.out, m.G, m.ldw, m.h, m.S, lo, hi, m.codes,
+                                           m.scales, m.offs, m.GL, m.R, tid);
+  } else {
+    run_side_work(side, ring, static_cast<int>(threadIdx.x - kCta), blockIdx.x, gridDim.x);
+  }
+}
+
+cudaError_t launch_scale_sweep_batched_side(const SweepDesc* d_dev, int64_t n, int64_t total_ctas,
+                                            bool weighted, int lo, int hi, const SideWork& side,
+                                            cudaStream_t stream) {
+  if (n == 0 || total_ctas == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>(total_ctas);
+  const int K = hi - lo + 1;
+  if (weighted) {
+    if (K == 16)
+      scale_sweep_batched_side_kernel<true, 16><<<blocks, kCta + 32, 0, stream>>>(d_dev, n, lo, hi, side);
+    else
+      scale_sweep_batched_side_kernel<true, 0><<<blocks, kCta + 32, 0, stream>>>(d_dev, n, lo, hi, side);
+  } else {
+    if (K == 16)
+      scale_sweep_batched_side_kernel<false, 16><<<blocks, kCta + 32, 0, stream>>>(d_dev, n, lo, hi, side);
+    else
+      scale_sweep_batched_side_kernel<false, 0><<<blocks, kCta + 32, 0, stream>>>(d_dev, n, lo, hi, side);
+  }
+  return cudaGetLastError();
+}
+
 int sweep_resident_ctas(bool weighted) {
   static const int ctas[2] = {
       resident_ctas(reinterpret_cast<const void*>(&scale_sweep_kernel<false, 0>), kCta),

@@ -25,16 +25,22 @@ constexpr int kSideRows = 8;     // rows per batch (the standalone kernel's run 
 constexpr int kSideBatches = 4;  // batches in flight per lane
 constexpr int kMaxSideJobs = 8;
 
-// One reduction's share of tasks [t0, t1) of its R x V task grid.
+// One reduction's share of tasks [t0, t1) of its task grid.
 struct SideJob {
   const uint16_t* A;   // bf16 [rows, ld]
   int64_t rows, ld;
   int64_t cols;        // elements per row (a multiple of 8)
-  int64_t R;           // row lanes of the task grid
+  int64_t R;           // kinds 0, 1: row lanes of the task grid (R x V tasks)
   int64_t t0, t1;      // task range
-  float* P;            // kind 0: partials [R, cols]
+  float* P;            // kinds 0, 2: partials
   uint32_t* amax;      // kind 1: the max word (bf16 bit pattern of |a|)
-  int kind;            // 0: diagonal Hessian, 1: absmax
+  // kind 2: expert-contiguous rows, as the grouped diagonal-Hessian kernel
+  // reads them: row offsets [E + 1], its slice plan (device), and its CTA size
+  const int64_t* off;
+  const int64_t* cstart;
+  int64_t E;
+  int block;
+  int kind;            // 0: diagonal Hessian, 1: absmax, 2: grouped diagonal Hessian
 };
 
 struct SideWork {
@@ -56,32 +62,38 @@ __device__ __forceinline__ void sq_acc_bf16x2(uint32_t w, float& s0, float& s1) 
       : "+f"(s0), "+f"(s1) : "r"(w));
 }
 
-// Task (r, v) of a job: runs of kSideRows rows through the ring, then the
-// remaining rows one by one, as the standalone kernels order them.
-__device__ __forceinline__ void side_task(const SideJob& j, int64_t r, int64_t v, SideRing& ring,
-                                          int lane) {
-  const uint16_t* col = j.A + v * 8;
-  const int64_t R = j.R;
-  const int64_t n = (j.rows - r + R - 1) / R;  // rows of this task (r < R <= rows)
+// The running maximum of eight sign-cleared bf16 patterns (two per 32 bits).
+__device__ __forceinline__ uint32_t absmax_bf16x8(uint32_t m, const uint4& q) {
+  return __vmaxu2(__vmaxu2(m, q.x & 0x7FFF7FFFu),
+                  __vmaxu2(__vmaxu2(q.y & 0x7FFF7FFFu, q.z & 0x7FFF7FFFu), q.w & 0x7FFF7FFFu));
+}
+
+// Rows t0, t0 + stride, ... below t_end of one 16-byte column (col; ld
+// elements per row): full runs of kSideRows rows through the ring, then the
+// remaining rows one by one, as the standalone kernels order them.  kSq: sums
+// of squares added into acc (a run summed first, then added); otherwise the
+// maximum of sign-cleared patterns into m.
+template <bool kSq>
+__device__ __forceinline__ void side_stream(const uint16_t* col, int64_t ld, int64_t t0,
+                                            int64_t stride, int64_t t_end, SideRing& ring,
+                                            int lane, float (&acc)[8], uint32_t& m) {
+  const int64_t n = t_end > t0 ? (t_end - t0 + stride - 1) / stride : 0;
   const int64_t runs = n / kSideRows;
   auto issue = [&](int64_t k) {
     const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
 #pragma unroll
     for (int u = 0; u < kSideRows; ++u)
-      cp_async16(&ring.v[slot + u][lane], col + (r + (k * kSideRows + u) * R) * j.ld);
+      cp_async16(&ring.v[slot + u][lane], col + (t0 + (k * kSideRows + u) * stride) * ld);
   };
 #pragma unroll
   for (int k = 0; k < kSideBatches; ++k) {
     if (k < runs) issue(k);
     cp_async_commit();
   }
-  if (j.kind == 0) {
-    float acc[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
-    for (int64_t k = 0; k < runs; ++k) {
-      cp_async_wait<kSideBatches - 1>();
-      const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
+  for (int64_t k = 0; k < runs; ++k) {
+    cp_async_wait<kSideBatches - 1>();
+    const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
+    if constexpr (kSq) {
       float s[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) s[c] = 0.0f;
@@ -95,42 +107,78 @@ __device__ __forceinline__ void side_task(const SideJob& j, int64_t r, int64_t v
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) acc[c] += s[c];
-      if (k + kSideBatches < runs) issue(k + kSideBatches);
-      cp_async_commit();
+    } else {
+#pragma unroll
+      for (int u = 0; u < kSideRows; ++u) m = absmax_bf16x8(m, ring.v[slot + u][lane]);
     }
-    cp_async_wait<0>();
-    for (int64_t t = r + runs * kSideRows * R; t < j.rows; t += R) {
-      const uint4 q = ld_stream_v4(col + t * j.ld);
+    if (k + kSideBatches < runs) issue(k + kSideBatches);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  for (int64_t t = t0 + runs * kSideRows * stride; t < t_end; t += stride) {
+    const uint4 q = ld_stream_v4(col + t * ld);
+    if constexpr (kSq) {
       sq_acc_bf16x2(q.x, acc[0], acc[1]);
       sq_acc_bf16x2(q.y, acc[2], acc[3]);
       sq_acc_bf16x2(q.z, acc[4], acc[5]);
       sq_acc_bf16x2(q.w, acc[6], acc[7]);
+    } else {
+      m = absmax_bf16x8(m, q);
     }
-    float4* dst = reinterpret_cast<float4*>(j.P + r * j.cols + v * 8);
-    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  } else {
-    uint32_t m = 0;
-    for (int64_t k = 0; k < runs; ++k) {
-      cp_async_wait<kSideBatches - 1>();
-      const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
+  }
+}
+
+__device__ __forceinline__ void store_partial(float* p, const float (&acc)[8]) {
+  float4* dst = reinterpret_cast<float4*>(p);
+  dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+// Task t of a job.  Kinds 0 and 1: t = r V + v covers rows r, r + R, ... of
+// vector v.  Kind 2: t = q V + v is slice q of the grouped kernel's plan for
+// vector v: the row lanes of that kernel's CTA one after another, each as that
+// lane streams it, then added in lane order as its CTA does.
+__device__ __forceinline__ void side_task(const SideJob& j, int64_t t, SideRing& ring, int lane) {
+  const int64_t V = j.cols / 8;
+  const int64_t q = t / V, v = t - q * V;
+  const uint16_t* col = j.A + v * 8;
+  float acc[8];
+  uint32_t m = 0;
 #pragma unroll
-      for (int u = 0; u < kSideRows; ++u) {
-        const uint4 q = ring.v[slot + u][lane];
-        m = __vmaxu2(__vmaxu2(m, q.x & 0x7FFF7FFFu),
-                     __vmaxu2(__vmaxu2(q.y & 0x7FFF7FFFu, q.z & 0x7FFF7FFFu), q.w & 0x7FFF7FFFu));
-      }
-      if (k + kSideBatches < runs) issue(k + kSideBatches);
-      cp_async_commit();
-    }
-    cp_async_wait<0>();
-    for (int64_t t = r + runs * kSideRows * R; t < j.rows; t += R) {
-      const uint4 q = ld_stream_v4(col + t * j.ld);
-      m = __vmaxu2(__vmaxu2(m, q.x & 0x7FFF7FFFu),
-                   __vmaxu2(__vmaxu2(q.y & 0x7FFF7FFFu, q.z & 0x7FFF7FFFu), q.w & 0x7FFF7FFFu));
-    }
+  for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+  if (j.kind == 0) {
+    side_stream<true>(col, j.ld, q, j.R, j.rows, ring, lane, acc, m);
+    store_partial(j.P + q * j.cols + v * 8, acc);
+  } else if (j.kind == 1) {
+    side_stream<false>(col, j.ld, q, j.R, j.rows, ring, lane, acc, m);
     m = max(m & 0xFFFFu, m >> 16);
     if (m != 0u) atomicMax(j.amax, m);
+  } else {
+    const int64_t E = j.E;
+    if (q >= j.cstart[E]) return;  // beyond the plan's slices
+    const int64_t target = j.cstart[E + 1];
+    int64_t a = 0, z = E - 1;       // expert: last e with cstart[e] <= q
+    while (a < z) {
+      const int64_t mid = (a + z + 1) >> 1;
+      if (j.cstart[mid] <= q) a = mid; else z = mid - 1;
+    }
+    int64_t r_lo = j.off[a], r_hi = j.off[a + 1];
+    r_lo = r_lo < 0 ? 0 : (r_lo > j.rows ? j.rows : r_lo);
+    r_hi = r_hi < r_lo ? r_lo : (r_hi > j.rows ? j.rows : r_hi);
+    const int64_t rb = r_lo + (q - j.cstart[a]) * target;
+    const int64_t re = (rb + target < r_hi) ? rb + target : r_hi;
+    const int64_t v0 = (v / 256) * 256;
+    const int64_t VLc = (V - v0) < 256 ? (V - v0) : 256;
+    const int64_t RL = j.block / VLc;
+    for (int64_t rl = 0; rl < RL; ++rl) {
+      float part[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) part[c] = 0.0f;
+      side_stream<true>(col, j.ld, rb + rl, RL, re, ring, lane, part, m);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = rl == 0 ? part[c] : acc[c] + part[c];
+    }
+    store_partial(j.P + q * j.cols + v * 8, acc);
   }
 }
 
@@ -148,10 +196,7 @@ __device__ __forceinline__ void run_side_work(const SideWork& w, SideRing& ring,
     }
     if (jb >= w.n) break;
     const SideJob& j = w.job[jb];
-    const int64_t t = j.t0 + (k - base);
-    const int64_t V = j.cols / 8;
-    const int64_t r = t / V;
-    side_task(j, r, t - r * V, ring, lane);
+    side_task(j, j.t0 + (k - base), ring, lane);
   }
 }
 

@@ -312,6 +312,59 @@ int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
                          void* const* sweep_events, void* stream);
 
 /* ------------------------------------------------------------------------
+ * A mixture-of-experts layer in one call: two batches of expert matrices, each
+ * batch reading one expert-contiguous calibration input (for example every
+ * expert's gate and up projections reading the routed tokens' hidden states,
+ * then every expert's down projection reading their activations).
+ *   first_input.h  = the grouped diagonal Hessian of first_input, as
+ *                    nvfp4_diag_hessian_grouped writes it (not accumulated);
+ *   S[0 .. n_first + n_second)  = the global scale of every matrix, first
+ *                    batch then second, as nvfp4_global_scale_batched writes
+ *                    it (amax and status too, both nullable);
+ *   the first batch's sweeps, then second_input.h, then the second batch's
+ *   sweeps, as nvfp4_scale_sweep_quantize_batched writes them.
+ * The bytes written equal those of the grouped and batched calls.  The
+ * second input's diagonal Hessian is streamed by a fifth warp in every CTA of
+ * the first batch's sweep, which is bound by FP32 arithmetic.
+ *
+ *   first, second  sweep descriptors as for nvfp4_scale_sweep_quantize_batched
+ *              (out, in > 0); descriptor i of `first` has S == S + i, of
+ *              `second` S == S + n_first + i.  Their h may point into the
+ *              inputs' h (the first batch into first_input.h, the second into
+ *              either), or be NULL for a whole batch (plain MSE).
+ *   first_input, second_input  X bf16 [total_tokens, ldx] with row_offsets
+ *              int64 [experts + 1] on the device (as for
+ *              nvfp4_diag_hessian_grouped); h float [experts, in], 16-byte
+ *              aligned (written).
+ *   workspace  device, 256-byte aligned, at least
+ *              nvfp4_quantize_grouped_layer_workspace_size(...) bytes (device
+ *              dependent; 0 for invalid arguments or no device).
+ *   sweep_events  NULL or 4 cudaEvent_t (as void*): recorded on `stream`
+ *              right before and after the first batch's sweep launch (with
+ *              what it streams) and the second's, for timing.
+ * Asynchronous on `stream`; descriptors are read on the host during the call.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const void* X;
+  const int64_t* row_offsets;
+  int64_t total_tokens, in, ldx;
+  float* h;
+} nvfp4_grouped_input;
+
+size_t nvfp4_quantize_grouped_layer_workspace_size(const nvfp4_sweep_desc* first, int64_t n_first,
+                                                   const nvfp4_sweep_desc* second, int64_t n_second,
+                                                   const nvfp4_grouped_input* first_input,
+                                                   const nvfp4_grouped_input* second_input,
+                                                   int64_t experts, float* S);
+int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
+                                 const nvfp4_sweep_desc* second, int64_t n_second,
+                                 const nvfp4_grouped_input* first_input,
+                                 const nvfp4_grouped_input* second_input, int64_t experts,
+                                 float q_max, int lo, int hi, float* S, float* amax, int* status,
+                                 void* workspace, size_t workspace_bytes,
+                                 void* const* sweep_events, void* stream);
+
+/* ------------------------------------------------------------------------
  * Online activation quantization (ScaleSweep summary, sec. 1-3 and
  * "Experimental Results": in the W+A settings the activations are NVFP4 too,
  * their scales chosen with the MSE objective and the [-3, +7] window).  One
