@@ -169,9 +169,10 @@ class ClockSampler:
 
 def build_layer(rank: int, device, name: str = "llama33_70b_mlp"):
     import torch
-    if name == "moe_grouped":
+    if name in ("moe_grouped", "moe_slice"):
         import workloads
-        wl = workloads.moe_grouped(device=device)
+        wl = (workloads.moe_grouped(device=device) if name == "moe_grouped" else
+              workloads.moe_grouped(tokens=32768, experts=16, device=device))
         Ws = {m.name: m.make(device) for m in wl.matrices}
         Xs = {k: c.make(device) for k, c in wl.calibs.items()}
         torch.cuda.synchronize()
@@ -446,7 +447,8 @@ class GroupedStep:
         self.side_bytes = Xs[k2].numel() * 2       # streamed beside the first batch's sweep
         self.carry_launches = 1
         self.carry_elems = sum(m.out * m.inp for m in first)
-        self.traffic_key = "scale_sweep_grouped_layer"   # no capture recorded: traffic null
+        self.traffic_key = "scale_sweep_grouped_layer"
+        self.plain_traffic_key = "scale_sweep_batched"
         self.layer_note = ("the first input's h and every matrix's S run first (rest); the second "
                            "input's h is streamed by a fifth warp in each CTA of the first batch's "
                            "sweep (carrying sweep)")
@@ -821,6 +823,8 @@ WORKLOADS = {
     "mlp_layer_slice": ("mlp_layer_slice (profiling size): gate/up 8192x4096, down 4096x8192 "
                         "bf16 N(0,0.015) 0.1% x10; X 16384 tokens x {4096, 8192} bf16 "
                         "lognormal(1.5) channel scales"),
+    "moe_slice": ("moe_slice (profiling size): 16 experts x {gate, up 768x2048; down 2048x768} "
+                  "bf16 N(0,0.02) 0.1% x10; 32768 tokens routed top-8 (Zipf 1.1)"),
     "moe_grouped": ("moe_grouped: 128 experts x {gate, up 768x2048; down 2048x768} bf16 N(0,0.02) "
                     "0.1% x10; 262144 tokens routed top-8 (Zipf 1.1), per-expert X slices and h; "
                     "grouped diag-Hessian + batched global scale + batched sweep"),
@@ -951,7 +955,7 @@ def main():
             dist.destroy_process_group()
         return
     wl, Ws, Xs = build_layer(rank, dev, args.workload)
-    if args.workload == "moe_grouped":
+    if args.workload in ("moe_grouped", "moe_slice"):
         step = GroupedStep(nv, wl, Ws, Xs, dev, serial=args.schedule == "serial",
                            layer=args.schedule in ("auto", "layer"))
     else:
@@ -1001,7 +1005,7 @@ def main():
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if args.e2e_steps > 0 and args.workload != "moe_grouped":
+    if args.e2e_steps > 0 and args.workload not in ("moe_grouped", "moe_slice"):
         hostW = {n: W.cpu().pin_memory() for n, W in Ws.items()}
         hostX = {k: X.cpu().pin_memory() for k, X in Xs.items()}
         hostC = {n: torch.empty_like(c, device="cpu").pin_memory() for n, c in step.codes.items()}
@@ -1095,7 +1099,8 @@ def main():
         # sweeps' from their capture (per algorithmic byte, side bytes
         # included), the last sweep's from the plain sweep's capture
         t_side = profiled_traffic(step.traffic_key, SWEEP_BYTES_PER_ELEM * step.carry_elems + side)
-        t_plain = profiled_traffic("scale_sweep", wl.weight_elems - step.carry_elems)
+        t_plain = profiled_traffic(getattr(step, "plain_traffic_key", "scale_sweep"),
+                                   wl.weight_elems - step.carry_elems)
         roofline["traffic"] = (None if t_side is None or t_plain is None
                                else (t_side + t_plain) / sweep_launches)
         roofline["traffic_note"] = ("DRAM read+write bytes per sweep launch, averaged over the "
