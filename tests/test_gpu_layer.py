@@ -3,6 +3,7 @@ every input, S (and status) of every weight, codes, scales and offsets of
 every sweep -- whether the reductions ride along earlier sweeps (shapes whose
 rows hold a multiple of 512 elements, long enough to hand rows out at run
 time) or run on their own.  Needs a B200."""
+import numpy as np
 import pytest
 import torch
 
@@ -144,3 +145,27 @@ def test_many_projections_fill_the_side_job_slots(nv):
     Xs = [workloads.calib(2048, 2048, 1.0, 650, DEV), workloads.calib(1536, 4096, 1.0, 651, DEV),
           workloads.calib(3000, 2048, 1.0, 652, DEV), workloads.calib(1024, 2048, 1.0, 653, DEV)]
     _check_same(nv, Ws, Xs, [k for _, _, k in shapes])
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3, 4])
+def test_random_layers(nv, seed):
+    """Random projections over random inputs (shapes a multiple of 16 wide,
+    some long enough to carry side work, some not; weighted and MSE weights;
+    random windows): the layer call equals the per-step calls."""
+    import workloads
+    rng = np.random.default_rng(seed)
+    nx = int(rng.integers(1, 4))
+    widths = [int(rng.choice([512, 1024, 2048, 4096, 1040])) for _ in range(nx)]
+    Xs = [workloads.calib(int(rng.integers(1, 3000)), w, 1.0, 700 + 10 * seed + k, DEV)
+          for k, w in enumerate(widths)]
+    nw = int(rng.integers(1, 7))
+    Ws, inputs = [], []
+    for j in range(nw):
+        k = int(rng.integers(-1, nx))
+        inp = widths[k] if k >= 0 else int(rng.choice([256, 2048]))
+        out = int(rng.choice([64, 700, 3000, 5000]))
+        Ws.append(workloads.weight(out, inp, 0.02, 0.001, 10.0, 800 + 10 * seed + j, DEV))
+        inputs.append(k)
+    lo = int(rng.integers(-12, 1))
+    hi = int(rng.integers(0, 16 + lo))
+    _check_same(nv, Ws, Xs, inputs, q_max=float(rng.choice([256.0, 448.0])), lo=lo, hi=hi)
