@@ -103,3 +103,20 @@ def test_moe_layer_at_the_benchmarked_size(nv):
     W1 = [Ws[f"e{e}.gate"] for e in range(E)] + [Ws[f"e{e}.up"] for e in range(E)]
     W2 = [Ws[f"e{e}.down"] for e in range(E)]
     _run_both(nv, W1, W2, X1, X2, wl.calibs["gu"].row_offsets)
+
+
+@pytest.mark.parametrize("seed", [5, 6, 7])
+def test_random_moe_layers(nv, seed):
+    """Random expert counts, routings (with empty experts), widths, windows
+    and objectives: the grouped layer call equals the grouped and batched
+    calls."""
+    rng = np.random.default_rng(seed)
+    E = int(rng.integers(1, 10))
+    counts = [int(c) if rng.random() > 0.2 else 0 for c in rng.integers(1, 4000, size=E)]
+    gu_in = int(rng.choice([512, 1024, 2048]))
+    gu_out = int(rng.choice([256, 768, 1040]))
+    W1, W2, X1, X2, offs = _moe(E, counts, gu_out, gu_in, 1000 + 37 * seed)
+    lo = int(rng.integers(-10, 1))
+    hi = int(rng.integers(0, 16 + lo))
+    _run_both(nv, W1, W2, X1, X2, offs, lo=lo, hi=hi, q_max=float(rng.choice([256.0, 448.0])),
+              weighted=bool(rng.random() > 0.3))
