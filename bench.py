@@ -444,14 +444,21 @@ class GroupedStep:
                                                             self.lx[1], self.E, self.lS)
         self.lws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
         self.lnb = nb
-        self.side_bytes = Xs[k2].numel() * 2       # streamed beside the first batch's sweep
+        # the call sweeps first whichever batch costs less; the other input's h
+        # is streamed beside that sweep
+        order = nv.nvfp4_quantize_grouped_layer_order(self.lfirst, self.lsecond, self.lx[0],
+                                                      self.lx[1], self.E, self.lS, LO, HI)
+        carrier, carried = (first, k2) if order == 0 else (second, k1)
+        self.layer_order = [k1, k2] if order == 0 else [k2, k1]
+        self.side_bytes = Xs[carried].numel() * 2  # streamed beside the carrying sweep
         self.carry_launches = 1
-        self.carry_elems = sum(m.out * m.inp for m in first)
+        self.carry_elems = sum(m.out * m.inp for m in carrier)
         self.traffic_key = "scale_sweep_grouped_layer"
         self.plain_traffic_key = "scale_sweep_batched"
-        self.layer_note = ("the first input's h and every matrix's S run first (rest); the second "
-                           "input's h is streamed by a fifth warp in each CTA of the first batch's "
-                           "sweep (carrying sweep)")
+        self.layer_note = (f"the {self.layer_order[0]} input's h and every matrix's S run first "
+                           f"(rest); the {carried} input's h is streamed by a fifth warp in each CTA "
+                           f"of the {self.layer_order[0]} batch's sweep (carrying sweep), then the "
+                           f"{carried} batch is swept")
 
     @property
     def launches_per_step(self):
@@ -498,8 +505,11 @@ class GroupedStep:
             if ev is not None:
                 b.record(stream)
                 ev.setdefault("layer_call", []).append((a, b))
-                ev.setdefault("scale_sweep", []).append((sev[0], sev[1]))
-                ev.setdefault("scale_sweep", []).append((sev[2], sev[3]))
+                # the carrying sweep (the batch swept first) is listed first
+                pairs = [(sev[0], sev[1]), (sev[2], sev[3])]
+                if self.layer_order[0] != self.keys[0]:
+                    pairs.reverse()
+                ev.setdefault("scale_sweep", []).extend(pairs)
             return
 
         def dh(k, s):

@@ -27,7 +27,7 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
     "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "quantize_layer_many",
     "LayerWeight", "LayerInput", "GroupedInput", "nvfp4_quantize_grouped_layer_workspace_size",
-    "nvfp4_quantize_grouped_layer",
+    "nvfp4_quantize_grouped_layer", "nvfp4_quantize_grouped_layer_order",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
     "nvfp4_scale_sweep_quantize", "nvfp4_dequantize", "nvfp4_quantize_activations",
     "quantize_activations", "nvfp4_blocked_scales_size", "nvfp4_scales_to_blocked",
@@ -99,6 +99,9 @@ _SIGS = {
     "nvfp4_quantize_grouped_layer_workspace_size": ([C.POINTER(SweepDesc), _i64, C.POINTER(SweepDesc),
                                                      _i64, C.POINTER(GroupedInput),
                                                      C.POINTER(GroupedInput), _i64, _vp], _sz),
+    "nvfp4_quantize_grouped_layer_order": ([C.POINTER(SweepDesc), _i64, C.POINTER(SweepDesc), _i64,
+                                            C.POINTER(GroupedInput), C.POINTER(GroupedInput), _i64,
+                                            _vp, _int, _int], _int),
     "nvfp4_quantize_grouped_layer": ([C.POINTER(SweepDesc), _i64, C.POINTER(SweepDesc), _i64,
                                       C.POINTER(GroupedInput), C.POINTER(GroupedInput), _i64, _f32,
                                       _int, _int, _vp, _vp, _vp, _vp, _sz, C.POINTER(_vp), _vp],
@@ -149,7 +152,9 @@ def _check(fn: str, st: int):
 
 
 def _ptr(t) -> int | None:
-    return None if t is None else t.data_ptr()
+    if t is None or isinstance(t, int):
+        return t
+    return t.data_ptr()
 
 
 def _stream(stream) -> int | None:
@@ -244,6 +249,18 @@ def nvfp4_quantize_grouped_layer_workspace_size(first, second, first_input, seco
     return lib().nvfp4_quantize_grouped_layer_workspace_size(
         fa, len(first), sa, len(second), C.byref(first_input), C.byref(second_input), experts,
         _ptr(S))
+
+
+def nvfp4_quantize_grouped_layer_order(first, second, first_input, second_input, experts, S,
+                                       lo, hi) -> int:
+    """0 if nvfp4_quantize_grouped_layer with these arguments sweeps `first`
+    first, 1 if it sweeps `second` first (host only, no CUDA call)."""
+    fa, sa = _sweep_array(first), _sweep_array(second)
+    r = lib().nvfp4_quantize_grouped_layer_order(
+        fa, len(first), sa, len(second), C.byref(first_input), C.byref(second_input), experts,
+        _ptr(S), int(lo), int(hi))
+    _check("nvfp4_quantize_grouped_layer_order", min(r, 0))
+    return r
 
 
 def nvfp4_quantize_grouped_layer(first, second, first_input, second_input, experts, q_max, lo, hi,

@@ -6,9 +6,11 @@
 // and launch.  No C++ exception crosses this boundary.
 #include "nvfp4hs.h"
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <functional>
 #include <vector>
 
 #include "nvfp4_kernels.cuh"
@@ -542,6 +544,49 @@ GroupedLayerLayout grouped_layer_layout(int64_t nf, int64_t ns, const nvfp4_grou
   return L;
 }
 
+// Which batch a grouped layer call sweeps first.  The input of the batch swept
+// first has its h computed on its own beforehand; the other input's h is
+// streamed beside that sweep.  Costs are estimated in HBM-byte equivalents:
+//   R(x)   = the bytes of input x (its reduction is bound by HBM);
+//   Sw(b)  = weight elements x candidates x 1.3 (a sweep, bound by FP32
+//            arithmetic, takes about 2.1e-13 s per element and candidate on
+//            B200, as long as 1.3 bytes take at the copy bandwidth);
+//   carrying R(x) beside Sw(b) takes max(Sw(b) + 0.38 R(x), R(x)) (a carrying
+//   sweep slows by about 38% of the streamed reduction's time on its own).
+// The call with a first is R(x_a) + carry(a, x_b) + Sw(b); the batch whose order
+// costs less goes first (a tie keeps the caller's order).  The second batch
+// may go first only if none of its h point into the first input's h, which
+// would not be ready yet.
+bool grouped_layer_second_first(const nvfp4_sweep_desc* first, int64_t nf,
+                                const nvfp4_sweep_desc* second, int64_t ns,
+                                const nvfp4_grouped_input& x1, const nvfp4_grouped_input& x2,
+                                int64_t experts, int lo, int hi) {
+  const float* h1_lo = x1.h;
+  const float* h1_hi = x1.h + experts * x1.in;
+  for (int64_t i = 0; i < ns; ++i) {
+    const float* h = second[i].h;
+    if (h != nullptr && std::less_equal<const float*>()(h1_lo, h) && std::less<const float*>()(h, h1_hi))
+      return false;
+  }
+  constexpr double kSweepBytes = 1.3, kCarry = 0.38;
+  const double K = static_cast<double>(hi - lo + 1);
+  auto sweep = [&](const nvfp4_sweep_desc* d, int64_t n) {
+    double e = 0.0;
+    for (int64_t i = 0; i < n; ++i) e += static_cast<double>(d[i].out) * static_cast<double>(d[i].in);
+    return e * K * kSweepBytes;
+  };
+  auto bytes = [](const nvfp4_grouped_input& x) {
+    return 2.0 * static_cast<double>(x.total_tokens) * static_cast<double>(x.in);
+  };
+  auto cost = [&](double ra, double swa, int64_t na, double rb, double swb) {
+    const double carry = na > 0 ? std::max(swa + kCarry * rb, rb) : rb;
+    return ra + carry + swb;
+  };
+  const double s1 = sweep(first, nf), s2 = sweep(second, ns);
+  const double r1 = bytes(x1), r2 = bytes(x2);
+  return cost(r2, s2, ns, r1, s1) < cost(r1, s1, nf, r2, s2);
+}
+
 }  // namespace
 
 extern "C" {
@@ -604,6 +649,23 @@ size_t nvfp4_quantize_grouped_layer_workspace_size(const nvfp4_sweep_desc* first
   return grouped_layer_layout(n_first, n_second, first_input, second_input, experts, md, sms).bytes;
 }
 
+int nvfp4_quantize_grouped_layer_order(const nvfp4_sweep_desc* first, int64_t n_first,
+                                       const nvfp4_sweep_desc* second, int64_t n_second,
+                                       const nvfp4_grouped_input* first_input,
+                                       const nvfp4_grouped_input* second_input, int64_t experts,
+                                       float* S, int lo, int hi) {
+  std::vector<nvfp4_matrix_desc> md;
+  bool w1 = false, w2 = false;
+  const int st = check_grouped_layer(first, n_first, second, n_second, first_input, second_input,
+                                     experts, S, &md, &w1, &w2);
+  if (st != NVFP4_OK) return st;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  return grouped_layer_second_first(first, n_first, second, n_second, *first_input, *second_input,
+                                    experts, lo, hi)
+             ? 1
+             : 0;
+}
+
 int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
                                  const nvfp4_sweep_desc* second, int64_t n_second,
                                  const nvfp4_grouped_input* first_input,
@@ -633,16 +695,30 @@ int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const nvfp4_grouped_input& x1 = *first_input;
   const nvfp4_grouped_input& x2 = *second_input;
+  // a: the batch swept first, its input's h computed on its own beforehand;
+  // b: the batch swept second, its input's h streamed beside a's sweep
+  const bool swap = grouped_layer_second_first(first, n_first, second, n_second, x1, x2, experts,
+                                               lo, hi);
+  const nvfp4_sweep_desc* da = swap ? second : first;
+  const nvfp4_sweep_desc* db = swap ? first : second;
+  const int64_t na = swap ? n_second : n_first, nb = swap ? n_first : n_second;
+  const bool wa = swap ? w2 : w1, wb = swap ? w1 : w2;
+  const nvfp4_grouped_input& xa = swap ? x2 : x1;
+  const nvfp4_grouped_input& xb = swap ? x1 : x2;
+  char* const gda = ws + (swap ? L.gd2 : L.gd1);
+  char* const gdb = ws + (swap ? L.gd1 : L.gd2);
+  const size_t swa = swap ? L.sw2 : L.sw1, swb = swap ? L.sw1 : L.sw2;
+  const int eva = swap ? 2 : 0, evb = swap ? 0 : 2;  // sweep_events pairs: first's, second's
   auto fail = [](cudaError_t e) { return e != cudaSuccess; };
   cudaError_t e;
-  // 1. h of the first input (the first batch needs it), the second input's
-  //    slice plan, and every matrix's S
-  if (fail(e = nvfp4::launch_diag_hessian_grouped(static_cast<const uint16_t*>(x1.X),
-                                                  x1.row_offsets, experts, x1.total_tokens, x1.in,
-                                                  x1.ldx, x1.h, 0, ws + L.gd1, sms, s)))
+  // 1. h of a's input (a's sweep needs it), b's input's slice plan, and every
+  //    matrix's S
+  if (fail(e = nvfp4::launch_diag_hessian_grouped(static_cast<const uint16_t*>(xa.X),
+                                                  xa.row_offsets, experts, xa.total_tokens, xa.in,
+                                                  xa.ldx, xa.h, 0, gda, sms, s)))
     return cuda_status(e);
-  const nvfp4::GroupedSide g2 = nvfp4::grouped_diag_side(experts, x2.in, ws + L.gd2, sms);
-  if (fail(e = nvfp4::launch_grouped_diag_plan(x2.row_offsets, experts, x2.total_tokens, g2, s)))
+  const nvfp4::GroupedSide gb = nvfp4::grouped_diag_side(experts, xb.in, gdb, sms);
+  if (fail(e = nvfp4::launch_grouped_diag_plan(xb.row_offsets, experts, xb.total_tokens, gb, s)))
     return cuda_status(e);
   const int64_t nm = static_cast<int64_t>(md.size());
   if (nm > 0) {
@@ -656,25 +732,25 @@ int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
                                                     status, partial, s)))
       return cuda_status(e);
   }
-  // 2. the first batch's sweep, its CTAs' fifth warp streaming the second
-  //    input's partials (the grouped kernel's tasks: slice x vector)
+  // 2. a's sweep, its CTAs' fifth warp streaming b's input's partials (the
+  //    grouped kernel's tasks: slice x vector)
   nvfp4::SideWork side{};
   side.n = 0;
   side.tasks = 0;
-  if (x2.total_tokens > 0) {
+  if (xb.total_tokens > 0) {
     nvfp4::SideJob& j = side.job[side.n++];
-    j.A = static_cast<const uint16_t*>(x2.X);
-    j.rows = x2.total_tokens;
-    j.ld = x2.ldx;
-    j.cols = x2.in;
-    j.P = g2.P;
-    j.off = x2.row_offsets;
-    j.cstart = g2.cstart;
+    j.A = static_cast<const uint16_t*>(xb.X);
+    j.rows = xb.total_tokens;
+    j.ld = xb.ldx;
+    j.cols = xb.in;
+    j.P = gb.P;
+    j.off = xb.row_offsets;
+    j.cstart = gb.cstart;
     j.E = experts;
-    j.block = g2.block;
+    j.block = gb.block;
     j.kind = 2;
     j.t0 = 0;
-    j.t1 = g2.cap * (x2.in / 8);
+    j.t1 = gb.cap * (xb.in / 8);
     side.tasks = j.t1;
   }
   auto record = [&](int k) -> cudaError_t {
@@ -696,22 +772,22 @@ int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
     return carry ? nvfp4::launch_scale_sweep_batched_side(dd, n, total, weighted, lo, hi, side, s)
                  : nvfp4::launch_scale_sweep_batched(dd, n, total, weighted, lo, hi, s);
   };
-  const bool carry = n_first > 0 && side.tasks > 0;
-  if (fail(e = record(0)) || fail(e = sweep_batch(first, n_first, w1, L.sw1, carry)) ||
-      fail(e = record(1)))
+  const bool carry = na > 0 && side.tasks > 0;
+  if (fail(e = record(eva)) || fail(e = sweep_batch(da, na, wa, swa, carry)) ||
+      fail(e = record(eva + 1)))
     return cuda_status(e);
-  if (!carry && x2.total_tokens > 0) {
+  if (!carry && xb.total_tokens > 0) {
     // nothing to carry it: the grouped partial pass on its own
-    if (fail(e = nvfp4::launch_diag_hessian_grouped(static_cast<const uint16_t*>(x2.X),
-                                                    x2.row_offsets, experts, x2.total_tokens,
-                                                    x2.in, x2.ldx, x2.h, 0, ws + L.gd2, sms, s)))
+    if (fail(e = nvfp4::launch_diag_hessian_grouped(static_cast<const uint16_t*>(xb.X),
+                                                    xb.row_offsets, experts, xb.total_tokens,
+                                                    xb.in, xb.ldx, xb.h, 0, gdb, sms, s)))
       return cuda_status(e);
-  } else if (fail(e = nvfp4::launch_grouped_diag_finalize(experts, x2.in, x2.h, 0, g2, s))) {
+  } else if (fail(e = nvfp4::launch_grouped_diag_finalize(experts, xb.in, xb.h, 0, gb, s))) {
     return cuda_status(e);
   }
-  // 3. the second batch's sweep
-  if (fail(e = record(2)) || fail(e = sweep_batch(second, n_second, w2, L.sw2, false)) ||
-      fail(e = record(3)))
+  // 3. b's sweep
+  if (fail(e = record(evb)) || fail(e = sweep_batch(db, nb, wb, swb, false)) ||
+      fail(e = record(evb + 1)))
     return cuda_status(e);
   return NVFP4_OK;
 }

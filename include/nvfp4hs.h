@@ -316,16 +316,21 @@ int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
  * batch reading one expert-contiguous calibration input (for example every
  * expert's gate and up projections reading the routed tokens' hidden states,
  * then every expert's down projection reading their activations).
- *   first_input.h  = the grouped diagonal Hessian of first_input, as
- *                    nvfp4_diag_hessian_grouped writes it (not accumulated);
+ *   first_input.h, second_input.h  = the grouped diagonal Hessian of each
+ *                    input, as nvfp4_diag_hessian_grouped writes it (not
+ *                    accumulated);
  *   S[0 .. n_first + n_second)  = the global scale of every matrix, first
  *                    batch then second, as nvfp4_global_scale_batched writes
  *                    it (amax and status too, both nullable);
- *   the first batch's sweeps, then second_input.h, then the second batch's
- *   sweeps, as nvfp4_scale_sweep_quantize_batched writes them.
- * The bytes written equal those of the grouped and batched calls.  The
- * second input's diagonal Hessian is streamed by a fifth warp in every CTA of
- * the first batch's sweep, which is bound by FP32 arithmetic.
+ *   both batches' sweeps, as nvfp4_scale_sweep_quantize_batched writes them.
+ * The bytes written equal those of the grouped and batched calls.  One batch
+ * is swept first, its input's h computed on its own beforehand; the other
+ * input's diagonal Hessian is streamed by a fifth warp in every CTA of that
+ * sweep, which is bound by FP32 arithmetic, and the other batch is swept last.
+ * The call picks the order with the lower estimated time (HBM bytes of the
+ * reduction run on its own against the sweeps' FP32 work; see
+ * nvfp4_quantize_grouped_layer_order).  `second` goes first only if none of
+ * its h point into first_input.h.  Either order writes the same bytes.
  *
  *   first, second  sweep descriptors as for nvfp4_scale_sweep_quantize_batched
  *              (out, in > 0); descriptor i of `first` has S == S + i, of
@@ -339,10 +344,16 @@ int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
  *   workspace  device, 256-byte aligned, at least
  *              nvfp4_quantize_grouped_layer_workspace_size(...) bytes (device
  *              dependent; 0 for invalid arguments or no device).
- *   sweep_events  NULL or 4 cudaEvent_t (as void*): recorded on `stream`
- *              right before and after the first batch's sweep launch (with
- *              what it streams) and the second's, for timing.
+ *   sweep_events  NULL or 4 cudaEvent_t (as void*): [0], [1] recorded on
+ *              `stream` right before and after the sweep launch of `first`,
+ *              [2], [3] around that of `second` (the one swept first includes
+ *              what it streams), for timing.
  * Asynchronous on `stream`; descriptors are read on the host during the call.
+ *
+ * nvfp4_quantize_grouped_layer_order returns which batch that call, with the
+ * same arguments, sweeps first: 0 for `first`, 1 for `second`, or a negative
+ * status.  It reads only the descriptors' sizes and h pointers on the host
+ * (no CUDA call).
  * ------------------------------------------------------------------------ */
 typedef struct {
   const void* X;
@@ -356,6 +367,11 @@ size_t nvfp4_quantize_grouped_layer_workspace_size(const nvfp4_sweep_desc* first
                                                    const nvfp4_grouped_input* first_input,
                                                    const nvfp4_grouped_input* second_input,
                                                    int64_t experts, float* S);
+int nvfp4_quantize_grouped_layer_order(const nvfp4_sweep_desc* first, int64_t n_first,
+                                       const nvfp4_sweep_desc* second, int64_t n_second,
+                                       const nvfp4_grouped_input* first_input,
+                                       const nvfp4_grouped_input* second_input, int64_t experts,
+                                       float* S, int lo, int hi);
 int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
                                  const nvfp4_sweep_desc* second, int64_t n_second,
                                  const nvfp4_grouped_input* first_input,

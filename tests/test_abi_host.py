@@ -245,3 +245,45 @@ def test_quantize_layer_validation(L):
         xa = (nv.LayerInput * 1)(X())
         assert L.nvfp4_quantize_layer_workspace_size(wa, 1, xa, 1) == 0
         assert call([W()], [X()]) == -6
+
+
+def test_grouped_layer_order(L):
+    """The grouped layer call sweeps first the batch whose order costs less:
+    with the 128-expert layer's sizes, the down projections (whose input is
+    the smaller) go first and the gate/up input's h is streamed beside their
+    sweep; passed the other way round, the caller's order stands.  A batch
+    whose h point into the other input's h never goes first.  Host only."""
+    import block_scale_search_b200 as nv
+    E, T = 128, 2_097_152
+    h1, h2 = 0x100000, 0x200000          # the two inputs' h [E, in]
+    S = 0x300000
+    x_gu = nv.GroupedInput(P, P, T, 2048, 2048, h1)
+    x_dn = nv.GroupedInput(P, P, T, 768, 768, h2)
+
+    def descs(shape, n, hbase, in_, s0):
+        return [nv.SweepDesc(P, shape[0], shape[1], shape[1], hbase + 4 * in_ * (i % E),
+                             S + 4 * (s0 + i), P, P, None) for i in range(n)]
+
+    gu = descs((768, 2048), 2 * E, h1, 2048, 0)
+    dn = descs((2048, 768), E, h2, 768, 2 * E)
+    assert nv.nvfp4_quantize_grouped_layer_order(gu, dn, x_gu, x_dn, E, S, -9, 6) == 1
+    # the other way round: the down batch is already first
+    dn0 = descs((2048, 768), E, h2, 768, 0)
+    gu1 = descs((768, 2048), 2 * E, h1, 2048, E)
+    assert nv.nvfp4_quantize_grouped_layer_order(dn0, gu1, x_dn, x_gu, E, S, -9, 6) == 0
+    # the second batch reading the first input's h cannot go first
+    dn_bad = descs((2048, 768), E, h1, 2048, 2 * E)
+    assert nv.nvfp4_quantize_grouped_layer_order(gu, dn_bad, x_gu, x_dn, E, S, -9, 6) == 0
+    # a small first input and a large sweep keep the caller's order even when
+    # the second input is larger: its reduction is carried at a fraction of its cost
+    x_small = nv.GroupedInput(P, P, 4096, 2048, 2048, h1)
+    x_big = nv.GroupedInput(P, P, 65536, 768, 768, h2)
+    assert nv.nvfp4_quantize_grouped_layer_order(gu, dn, x_small, x_big, E, S, -9, 6) == 0
+    # an empty first batch cannot carry anything: the second goes first
+    assert nv.nvfp4_quantize_grouped_layer_order([], descs((2048, 768), E, h2, 768, 0), x_gu, x_dn,
+                                                 E, S, -9, 6) == 1
+    # invalid arguments: the validation's status
+    with pytest.raises(nv.NVFP4Error):
+        nv.nvfp4_quantize_grouped_layer_order(gu, dn, x_gu, x_dn, E, S, -10, 6)
+    with pytest.raises(nv.NVFP4Error):
+        nv.nvfp4_quantize_grouped_layer_order(gu, dn, x_gu, x_dn, E, S + 4, -9, 6)

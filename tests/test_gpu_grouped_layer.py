@@ -1,7 +1,9 @@
 """nvfp4_quantize_grouped_layer writes exactly what the grouped and batched
 calls write: both inputs' per-expert h, every matrix's S, amax and status,
-and both batches' codes, scales and offsets -- with the second input's
-diagonal Hessian streamed beside the first batch's sweep.  Needs a B200."""
+and both batches' codes, scales and offsets -- with one input's diagonal
+Hessian streamed beside the other batch's sweep, in whichever order the call
+picks (each case runs with the batches passed both ways round).  Needs a
+B200."""
 import numpy as np
 import pytest
 import torch
@@ -18,6 +20,9 @@ def nv():
 
 
 def _run_both(nv, W1, W2, X1, X2, offs, lo=-9, hi=6, q_max=448.0, weighted=True):
+    """Compare the grouped layer call, with the batches passed in the given
+    order, against the grouped and batched calls; returns which batch the
+    call swept first (0: W1's, 1: W2's)."""
     E = len(offs) - 1
     off_d = torch.as_tensor(offs, dtype=torch.int64, device=DEV)
     # reference: the grouped and batched calls
@@ -57,6 +62,7 @@ def _run_both(nv, W1, W2, X1, X2, offs, lo=-9, hi=6, q_max=448.0, weighted=True)
     nb = nv.nvfp4_quantize_grouped_layer_workspace_size(d1, d2, x1, x2, E, gS)
     assert nb > 0
     ws = torch.empty(nb, dtype=torch.uint8, device=DEV)
+    order = nv.nvfp4_quantize_grouped_layer_order(d1, d2, x1, x2, E, gS, lo, hi)
     nv.nvfp4_quantize_grouped_layer(d1, d2, x1, x2, E, q_max, lo, hi, gS, gA, gst, ws, nb)
     torch.cuda.synchronize()
     assert torch.equal(g1.view(torch.int32), h1.view(torch.int32))
@@ -66,6 +72,13 @@ def _run_both(nv, W1, W2, X1, X2, offs, lo=-9, hi=6, q_max=448.0, weighted=True)
     for got, want in zip(outs, list(ref1) + list(ref2)):
         for a, b in zip(got, want):
             assert torch.equal(a, b)
+    return order
+
+
+def _run_both_orders(nv, W1, W2, X1, X2, offs, **kw):
+    """The call with the batches passed either way round; returns the two
+    orders it chose."""
+    return (_run_both(nv, W1, W2, X1, X2, offs, **kw), _run_both(nv, W2, W1, X2, X1, offs, **kw))
 
 
 def _moe(E, counts, gu_out, gu_in, seed):
@@ -82,13 +95,14 @@ def _moe(E, counts, gu_out, gu_in, seed):
 def test_small_moe_layer(nv):
     E = 6
     W1, W2, X1, X2, offs = _moe(E, [700, 0, 3000, 17, 1200, 5000], 768, 2048, 901)
-    _run_both(nv, W1, W2, X1, X2, offs)
+    # the down batch (the smaller input) goes first whichever way it is passed
+    assert _run_both_orders(nv, W1, W2, X1, X2, offs) == (1, 0)
 
 
 def test_small_moe_layer_mse_window(nv):
     E = 4
     W1, W2, X1, X2, offs = _moe(E, [900, 2100, 0, 40], 768, 2048, 931)
-    _run_both(nv, W1, W2, X1, X2, offs, lo=-3, hi=7, q_max=256.0, weighted=False)
+    _run_both_orders(nv, W1, W2, X1, X2, offs, lo=-3, hi=7, q_max=256.0, weighted=False)
 
 
 def test_moe_layer_at_the_benchmarked_size(nv):
@@ -102,7 +116,7 @@ def test_moe_layer_at_the_benchmarked_size(nv):
     E = wl.experts
     W1 = [Ws[f"e{e}.gate"] for e in range(E)] + [Ws[f"e{e}.up"] for e in range(E)]
     W2 = [Ws[f"e{e}.down"] for e in range(E)]
-    _run_both(nv, W1, W2, X1, X2, wl.calibs["gu"].row_offsets)
+    assert _run_both_orders(nv, W1, W2, X1, X2, wl.calibs["gu"].row_offsets) == (1, 0)
 
 
 @pytest.mark.parametrize("seed", [5, 6, 7])
@@ -118,5 +132,5 @@ def test_random_moe_layers(nv, seed):
     W1, W2, X1, X2, offs = _moe(E, counts, gu_out, gu_in, 1000 + 37 * seed)
     lo = int(rng.integers(-10, 1))
     hi = int(rng.integers(0, 16 + lo))
-    _run_both(nv, W1, W2, X1, X2, offs, lo=lo, hi=hi, q_max=float(rng.choice([256.0, 448.0])),
-              weighted=bool(rng.random() > 0.3))
+    _run_both_orders(nv, W1, W2, X1, X2, offs, lo=lo, hi=hi,
+                     q_max=float(rng.choice([256.0, 448.0])), weighted=bool(rng.random() > 0.3))
