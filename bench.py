@@ -175,12 +175,14 @@ def build_layer(rank: int, device, name: str = "llama33_70b_mlp"):
               workloads.moe_grouped(tokens=32768, experts=16, device=device))
         Ws = {m.name: m.make(device) for m in wl.matrices}
         Xs = {k: c.make(device) for k, c in wl.calibs.items()}
-        torch.cuda.synchronize()
+        if torch.device(device).type == "cuda":
+            torch.cuda.synchronize()
         return wl, Ws, Xs
     wl = rank_workload(rank, name)
     Ws = {m.name: m.make(device) for m in wl.matrices}
     Xs = {k: c.make(device) for k, c in wl.calibs.items()}
-    torch.cuda.synchronize()
+    if torch.device(device).type == "cuda":   # the oracle arm also runs on a host without a GPU
+        torch.cuda.synchronize()
     return wl, Ws, Xs
 
 
