@@ -220,14 +220,17 @@ class Step:
         self.layer_x = [nv.LayerInput(Xs[k].data_ptr(), Xs[k].shape[0], Xs[k].shape[1],
                                       Xs[k].stride(0), self.h[k].data_ptr()) for k in keys]
         self.layer_arrays = nv._layer_arrays(self.layer_w, self.layer_x)
-        # what the layer call's sweeps carry here: every reduction but the
-        # first weight's S and its input's h, in the sweeps before the last
-        first = wl.matrices[0]
+        # the order the call sweeps the weights in, and what its sweeps carry:
+        # every reduction but the first swept weight's S and its input's h, in
+        # the sweeps before the last
+        self.sweep_order = nv.nvfp4_quantize_layer_order(self.layer_w, self.layer_x, LO, HI)
+        swept = [wl.matrices[j] for j in self.sweep_order]
+        first = swept[0]
         fx = wl.calibs[first.x_key]
         self.side_bytes = (wl.calib_bytes - 2 * fx.tokens * fx.inp
                            + 2 * (wl.weight_elems - first.out * first.inp))
         self.carry_launches = len(wl.matrices) - 1
-        self.carry_elems = sum(m.out * m.inp for m in wl.matrices[:-1])
+        self.carry_elems = sum(m.out * m.inp for m in swept[:-1])
         self.traffic_key = "scale_sweep_layer"
         self.layer_note = ("the first weight's S and its input's h run first on their own (rest); "
                            "the other weights' S and the other inputs' h are streamed by a fifth "
@@ -279,7 +282,7 @@ class Step:
             if ev is not None:
                 b.record(main)
                 ev.setdefault("layer_call", []).append((a, b))
-                for j in range(len(self.mats)):
+                for j in self.sweep_order:   # carrying sweeps first
                     ev.setdefault("scale_sweep", []).append((sev[2 * j], sev[2 * j + 1]))
             if io is not None:
                 e = torch.cuda.Event()

@@ -25,7 +25,8 @@ __all__ = [
     "nvfp4_global_scale_batched", "nvfp4_scale_sweep_quantize_batched_workspace_size",
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
-    "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "quantize_layer_many",
+    "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "nvfp4_quantize_layer_order",
+    "quantize_layer_many",
     "LayerWeight", "LayerInput", "GroupedInput", "nvfp4_quantize_grouped_layer_workspace_size",
     "nvfp4_quantize_grouped_layer", "nvfp4_quantize_grouped_layer_order",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
@@ -108,6 +109,8 @@ _SIGS = {
                                      _int),
     "nvfp4_quantize_layer_workspace_size": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput),
                                              _int], _sz),
+    "nvfp4_quantize_layer_order": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput), _int, _int,
+                                    _int, C.POINTER(_int)], _int),
     "nvfp4_quantize_layer": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput), _int, _f32, _int,
                               _int, _vp, _sz, C.POINTER(_vp), _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
@@ -219,6 +222,16 @@ def nvfp4_quantize_layer_workspace_size(weights, inputs) -> int:
     """weights: list of LayerWeight, inputs: list of LayerInput."""
     wa, xa = _layer_arrays(weights, inputs)
     return lib().nvfp4_quantize_layer_workspace_size(wa, len(weights), xa, len(inputs))
+
+
+def nvfp4_quantize_layer_order(weights, inputs, lo, hi) -> list[int]:
+    """The order nvfp4_quantize_layer sweeps these weights in: element j is the
+    index of the weight swept j-th (needs the device for its SM count)."""
+    wa, xa = _layer_arrays(weights, inputs)
+    order = (_int * max(1, len(weights)))()
+    _check("nvfp4_quantize_layer_order", lib().nvfp4_quantize_layer_order(
+        wa, len(weights), xa, len(inputs), int(lo), int(hi), order))
+    return [int(order[j]) for j in range(len(weights))]
 
 
 def nvfp4_quantize_layer(weights, inputs, q_max, lo, hi, workspace, workspace_bytes,

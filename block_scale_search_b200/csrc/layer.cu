@@ -8,7 +8,10 @@
 // bit: the side reductions (side_reduce.cuh) write the standalone kernels'
 // partials in their order, and the standalone finalize kernels run on them.
 //
-// Schedule, on one stream, for weights w_0 .. w_{n-1} in the caller's order:
+// The weights are swept in the order with the lowest estimated time (every
+// permutation for up to six weights, plan_cost below; ties keep the caller's
+// order); every order writes the same bytes.  Schedule, on one stream, for
+// the weights w_0 .. w_{n-1} in that order:
 //   * a reduction's deadline is the first sweep that needs it: S of w_j is
 //     needed by sweep j, h of an input by the first sweep of a weight using it
 //     (inputs no weight uses: after the last sweep);
@@ -153,15 +156,71 @@ Plan make_plan(const LayerWeight* w, int nw, const LayerInput* x, int nx, int sm
   return P;
 }
 
+// A plan's time as HBM-byte equivalents: a reduction run on its own costs its
+// bytes; a sweep of E weight elements and K candidates costs 1.3 E K (about
+// 2.1e-13 s per element and candidate on B200, as long as 1.3 bytes take at
+// the copy bandwidth), and carrying C bytes beside it max(that + 0.38 C, C)
+// (a carrying sweep slows by about 38% of the carried reductions' own time).
+double plan_cost(const Plan& P, const LayerWeight* w, int nw, int K) {
+  constexpr double kSweepBytes = 1.3, kCarry = 0.38;
+  double cost = 0.0;
+  for (const Reduction& r : P.red)
+    if (r.standalone) cost += r.bytes;
+  for (int j = 0; j < nw; ++j) {
+    double carried = 0.0;
+    for (const Share& s : P.shares[j]) {
+      const Reduction& r = P.red[s.red];
+      if (!r.standalone && r.tasks > 0)
+        carried += r.bytes * static_cast<double>(s.t1 - s.t0) / static_cast<double>(r.tasks);
+    }
+    const double sweep =
+        static_cast<double>(w[j].out) * static_cast<double>(w[j].in) * K * kSweepBytes;
+    cost += std::max(sweep + kCarry * carried, carried);
+  }
+  return cost;
+}
+
 }  // namespace
 
 size_t layer_workspace_bytes(const LayerWeight* w, int nw, const LayerInput* x, int nx, int sms) {
+  // the same for every order of the weights: each reduction's workspace is
+  // sized and aligned on its own
   return make_plan(w, nw, x, nx, sms).bytes;
 }
 
-cudaError_t quantize_layer(const LayerWeight* w, int nw, const LayerInput* x, int nx, float q_max,
-                           int lo, int hi, void* workspace, int sms, const cudaEvent_t* events,
-                           cudaStream_t stream) {
+std::vector<int> layer_sweep_order(const LayerWeight* w, int nw, const LayerInput* x, int nx,
+                                   int sms, int lo, int hi) {
+  std::vector<int> perm(static_cast<size_t>(std::max(nw, 0)));
+  for (int j = 0; j < nw; ++j) perm[j] = j;
+  std::vector<int> best = perm;
+  if (nw < 2 || nw > kMaxOrderedWeights) return best;
+  const int K = hi - lo + 1;
+  std::vector<LayerWeight> wp(static_cast<size_t>(nw));
+  double best_cost = 0.0;
+  bool first = true;
+  // the caller's order is the first permutation; another must be cheaper by
+  // more than rounding to replace it
+  do {
+    for (int j = 0; j < nw; ++j) wp[j] = w[perm[j]];
+    const double c = plan_cost(make_plan(wp.data(), nw, x, nx, sms), wp.data(), nw, K);
+    if (first || c < best_cost * (1.0 - 1e-9)) {
+      best_cost = c;
+      best = perm;
+      first = false;
+    }
+  } while (std::next_permutation(perm.begin(), perm.end()));
+  return best;
+}
+
+cudaError_t quantize_layer(const LayerWeight* w_caller, int nw, const LayerInput* x, int nx,
+                           float q_max, int lo, int hi, void* workspace, int sms,
+                           const cudaEvent_t* events, cudaStream_t stream) {
+  // the weights in the order they are swept; events stay indexed by the
+  // caller's order
+  const std::vector<int> perm = layer_sweep_order(w_caller, nw, x, nx, sms, lo, hi);
+  std::vector<LayerWeight> wv(static_cast<size_t>(nw));
+  for (int j = 0; j < nw; ++j) wv[j] = w_caller[perm[j]];
+  const LayerWeight* w = wv.data();
   Plan P = make_plan(w, nw, x, nx, sms);
   char* ws = static_cast<char*>(workspace);
   uint32_t* words = reinterpret_cast<uint32_t*>(ws + P.amax_off);
@@ -198,7 +257,7 @@ cudaError_t quantize_layer(const LayerWeight* w, int nw, const LayerInput* x, in
     const LayerWeight& m = w[j];
     const float* h = m.input >= 0 ? x[m.input].h : nullptr;
     bool carried = false;
-    if (events != nullptr && !ok(cudaEventRecord(events[2 * j], stream))) return e;
+    if (events != nullptr && !ok(cudaEventRecord(events[2 * perm[j]], stream))) return e;
     if (!P.shares[j].empty()) {
       SideWork sw{};
       sw.n = 0;
@@ -239,7 +298,7 @@ cudaError_t quantize_layer(const LayerWeight* w, int nw, const LayerInput* x, in
                                  m.offs, sp, stream)))
         return e;
     }
-    if (events != nullptr && !ok(cudaEventRecord(events[2 * j + 1], stream))) return e;
+    if (events != nullptr && !ok(cudaEventRecord(events[2 * perm[j] + 1], stream))) return e;
     if (!carried) {
       // this sweep's shares: their reductions run whole, now
       for (const Share& s : P.shares[j])

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <vector>
 #include <cuda_runtime.h>
 
 #include "nvfp4_device.cuh"
@@ -133,6 +134,12 @@ struct LayerInput {
   float* h;
 };
 size_t layer_workspace_bytes(const LayerWeight* w, int nw, const LayerInput* x, int nx, int sms);
+// The order quantize_layer sweeps the weights in (indices into w): the
+// permutation with the lowest estimated time, for up to kMaxOrderedWeights
+// weights; the caller's order otherwise and on ties.
+constexpr int kMaxOrderedWeights = 6;
+std::vector<int> layer_sweep_order(const LayerWeight* w, int nw, const LayerInput* x, int nx,
+                                   int sms, int lo, int hi);
 cudaError_t quantize_layer(const LayerWeight* w, int nw, const LayerInput* x, int nx, float q_max,
                            int lo, int hi, void* workspace, int sms, const cudaEvent_t* events,
                            cudaStream_t stream);

@@ -199,6 +199,23 @@ size_t nvfp4_quantize_layer_workspace_size(const nvfp4_layer_weight* weights, in
   return nvfp4::layer_workspace_bytes(wv.data(), n_weights, xv.data(), n_inputs, sms);
 }
 
+int nvfp4_quantize_layer_order(const nvfp4_layer_weight* weights, int n_weights,
+                               const nvfp4_layer_input* inputs, int n_inputs, int lo, int hi,
+                               int* order) {
+  std::vector<nvfp4::LayerWeight> wv;
+  std::vector<nvfp4::LayerInput> xv;
+  const int st = check_layer(weights, n_weights, inputs, n_inputs, &wv, &xv);
+  if (st != NVFP4_OK) return st;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  if (order == nullptr && n_weights > 0) return NVFP4_ERR_INVALID_ARG;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  const std::vector<int> perm =
+      nvfp4::layer_sweep_order(wv.data(), n_weights, xv.data(), n_inputs, sms, lo, hi);
+  for (int j = 0; j < n_weights; ++j) order[j] = perm[j];
+  return NVFP4_OK;
+}
+
 int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
                          const nvfp4_layer_input* inputs, int n_inputs, float q_max, int lo,
                          int hi, void* workspace, size_t workspace_bytes,

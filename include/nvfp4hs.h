@@ -256,14 +256,19 @@ int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n,
  * sweep of nvfp4_scale_sweep_quantize with the h of its input (input = -1:
  * plain MSE).  The bytes written equal those of the per-step calls.
  *
- * The library orders the work itself: weight 0's S and its input's h first;
- * the other reductions, which are bound by HBM bandwidth, are streamed by an
- * extra warp in each CTA of earlier sweeps, which are bound by FP32
- * arithmetic (H-Scale summary, sec. 4 "Efficiency and Hardware Deployment":
- * the added cost is the offline search and one activation pass).  Weights are swept in the order
- * given; a reduction that no earlier sweep can carry (the sweep's row length
- * is not a multiple of 512 elements, or it is short) runs on its own before
- * it is needed.
+ * The library orders the work itself: the first weight swept has its S and
+ * its input's h computed first; the other reductions, which are bound by HBM
+ * bandwidth, are streamed by an extra warp in each CTA of earlier sweeps,
+ * which are bound by FP32 arithmetic (H-Scale summary, sec. 4 "Efficiency
+ * and Hardware Deployment": the added cost is the offline search and one
+ * activation pass).  A reduction that no earlier sweep can carry (the
+ * sweep's row length is not a multiple of 512 elements, or it is short) runs
+ * on its own before it is needed.  For up to six weights the sweep order is
+ * the permutation with the lowest estimated time (HBM bytes of the
+ * reductions run on their own against the sweeps' FP32 work); ties, and more
+ * weights, keep the order given.  Every order writes the same bytes.
+ * nvfp4_quantize_layer_order writes the order chosen: order[j] = the index of
+ * the weight swept j-th (it needs the device, for its SM count; no launch).
  *
  *   weights    n_weights descriptors: W bf16 [out, ldw] (16-byte aligned,
  *              ldw % 8 == 0, in % 16 == 0, out and in > 0); input in
@@ -306,6 +311,9 @@ typedef struct {
 
 size_t nvfp4_quantize_layer_workspace_size(const nvfp4_layer_weight* weights, int n_weights,
                                            const nvfp4_layer_input* inputs, int n_inputs);
+int nvfp4_quantize_layer_order(const nvfp4_layer_weight* weights, int n_weights,
+                               const nvfp4_layer_input* inputs, int n_inputs, int lo, int hi,
+                               int* order);
 int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
                          const nvfp4_layer_input* inputs, int n_inputs, float q_max, int lo,
                          int hi, void* workspace, size_t workspace_bytes,

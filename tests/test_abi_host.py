@@ -238,6 +238,14 @@ def test_quantize_layer_validation(L):
     assert call([W()], [X()], q=float("nan")) == -1
     assert call([W()], [X()], lo=-10, hi=6) == -4          # window over 16
     assert L.nvfp4_quantize_layer(None, 1, None, 0, 448.0, -9, 6, ws, 1 << 30, None, None) == -1
+    # the order query validates as the call does
+    order = (C.c_int * 1)()
+    wa1 = (nv.LayerWeight * 1)(W())
+    xa1 = (nv.LayerInput * 1)(X())
+    assert L.nvfp4_quantize_layer_order(wa1, 1, xa1, 1, -10, 6, order) == -4
+    assert L.nvfp4_quantize_layer_order(wa1, 1, xa1, 1, -9, 6, None) == -1
+    wbad = (nv.LayerWeight * 1)(W(input=1))
+    assert L.nvfp4_quantize_layer_order(wbad, 1, xa1, 1, -9, 6, order) == -1
     # no device here: the workspace query returns 0 and a valid call a CUDA error
     import torch
     if not torch.cuda.is_available():
@@ -245,6 +253,7 @@ def test_quantize_layer_validation(L):
         xa = (nv.LayerInput * 1)(X())
         assert L.nvfp4_quantize_layer_workspace_size(wa, 1, xa, 1) == 0
         assert call([W()], [X()]) == -6
+        assert L.nvfp4_quantize_layer_order(wa, 1, xa, 1, -9, 6, order) == -6
 
 
 def test_grouped_layer_order(L):

@@ -169,3 +169,31 @@ def test_random_layers(nv, seed):
     lo = int(rng.integers(-12, 1))
     hi = int(rng.integers(0, 16 + lo))
     _check_same(nv, Ws, Xs, inputs, q_max=float(rng.choice([256.0, 448.0])), lo=lo, hi=hi)
+
+
+def _order(nv, Ws, Xs, inputs, lo=-9, hi=6):
+    """The sweep order the layer call picks for these shapes (descriptors
+    with placeholder outputs; nothing is launched)."""
+    wd = [nv.LayerWeight(W.data_ptr(), *W.shape, W.stride(0), k, W.data_ptr(), None, None,
+                         W.data_ptr(), W.data_ptr(), None) for W, k in zip(Ws, inputs)]
+    xd = [nv.LayerInput(X.data_ptr(), *X.shape, X.stride(0), X.data_ptr()) for X in Xs]
+    return nv.nvfp4_quantize_layer_order(wd, xd, lo, hi)
+
+
+def test_sweep_order_is_chosen_and_writes_the_same_bytes(nv):
+    """The call sweeps the weights in the order with the lowest estimated time.
+    Given gate, up, down, it keeps that order. Given down first, it sweeps a
+    projection reading the smaller gate/up input first, and writes the per-step
+    calls' bytes all the same."""
+    Ws, Xs, inputs = _mlp(3072, 2048, 2048, 4096, 31)
+    assert _order(nv, Ws, Xs, inputs) == [0, 1, 2]
+    given = [2, 0, 1]                      # down, gate, up
+    Ws2 = [Ws[i] for i in given]
+    in2 = [inputs[i] for i in given]
+    o2 = _order(nv, Ws2, Xs, in2)
+    assert sorted(o2) == [0, 1, 2] and o2[0] in (1, 2)
+    _check_same(nv, Ws2, Xs, in2)
+    # and at the benchmarked size, in the bench's order
+    Wb, Xb, ib = _mlp(28672, 8192, 8192, 65536, 4)
+    assert _order(nv, Wb, Xb, ib) == [0, 1, 2]
+    assert _order(nv, [Wb[2], Wb[0], Wb[1]], Xb, [1, 0, 0])[0] in (1, 2)
