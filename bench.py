@@ -369,12 +369,14 @@ class Step:
 
 
 class GroupedStep:
-    """Mixture-of-experts layer: one grouped diag-Hessian launch per
-    calibration tensor, one batched global scale for all matrices, and the
-    batched sweep -- one launch for all matrices (serial), or one per
-    calibration input with the later inputs' h on a second stream beside the
-    first batch (overlapped, the default).  Descriptor tables are built once;
-    run() calls the C ABI."""
+    """Mixture-of-experts layer.  Default (layer): one
+    nvfp4_quantize_grouped_layer call, which sweeps first the batch whose
+    order costs less and streams the other input's grouped h beside that
+    sweep.  Otherwise one grouped diag-Hessian launch per calibration tensor,
+    one batched global scale for all matrices, and the batched sweep: one
+    launch for all matrices (serial), or one per calibration input with the
+    later inputs' h on a second stream beside the first batch (overlapped).
+    Descriptor tables are built once; run() calls the C ABI."""
 
     def __init__(self, nv, wl, Ws, Xs, device, serial=False, layer=False):
         import ctypes as C
