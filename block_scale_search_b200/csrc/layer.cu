@@ -8,9 +8,10 @@
 // bit: the side reductions (side_reduce.cuh) write the standalone kernels'
 // partials in their order, and the standalone finalize kernels run on them.
 //
-// The weights are swept in the order with the lowest estimated time (every
-// permutation for up to six weights, plan_cost below; ties keep the caller's
-// order); every order writes the same bytes.  Schedule, on one stream, for
+// The weights are swept in the order with the lowest estimated time
+// (plan_cost below: every permutation for up to four weights, otherwise each
+// weight first with the others in the caller's order; ties keep the
+// caller's order); every order writes the same bytes.  Schedule, on one stream, for
 // the weights w_0 .. w_{n-1} in that order:
 //   * a reduction's deadline is the first sweep that needs it: S of w_j is
 //     needed by sweep j, h of an input by the first sweep of a weight using it
@@ -193,22 +194,35 @@ std::vector<int> layer_sweep_order(const LayerWeight* w, int nw, const LayerInpu
   std::vector<int> perm(static_cast<size_t>(std::max(nw, 0)));
   for (int j = 0; j < nw; ++j) perm[j] = j;
   std::vector<int> best = perm;
-  if (nw < 2 || nw > kMaxOrderedWeights) return best;
+  if (nw < 2) return best;
   const int K = hi - lo + 1;
   std::vector<LayerWeight> wp(static_cast<size_t>(nw));
   double best_cost = 0.0;
   bool first = true;
-  // the caller's order is the first permutation; another must be cheaper by
-  // more than rounding to replace it
-  do {
-    for (int j = 0; j < nw; ++j) wp[j] = w[perm[j]];
+  // the caller's order is tried first; another must be cheaper by more than
+  // rounding to replace it
+  auto consider = [&](const std::vector<int>& order) {
+    for (int j = 0; j < nw; ++j) wp[j] = w[order[j]];
     const double c = plan_cost(make_plan(wp.data(), nw, x, nx, sms), wp.data(), nw, K);
     if (first || c < best_cost * (1.0 - 1e-9)) {
       best_cost = c;
-      best = perm;
+      best = order;
       first = false;
     }
-  } while (std::next_permutation(perm.begin(), perm.end()));
+  };
+  if (nw <= kMaxOrderedWeights) {
+    do consider(perm);
+    while (std::next_permutation(perm.begin(), perm.end()));
+  } else {
+    // the first weight fixes the standalone prologue, where orders differ
+    // most: each weight first, the others in the caller's order
+    for (int f = 0; f < nw; ++f) {
+      std::vector<int> order{f};
+      for (int j = 0; j < nw; ++j)
+        if (j != f) order.push_back(j);
+      consider(order);
+    }
+  }
   return best;
 }
 

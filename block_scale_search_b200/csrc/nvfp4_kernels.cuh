@@ -135,9 +135,10 @@ struct LayerInput {
 };
 size_t layer_workspace_bytes(const LayerWeight* w, int nw, const LayerInput* x, int nx, int sms);
 // The order quantize_layer sweeps the weights in (indices into w): the
-// permutation with the lowest estimated time, for up to kMaxOrderedWeights
-// weights; the caller's order otherwise and on ties.
-constexpr int kMaxOrderedWeights = 6;
+// permutation with the lowest estimated time for up to kMaxOrderedWeights
+// weights; for more, the best choice of the first weight with the others in
+// the caller's order.  Ties keep the caller's order.
+constexpr int kMaxOrderedWeights = 4;
 std::vector<int> layer_sweep_order(const LayerWeight* w, int nw, const LayerInput* x, int nx,
                                    int sms, int lo, int hi);
 cudaError_t quantize_layer(const LayerWeight* w, int nw, const LayerInput* x, int nx, float q_max,

@@ -263,10 +263,11 @@ int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n,
  * and Hardware Deployment": the added cost is the offline search and one
  * activation pass).  A reduction that no earlier sweep can carry (the
  * sweep's row length is not a multiple of 512 elements, or it is short) runs
- * on its own before it is needed.  For up to six weights the sweep order is
- * the permutation with the lowest estimated time (HBM bytes of the
- * reductions run on their own against the sweeps' FP32 work); ties, and more
- * weights, keep the order given.  Every order writes the same bytes.
+ * on its own before it is needed.  The sweep order is the one with the
+ * lowest estimated time (HBM bytes of the reductions run on their own
+ * against the sweeps' FP32 work): among all permutations for up to four
+ * weights; for more, each weight is tried first with the others in the order
+ * given.  Ties keep the order given.  Every order writes the same bytes.
  * nvfp4_quantize_layer_order writes the order chosen: order[j] = the index of
  * the weight swept j-th (it needs the device, for its SM count; no launch).
  *
