@@ -947,8 +947,8 @@ def main():
                     help="layer: one nvfp4_quantize_layer call per step, which streams the "
                          "HBM-bound reductions beside the FP32-bound sweeps; serial: the per-step "
                          "calls on one stream in the order h, S, sweep; overlapped: the per-step "
-                         "calls with later weights' S and h on a second stream; auto: layer for "
-                         "a dense layer, serial for the MoE layer (grouped calls)")
+                         "calls with later weights' S and h on a second stream; auto: layer "
+                         "(nvfp4_quantize_grouped_layer for the MoE layer)")
     ap.add_argument("--workload", default="llama33_70b_mlp",
                     choices=list(WORKLOADS) + ["act_llama33_70b"])
     args = ap.parse_args()
