@@ -62,6 +62,15 @@ __device__ __forceinline__ void sq_acc_bf16x2(uint32_t w, float& s0, float& s1) 
       : "+f"(s0), "+f"(s1) : "r"(w));
 }
 
+// x^2 + 0 for the two bf16 halves of w: the same single rounding as
+// sq_acc_bf16x2 on zeroed sums, without registers to zero.
+__device__ __forceinline__ void sq_first_bf16x2(uint32_t w, float& s0, float& s1) {
+  asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, l, l, 0f00000000;\n\t"
+      "fma.rn.f32.bf16 %1, h, h, 0f00000000; }"
+      : "=f"(s0), "=f"(s1) : "r"(w));
+}
+
 // The running maximum of eight sign-cleared bf16 patterns (two per 32 bits).
 __device__ __forceinline__ uint32_t absmax_bf16x8(uint32_t m, const uint4& q) {
   return __vmaxu2(__vmaxu2(m, q.x & 0x7FFF7FFFu),
@@ -79,11 +88,16 @@ __device__ __forceinline__ void side_stream(const uint16_t* col, int64_t ld, int
                                             int lane, float (&acc)[8], uint32_t& m) {
   const int64_t n = t_end > t0 ? (t_end - t0 + stride - 1) / stride : 0;
   const int64_t runs = n / kSideRows;
+  // rows are issued in order: a running pointer advanced by one row stride
+  const int64_t step = stride * ld;
+  const uint16_t* next_row = col + t0 * ld;
   auto issue = [&](int64_t k) {
     const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
 #pragma unroll
-    for (int u = 0; u < kSideRows; ++u)
-      cp_async16(&ring.v[slot + u][lane], col + (t0 + (k * kSideRows + u) * stride) * ld);
+    for (int u = 0; u < kSideRows; ++u) {
+      cp_async16(&ring.v[slot + u][lane], next_row);
+      next_row += step;
+    }
   };
 #pragma unroll
   for (int k = 0; k < kSideBatches; ++k) {
@@ -95,10 +109,15 @@ __device__ __forceinline__ void side_stream(const uint16_t* col, int64_t ld, int
     const int slot = static_cast<int>(k % kSideBatches) * kSideRows;
     if constexpr (kSq) {
       float s[8];
+      {
+        const uint4 q = ring.v[slot][lane];
+        sq_first_bf16x2(q.x, s[0], s[1]);
+        sq_first_bf16x2(q.y, s[2], s[3]);
+        sq_first_bf16x2(q.z, s[4], s[5]);
+        sq_first_bf16x2(q.w, s[6], s[7]);
+      }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) s[c] = 0.0f;
-#pragma unroll
-      for (int u = 0; u < kSideRows; ++u) {
+      for (int u = 1; u < kSideRows; ++u) {
         const uint4 q = ring.v[slot + u][lane];
         sq_acc_bf16x2(q.x, s[0], s[1]);
         sq_acc_bf16x2(q.y, s[2], s[3]);
@@ -115,8 +134,8 @@ __device__ __forceinline__ void side_stream(const uint16_t* col, int64_t ld, int
     cp_async_commit();
   }
   cp_async_wait<0>();
-  for (int64_t t = t0 + runs * kSideRows * stride; t < t_end; t += stride) {
-    const uint4 q = ld_stream_v4(col + t * ld);
+  for (int64_t t = t0 + runs * kSideRows * stride; t < t_end; t += stride, next_row += step) {
+    const uint4 q = ld_stream_v4(next_row);
     if constexpr (kSq) {
       sq_acc_bf16x2(q.x, acc[0], acc[1]);
       sq_acc_bf16x2(q.y, acc[2], acc[3]);
