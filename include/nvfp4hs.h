@@ -267,7 +267,9 @@ int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n,
  * lowest estimated time (HBM bytes of the reductions run on their own
  * against the sweeps' FP32 work): among all permutations for up to four
  * weights; for more, each weight is tried first with the others in the order
- * given.  Ties keep the order given.  Every order writes the same bytes.
+ * given.  Ties keep the order given.  Every order writes the same bytes as
+ * long as no two weights' outputs (S, amax, status, codes, scales,
+ * chosen_offset) overlap each other or any input, which the call requires.
  * nvfp4_quantize_layer_order writes the order chosen: order[j] = the index of
  * the weight swept j-th (it needs the device, for its SM count; no launch).
  *
@@ -339,7 +341,8 @@ int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
  * The call picks the order with the lower estimated time (HBM bytes of the
  * reduction run on its own against the sweeps' FP32 work; see
  * nvfp4_quantize_grouped_layer_order).  `second` goes first only if none of
- * its h point into first_input.h.  Either order writes the same bytes.
+ * its h point into first_input.h.  Either order writes the same bytes, as
+ * long as no matrix's outputs overlap another's or any input (required).
  *
  *   first, second  sweep descriptors as for nvfp4_scale_sweep_quantize_batched
  *              (out, in > 0); descriptor i of `first` has S == S + i, of
