@@ -36,6 +36,7 @@ SWEEP_BYTES_PER_ELEM = 2 + 0.5 + 1 / 16   # read bf16 W; write 4-bit code + 1/16
 # h*e and the accumulation (h e) e -- five FP32 lane operations.
 SWEEP_OPS_PER_ELEM_CAND = 5
 SMS, LANES_PER_SM = 148, 128
+ISSUE_PER_SM = 4          # warp instructions per SM per cycle (4 schedulers)
 # Online activation quantization (W+A settings): plain MSE, so no weighting
 # multiply -- four FP32 lane operations per element and candidate.
 ACT_LO, ACT_HI, ACT_Q = -3, 7, 256.0
@@ -556,10 +557,10 @@ class GroupedStep:
             sw(*self.part[k], stream)
 
 
-def profiled_traffic(kernel: str, units_per_launch: float):
-    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json),
-    scaled by the units one launch processes; None when the kernel's source has
-    changed since the capture."""
+def _profiled_record(kernel: str):
+    """The committed ncu record of a kernel (profiles/traffic.json), or None when
+    any file the kernel is compiled from has changed since the capture: sha1
+    over the listed sources' bytes, concatenated in order."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
@@ -568,8 +569,6 @@ def profiled_traffic(kernel: str, units_per_launch: float):
         d = json.load(f).get(kernel)
     if not d:
         return None
-    # the capture is void once any file the kernel is compiled from has changed:
-    # sha1 over the listed sources' bytes, concatenated in order
     srcs = [os.path.join(ROOT, x) for x in d.get("sources", [d.get("source", "")])]
     if not all(os.path.exists(x) for x in srcs):
         return None
@@ -577,9 +576,23 @@ def profiled_traffic(kernel: str, units_per_launch: float):
     for x in srcs:
         with open(x, "rb") as f:
             h.update(f.read())
-    if h.hexdigest() != d["source_sha1"]:
+    return d if h.hexdigest() == d["source_sha1"] else None
+
+
+def profiled_traffic(kernel: str, units_per_launch: float):
+    """DRAM bytes per launch from the committed ncu capture, scaled by the units
+    one launch processes; None when the kernel's source has changed since."""
+    d = _profiled_record(kernel)
+    return None if d is None else d["dram_bytes_per_unit"] * units_per_launch
+
+
+def profiled_warp_inst(kernel: str, units_per_launch: float):
+    """Warp instructions per launch from the committed ncu capture
+    (sm__inst_executed.sum), scaled by units; None if absent or stale."""
+    d = _profiled_record(kernel)
+    if d is None or "warp_inst_per_unit" not in d:
         return None
-    return d["dram_bytes_per_unit"] * units_per_launch
+    return d["warp_inst_per_unit"] * units_per_launch
 
 
 def kernel_bytes(wl):
@@ -909,18 +922,33 @@ def dominant_roofline(kern, wl, clocks, traffic_key=None):
     launches = kern[dom]["launch_pairs_per_step"]
     per_launch_s = kern[dom]["ms_per_step"] / launches * 1e-3
     if dom == "scale_sweep":
-        # compute-bound: FP32 lane operations the definition needs, against
-        # 148 SMs x 128 FP32 lanes x the SM clock sampled during the run
-        ops = SWEEP_OPS_PER_ELEM_CAND * (HI - LO + 1) * wl.weight_elems / launches
+        # graded on HBM: 2.5625 algorithmic bytes per weight element against the
+        # measured copy peak.  Its binding resource is instruction issue (FP32
+        # and ALU pipes), so two compute fractions ride along: issue_frac, the
+        # warp instructions the committed capture counts per element against 4
+        # issue slots per SM per cycle at the clock sampled during the run, and
+        # the older model of 5 FP32 lane operations per element and candidate.
+        achieved = kb[dom] / launches / per_launch_s / 1e9
         clk = (clocks or {}).get("sm_mhz") or 1965.0
+        wi = profiled_warp_inst(dom, wl.weight_elems / launches)
+        issue_slots = SMS * ISSUE_PER_SM * clk * 1e6 * per_launch_s
+        ops = SWEEP_OPS_PER_ELEM_CAND * (HI - LO + 1) * wl.weight_elems / launches
         peak_top = SMS * LANES_PER_SM * clk * 1e6 / 1e12
-        achieved = ops / per_launch_s / 1e12
-        return {"kernel": dom, "bound": "alu", "achieved": round(achieved, 2),
-                "peak": round(peak_top, 2), "unit": "TOP/s",
-                "peak_source": f"148 SMs x 128 FP32 lanes x {clk:.0f} MHz (sampled SM clock)",
-                "frac": round(achieved / peak_top, 4),
-                "ops_per_unit": f"{SWEEP_OPS_PER_ELEM_CAND} FP32 ops per weight element per candidate",
-                "hbm_frac_of_measured": kern[dom][f"frac_of_{peak_kind}"],
+        return {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS copy)", "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                "binding_resource": "instruction issue (FP32 FMA and ALU pipes)",
+                "issue_frac": None if wi is None else round(wi / issue_slots, 4),
+                "issue_note": ("warp instructions per launch from the committed ncu capture "
+                               "(sm__inst_executed.sum per weight element x elements) / "
+                               f"(148 SMs x {ISSUE_PER_SM} issue slots x {clk:.0f} MHz sampled "
+                               "x launch time); null once the sweep's sources change"),
+                "alu_model": {"achieved_top_s": round(ops / per_launch_s / 1e12, 2),
+                              "peak_top_s": round(peak_top, 2),
+                              "frac": round(ops / per_launch_s / 1e12 / peak_top, 4),
+                              "ops_per_unit": f"{SWEEP_OPS_PER_ELEM_CAND} FP32 lane ops per "
+                                              "weight element per candidate (definitional)"},
                 "traffic": profiled_traffic(traffic_key or dom, wl.weight_elems / launches),
                 "traffic_note": "DRAM read+write bytes per launch, from the committed ncu "
                                 "capture on the profiling-size layer, scaled by elements"}

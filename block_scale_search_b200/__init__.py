@@ -38,7 +38,7 @@ __all__ = [
 
 STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_INVALID_ARG", -2: "NVFP4_ERR_SHAPE",
           -3: "NVFP4_ERR_ALIGN", -4: "NVFP4_ERR_WINDOW", -5: "NVFP4_ERR_NONFINITE",
-          -6: "NVFP4_ERR_CUDA", -7: "NVFP4_ERR_WORKSPACE"}
+          -6: "NVFP4_ERR_CUDA", -7: "NVFP4_ERR_WORKSPACE", -8: "NVFP4_ERR_CAPTURE"}
 
 
 class NVFP4Error(RuntimeError):
@@ -522,6 +522,54 @@ def quantize_layer_many(Ws, Xs, inputs, q_max: float = 448.0, lo: int = -9, hi: 
     wsv = ws[base:base + nb]
     nvfp4_quantize_layer(wd, xd, q_max, lo, hi, wsv, nb, stream)
     return outs, hs
+
+
+def quantize_grouped_layer(first, second, first_input, second_input, row_offsets,
+                           q_max: float = 448.0, lo: int = -9, hi: int = 6, weighted: bool = True,
+                           want_offsets: bool = False, stream=None):
+    """A mixture-of-experts layer in one call (nvfp4_quantize_grouped_layer).
+    first, second: lists of (W, expert) -- bf16 weights and the expert whose
+    row of the first (resp. second) input's h weights them; first_input,
+    second_input: expert-contiguous bf16 inputs; row_offsets: int64 CUDA
+    tensor [E+1].  weighted=False sweeps both batches with plain MSE.
+    Returns (outputs of first, outputs of second, h1 [E, in1], h2 [E, in2],
+    S, amax, status), each output (codes, scales, offsets or None), S etc.
+    device [n_first + n_second]."""
+    X1 = _bf16_2d(first_input, "X")
+    X2 = _bf16_2d(second_input, "X")
+    dev = X1.device
+    E = row_offsets.numel() - 1
+    h1 = torch.empty(E, X1.shape[1], dtype=torch.float32, device=dev)
+    h2 = torch.empty(E, X2.shape[1], dtype=torch.float32, device=dev)
+    n = len(first) + len(second)
+    S = torch.empty(n, dtype=torch.float32, device=dev)
+    amax = torch.empty(n, dtype=torch.float32, device=dev)
+    status = torch.empty(n, dtype=torch.int32, device=dev)
+    descs, outs = ([], []), ([], [])
+    for b, (batch, hb) in enumerate(((first, h1), (second, h2))):
+        for W, e in batch:
+            W = _bf16_2d(W, "W")
+            o, k = W.shape
+            i = len(descs[0]) if b == 0 else len(first) + len(descs[1])
+            codes = torch.empty(o, k // 2, dtype=torch.uint8, device=dev)
+            scales = torch.empty(o, k // 16, dtype=torch.uint8, device=dev)
+            offs = torch.empty(o, k // 16, dtype=torch.int8, device=dev) if want_offsets else None
+            descs[b].append(SweepDesc(W.data_ptr(), o, k, W.stride(0),
+                                      hb[e].data_ptr() if weighted else None,
+                                      S[i:i + 1].data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                                      _ptr(offs)))
+            outs[b].append((codes, scales, offs))
+    x1 = GroupedInput(X1.data_ptr(), row_offsets.data_ptr(), X1.shape[0], X1.shape[1],
+                      X1.stride(0), h1.data_ptr())
+    x2 = GroupedInput(X2.data_ptr(), row_offsets.data_ptr(), X2.shape[0], X2.shape[1],
+                      X2.stride(0), h2.data_ptr())
+    nb = nvfp4_quantize_grouped_layer_workspace_size(descs[0], descs[1], x1, x2, E, S)
+    if nb == 0:
+        raise NVFP4Error("nvfp4_quantize_grouped_layer_workspace_size", -1)
+    ws = _workspace(nb, dev)
+    nvfp4_quantize_grouped_layer(descs[0], descs[1], x1, x2, E, q_max, lo, hi, S, amax, status,
+                                 ws, nb, stream=stream)
+    return outs[0], outs[1], h1, h2, S, amax, status
 
 
 def diag_hessian_grouped(X: torch.Tensor, row_offsets: torch.Tensor, h: torch.Tensor | None = None,

@@ -11,53 +11,49 @@
 // the process exits; a problem whose partials would not fit is rejected.
 //
 // The array's name in host code is only a host-side stand-in, so its device
-// address is looked up with cudaGetSymbolAddress, once per device, on the
-// first call made while that device is current.  All calls share the one
-// array: calls whose work overlaps on the GPU (different streams, no ordering)
-// race on it.  Nothing in it has to start at zero -- every launch writes each
-// slot that it later reads -- so nothing is cleared.
+// address comes from cudaGetSymbolAddress, with the caller's device current.
+// The lookup is repeated on every call (it is a cheap host call): a cached
+// address would belong to the context it was taken in and would go stale after
+// cudaDeviceReset or under another context on the same device.  The first call
+// on a device also makes the runtime load this library's device code there, so
+// it should come before any stream capture.  All calls share the one array:
+// calls whose work overlaps on the GPU (different streams, no ordering) race on
+// it.  Nothing in it has to start at zero -- every launch writes each slot that
+// it later reads -- so nothing is cleared.
 #include "nvfp4hs.h"
 
 #include <cmath>
-#include <mutex>
 
 #include "nvfp4_kernels.cuh"
 
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 64 * 1024;
-constexpr int kMaxDevices = 128;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (set up once per
-// device); nullptr with *err set if the lookup fails.
+// Device address of the scratch array in the current context; nullptr with
+// *err set on failure (the runtime's last-error state is then cleared, so a
+// later call does not see this one's error).
 void* scratch_on_current_device(cudaError_t* err) {
-  int dev = 0;
-  *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return nullptr;
-  if (dev < 0 || dev >= kMaxDevices) {
-    *err = cudaErrorInvalidDevice;
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (*err != cudaSuccess) {
+    cudaGetLastError();
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (*err != cudaSuccess) return nullptr;
-    g_scratch_addr[dev] = p;
-  }
-  *err = cudaSuccess;
-  return g_scratch_addr[dev];
+  return p;
 }
 
-int current_sms() {
+// SM count of the current device; 0 with *err set on failure.
+int current_sms(cudaError_t* err) {
   int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  *err = cudaGetDevice(&dev);
+  if (*err == cudaSuccess) *err = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (*err != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
   return n;
 }
 
@@ -78,18 +74,14 @@ extern "C" int nvfp4_global_scale_noalloc(const void* W, int64_t out, int64_t in
   if (S == nullptr || !std::isfinite(q_max) || !(q_max > 0.0f)) return NVFP4_ERR_INVALID_ARG;
   if (!is_aligned(S, 4) || !is_aligned(amax, 4) || !is_aligned(status, 4)) return NVFP4_ERR_ALIGN;
 
-  const int sms = current_sms();
-  if (sms <= 0) {
-    cudaGetLastError();
-    return NVFP4_ERR_CUDA;
-  }
+  cudaError_t err = cudaSuccess;
+  const int sms = current_sms(&err);
+  if (sms <= 0) return nvfp4::record_cuda_status(err == cudaSuccess ? cudaErrorNoDevice : err);
   const nvfp4::LanePlan p = nvfp4::global_scale_plan(out, in, sms);
   if (nvfp4::global_scale_workspace_bytes(p) > kNoAllocScratchBytes) return NVFP4_ERR_WORKSPACE;
-  cudaError_t err = cudaSuccess;
   void* scratch = scratch_on_current_device(&err);
-  if (scratch == nullptr) return NVFP4_ERR_CUDA;
-  const cudaError_t e = nvfp4::launch_global_scale(
+  if (scratch == nullptr) return nvfp4::record_cuda_status(err);
+  return nvfp4::record_cuda_status(nvfp4::launch_global_scale(
       static_cast<const uint16_t*>(W), out, ldw, q_max, S, amax, status,
-      static_cast<uint32_t*>(scratch), p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+      static_cast<uint32_t*>(scratch), p, static_cast<cudaStream_t>(stream)));
 }

@@ -278,6 +278,8 @@ cudaError_t quantize_layer(const LayerWeight* w_caller, int nw, const LayerInput
       sw.tasks = 0;
       for (const Share& s : P.shares[j]) {
         const Reduction& r = P.red[s.red];
+        // an earlier carrier that could not carry ran this reduction whole
+        if (r.standalone) continue;
         SideJob& jb = sw.job[sw.n++];
         if (r.kind == 0) {
           const LayerInput& in = x[r.idx];
@@ -302,7 +304,8 @@ cudaError_t quantize_layer(const LayerWeight* w_caller, int nw, const LayerInput
         jb.t1 = s.t1;
         sw.tasks += s.t1 - s.t0;
       }
-      if (!ok(launch_scale_sweep_side(m.W, m.out, m.in, m.ldw, h, m.S, lo, hi, m.codes, m.scales,
+      if (sw.n > 0 &&
+          !ok(launch_scale_sweep_side(m.W, m.out, m.in, m.ldw, h, m.S, lo, hi, m.codes, m.scales,
                                       m.offs, sw, sms, &carried, stream)))
         return e;
     }

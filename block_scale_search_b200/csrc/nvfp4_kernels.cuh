@@ -162,4 +162,9 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               int64_t out, int64_t in, float* W_out, int num_sms,
                               cudaStream_t stream);
 
+// Maps a CUDA error to the entry points' status: NVFP4_OK for cudaSuccess,
+// otherwise NVFP4_ERR_CUDA, with the code kept for nvfp4_last_cuda_error()
+// (per host thread).  Defined with the entry points in nvfp4hs_capi.cu.
+int record_cuda_status(cudaError_t e);
+
 }  // namespace nvfp4

@@ -30,6 +30,19 @@ int cuda_status(cudaError_t e) {
   return NVFP4_ERR_CUDA;
 }
 
+// NVFP4_ERR_CAPTURE when `s` is being captured into a CUDA graph, else
+// NVFP4_OK.  The batched and grouped calls stage their descriptor tables
+// from host memory that is gone once they return; a graph replay would read
+// it later, so those calls refuse a capturing stream instead.
+int refuse_capture(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_OK;  // let the call's own CUDA calls report the stream's state
+  }
+  return cs == cudaStreamCaptureStatusNone ? NVFP4_OK : NVFP4_ERR_CAPTURE;
+}
+
 // SM count of the current device, cached per device ordinal (0 on failure).
 int current_sm_count() {
   static std::atomic<int> cache[128];
@@ -112,6 +125,10 @@ int resident_ctas(const void* kernel, int threads_per_cta) {
   }
   return n > 0 ? n : 1;
 }
+}  // namespace nvfp4
+
+namespace nvfp4 {
+int record_cuda_status(cudaError_t e) { return cuda_status(e); }
 }  // namespace nvfp4
 
 extern "C" {
@@ -471,6 +488,7 @@ int nvfp4_global_scale_batched(const nvfp4_matrix_desc* descs, int64_t n, float 
   if (!aligned(S, 4) || !aligned(amax, 4) || !aligned(status, 4)) return NVFP4_ERR_ALIGN;
   if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  if ((st = refuse_capture(static_cast<cudaStream_t>(stream))) != NVFP4_OK) return st;
   const int sms = current_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorNoDevice);
   const GsBatchPlan p = plan_global_scale_batch(descs, n, sms);
@@ -637,6 +655,7 @@ int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n,
   if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
   if (workspace_bytes < round256(static_cast<size_t>(n) * sizeof(nvfp4::SweepDesc)))
     return NVFP4_ERR_WORKSPACE;
+  if (const int cst = refuse_capture(static_cast<cudaStream_t>(stream)); cst != NVFP4_OK) return cst;
   const int sms = current_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorNoDevice);
   const bool weighted = any_h;
@@ -703,6 +722,7 @@ int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
       if (sweep_events[k] == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  if ((st = refuse_capture(static_cast<cudaStream_t>(stream))) != NVFP4_OK) return st;
   const int sms = current_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorNoDevice);
   const GroupedLayerLayout L =

@@ -54,7 +54,8 @@ typedef enum nvfp4_status {
     NVFP4_ERR_WINDOW = -4,       /* lo/hi outside the supported sweep window            */
     NVFP4_ERR_NONFINITE = -5,    /* written to a device status word: Inf/NaN in W       */
     NVFP4_ERR_CUDA = -6,         /* a CUDA runtime call or kernel launch failed         */
-    NVFP4_ERR_WORKSPACE = -7     /* workspace NULL or smaller than the queried size     */
+    NVFP4_ERR_WORKSPACE = -7,    /* workspace NULL or smaller than the queried size     */
+    NVFP4_ERR_CAPTURE = -8       /* a call that stages host tables, on a capturing stream */
 } nvfp4_status;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -112,9 +113,13 @@ int nvfp4_global_scale(const void* W, int64_t out, int64_t in, int64_t ldw, floa
  * a pre-planned memory pool -- the per-CTA partial maxima go to a 64 KiB
  * array compiled into the library, which every GPU that loads the library
  * holds until the process exits.  Nothing is allocated.
- *   - The first call on a device, made while that device is current, looks up
- *     the array's device address (cudaGetSymbolAddress); make that first call
- *     before any stream capture.
+ *   - Every call looks up the array's device address in the current context
+ *     (cudaGetSymbolAddress), so a cudaDeviceReset or another context on the
+ *     same device never leaves it a stale address.  The first call on a device
+ *     also makes the runtime load the library's device code there: make that
+ *     first call before any stream capture.
+ *   - CUDA failures (device query, address lookup, launch) return
+ *     NVFP4_ERR_CUDA with the code kept for nvfp4_last_cuda_error().
  *   - All calls share the array: calls that overlap on the GPU (different
  *     streams without ordering between them) race and must not be issued.
  *   - The array needs no initialisation; it is not cleared.
@@ -220,7 +225,10 @@ typedef struct nvfp4_matrix_desc {
  *   workspace    at least nvfp4_global_scale_batched_workspace_size(descs, n)
  *                bytes, 256-byte aligned: a device copy of the table plus one
  *                partial maximum per CTA.
- * Each descriptor is checked as nvfp4_global_scale checks its arguments. */
+ * Each descriptor is checked as nvfp4_global_scale checks its arguments.
+ * The table is staged from host memory, so the call cannot be captured into
+ * a CUDA graph: on a capturing stream it returns NVFP4_ERR_CAPTURE and
+ * enqueues nothing. */
 size_t nvfp4_global_scale_batched_workspace_size(const nvfp4_matrix_desc* descs, int64_t n);
 int nvfp4_global_scale_batched(const nvfp4_matrix_desc* descs, int64_t n, float q_max, float* S,
                                float* amax, int* status, void* workspace,
@@ -242,7 +250,8 @@ typedef struct nvfp4_sweep_desc {
  *   descs        HOST array of n descriptors (read before the call returns).
  *   workspace    at least nvfp4_scale_sweep_quantize_batched_workspace_size(n)
  *                bytes, 256-byte aligned (a device copy of the table).
- * A batch mixing NULL and non-NULL h returns NVFP4_ERR_INVALID_ARG. */
+ * A batch mixing NULL and non-NULL h returns NVFP4_ERR_INVALID_ARG.  As for
+ * nvfp4_global_scale_batched, a capturing stream returns NVFP4_ERR_CAPTURE. */
 size_t nvfp4_scale_sweep_quantize_batched_workspace_size(int64_t n);
 int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n, int lo, int hi,
                                        void* workspace, size_t workspace_bytes, void* stream);
@@ -360,7 +369,9 @@ int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
  *              `stream` right before and after the sweep launch of `first`,
  *              [2], [3] around that of `second` (the one swept first includes
  *              what it streams), for timing.
- * Asynchronous on `stream`; descriptors are read on the host during the call.
+ * Asynchronous on `stream`; descriptors are read on the host during the call
+ * and staged from host memory, so a capturing stream returns
+ * NVFP4_ERR_CAPTURE with nothing enqueued.
  *
  * nvfp4_quantize_grouped_layer_order returns which batch that call, with the
  * same arguments, sweeps first: 0 for `first`, 1 for `second`, or a negative

@@ -7,10 +7,26 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+# per-matrix parity figures collected by the full-size tests, printed in the
+# run's summary (they pass silently otherwise)
+_REPORT: list[str] = []
+
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size workload checks")
+
+
+def pytest_terminal_summary(terminalreporter):
+    if _REPORT:
+        terminalreporter.section("parity per matrix")
+        for line in _REPORT:
+            terminalreporter.write_line(line)
+
+
+@pytest.fixture(scope="session")
+def parity_report():
+    return _REPORT.append
 
 
 @pytest.fixture(scope="session")

@@ -34,6 +34,10 @@ def test_native_line():
     r = d["roofline"]
     assert r["bound"] in ("hbm", "alu", "tensor") and r["achieved"] > 0 and r["peak"] > 0
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-3 and "traffic" in r
+    if r["kernel"] == "scale_sweep":
+        # graded on HBM bytes, with the issue-slot fraction and the lane-op model beside it
+        assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+        assert "issue_frac" in r and r["alu_model"]["frac"] > 0
     c = d["cpu_baseline"]
     assert c["kind"] == "oracle" and c["value"] > 0 and c["cores"] >= 1 and c["sample"]
     e = d["e2e"]

@@ -129,3 +129,55 @@ def test_moe_layer_through_grouped_calls(orc, nv):
         gc, gs = outs[i][0].cpu().numpy(), outs[i][1].cpu().numpy()
         w, hh, _, _ = matrix_groups(bits, gc, gs, hn)
         assert_parity(compare_groups(orc, w, hh, float(S_ref), gc, gs, rc, rs), m.name)
+
+
+def test_batched_calls_refuse_stream_capture(nv):
+    """The batched S, batched sweep and grouped layer calls stage host tables,
+    which a graph replay could not read: on a capturing stream they return
+    NVFP4_ERR_CAPTURE and enqueue nothing; the capture itself stays usable."""
+    import workloads
+    Ws = [workloads.weight(64, 256, 0.02, 0.0, 1.0, 70 + i, DEV) for i in range(2)]
+    mdesc = [nv.MatrixDesc(W.data_ptr(), 64, 256, 256) for W in Ws]
+    S = torch.zeros(2, device=DEV)
+    amax = torch.zeros(2, device=DEV)
+    status = torch.zeros(2, dtype=torch.int32, device=DEV)
+    gws = torch.empty(nv.nvfp4_global_scale_batched_workspace_size(mdesc), dtype=torch.uint8,
+                      device=DEV)
+    codes = [torch.empty(64, 128, dtype=torch.uint8, device=DEV) for _ in Ws]
+    scales = [torch.empty(64, 16, dtype=torch.uint8, device=DEV) for _ in Ws]
+    sdesc = [nv.SweepDesc(W.data_ptr(), 64, 256, 256, None, S[i:i + 1].data_ptr(),
+                          codes[i].data_ptr(), scales[i].data_ptr(), None) for i, W in enumerate(Ws)]
+    sws = torch.empty(nv.nvfp4_scale_sweep_quantize_batched_workspace_size(2), dtype=torch.uint8,
+                      device=DEV)
+    X = workloads.calib(32, 256, 1.0, 72, DEV)
+    off = torch.tensor([0, 16, 32], dtype=torch.int64, device=DEV)
+    h1 = torch.empty(2, 256, device=DEV)
+    h2 = torch.empty(2, 256, device=DEV)
+    x1 = nv.GroupedInput(X.data_ptr(), off.data_ptr(), 32, 256, 256, h1.data_ptr())
+    x2 = nv.GroupedInput(X.data_ptr(), off.data_ptr(), 32, 256, 256, h2.data_ptr())
+    gl = [nv.SweepDesc(W.data_ptr(), 64, 256, 256, h1[i].data_ptr(), S[i:i + 1].data_ptr(),
+                       codes[i].data_ptr(), scales[i].data_ptr(), None) for i, W in enumerate(Ws)]
+    nb = nv.nvfp4_quantize_grouped_layer_workspace_size(gl[:1], gl[1:], x1, x2, 2, S)
+    lws = torch.empty(nb, dtype=torch.uint8, device=DEV)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    got = []
+    with torch.cuda.graph(g, stream=s):
+        for call in (lambda: nv.nvfp4_global_scale_batched(mdesc, 448.0, S, amax, status, gws,
+                                                           gws.numel(), s),
+                     lambda: nv.nvfp4_scale_sweep_quantize_batched(sdesc, -9, 6, sws, sws.numel(),
+                                                                   s),
+                     lambda: nv.nvfp4_quantize_grouped_layer(gl[:1], gl[1:], x1, x2, 2, 448.0, -9,
+                                                             6, S, amax, status, lws, nb,
+                                                             stream=s)):
+            try:
+                call()
+                got.append(0)
+            except nv.NVFP4Error as e:
+                got.append(e.status)
+        S.add_(1.0)  # the capture goes on after the refusals
+    assert got == [-8, -8, -8]
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(S.cpu(), torch.ones(2))
