@@ -25,6 +25,7 @@
 #include <cmath>
 
 #include "nvfp4_kernels.cuh"
+#include "nvtx_range.cuh"
 
 namespace {
 
@@ -64,6 +65,7 @@ bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t
 extern "C" int nvfp4_global_scale_noalloc(const void* W, int64_t out, int64_t in, int64_t ldw,
                                           float q_max, float* S, float* amax, int* status,
                                           void* stream) {
+  NVFP4_RANGE("nvfp4_global_scale_noalloc");
   // the same argument checks as nvfp4_global_scale, before any CUDA call
   if (out < 0 || in < 0) return NVFP4_ERR_INVALID_ARG;
   if (W == nullptr && out > 0 && in > 0) return NVFP4_ERR_INVALID_ARG;

@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "nvfp4_kernels.cuh"
+#include "nvtx_range.cuh"
 #include "row_counters.cuh"
 #include "side_reduce.cuh"
 
@@ -147,6 +148,7 @@ size_t nvfp4_diag_hessian_workspace_size(int64_t tokens, int64_t in) {
 
 int nvfp4_diag_hessian(const void* X, int64_t tokens, int64_t in, int64_t ldx, float* h,
                        int accumulate, void* workspace, size_t workspace_bytes, void* stream) {
+  NVFP4_RANGE("nvfp4_diag_hessian");
   int st = check_diag_hessian(X, tokens, in, ldx, h, accumulate);
   if (st != NVFP4_OK) return st;
   if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
@@ -170,6 +172,7 @@ size_t nvfp4_global_scale_workspace_size(int64_t out, int64_t in) {
 int nvfp4_global_scale(const void* W, int64_t out, int64_t in, int64_t ldw, float q_max,
                        float* S, float* amax, int* status, void* workspace,
                        size_t workspace_bytes, void* stream) {
+  NVFP4_RANGE("nvfp4_global_scale");
   int st = check_matrix(W, out, in, ldw, 8);
   if (st != NVFP4_OK) return st;
   if (S == nullptr || !std::isfinite(q_max) || !(q_max > 0.0f)) return NVFP4_ERR_INVALID_ARG;
@@ -190,6 +193,7 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
                                const float* h, const float* S, int lo, int hi,
                                uint8_t* codes, uint8_t* scales, int8_t* chosen_offset,
                                void* stream) {
+  NVFP4_RANGE("nvfp4_scale_sweep_quantize");
   int st = check_matrix(W, out, in, ldw, 16);
   if (st != NVFP4_OK) return st;
   const bool empty = out == 0 || in == 0;
@@ -237,6 +241,7 @@ int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
                          const nvfp4_layer_input* inputs, int n_inputs, float q_max, int lo,
                          int hi, void* workspace, size_t workspace_bytes,
                          void* const* sweep_events, void* stream) {
+  NVFP4_RANGE("nvfp4_quantize_layer");
   std::vector<nvfp4::LayerWeight> wv;
   std::vector<nvfp4::LayerInput> xv;
   int st = check_layer(weights, n_weights, inputs, n_inputs, &wv, &xv);
@@ -266,6 +271,7 @@ int nvfp4_debug_row_counters(void** ptr, size_t* bytes) {
 int nvfp4_scale_sweep_quantize_full(const void* W, int64_t out, int64_t in, int64_t ldw,
                                     const float* h, const float* S, uint8_t* codes,
                                     uint8_t* scales, int8_t* chosen_offset, void* stream) {
+  NVFP4_RANGE("nvfp4_scale_sweep_quantize_full");
   int st = check_matrix(W, out, in, ldw, 16);
   if (st != NVFP4_OK) return st;
   const bool empty = out == 0 || in == 0;
@@ -284,6 +290,7 @@ int nvfp4_quantize_activations(const void* A, int64_t tokens, int64_t in, int64_
                                float q_max, int lo, int hi, float* S, uint8_t* codes,
                                uint8_t* scales, int8_t* chosen_offset, int* status,
                                void* stream) {
+  NVFP4_RANGE("nvfp4_quantize_activations");
   int st = check_matrix(A, tokens, in, lda, 16);
   if (st != NVFP4_OK) return st;
   if (!std::isfinite(q_max) || !(q_max > 0.0f)) return NVFP4_ERR_INVALID_ARG;
@@ -312,6 +319,7 @@ size_t nvfp4_blocked_scales_size(int64_t rows, int64_t cols) {
 
 int nvfp4_scales_to_blocked(const uint8_t* scales, int64_t rows, int64_t cols, int64_t ld,
                             uint8_t* out, void* stream) {
+  NVFP4_RANGE("nvfp4_scales_to_blocked");
   if (rows < 0 || cols < 0) return NVFP4_ERR_INVALID_ARG;
   if (ld < cols || rows > kMaxDim || cols > kMaxDim || ld > kMaxDim) return NVFP4_ERR_SHAPE;
   if (rows == 0 || cols == 0) return NVFP4_OK;
@@ -325,6 +333,7 @@ int nvfp4_scales_to_blocked(const uint8_t* scales, int64_t rows, int64_t cols, i
 
 int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* S, int64_t out,
                      int64_t in, float* W_out, void* stream) {
+  NVFP4_RANGE("nvfp4_dequantize");
   if (out < 0 || in < 0) return NVFP4_ERR_INVALID_ARG;
   if (in % 16 != 0 || out > kMaxDim || in > kMaxDim) return NVFP4_ERR_SHAPE;
   if (out == 0 || in == 0) return NVFP4_OK;
@@ -353,6 +362,7 @@ int nvfp4_diag_hessian_grouped(const void* X, const int64_t* row_offsets, int64_
                                int64_t total_tokens, int64_t in, int64_t ldx, float* h,
                                int accumulate, void* workspace, size_t workspace_bytes,
                                void* stream) {
+  NVFP4_RANGE("nvfp4_diag_hessian_grouped");
   int st = check_diag_hessian(X, total_tokens, in, ldx, h, accumulate);
   if (st != NVFP4_OK) return st;
   if (row_offsets == nullptr || experts <= 0) return NVFP4_ERR_INVALID_ARG;
@@ -481,6 +491,7 @@ size_t nvfp4_global_scale_batched_workspace_size(const nvfp4_matrix_desc* descs,
 int nvfp4_global_scale_batched(const nvfp4_matrix_desc* descs, int64_t n, float q_max, float* S,
                                float* amax, int* status, void* workspace, size_t workspace_bytes,
                                void* stream) {
+  NVFP4_RANGE("nvfp4_global_scale_batched");
   int st = check_batch(descs, n, 8);
   if (st != NVFP4_OK) return st;
   if (n == 0) return NVFP4_OK;
@@ -633,6 +644,7 @@ size_t nvfp4_scale_sweep_quantize_batched_workspace_size(int64_t n) {
 
 int nvfp4_scale_sweep_quantize_batched(const nvfp4_sweep_desc* descs, int64_t n, int lo, int hi,
                                        void* workspace, size_t workspace_bytes, void* stream) {
+  NVFP4_RANGE("nvfp4_scale_sweep_quantize_batched");
   if (n < 0 || (n > 0 && descs == nullptr)) return NVFP4_ERR_INVALID_ARG;
   if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
   bool any_h = false, all_h = true;
@@ -709,6 +721,7 @@ int nvfp4_quantize_grouped_layer(const nvfp4_sweep_desc* first, int64_t n_first,
                                  float q_max, int lo, int hi, float* S, float* amax, int* status,
                                  void* workspace, size_t workspace_bytes,
                                  void* const* sweep_events, void* stream) {
+  NVFP4_RANGE("nvfp4_quantize_grouped_layer");
   std::vector<nvfp4_matrix_desc> md;
   bool w1 = false, w2 = false;
   int st = check_grouped_layer(first, n_first, second, n_second, first_input, second_input,

@@ -296,3 +296,22 @@ def test_grouped_layer_order(L):
         nv.nvfp4_quantize_grouped_layer_order(gu, dn, x_gu, x_dn, E, S, -10, 6)
     with pytest.raises(nv.NVFP4Error):
         nv.nvfp4_quantize_grouped_layer_order(gu, dn, x_gu, x_dn, E, S + 4, -9, 6)
+
+
+def test_every_launching_entry_point_opens_an_nvtx_range():
+    """Each entry point that enqueues GPU work opens a named NVTX range first
+    (a profiler timeline then shows which call launched which kernels); the
+    size and order queries, which launch nothing, need none."""
+    import re
+    csrc = os.path.join(ROOT, "block_scale_search_b200", "csrc")
+    found = {}
+    for fn in ("nvfp4hs_capi.cu", "global_scale_noalloc.cu"):
+        src = open(os.path.join(csrc, fn)).read()
+        for m in re.finditer(r"\n(?:extern \"C\" )?int (nvfp4_\w+)\((?:.|\n)*?\) \{\n(.*)\n", src):
+            found[m.group(1)] = m.group(2).strip()
+    queries = {"nvfp4_version", "nvfp4_last_cuda_error", "nvfp4_quantize_layer_order",
+               "nvfp4_quantize_grouped_layer_order", "nvfp4_debug_row_counters"}
+    launching = {k: v for k, v in found.items() if k not in queries}
+    assert len(launching) == 13, sorted(launching)
+    for name, first in launching.items():
+        assert first == f'NVFP4_RANGE("{name}");', (name, first)
