@@ -237,6 +237,21 @@ class Step:
                            "the other weights' S and the other inputs' h are streamed by a fifth "
                            "warp in each CTA of the earlier sweeps (carrying sweeps)")
         nb = nv.nvfp4_quantize_layer_workspace_size(self.layer_w, self.layer_x)
+        # several layers (workloads listing their layers): the multi-layer call
+        # over the same descriptors, each layer's input indices its own
+        self.layers = None
+        if wl.extra.get("layers"):
+            self.layers = []
+            for names in wl.extra["layers"]:
+                lk = list(dict.fromkeys(self.x_of[n] for n in names))
+                lw = [self.layer_w[self.mats.index(n)] for n in names]
+                lw = [nv.LayerWeight(d.W, d.out, d.inp, d.ldw, lk.index(self.x_of[n]), d.S, d.amax,
+                                     d.status, d.codes, d.scales, d.chosen_offset)
+                      for d, n in zip(lw, names)]
+                lx = [self.layer_x[keys.index(k)] for k in lk]
+                self.layers.append((lw, lx))
+            assert [n for names in wl.extra["layers"] for n in names] == self.mats
+            nb = nv.nvfp4_quantize_layers_workspace_size(self.layers)
         self.layer_ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=device)
         self.layer_nb = nb
 
@@ -277,9 +292,13 @@ class Step:
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record(main)
-            wa, xa = self.layer_arrays
-            nv.nvfp4_quantize_layer(wa, xa, self.wl.q_max, LO, HI, self.layer_ws, self.layer_nb,
-                                    sweep_events=sev, stream=main)
+            if self.layers is not None:
+                nv.nvfp4_quantize_layers(self.layers, self.wl.q_max, LO, HI, self.layer_ws,
+                                         self.layer_nb, sweep_events=sev, stream=main)
+            else:
+                wa, xa = self.layer_arrays
+                nv.nvfp4_quantize_layer(wa, xa, self.wl.q_max, LO, HI, self.layer_ws,
+                                        self.layer_nb, sweep_events=sev, stream=main)
             if ev is not None:
                 b.record(main)
                 ev.setdefault("layer_call", []).append((a, b))
@@ -850,6 +869,9 @@ WORKLOADS = {
                         "channel scales"),
     "mlp_slice": ("mlp_slice (profiling size): W 8192x8192 bf16 N(0,0.015) 0.1% x10; X 16384 x "
                   "8192 bf16 lognormal(1.5) channel scales"),
+    "llama33_70b_mlp_x2": ("llama33_70b_mlp_x2: two consecutive Llama-3.3-70B-shaped MLP layers "
+                           "(each gate/up 28672x8192, down 8192x28672 bf16 N(0,0.015) 0.1% x10; X "
+                           "65536 tokens, lognormal(1.5)) in one nvfp4_quantize_layers call"),
     "mlp_layer_slice": ("mlp_layer_slice (profiling size): gate/up 8192x4096, down 4096x8192 "
                         "bf16 N(0,0.015) 0.1% x10; X 16384 tokens x {4096, 8192} bf16 "
                         "lognormal(1.5) channel scales"),

@@ -26,7 +26,8 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
     "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "nvfp4_quantize_layer_order",
-    "quantize_layer_many",
+    "quantize_layer_many", "Layer", "nvfp4_quantize_layers_workspace_size",
+    "nvfp4_quantize_layers", "quantize_layers_many", "quantize_grouped_layer",
     "LayerWeight", "LayerInput", "GroupedInput", "nvfp4_quantize_grouped_layer_workspace_size",
     "nvfp4_quantize_grouped_layer", "nvfp4_quantize_grouped_layer_order",
     "diag_hessian_grouped", "global_scale_batched", "scale_sweep_quantize_batched",
@@ -80,6 +81,12 @@ class LayerInput(C.Structure):
     _fields_ = [("X", _vp), ("tokens", _i64), ("inp", _i64), ("ldx", _i64), ("h", _vp)]
 
 
+class Layer(C.Structure):
+    """nvfp4_layer: one layer's weight and input descriptors"""
+    _fields_ = [("weights", C.POINTER(LayerWeight)), ("n_weights", _int),
+                ("inputs", C.POINTER(LayerInput)), ("n_inputs", _int)]
+
+
 class GroupedInput(C.Structure):
     """nvfp4_grouped_input"""
     _fields_ = [("X", _vp), ("row_offsets", _vp), ("total_tokens", _i64), ("inp", _i64),
@@ -113,6 +120,9 @@ _SIGS = {
                                     _int, C.POINTER(_int)], _int),
     "nvfp4_quantize_layer": ([C.POINTER(LayerWeight), _int, C.POINTER(LayerInput), _int, _f32, _int,
                               _int, _vp, _sz, C.POINTER(_vp), _vp], _int),
+    "nvfp4_quantize_layers_workspace_size": ([C.POINTER(Layer), _int], _sz),
+    "nvfp4_quantize_layers": ([C.POINTER(Layer), _int, _f32, _int, _int, _vp, _sz, C.POINTER(_vp),
+                               _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
     "nvfp4_blocked_scales_size": ([_i64, _i64], _sz),
     "nvfp4_scales_to_blocked": ([_vp, _i64, _i64, _i64, _vp, _vp], _int),
@@ -250,6 +260,34 @@ def nvfp4_quantize_layer(weights, inputs, q_max, lo, hi, workspace, workspace_by
     _check("nvfp4_quantize_layer", lib().nvfp4_quantize_layer(
         wa, len(weights), xa, len(inputs), float(q_max), int(lo), int(hi), _ptr(workspace),
         workspace_bytes, ev, _stream(stream)))
+
+
+def _layers_array(layers):
+    """layers: list of (weights, inputs) lists of LayerWeight / LayerInput.
+    Returns the ctypes array and the per-layer arrays it points into (which
+    must outlive the call)."""
+    keep = [_layer_arrays(w, x) for w, x in layers]
+    arr = (Layer * max(1, len(layers)))(*[Layer(wa, len(w), xa, len(x))
+                                          for (wa, xa), (w, x) in zip(keep, layers)])
+    return arr, keep
+
+
+def nvfp4_quantize_layers_workspace_size(layers) -> int:
+    arr, _keep = _layers_array(layers)
+    return lib().nvfp4_quantize_layers_workspace_size(arr, len(layers))
+
+
+def nvfp4_quantize_layers(layers, q_max, lo, hi, workspace, workspace_bytes, sweep_events=None,
+                          stream=None):
+    """layers: list of (weights, inputs), as for nvfp4_quantize_layer; a weight's
+    input indexes its own layer's inputs."""
+    arr, _keep = _layers_array(layers)
+    ev = None
+    if sweep_events is not None:
+        ev = (_vp * len(sweep_events))(*[e.cuda_event for e in sweep_events])
+    _check("nvfp4_quantize_layers", lib().nvfp4_quantize_layers(
+        arr, len(layers), float(q_max), int(lo), int(hi), _ptr(workspace), workspace_bytes, ev,
+        _stream(stream)))
 
 
 def _sweep_array(descs):
@@ -570,6 +608,44 @@ def quantize_grouped_layer(first, second, first_input, second_input, row_offsets
     nvfp4_quantize_grouped_layer(descs[0], descs[1], x1, x2, E, q_max, lo, hi, S, amax, status,
                                  ws, nb, stream=stream)
     return outs[0], outs[1], h1, h2, S, amax, status
+
+
+def quantize_layers_many(layers, q_max: float = 448.0, lo: int = -9, hi: int = 6,
+                         want_offsets: bool = False, stream=None):
+    """Several consecutive layers in one call (nvfp4_quantize_layers).  layers:
+    list of (Ws, Xs, inputs) as for quantize_layer_many.  Returns, per layer,
+    (list of (codes, scales, S, offsets or None, status) per weight, list of h
+    per input)."""
+    descs, outs = [], []
+    for Ws, Xs, inputs in layers:
+        Ws = [_bf16_2d(W, "W") for W in Ws]
+        Xs = [_bf16_2d(X, "X") for X in Xs]
+        dev = (Ws or Xs)[0].device
+        hs = [torch.empty(X.shape[1], dtype=torch.float32, device=dev) for X in Xs]
+        lo_, wd = [], []
+        for W, k in zip(Ws, inputs):
+            o, n = W.shape
+            codes = torch.empty(o, n // 2, dtype=torch.uint8, device=dev)
+            scales = torch.empty(o, n // 16, dtype=torch.uint8, device=dev)
+            S = torch.empty(1, dtype=torch.float32, device=dev)
+            status = torch.empty(1, dtype=torch.int32, device=dev)
+            offs = torch.empty(o, n // 16, dtype=torch.int8, device=dev) if want_offsets else None
+            wd.append(LayerWeight(W.data_ptr(), o, n, W.stride(0), int(k), S.data_ptr(), None,
+                                  status.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                                  _ptr(offs)))
+            lo_.append((codes, scales, S, offs, status))
+        xd = [LayerInput(X.data_ptr(), X.shape[0], X.shape[1], X.stride(0), h.data_ptr())
+              for X, h in zip(Xs, hs)]
+        descs.append((wd, xd))
+        outs.append((lo_, hs))
+    nb = nvfp4_quantize_layers_workspace_size(descs)
+    if nb == 0:
+        raise NVFP4Error("nvfp4_quantize_layers_workspace_size", -1)
+    dev = outs[0][0][0][0].device if outs and outs[0][0] else outs[0][1][0].device
+    ws = torch.empty(nb + 256, dtype=torch.uint8, device=dev)
+    base = (-ws.data_ptr()) % 256
+    nvfp4_quantize_layers(descs, q_max, lo, hi, ws[base:base + nb], nb, stream=stream)
+    return outs
 
 
 def diag_hessian_grouped(X: torch.Tensor, row_offsets: torch.Tensor, h: torch.Tensor | None = None,

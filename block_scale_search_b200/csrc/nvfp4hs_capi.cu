@@ -210,6 +210,66 @@ int nvfp4_scale_sweep_quantize(const void* W, int64_t out, int64_t in, int64_t l
                                                static_cast<cudaStream_t>(stream)));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Several layers' descriptors as one: inputs appended layer by layer, each
+// weight's input index moved by its layer's first input.
+int flatten_layers(const nvfp4_layer* layers, int n_layers, std::vector<nvfp4_layer_weight>* w,
+                   std::vector<nvfp4_layer_input>* x) {
+  if (n_layers < 0 || (n_layers > 0 && layers == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  int64_t nw = 0, nx = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    const nvfp4_layer& L = layers[l];
+    if (L.n_weights < 0 || L.n_inputs < 0 || (L.n_weights > 0 && L.weights == nullptr) ||
+        (L.n_inputs > 0 && L.inputs == nullptr))
+      return NVFP4_ERR_INVALID_ARG;
+    nw += L.n_weights;
+    nx += L.n_inputs;
+  }
+  if (nw > (1 << 20) || nx > (1 << 20)) return NVFP4_ERR_INVALID_ARG;
+  w->clear();
+  x->clear();
+  for (int l = 0; l < n_layers; ++l) {
+    const nvfp4_layer& L = layers[l];
+    const int base = static_cast<int>(x->size());
+    for (int k = 0; k < L.n_inputs; ++k) x->push_back(L.inputs[k]);
+    for (int j = 0; j < L.n_weights; ++j) {
+      nvfp4_layer_weight d = L.weights[j];
+      if (d.input < -1 || d.input >= L.n_inputs) return NVFP4_ERR_INVALID_ARG;
+      if (d.input >= 0) d.input += base;
+      w->push_back(d);
+    }
+  }
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_quantize_layers_workspace_size(const nvfp4_layer* layers, int n_layers) {
+  std::vector<nvfp4_layer_weight> w;
+  std::vector<nvfp4_layer_input> x;
+  if (flatten_layers(layers, n_layers, &w, &x) != NVFP4_OK) return 0;
+  return nvfp4_quantize_layer_workspace_size(w.data(), static_cast<int>(w.size()), x.data(),
+                                             static_cast<int>(x.size()));
+}
+
+int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, int lo, int hi,
+                          void* workspace, size_t workspace_bytes, void* const* sweep_events,
+                          void* stream) {
+  NVFP4_RANGE("nvfp4_quantize_layers");
+  std::vector<nvfp4_layer_weight> w;
+  std::vector<nvfp4_layer_input> x;
+  const int st = flatten_layers(layers, n_layers, &w, &x);
+  if (st != NVFP4_OK) return st;
+  return nvfp4_quantize_layer(w.data(), static_cast<int>(w.size()), x.data(),
+                              static_cast<int>(x.size()), q_max, lo, hi, workspace,
+                              workspace_bytes, sweep_events, stream);
+}
+
 size_t nvfp4_quantize_layer_workspace_size(const nvfp4_layer_weight* weights, int n_weights,
                                            const nvfp4_layer_input* inputs, int n_inputs) {
   std::vector<nvfp4::LayerWeight> wv;

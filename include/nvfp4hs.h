@@ -332,6 +332,36 @@ int nvfp4_quantize_layer(const nvfp4_layer_weight* weights, int n_weights,
                          void* const* sweep_events, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Several consecutive layers in one call (H-Scale summary, sec. 4
+ * "Efficiency and Hardware Deployment": the added cost is one activation pass
+ * and the offline search, which a model-wide pass should pay once).  Each
+ * layer is the argument set of nvfp4_quantize_layer, its weights' `input`
+ * indexing its own inputs.  The call is nvfp4_quantize_layer over all the
+ * layers' weights (in layer order) and inputs together: the results are the
+ * per-step calls' bytes, and the reductions of a later layer -- its inputs'
+ * h and its weights' S -- are streamed beside the sweeps of earlier layers,
+ * so that only the first swept weight's S and its input's h run on their own
+ * (in a single-layer call, each layer would run those two alone and its last
+ * sweep would carry nothing).
+ *   layers       n_layers HOST descriptors (read during the call).
+ *   sweep_events NULL or 2 * (total weights) events, weights counted across
+ *                the layers in order, as for nvfp4_quantize_layer.
+ * Workspace, alignment, status and error rules are nvfp4_quantize_layer's;
+ * an `input` outside its own layer's inputs returns NVFP4_ERR_INVALID_ARG.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const nvfp4_layer_weight* weights;
+  int n_weights;
+  const nvfp4_layer_input* inputs;
+  int n_inputs;
+} nvfp4_layer;
+
+size_t nvfp4_quantize_layers_workspace_size(const nvfp4_layer* layers, int n_layers);
+int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, int lo, int hi,
+                          void* workspace, size_t workspace_bytes, void* const* sweep_events,
+                          void* stream);
+
+/* ------------------------------------------------------------------------
  * A mixture-of-experts layer in one call: two batches of expert matrices, each
  * batch reading one expert-contiguous calibration input (for example every
  * expert's gate and up projections reading the routed tokens' hidden states,

@@ -256,6 +256,34 @@ def test_quantize_layer_validation(L):
         assert L.nvfp4_quantize_layer_order(wa, 1, xa, 1, -9, 6, order) == -6
 
 
+def test_quantize_layers_validation(L):
+    """The multi-layer call checks each layer's descriptors as the one-layer
+    call does, with input indices local to their layer."""
+    import block_scale_search_b200 as nv
+    W = lambda **k: nv.LayerWeight(**{**dict(W=P, out=64, inp=256, ldw=256, input=0, S=P, amax=None,
+                                            status=None, codes=P, scales=P, chosen_offset=None), **k})
+    X = lambda **k: nv.LayerInput(**{**dict(X=P, tokens=32, inp=256, ldx=256, h=P), **k})
+
+    def call(layers, n=None, q=448.0, lo=-9, hi=6):
+        arr, _keep = nv._layers_array(layers)
+        return L.nvfp4_quantize_layers(arr, len(layers) if n is None else n, q, lo, hi, P, 1 << 30,
+                                       None, None)
+
+    assert L.nvfp4_quantize_layers(None, 1, 448.0, -9, 6, P, 1 << 30, None, None) == -1
+    assert call([([W()], [X()])], n=-1) == -1
+    # layer 1's weight names its own input 1, which layer 1 does not have
+    assert call([([W()], [X()]), ([W(input=1)], [X()])]) == -1
+    assert call([([W()], [X()]), ([W(input=0, inp=128, ldw=128)], [X()])]) == -2
+    assert call([([W()], [X()]), ([W()], [X(h=P + 4)])]) == -3
+    assert call([([W()], [X()])], lo=-10) == -4
+    assert call([]) == 0                                    # nothing to do
+    import torch
+    if not torch.cuda.is_available():
+        arr, _keep = nv._layers_array([([W()], [X()]), ([W(), W(input=-1)], [X()])])
+        assert L.nvfp4_quantize_layers_workspace_size(arr, 2) == 0
+        assert call([([W()], [X()]), ([W(), W(input=-1)], [X()])]) == -6
+
+
 def test_grouped_layer_order(L):
     """The grouped layer call sweeps first the batch whose order costs less:
     with the 128-expert layer's sizes, the down projections (whose input is
@@ -312,6 +340,6 @@ def test_every_launching_entry_point_opens_an_nvtx_range():
     queries = {"nvfp4_version", "nvfp4_last_cuda_error", "nvfp4_quantize_layer_order",
                "nvfp4_quantize_grouped_layer_order", "nvfp4_debug_row_counters"}
     launching = {k: v for k, v in found.items() if k not in queries}
-    assert len(launching) == 13, sorted(launching)
+    assert len(launching) == 14, sorted(launching)
     for name, first in launching.items():
         assert first == f'NVFP4_RANGE("{name}");', (name, first)

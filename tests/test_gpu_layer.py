@@ -197,3 +197,27 @@ def test_sweep_order_is_chosen_and_writes_the_same_bytes(nv):
     Wb, Xb, ib = _mlp(28672, 8192, 8192, 65536, 4)
     assert _order(nv, Wb, Xb, ib) == [0, 1, 2]
     assert _order(nv, [Wb[2], Wb[0], Wb[1]], Xb, [1, 0, 0])[0] in (1, 2)
+
+
+def test_two_layers_in_one_call(orc, nv):
+    """nvfp4_quantize_layers: two MLP layers in one call (the second layer's h
+    and S streamed beside the first layer's sweeps) write the per-step calls'
+    bytes, and every group matches the oracle fed the same h."""
+    from parity import assert_parity, check_h, compare_groups, matrix_groups, to_bits
+    layers = [_mlp(3072, 2048, 2048, 4096, 51), _mlp(3072, 2048, 2048, 4096, 61)]
+    got = nv.quantize_layers_many(layers, want_offsets=True)
+    torch.cuda.synchronize()
+    for (Ws, Xs, inputs), (outs, hs) in zip(layers, got):
+        ref, href = _per_step(nv, Ws, Xs, inputs, 448.0, -9, 6)
+        for a, b, X in zip(hs, href, Xs):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+            check_h(a.cpu().numpy(), orc.parallel_diag_hessian(X.cpu()))
+        for W, k, (c, s, S, o, st), (rc, rs, rS, ro, rst) in zip(Ws, inputs, outs, ref):
+            assert torch.equal(S.view(torch.int32), rS.view(torch.int32)) and int(st.item()) == 0
+            assert torch.equal(c, rc) and torch.equal(s, rs) and torch.equal(o, ro)
+            bits = to_bits(W)
+            h = hs[k].cpu().numpy()
+            rcodes, rscales, _ = orc.parallel_sweep_quantize(bits, h, float(S.item()), -9, 6)
+            gc, gs = c.cpu().numpy(), s.cpu().numpy()
+            w, hh, _, _ = matrix_groups(bits, gc, gs, h)
+            assert_parity(compare_groups(orc, w, hh, float(S.item()), gc, gs, rcodes, rscales))

@@ -197,6 +197,23 @@ def llama33_70b_mlp(seed_offset: int = 0) -> Workload:
     return Workload("llama33_70b_mlp", 448.0, mats, cal, [Run(-9, 6, True)])
 
 
+def llama33_70b_mlp_x2(seed_offset: int = 0, layers: int = 2) -> Workload:
+    """Consecutive Llama-3.3-70B-shaped MLP layers, quantized in one call: layer
+    0 is llama33_70b_mlp (same seeds), each further layer its own draw."""
+    mats, cal, groups = [], {}, []
+    for l in range(layers):
+        one = llama33_70b_mlp(seed_offset) if l == 0 else llama33_70b_mlp(seed_offset + 1000 * l)
+        groups.append([])
+        for m in one.matrices:
+            mats.append(Matrix(f"L{l}.{m.name}", m.out, m.inp, f"L{l}.{m.x_key}", m.seed, m.std,
+                               m.outlier_frac, m.outlier_mult))
+            groups[-1].append(mats[-1].name)
+        for k, c in one.calibs.items():
+            cal[f"L{l}.{k}"] = Calib(f"L{l}.{k}", c.tokens, c.inp, c.sigma, c.seed, c.dist)
+    return Workload(f"llama33_70b_mlp_x{layers}", 448.0, mats, cal, [Run(-9, 6, True)],
+                    extra={"layers": groups})
+
+
 def mlp_layer_slice(seed_offset: int = 0) -> Workload:
     """A whole 70B-MLP-like layer at profiling size: gate/up 8192x4096, down
     4096x8192, N(0,0.015), 0.1% x10; X 16384 tokens x {4096, 8192},
@@ -239,4 +256,4 @@ def moe_grouped(tokens: int = 262144, experts: int = 128, device="cpu") -> Workl
 
 ALL = {"single_layer": single_layer, "square_layer": square_layer, "llama3_8b": llama3_8b,
        "llama33_70b_mlp": llama33_70b_mlp, "mlp_slice": mlp_slice, "moe_grouped": moe_grouped,
-       "mlp_layer_slice": mlp_layer_slice}
+       "mlp_layer_slice": mlp_layer_slice, "llama33_70b_mlp_x2": llama33_70b_mlp_x2}
