@@ -26,7 +26,7 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
     "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "nvfp4_quantize_layer_order",
-    "quantize_layer_many", "Layer", "nvfp4_quantize_layers_workspace_size",
+    "quantize_layer_many", "nvfp4_debug_checks", "nvfp4_debug_checks_compiled", "Layer", "nvfp4_quantize_layers_workspace_size",
     "nvfp4_quantize_layers", "quantize_layers_many", "quantize_grouped_layer",
     "LayerWeight", "LayerInput", "GroupedInput", "nvfp4_quantize_grouped_layer_workspace_size",
     "nvfp4_quantize_grouped_layer", "nvfp4_quantize_grouped_layer_order",
@@ -96,6 +96,8 @@ class GroupedInput(C.Structure):
 _SIGS = {
     "nvfp4_version": ([], _int),
     "nvfp4_last_cuda_error": ([], _int),
+    "nvfp4_debug_checks_compiled": ([], _int),
+    "nvfp4_debug_checks": ([C.POINTER(C.c_ulonglong), C.POINTER(C.c_uint), _int], _int),
     "nvfp4_diag_hessian_workspace_size": ([_i64, _i64], _sz),
     "nvfp4_diag_hessian": ([_vp, _i64, _i64, _i64, _vp, _int, _vp, _sz, _vp], _int),
     "nvfp4_global_scale_workspace_size": ([_i64, _i64], _sz),
@@ -147,7 +149,9 @@ def lib(path: str | None = None):
     global _lib
     with _lock:
         if _lib is None:
-            p = path or LIB_PATH
+            # NVFP4HS_LIB selects another build of the library, e.g. the
+            # bounds-checked libnvfp4hs_checked.so next to it
+            p = path or os.environ.get("NVFP4HS_LIB") or LIB_PATH
             if not os.path.exists(p):
                 raise ImportError(f"libnvfp4hs.so not built at {p}; run __graft_entry__.build()")
             L = C.CDLL(p)
@@ -328,6 +332,20 @@ def nvfp4_quantize_grouped_layer(first, second, first_input, second_input, exper
         fa, len(first), sa, len(second), C.byref(first_input), C.byref(second_input), experts,
         float(q_max), int(lo), int(hi), _ptr(S), _ptr(amax), _ptr(status), _ptr(workspace),
         workspace_bytes, ev, _stream(stream)))
+
+
+def nvfp4_debug_checks_compiled() -> bool:
+    """Whether this build of the library checks its global accesses."""
+    return bool(lib().nvfp4_debug_checks_compiled())
+
+
+def nvfp4_debug_checks(reset: bool = False):
+    """(failed checks, first failure) of a bounds-checked build; (0, 0) for a
+    build without checks (see nvfp4_debug_checks_compiled)."""
+    first, count = C.c_ulonglong(0), C.c_uint(0)
+    _check("nvfp4_debug_checks", lib().nvfp4_debug_checks(C.byref(first), C.byref(count),
+                                                          int(bool(reset))))
+    return count.value, first.value
 
 
 def nvfp4_debug_row_counters():

@@ -4,6 +4,7 @@
 // the product of the FP32 global scale and the E4M3 local scale.  g * v is
 // exact in FP32 (at most 6 significant bits), so the one rounding is the final
 // multiply by S.  One thread per group: 9 bytes in, 64 bytes out.
+#include "checks.cuh"
 #include "nvfp4_kernels.cuh"
 
 namespace nvfp4 {
@@ -14,8 +15,9 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
   const float S = *Sp;
   for (int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; gi < ngroups;
        gi += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint2 c = *reinterpret_cast<const uint2*>(codes + gi * 8);
-    const int sc = scales[gi];
+    const uint2 c = *checked(reinterpret_cast<const uint2*>(codes + gi * 8), codes, ngroups * 8,
+                             kSiteDequantIn);
+    const int sc = *checked(scales + gi, scales, ngroups, kSiteDequantIn);
     const float v = (sc == 0 || sc > 126) ? (sc == 0 ? 0.0f : __uint_as_float(0x7FC00000u))
                                           : e4m3_value(sc);
     const uint32_t w[2] = {c.x, c.y};
@@ -31,7 +33,9 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
     }
     float4* o = reinterpret_cast<float4*>(out + gi * 16);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+    for (int i = 0; i < 4; ++i)
+      *checked(o + i, out, ngroups * 64, kSiteDequantOut) =
+          make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
   }
 }
 

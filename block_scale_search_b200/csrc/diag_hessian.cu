@@ -15,6 +15,7 @@
 //     per-lane accumulator, and writes it to partials[r, col];
 //   * a second kernel adds the R partials of each column in FP64 in a fixed
 //     order (deterministic) and rounds once to FP32.
+#include "checks.cuh"
 #include "nvfp4_kernels.cuh"
 
 namespace nvfp4 {
@@ -27,6 +28,10 @@ diag_hessian_partial_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t i
   if (tid >= R * VL) return;
   const int64_t r = tid / VL;
   const int64_t vl = tid - r * VL;
+  const int64_t xbytes = extent_bytes(T, in, ldx, 2);
+  auto ldx16 = [&](const uint16_t* p) {
+    return ld_stream_v4(checked(reinterpret_cast<const uint4*>(p), X, xbytes, kSiteDiagX));
+  };
   for (int64_t v = vl; v < V; v += VL) {
     float acc[8];
 #pragma unroll
@@ -36,7 +41,7 @@ diag_hessian_partial_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t i
     for (; t + (U - 1) * R < T; t += U * R) {
       uint4 q[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) q[u] = ld_stream_v4(col + (t + u * R) * ldx);
+      for (int u = 0; u < U; ++u) q[u] = ldx16(col + (t + u * R) * ldx);
       float s[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) s[c] = 0.0f;
@@ -54,7 +59,7 @@ diag_hessian_partial_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t i
       for (int c = 0; c < 8; ++c) acc[c] += s[c];
     }
     for (; t < T; t += R) {
-      const uint4 q = ld_stream_v4(col + t * ldx);
+      const uint4 q = ldx16(col + t * ldx);
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -64,8 +69,9 @@ diag_hessian_partial_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t i
       }
     }
     float4* dst = reinterpret_cast<float4*>(P + r * in + v * 8);
-    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    const int64_t pbytes = R * in * 4;
+    *checked(dst, P, pbytes, kSiteDiagPartial) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *checked(dst + 1, P, pbytes, kSiteDiagPartial) = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
@@ -81,14 +87,15 @@ diag_hessian_finalize_kernel(const float* __restrict__ P, int64_t R, int64_t in,
   const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + c;
   double s = 0.0;
   if (j < in)
-    for (int64_t r = g; r < R; r += 8) s += P[r * in + j];
+    for (int64_t r = g; r < R; r += 8) s += *checked(&P[r * in + j], P, R * in * 4, kSiteDiagPartial);
   part[g][c] = s;
   __syncthreads();
   if (g == 0 && j < in) {
     const double t = ((part[0][c] + part[1][c]) + (part[2][c] + part[3][c])) +
                      ((part[4][c] + part[5][c]) + (part[6][c] + part[7][c]));
-    const double base = accumulate ? static_cast<double>(h[j]) : 0.0;
-    h[j] = static_cast<float>(base + t);
+    float* hj = checked(&h[j], h, in * 4, kSiteDiagH);
+    const double base = accumulate ? static_cast<double>(*hj) : 0.0;
+    *hj = static_cast<float>(base + t);
   }
 }
 

@@ -11,6 +11,7 @@
 // non-finite input surfaces as amax >= 0x7F80 and is reported, not hidden.
 // Same lane layout as the diagonal-Hessian kernel; per-CTA maxima go to the
 // workspace and one CTA finishes the reduction and the division.
+#include "checks.cuh"
 #include "nvfp4_kernels.cuh"
 
 namespace nvfp4 {
@@ -23,6 +24,10 @@ absmax_partial_kernel(const uint16_t* __restrict__ W, int64_t rows, int64_t ldw,
                       int64_t VL, int64_t R, uint32_t* __restrict__ partial) {
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   uint32_t m = 0;
+  const int64_t wbytes = extent_bytes(rows, V * 8, ldw, 2);
+  auto ldw16 = [&](const uint16_t* p) {
+    return ld_stream_v4(checked(reinterpret_cast<const uint4*>(p), W, wbytes, kSiteAbsmaxW));
+  };
   if (tid < R * VL) {
     const int64_t r = tid / VL;
     const int64_t vl = tid - r * VL;
@@ -32,7 +37,7 @@ absmax_partial_kernel(const uint16_t* __restrict__ W, int64_t rows, int64_t ldw,
       for (; t + (U - 1) * R < rows; t += U * R) {
         uint4 q[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) q[u] = ld_stream_v4(col + (t + u * R) * ldw);
+        for (int u = 0; u < U; ++u) q[u] = ldw16(col + (t + u * R) * ldw);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           m = umax_u16x2(m, q[u].x & 0x7FFF7FFFu);
@@ -42,7 +47,7 @@ absmax_partial_kernel(const uint16_t* __restrict__ W, int64_t rows, int64_t ldw,
         }
       }
       for (; t < rows; t += R) {
-        const uint4 q = ld_stream_v4(col + t * ldw);
+        const uint4 q = ldw16(col + t * ldw);
         m = umax_u16x2(m, q.x & 0x7FFF7FFFu);
         m = umax_u16x2(m, q.y & 0x7FFF7FFFu);
         m = umax_u16x2(m, q.z & 0x7FFF7FFFu);
@@ -60,7 +65,9 @@ absmax_partial_kernel(const uint16_t* __restrict__ W, int64_t rows, int64_t ldw,
     m = threadIdx.x < (blockDim.x >> 5) ? sm[threadIdx.x] : 0u;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (threadIdx.x == 0) partial[blockIdx.x] = m;
+    if (threadIdx.x == 0)
+      *checked(partial + blockIdx.x, partial, static_cast<int64_t>(gridDim.x) * 4,
+               kSiteAbsmaxPartial) = m;
   }
 }
 
@@ -68,7 +75,9 @@ __global__ void __launch_bounds__(256)
 global_scale_finalize_kernel(const uint32_t* __restrict__ partial, int n, float q_max, float* S,
                              float* amax, int* status) {
   uint32_t m = 0;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) m = max(m, partial[i]);
+  for (int i = threadIdx.x; i < n; i += blockDim.x)
+    m = max(m, *checked(partial + i, partial, static_cast<int64_t>(n) * 4, kSiteAbsmaxPartial));
+
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   __shared__ uint32_t sm[8];

@@ -13,6 +13,7 @@
 #include <functional>
 #include <vector>
 
+#include "checks.cuh"
 #include "nvfp4_kernels.cuh"
 #include "nvtx_range.cuh"
 #include "row_counters.cuh"
@@ -130,6 +131,36 @@ int resident_ctas(const void* kernel, int threads_per_cta) {
 
 namespace nvfp4 {
 int record_cuda_status(cudaError_t e) { return cuda_status(e); }
+
+// The checked build's per-translation-unit records (checks.cuh).
+namespace {
+std::vector<cudaError_t (*)(CheckState*, bool)>& check_readers() {
+  static std::vector<cudaError_t (*)(CheckState*, bool)> v;
+  return v;
+}
+}  // namespace
+
+int register_check_reader(cudaError_t (*reader)(CheckState*, bool)) {
+  check_readers().push_back(reader);
+  return static_cast<int>(check_readers().size());
+}
+
+bool checks_compiled() {
+#ifdef NVFP4HS_CHECKS
+  return true;
+#else
+  return false;
+#endif
+}
+
+cudaError_t collect_checks(CheckState* out, bool reset) {
+  *out = CheckState{};
+  for (auto* reader : check_readers()) {
+    const cudaError_t e = reader(out, reset);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 }  // namespace nvfp4
 
 extern "C" {
@@ -137,6 +168,22 @@ extern "C" {
 int nvfp4_version(void) { return 100; }  // 0.1.0
 
 int nvfp4_last_cuda_error(void) { return g_last_cuda_error; }
+
+int nvfp4_debug_checks_compiled(void) { return nvfp4::checks_compiled() ? 1 : 0; }
+
+int nvfp4_debug_checks(unsigned long long* first, unsigned int* count, int reset) {
+  if (first == nullptr || count == nullptr || (reset != 0 && reset != 1))
+    return NVFP4_ERR_INVALID_ARG;
+  nvfp4::CheckState st{};
+  const cudaError_t e = nvfp4::collect_checks(&st, reset != 0);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_status(e);
+  }
+  *first = st.first;
+  *count = st.count;
+  return NVFP4_OK;
+}
 
 size_t nvfp4_diag_hessian_workspace_size(int64_t tokens, int64_t in) {
   if (tokens < 0 || in <= 0 || in % 8 != 0 || in > kMaxDim) return 0;

@@ -36,6 +36,7 @@
 #include <algorithm>
 #include <type_traits>
 
+#include "checks.cuh"
 #include "nvfp4_kernels.cuh"
 #include "row_counters.cuh"
 #include "side_reduce.cuh"
@@ -64,10 +65,12 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
   const ScaleConsts sc = scale_consts(*Sp);
   const int64_t half_in = G * 8;
 
+  const int64_t wbytes = extent_bytes(out, G * 16, ldw, 2);
   auto issue = [&](int64_t gg, int64_t rr, int b) {
     const uint16_t* src = W + rr * ldw + gg * 16;
-    cp_async16(&wbuf[b][0][lane], src);
-    cp_async16(&wbuf[b][1][lane], src + 8);
+    cp_async16(&wbuf[b][0][lane], checked(reinterpret_cast<const uint4*>(src), W, wbytes, kSiteSweepW));
+    cp_async16(&wbuf[b][1][lane],
+               checked(reinterpret_cast<const uint4*>(src + 8), W, wbytes, kSiteSweepW));
   };
   int buf = 0;
   if (gl < G && r0 < out) issue(gl, r0, 0);
@@ -78,7 +81,7 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
     float hs = 1.0f, hsum = 16.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) h2[i] = f2_pack(1.0f, 1.0f);
-    if constexpr (kWeighted) group_weights(h, g, h2, hs, hsum);
+    if constexpr (kWeighted) group_weights(h, g, h2, hs, hsum, G);
 
     for (int64_t r = r0; r < out; r += R) {
       const unsigned amask = __activemask();
@@ -95,10 +98,11 @@ __device__ __forceinline__ void sweep_matrix(SweepSmem<kMaxK>& sm, const uint16_
       sweep_group<kWeighted, kFull, kMaxK, kK>(
           sm, amask, cur, h2, hs, hsum, h, g, sc, lo, K, [&](uint2 c, uint8_t s, int8_t o) {
             const int64_t gi = r * G + g;
-            *reinterpret_cast<uint2*>(codes + r * half_in + g * 8) = c;
-            scales[gi] = s;
-            if (offs) offs[gi] = o;
-          });
+            *checked(reinterpret_cast<uint2*>(codes + r * half_in + g * 8), codes, out * half_in,
+                     kSiteSweepCodes) = c;
+            *checked(scales + gi, scales, out * G, kSiteSweepScales) = s;
+            if (offs) *checked(offs + gi, offs, out * G, kSiteSweepOffs) = o;
+          }, G);
     }
   }
   cp_async_wait<0>();
@@ -130,16 +134,18 @@ __device__ __forceinline__ void sweep_rows_dynamic(SweepSmem<16>& sm, const uint
   const int lane = threadIdx.x;
   const ScaleConsts sc = scale_consts(*Sp);
   const int64_t half_in = G * 8;
+  const int64_t wbytes = extent_bytes(out, G * 16, ldw, 2);
   auto issue = [&](int64_t rr, int b) {
     const uint16_t* src = W + rr * ldw + g * 16;
-    cp_async16(&wbuf[b][0][lane], src);
-    cp_async16(&wbuf[b][1][lane], src + 8);
+    cp_async16(&wbuf[b][0][lane], checked(reinterpret_cast<const uint4*>(src), W, wbytes, kSiteSweepW));
+    cp_async16(&wbuf[b][1][lane],
+               checked(reinterpret_cast<const uint4*>(src + 8), W, wbytes, kSiteSweepW));
   };
   f32x2_t h2[8];
   float hs = 1.0f, hsum = 16.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) h2[i] = f2_pack(1.0f, 1.0f);
-  if constexpr (kWeighted) group_weights(h, g, h2, hs, hsum);
+  if constexpr (kWeighted) group_weights(h, g, h2, hs, hsum, G);
   // rows fit in 32 bits here (out <= 2^23), which keeps the loop's state small
   int r = static_cast<int>(r0) * kRowChunk;
   int end = r + kRowChunk;
@@ -164,10 +170,11 @@ __device__ __forceinline__ void sweep_rows_dynamic(SweepSmem<16>& sm, const uint
     sweep_group<kWeighted, false, 16, kK>(
         sm, 0xFFFFFFFFu, cur, h2, hs, hsum, h, g, sc, lo, K, [&](uint2 cw, uint8_t sb, int8_t o) {
           const int64_t gi = static_cast<int64_t>(r) * G + g;
-          *reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * half_in + g * 8) = cw;
-          scales[gi] = sb;
-          if (offs) offs[gi] = o;
-        });
+          *checked(reinterpret_cast<uint2*>(codes + static_cast<int64_t>(r) * half_in + g * 8),
+                   codes, out * half_in, kSiteSweepCodes) = cw;
+          *checked(scales + gi, scales, out * G, kSiteSweepScales) = sb;
+          if (offs) *checked(offs + gi, offs, out * G, kSiteSweepOffs) = o;
+        }, G);
     r = nr;
   }
   cp_async_wait<0>();

@@ -37,6 +37,7 @@
 //     being a tie to the even code.
 #pragma once
 
+#include "checks.cuh"
 #include "nvfp4_device.cuh"
 
 namespace nvfp4 {
@@ -151,13 +152,14 @@ __device__ __forceinline__ float weight_scale(float hmax) {
 // The group's weights h' = h * hs as eight pairs, hs from weight_scale, and
 // their sum (which bounds sum h' y^2 by sum h' * max y^2 for the guard).
 __device__ __forceinline__ void group_weights(const float* __restrict__ h, int64_t g,
-                                              f32x2_t (&h2)[8], float& hs, float& hsum) {
+                                              f32x2_t (&h2)[8], float& hs, float& hsum,
+                                              int64_t G = 0) {
   const float4* hp = reinterpret_cast<const float4*>(h + g * 16);
   float4 hv[4];
   float hmax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    hv[i] = hp[i];
+    hv[i] = *checked(hp + i, h, G * 64, kSiteSweepH);
     hmax = fmaxf(fmaxf(fmaxf(hmax, hv[i].x), fmaxf(hv[i].y, hv[i].z)), hv[i].w);
   }
   hs = weight_scale(hmax);
@@ -303,7 +305,8 @@ template <bool kWeighted, bool kFull, int kMaxK, int kK, int kThreads, typename 
 __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK, kThreads>& sm, unsigned amask, int cur,
                                             const f32x2_t (&h2)[8], float hs, float hsum,
                                             const float* __restrict__ h, int64_t g,
-                                            const ScaleConsts& sc, int lo, int K, Store&& store) {
+                                            const ScaleConsts& sc, int lo, int K, Store&& store,
+                                            int64_t G = 0) {
   const CandEntry* tab = sm.tab;
   auto& Lsm = sm.Lsm;
   auto& wbuf = sm.wbuf;
@@ -442,7 +445,8 @@ __device__ __forceinline__ void sweep_group(SweepSmem<kMaxK, kThreads>& sm, unsi
           const uint32_t word = wf[((j >> 3) * kThreads + tx) * 4 + ((j >> 1) & 3)];
           const float aj = fabsf((j & 1) ? bf16_hi(word) : bf16_lo(word));
           const float yj = (sc.tiny_s ? aj * sc.p : aj) * sc.inv_sp;
-          const float hj = kWeighted ? h[g_f * 16 + j] * hs_f : 1.0f;
+          const float hj = kWeighted ? *checked(&h[g_f * 16 + j], h, G * 64, kSiteSweepH) * hs_f
+                                     : 1.0f;
           const uint32_t k = exact_e2m1_one(yj * ivl, aj, t.v, S);
           const double q = static_cast<double>(e2m1_nibble_value(k));
           const double d = fma(-q, vS, static_cast<double>(aj));  // exact

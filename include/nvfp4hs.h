@@ -61,6 +61,20 @@ typedef enum nvfp4_status {
 /* Library version (major*10000 + minor*100 + patch). */
 int nvfp4_version(void);
 
+/* Bounds checks (debugging aid; no counterpart on the pages).  A library built
+ * with -DNVFP4HS_CHECKS checks every global-memory address of the per-step
+ * kernels (diagonal Hessian, global scale, sweep, dequantize) against the
+ * extent of its buffer that the call's size arguments imply; an address
+ * outside is counted, the first is recorded, and the access goes to a dummy
+ * buffer instead (no fault, no write to memory the call does not own).
+ * nvfp4_debug_checks_compiled() is 1 in such a build, 0 otherwise.
+ * nvfp4_debug_checks() synchronises with the device, writes the number of
+ * failed checks and the first one ((site << 48) | (byte offset + 1); 0 when
+ * none), and clears them if reset is 1; in a build without checks it writes
+ * zeros. */
+int nvfp4_debug_checks_compiled(void);
+int nvfp4_debug_checks(unsigned long long* first, unsigned int* count, int reset);
+
 /* The cudaError_t behind the calling thread's most recent NVFP4_ERR_CUDA. */
 int nvfp4_last_cuda_error(void);
 

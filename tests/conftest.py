@@ -17,6 +17,21 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: full-size workload checks")
 
 
+def pytest_sessionfinish(session, exitstatus):
+    """Under a bounds-checked build of the library (NVFP4HS_LIB pointing at
+    libnvfp4hs_checked.so), a run with any failed check fails."""
+    import os
+    if not os.environ.get("NVFP4HS_LIB"):
+        return
+    import block_scale_search_b200 as nv
+    if nv._lib is None or not nv.lib().nvfp4_debug_checks_compiled():
+        return
+    count, first = nv.nvfp4_debug_checks()
+    _REPORT.append(f"bounds checks: {count} failed (first record {first:#x})")
+    if count:
+        session.exitstatus = 1
+
+
 def pytest_terminal_summary(terminalreporter):
     if _REPORT:
         terminalreporter.section("parity per matrix")

@@ -338,8 +338,26 @@ def test_every_launching_entry_point_opens_an_nvtx_range():
         for m in re.finditer(r"\n(?:extern \"C\" )?int (nvfp4_\w+)\((?:.|\n)*?\) \{\n(.*)\n", src):
             found[m.group(1)] = m.group(2).strip()
     queries = {"nvfp4_version", "nvfp4_last_cuda_error", "nvfp4_quantize_layer_order",
+               "nvfp4_debug_checks_compiled", "nvfp4_debug_checks",
                "nvfp4_quantize_grouped_layer_order", "nvfp4_debug_row_counters"}
     launching = {k: v for k, v in found.items() if k not in queries}
     assert len(launching) == 14, sorted(launching)
     for name, first in launching.items():
         assert first == f'NVFP4_RANGE("{name}");', (name, first)
+
+
+def test_checked_build_loads_and_exports_the_same_entry_points():
+    """The bounds-checked variant is built beside the library (CPU compile),
+    exports every entry point the header declares, and says which it is."""
+    import ctypes as C
+    from block_scale_search_b200 import _build
+    path = _build.build(checked=True)
+    Lc = C.CDLL(path)
+    Lp = C.CDLL(_build.LIB)
+    for name in declared_functions():
+        assert hasattr(Lc, name), name
+    assert Lc.nvfp4_debug_checks_compiled() == 1 and Lp.nvfp4_debug_checks_compiled() == 0
+    first, count = C.c_ulonglong(7), C.c_uint(7)
+    assert Lp.nvfp4_debug_checks(C.byref(first), C.byref(count), 0) == 0
+    assert first.value == 0 and count.value == 0            # nothing recorded without checks
+    assert Lp.nvfp4_debug_checks(None, C.byref(count), 0) == -1
