@@ -81,6 +81,15 @@ def lib():
             L.orc_quantize_activations.restype = C.c_int
             L.orc_dequantize.argtypes = [u8p, u8p, C.c_float, i64, i64, f32p]
             L.orc_dequantize.restype = None
+            L.orc_sweep_group_f32_list.argtypes = [f32p, f32p, i64, C.c_float, C.c_int, C.c_int,
+                                                   u8p, u8p, i8p, f64p]
+            L.orc_sweep_group_f32_list.restype = None
+            L.orc_group_loss_f32.argtypes = [f32p, f32p, C.c_float, C.c_int]
+            L.orc_group_loss_f32.restype = C.c_double
+            L.orc_base_code_f32.argtypes = [f32p, C.c_float]
+            L.orc_base_code_f32.restype = C.c_int
+            L.orc_e2m1_quantize_list.argtypes = [f32p, f64p, i64, u8p]
+            L.orc_e2m1_quantize_list.restype = None
             _lib = L
     return _lib
 
@@ -242,6 +251,38 @@ def dequantize(codes, scales, S: float) -> np.ndarray:
     lib().orc_dequantize(_p(codes, C.c_uint8), _p(scales, C.c_uint8), float(S), o, half * 2,
                          _p(out, C.c_float))
     return out
+
+
+def sweep_group_f32_list(w, h, S: float, lo: int, hi: int):
+    """The windowed sweep of n FP32 groups w[n,16] (h[n,16] or None): (codes
+    [n,8], scales [n], offsets [n], losses [n])."""
+    w = np.ascontiguousarray(w, dtype=np.float32).reshape(-1, 16)
+    n = w.shape[0]
+    h = None if h is None else np.ascontiguousarray(h, dtype=np.float32).reshape(n, 16)
+    codes = np.zeros((n, 8), np.uint8)
+    scales = np.zeros(n, np.uint8)
+    offs = np.zeros(n, np.int8)
+    loss = np.zeros(n, np.float64)
+    lib().orc_sweep_group_f32_list(_p(w, C.c_float), None if h is None else _p(h, C.c_float), n,
+                                   float(S), int(lo), int(hi), _p(codes, C.c_uint8),
+                                   _p(scales, C.c_uint8), _p(offs, C.c_int8),
+                                   _p(loss, C.c_double))
+    return codes, scales, offs, loss
+
+
+def group_loss_f32(w, h, S: float, code: int) -> float:
+    w = np.ascontiguousarray(w, dtype=np.float32).reshape(16)
+    hp = None if h is None else _p(np.ascontiguousarray(h, dtype=np.float32).reshape(16), C.c_float)
+    return lib().orc_group_loss_f32(_p(w, C.c_float), hp, float(S), int(code))
+
+
+def e2m1_quantize_list(w, vS) -> np.ndarray:
+    """Nibbles of FP32 values w[n] at their own exact scales vS[n] (0: nibble 0)."""
+    w = np.ascontiguousarray(w, dtype=np.float32).reshape(-1)
+    vS = np.ascontiguousarray(vS, dtype=np.float64).reshape(-1)
+    nib = np.zeros(w.size, np.uint8)
+    lib().orc_e2m1_quantize_list(_p(w, C.c_float), _p(vS, C.c_double), w.size, _p(nib, C.c_uint8))
+    return nib
 
 
 # ---------------------------------------------------------- threaded drivers

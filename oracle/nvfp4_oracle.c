@@ -72,19 +72,48 @@ static int bf16_is_finite(uint16_t b) { return (b & 0x7F80u) != 0x7F80u; }
 
 /* ---- objective ---------------------------------------------------------- */
 
-double orc_group_loss(const uint16_t* w, const float* h, float S, int code) {
+/* The loss of a group given its 16 magnitudes a[j] (exact doubles of bf16 or
+ * FP32 values). */
+static double group_loss_abs(const double* a, const float* h, float S, int code) {
     double v = orc_e4m3_value(code);
     if (v < 0.0) return NAN;
     double vS = v * (double)S;                         /* exact: 4 x 24 bits */
     double L = 0.0;
     for (int j = 0; j < 16; ++j) {
-        double a = fabs(bf16_to_double(w[j]));
-        double q = (vS > 0.0) ? kGrid[orc_e2m1_index(a, vS)] : 0.0;
-        double d = a - q * vS;                         /* exact */
+        double q = (vS > 0.0) ? kGrid[orc_e2m1_index(a[j], vS)] : 0.0;
+        double d = a[j] - q * vS;                      /* exact: a and q*vS within a factor 2 */
         double hj = h ? (double)h[j] : 1.0;
         L += hj * (d * d);
     }
     return L;
+}
+
+static void abs_bf16(const uint16_t* w, double* a, int* neg) {
+    for (int j = 0; j < 16; ++j) {
+        a[j] = fabs(bf16_to_double(w[j]));
+        neg[j] = (w[j] & 0x8000u) != 0;
+    }
+}
+
+static void abs_f32(const float* w, double* a, int* neg) {
+    for (int j = 0; j < 16; ++j) {
+        a[j] = fabs((double)w[j]);
+        neg[j] = signbit(w[j]) != 0;
+    }
+}
+
+double orc_group_loss(const uint16_t* w, const float* h, float S, int code) {
+    double a[16];
+    int neg[16];
+    abs_bf16(w, a, neg);
+    return group_loss_abs(a, h, S, code);
+}
+
+double orc_group_loss_f32(const float* w, const float* h, float S, int code) {
+    double a[16];
+    int neg[16];
+    abs_f32(w, a, neg);
+    return group_loss_abs(a, h, S, code);
 }
 
 /* ---- calibration statistic: diagonal Hessian ----------------------------- */
@@ -131,12 +160,12 @@ int orc_global_scale(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
 
 /* ---- the windowed scale sweep ------------------------------------------- */
 
-int orc_base_code(const uint16_t* w, float S) {
+/* Base code from the group's magnitudes; a[j] are exact values of FP32 (or
+ * bf16) numbers, so their maximum is an FP32 value. */
+static int base_code_abs(const double* a16, float S) {
     double a = 0.0;
-    for (int j = 0; j < 16; ++j) {
-        double x = fabs(bf16_to_double(w[j]));
-        if (x > a) a = x;
-    }
+    for (int j = 0; j < 16; ++j)
+        if (a16[j] > a) a = a16[j];
     if (a == 0.0) return 0;
     float t = (float)a / 6.0f;                         /* fl32(a / 6) */
     float u = t / S;                                   /* fl32(. / S) */
@@ -146,11 +175,25 @@ int orc_base_code(const uint16_t* w, float S) {
     return b;
 }
 
+int orc_base_code(const uint16_t* w, float S) {
+    double a[16];
+    int neg[16];
+    abs_bf16(w, a, neg);
+    return base_code_abs(a, S);
+}
+
+int orc_base_code_f32(const float* w, float S) {
+    double a[16];
+    int neg[16];
+    abs_f32(w, a, neg);
+    return base_code_abs(a, S);
+}
+
 static int clamp_code(int c) { return c < 1 ? 1 : (c > 126 ? 126 : c); }
 
-void orc_sweep_group(const uint16_t* w, const float* h, float S, int lo, int hi,
-                     uint8_t* codes8, uint8_t* scale, int8_t* offset, double* loss) {
-    int b = orc_base_code(w, S);
+static void sweep_group_abs(const double* a, const int* neg, const float* h, float S, int lo,
+                            int hi, uint8_t* codes8, uint8_t* scale, int8_t* offset, double* loss) {
+    int b = base_code_abs(a, S);
     uint8_t nib[16];
     if (b == 0) {                                      /* all-zero group */
         if (codes8) memset(codes8, 0, 8);
@@ -163,21 +206,54 @@ void orc_sweep_group(const uint16_t* w, const float* h, float S, int lo, int hi,
     int bc = b, bk = 0;
     for (int k = lo; k <= hi; ++k) {                   /* ascending offsets */
         int c = clamp_code(b + k);
-        double L = orc_group_loss(w, h, S, c);
+        double L = group_loss_abs(a, h, S, c);
         if (L < best) { best = L; bc = c; bk = k; }    /* strict: ties keep lowest offset */
     }
     double vS = orc_e4m3_value(bc) * (double)S;
     for (int j = 0; j < 16; ++j) {
-        double x = bf16_to_double(w[j]);
-        int k = orc_e2m1_index(fabs(x), vS);
-        int neg = (w[j] & 0x8000u) != 0;
-        nib[j] = (uint8_t)((k != 0 && neg) ? (8 | k) : k);
+        int k = orc_e2m1_index(a[j], vS);
+        nib[j] = (uint8_t)((k != 0 && neg[j]) ? (8 | k) : k);
     }
     if (codes8)
         for (int i = 0; i < 8; ++i) codes8[i] = (uint8_t)(nib[2 * i] | (nib[2 * i + 1] << 4));
     if (scale) *scale = (uint8_t)bc;
     if (offset) *offset = (int8_t)bk;
     if (loss) *loss = best;
+}
+
+void orc_sweep_group(const uint16_t* w, const float* h, float S, int lo, int hi,
+                     uint8_t* codes8, uint8_t* scale, int8_t* offset, double* loss) {
+    double a[16];
+    int neg[16];
+    abs_bf16(w, a, neg);
+    sweep_group_abs(a, neg, h, S, lo, hi, codes8, scale, offset, loss);
+}
+
+void orc_sweep_group_f32(const float* w, const float* h, float S, int lo, int hi,
+                         uint8_t* codes8, uint8_t* scale, int8_t* offset, double* loss) {
+    double a[16];
+    int neg[16];
+    abs_f32(w, a, neg);
+    sweep_group_abs(a, neg, h, S, lo, hi, codes8, scale, offset, loss);
+}
+
+void orc_sweep_group_f32_list(const float* w, const float* h, int64_t n, float S, int lo, int hi,
+                              uint8_t* codes, uint8_t* scales, int8_t* offsets, double* losses) {
+    for (int64_t i = 0; i < n; ++i)
+        orc_sweep_group_f32(w + 16 * i, h ? h + 16 * i : NULL, S, lo, hi, codes + 8 * i,
+                            scales + i, offsets ? offsets + i : NULL, losses ? losses + i : NULL);
+}
+
+/* E2M1 nibbles (sign << 3 | magnitude index; +0 for a zero magnitude) of n FP32
+ * values w[i], each at its own scale vS[i] > 0 (an exact double); vS[i] == 0
+ * gives nibble 0.  The quantization step of a quantizer that has already chosen
+ * its scales, e.g. inside GPTQ's column loop. */
+void orc_e2m1_quantize_list(const float* w, const double* vS, int64_t n, uint8_t* nib) {
+    for (int64_t i = 0; i < n; ++i) {
+        if (!(vS[i] > 0.0)) { nib[i] = 0; continue; }
+        int k = orc_e2m1_index(fabs((double)w[i]), vS[i]);
+        nib[i] = (uint8_t)((k != 0 && signbit(w[i])) ? (8 | k) : k);
+    }
 }
 
 void orc_sweep_quantize(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,

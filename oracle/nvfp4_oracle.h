@@ -85,6 +85,21 @@ int orc_base_code(const uint16_t* w_bf16, float S);
 void orc_sweep_group(const uint16_t* w_bf16, const float* h, float S, int lo, int hi,
                      uint8_t* codes8, uint8_t* scale, int8_t* offset, double* loss);
 
+/* FP32-input forms, for quantizers whose weights are FP32 values rather than
+ * bf16 -- GPTQ's error-updated columns ([H-Scale] sec. B "GPTQ Integration":
+ * H-Scale replaces GPTQ's local quantization call).  The same definitions with
+ * w_j an FP32 number: exact E2M1 decisions, base code from fl32(fl32(a/6)/S),
+ * loss in double. */
+double orc_group_loss_f32(const float* w, const float* h, float S, int code);
+int orc_base_code_f32(const float* w, float S);
+void orc_sweep_group_f32(const float* w, const float* h, float S, int lo, int hi,
+                         uint8_t* codes8, uint8_t* scale, int8_t* offset, double* loss);
+void orc_sweep_group_f32_list(const float* w, const float* h, int64_t n, float S, int lo, int hi,
+                              uint8_t* codes, uint8_t* scales, int8_t* offsets, double* losses);
+/* Nibbles of n FP32 values, each at an already chosen scale vS[i] (exact
+ * double; 0 gives nibble 0). */
+void orc_e2m1_quantize_list(const float* w, const double* vS, int64_t n, uint8_t* nib);
+
 /* Whole matrix: W[out, in] bf16 row stride ldw, h[in] or NULL.
  * codes[out, in/2], scales[out, in/16], offsets[out, in/16] (NULL allowed). */
 void orc_sweep_quantize(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,

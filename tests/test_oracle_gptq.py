@@ -1,0 +1,112 @@
+"""Pins of the GPTQ oracle with the H-Scale local call (H-Scale summary, sec. B
+"GPTQ Integration"): each checks it against something other than itself --
+the standalone sweep where GPTQ has nothing to propagate, the bf16 oracle on
+values both can hold, the damped least-squares re-fit that GPTQ's update is,
+and the expected gain on correlated inputs."""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import gptq
+
+
+def _w(out, n, seed, frac=0.01):
+    import workloads
+    return workloads.weight(out, n, 0.02, frac, 10.0, seed)
+
+
+def test_uncorrelated_inputs_reduce_to_the_sweep():
+    """X = 2 I: H = 4 I, U is diagonal, nothing propagates, and GPTQ with the
+    local call is the standalone windowed sweep with h = 4."""
+    import torch
+    n = 256
+    W = _w(96, n, 1)
+    X = (2.0 * torch.eye(n)).to(torch.bfloat16)
+    codes, scales, S, _, h = gptq.gptq_hscale(W, X, lo=-9, hi=6)
+    assert np.all(h == 4.0)
+    rc, rs, _ = oracle.sweep_quantize(W, h, float(S), -9, 6)
+    np.testing.assert_array_equal(scales, rs)
+    np.testing.assert_array_equal(codes, rc)
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+def test_fp32_local_call_equals_the_bf16_sweep_on_bf16_values(weighted):
+    rng = np.random.default_rng(3)
+    W = _w(200, 512, 4, frac=0.02)
+    bits = oracle._bf16_bits(W).reshape(-1, 16)
+    bits[5] = 0                                     # an all-zero group
+    bits[6, :8] = 0x8000                            # negative zeros
+    h = rng.lognormal(0.0, 1.5, size=bits.shape).astype(np.float32) if weighted else None
+    S = float(oracle.global_scale(bits.reshape(200, 512), 448.0)[0])
+    rc, rs, ro, rl = oracle.sweep_groups(bits, h, S, -9, 6)
+    f = gptq.bf16_to_f64(bits).astype(np.float32)
+    fc, fs, fo, fl = oracle.sweep_group_f32_list(f, h, S, -9, 6)
+    np.testing.assert_array_equal(fc, rc)
+    np.testing.assert_array_equal(fs, rs)
+    np.testing.assert_array_equal(fo, ro)
+    np.testing.assert_array_equal(fl, rl)
+
+
+def test_propagation_is_the_damped_least_squares_refit():
+    """After column j, GPTQ's remaining columns minimise the damped output
+    error with the quantized columns held fixed: V = W_> + A H_<> H_>>^-1,
+    A = W_<= - Q_<=, computed here by a linear solve on the damped H (no
+    Cholesky, no inverse)."""
+    import torch
+    import workloads
+    n = 64
+    W = _w(12, n, 7)
+    Z = workloads.calib(200, n, 1.0, 8).float()
+    X = (Z @ (torch.eye(n) + 0.3 * torch.randn(n, n, generator=torch.Generator().manual_seed(9)))
+         ).to(torch.bfloat16)
+    _, _, Hd = gptq.inverse_cholesky_upper(oracle._bf16_bits(X))
+    W0 = gptq.bf16_to_f64(oracle._bf16_bits(W))
+    seen = []
+
+    def trace(j, Wc, Q):
+        if j in (0, 5, 15, 16, 40, 62):
+            A = W0[:, :j + 1] - Q[:, :j + 1]
+            V = W0[:, j + 1:] + np.linalg.solve(Hd[j + 1:, j + 1:], (A @ Hd[:j + 1, j + 1:]).T).T
+            np.testing.assert_allclose(Wc[:, j + 1:], V, rtol=1e-9, atol=1e-12)
+            seen.append(j)
+
+    gptq.gptq_hscale(W, X, trace=trace)
+    assert seen == [0, 5, 15, 16, 40, 62]
+
+
+@pytest.mark.parametrize("seed", [11, 12, 13])
+def test_correlated_inputs_lower_the_output_error(seed):
+    """On inputs with correlated channels GPTQ's propagation lowers the layer
+    output error below the standalone sweep's (the reason to combine them)."""
+    import torch
+    import workloads
+    n = 128
+    W = _w(64, n, seed)
+    Z = workloads.calib(512, n, 1.0, seed + 100).float()
+    mix = torch.eye(n) + 0.5 * torch.randn(n, n, generator=torch.Generator().manual_seed(seed))
+    X = (Z @ mix).to(torch.bfloat16)
+    codes, scales, S, Q, h = gptq.gptq_hscale(W, X)
+    rc, rs, _ = oracle.sweep_quantize(W, h, float(S), -9, 6)
+    nib = np.stack([rc & 15, rc >> 4], -1).reshape(64, n)
+    Qr = gptq.decode(nib, np.repeat(rs, 16, 1), float(S))
+    Wf = gptq.bf16_to_f64(oracle._bf16_bits(W))
+    Xf = gptq.bf16_to_f64(oracle._bf16_bits(X))
+    e_gptq = np.sum((Xf @ (Wf - Q).T) ** 2)
+    e_sweep = np.sum((Xf @ (Wf - Qr).T) ** 2)
+    assert e_gptq < 0.95 * e_sweep, (e_gptq, e_sweep)
+    # what the codes decode to is what GPTQ reconstructed
+    qn = np.stack([codes & 15, codes >> 4], -1).reshape(64, n)
+    np.testing.assert_array_equal(gptq.decode(qn, np.repeat(scales, 16, 1), float(S)), Q)
+
+
+def test_dead_columns_quantize_to_zero():
+    import workloads
+    n = 64
+    W = _w(32, n, 21)
+    X = workloads.calib(100, n, 1.0, 22)
+    X[:, 17] = 0
+    X[:, 40:48] = 0
+    codes, scales, S, Q, h = gptq.gptq_hscale(W, X)
+    assert np.all(Q[:, 17] == 0) and np.all(Q[:, 40:48] == 0)
+    nib = np.stack([codes & 15, codes >> 4], -1).reshape(32, n)
+    assert np.all(nib[:, 17] == 0) and np.all(nib[:, 40:48] == 0)
