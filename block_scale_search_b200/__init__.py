@@ -26,7 +26,8 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_batched", "MatrixDesc", "SweepDesc",
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
     "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "nvfp4_quantize_layer_order",
-    "quantize_layer_many", "nvfp4_debug_checks", "nvfp4_debug_checks_compiled", "Layer", "nvfp4_quantize_layers_workspace_size",
+    "quantize_layer_many", "nvfp4_gptq_workspace_size", "nvfp4_gptq_quantize", "gptq_quantize",
+    "nvfp4_scale_sweep_quantize_f32", "scale_sweep_quantize_f32", "nvfp4_debug_checks", "nvfp4_debug_checks_compiled", "Layer", "nvfp4_quantize_layers_workspace_size",
     "nvfp4_quantize_layers", "quantize_layers_many", "quantize_grouped_layer",
     "LayerWeight", "LayerInput", "GroupedInput", "nvfp4_quantize_grouped_layer_workspace_size",
     "nvfp4_quantize_grouped_layer", "nvfp4_quantize_grouped_layer_order",
@@ -39,7 +40,8 @@ __all__ = [
 
 STATUS = {0: "NVFP4_OK", -1: "NVFP4_ERR_INVALID_ARG", -2: "NVFP4_ERR_SHAPE",
           -3: "NVFP4_ERR_ALIGN", -4: "NVFP4_ERR_WINDOW", -5: "NVFP4_ERR_NONFINITE",
-          -6: "NVFP4_ERR_CUDA", -7: "NVFP4_ERR_WORKSPACE", -8: "NVFP4_ERR_CAPTURE"}
+          -6: "NVFP4_ERR_CUDA", -7: "NVFP4_ERR_WORKSPACE", -8: "NVFP4_ERR_CAPTURE",
+          -9: "NVFP4_ERR_NUMERIC"}
 
 
 class NVFP4Error(RuntimeError):
@@ -126,6 +128,11 @@ _SIGS = {
     "nvfp4_quantize_layers": ([C.POINTER(Layer), _int, _f32, _int, _int, _vp, _sz, C.POINTER(_vp),
                                _vp], _int),
     "nvfp4_dequantize": ([_vp, _vp, _vp, _i64, _i64, _vp, _vp], _int),
+    "nvfp4_gptq_workspace_size": ([_i64, _i64, _i64], _sz),
+    "nvfp4_gptq_quantize": ([_vp, _i64, _i64, _i64, _vp, _i64, _i64, _f32, _int, _int, _f32, _int,
+                             _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
+    "nvfp4_scale_sweep_quantize_f32": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp],
+                                       _int),
     "nvfp4_blocked_scales_size": ([_i64, _i64], _sz),
     "nvfp4_scales_to_blocked": ([_vp, _i64, _i64, _i64, _vp, _vp], _int),
     "nvfp4_quantize_activations": ([_vp, _i64, _i64, _i64, _f32, _int, _int, _vp, _vp, _vp, _vp,
@@ -332,6 +339,24 @@ def nvfp4_quantize_grouped_layer(first, second, first_input, second_input, exper
         fa, len(first), sa, len(second), C.byref(first_input), C.byref(second_input), experts,
         float(q_max), int(lo), int(hi), _ptr(S), _ptr(amax), _ptr(status), _ptr(workspace),
         workspace_bytes, ev, _stream(stream)))
+
+
+def nvfp4_gptq_workspace_size(out: int, inp: int, tokens: int) -> int:
+    return lib().nvfp4_gptq_workspace_size(out, inp, tokens)
+
+
+def nvfp4_gptq_quantize(W, out, inp, ldw, X, tokens, ldx, q_max, lo, hi, damp, weighted, codes,
+                        scales, S, h, status, workspace, workspace_bytes, stream=None):
+    _check("nvfp4_gptq_quantize", lib().nvfp4_gptq_quantize(
+        _ptr(W), out, inp, ldw, _ptr(X), tokens, ldx, float(q_max), int(lo), int(hi), float(damp),
+        int(bool(weighted)), _ptr(codes), _ptr(scales), _ptr(S), _ptr(h), _ptr(status),
+        _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def nvfp4_scale_sweep_quantize_f32(W, out, inp, ldw, h, S, lo, hi, codes, scales, stream=None):
+    _check("nvfp4_scale_sweep_quantize_f32", lib().nvfp4_scale_sweep_quantize_f32(
+        _ptr(W), out, inp, ldw, _ptr(h), _ptr(S), int(lo), int(hi), _ptr(codes), _ptr(scales),
+        _stream(stream)))
 
 
 def nvfp4_debug_checks_compiled() -> bool:
@@ -626,6 +651,41 @@ def quantize_grouped_layer(first, second, first_input, second_input, row_offsets
     nvfp4_quantize_grouped_layer(descs[0], descs[1], x1, x2, E, q_max, lo, hi, S, amax, status,
                                  ws, nb, stream=stream)
     return outs[0], outs[1], h1, h2, S, amax, status
+
+
+def gptq_quantize(W: torch.Tensor, X: torch.Tensor, q_max: float = 448.0, lo: int = -9, hi: int = 6,
+                  damp: float = 0.01, weighted: bool = True, stream=None):
+    """GPTQ with the H-Scale local call (nvfp4_gptq_quantize).  Returns (codes,
+    scales, S, h, status)."""
+    W = _bf16_2d(W, "W")
+    X = _bf16_2d(X, "X")
+    o, n = W.shape
+    dev = W.device
+    codes = torch.empty(o, n // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(o, n // 16, dtype=torch.uint8, device=dev)
+    S = torch.empty(1, dtype=torch.float32, device=dev)
+    h = torch.empty(n, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nb = nvfp4_gptq_workspace_size(o, n, X.shape[0])
+    if nb == 0:
+        raise NVFP4Error("nvfp4_gptq_workspace_size", -1)
+    ws = torch.empty(nb + 256, dtype=torch.uint8, device=dev)
+    base = (-ws.data_ptr()) % 256
+    nvfp4_gptq_quantize(W, o, n, W.stride(0), X, X.shape[0], X.stride(0), q_max, lo, hi, damp,
+                        weighted, codes, scales, S, h, status, ws[base:base + nb], nb, stream)
+    return codes, scales, S, h, status
+
+
+def scale_sweep_quantize_f32(W: torch.Tensor, h: torch.Tensor | None, S: torch.Tensor,
+                             lo: int = -9, hi: int = 6, stream=None):
+    """The windowed sweep of an FP32 matrix (GPTQ's local call on its own)."""
+    if W.dtype != torch.float32 or W.dim() != 2 or W.stride(1) != 1:
+        raise ValueError("W must be a 2-D float32 CUDA tensor with unit inner stride")
+    o, n = W.shape
+    codes = torch.empty(o, n // 2, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(o, n // 16, dtype=torch.uint8, device=W.device)
+    nvfp4_scale_sweep_quantize_f32(W, o, n, W.stride(0), h, S, lo, hi, codes, scales, stream)
+    return codes, scales
 
 
 def quantize_layers_many(layers, q_max: float = 448.0, lo: int = -9, hi: int = 6,

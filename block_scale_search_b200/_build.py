@@ -22,6 +22,11 @@ NVCC_FLAGS = [
 ]
 
 
+# GEMMs (X^T X and GPTQ's batch updates) and the Cholesky factorizations of
+# the GPTQ path come from cuBLAS and cuSOLVER
+LIBS = ["-lcublas", "-lcusolver"]
+
+
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
@@ -41,7 +46,7 @@ def build(force: bool = False, verbose: bool = False, checked: bool = False) -> 
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc, *NVCC_FLAGS, *(["-DNVFP4HS_CHECKS"] if checked else []), "-I", INCLUDE, "-I",
-           CSRC, *sources(), "-o", tmp]
+           CSRC, *sources(), *LIBS, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)

@@ -162,6 +162,18 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               int64_t out, int64_t in, float* W_out, int num_sms,
                               cudaStream_t stream);
 
+// H-Scale as GPTQ's local quantizer (gptq.cu).
+size_t gptq_workspace_bytes(int64_t out, int64_t in, int64_t tokens, int sms);
+cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw, const uint16_t* X,
+                        int64_t tokens, int64_t ldx, float q_max, int lo, int hi, float damp,
+                        bool weighted, uint8_t* codes, uint8_t* scales, float* S, float* h,
+                        int* status, void* workspace, size_t workspace_bytes, int sms,
+                        cudaStream_t stream);
+// The windowed sweep of an FP32 matrix (GPTQ's local call on its own).
+cudaError_t launch_sweep_f32(const float* W, int64_t out, int64_t in, int64_t ldw, const float* h,
+                             const float* S, int lo, int hi, uint8_t* codes, uint8_t* scales,
+                             int num_sms, cudaStream_t stream);
+
 // Maps a CUDA error to the entry points' status: NVFP4_OK for cudaSuccess,
 // otherwise NVFP4_ERR_CUDA, with the code kept for nvfp4_last_cuda_error()
 // (per host thread).  Defined with the entry points in nvfp4hs_capi.cu.

@@ -296,6 +296,67 @@ int flatten_layers(const nvfp4_layer* layers, int n_layers, std::vector<nvfp4_la
 
 extern "C" {
 
+size_t nvfp4_gptq_workspace_size(int64_t out, int64_t in, int64_t tokens) {
+  if (out <= 0 || in <= 0 || tokens < 0 || in % 16 != 0 || in >= (int64_t{1} << 31) ||
+      out > kMaxDim || tokens > kMaxDim)
+    return 0;
+  const int sms = current_sm_count();
+  if (sms <= 0) return 0;
+  return nvfp4::gptq_workspace_bytes(out, in, tokens, sms);
+}
+
+int nvfp4_gptq_quantize(const void* W, int64_t out, int64_t in, int64_t ldw, const void* X,
+                        int64_t tokens, int64_t ldx, float q_max, int lo, int hi, float damp,
+                        int weighted, uint8_t* codes, uint8_t* scales, float* S, float* h,
+                        int* status, void* workspace, size_t workspace_bytes, void* stream) {
+  NVFP4_RANGE("nvfp4_gptq_quantize");
+  if (W == nullptr || codes == nullptr || scales == nullptr || S == nullptr || h == nullptr ||
+      (X == nullptr && tokens > 0))
+    return NVFP4_ERR_INVALID_ARG;
+  if (out <= 0 || in <= 0 || tokens < 0 || (weighted != 0 && weighted != 1))
+    return NVFP4_ERR_INVALID_ARG;
+  if (in % 16 != 0 || ldw < in || ldx < in || in >= (int64_t{1} << 31) || out > kMaxDim ||
+      tokens > kMaxDim || ldw > kMaxDim || ldx > kMaxDim || tokens * ldx > (int64_t{1} << 31) * 64)
+    return NVFP4_ERR_SHAPE;
+  if (!std::isfinite(q_max) || !(q_max > 0.0f) || !std::isfinite(damp) || damp < 0.0f)
+    return NVFP4_ERR_INVALID_ARG;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  if (!aligned(W, 2) || !aligned(X, 16) || ldx % 8 != 0 || !aligned(codes, 8) || !aligned(S, 4) ||
+      !aligned(h, 16) || !aligned(status, 4))
+    return NVFP4_ERR_ALIGN;
+  if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  const size_t need = nvfp4::gptq_workspace_bytes(out, in, tokens, sms);
+  if (need == 0) return cuda_status(cudaErrorUnknown);
+  if (workspace_bytes < need) return NVFP4_ERR_WORKSPACE;
+  return cuda_status(nvfp4::launch_gptq(
+      static_cast<const uint16_t*>(W), out, in, ldw, static_cast<const uint16_t*>(X), tokens, ldx,
+      q_max, lo, hi, damp, weighted != 0, codes, scales, S, h, status, workspace, workspace_bytes,
+      sms, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_scale_sweep_quantize_f32(const float* W, int64_t out, int64_t in, int64_t ldw,
+                                   const float* h, const float* S, int lo, int hi,
+                                   uint8_t* codes, uint8_t* scales, void* stream) {
+  NVFP4_RANGE("nvfp4_scale_sweep_quantize_f32");
+  if (out < 0 || in < 0) return NVFP4_ERR_INVALID_ARG;
+  const bool empty = out == 0 || in == 0;
+  if (!empty && (W == nullptr || S == nullptr || codes == nullptr || scales == nullptr))
+    return NVFP4_ERR_INVALID_ARG;
+  if (in % 16 != 0 || ldw < in || out > kMaxDim || in > kMaxDim || ldw > kMaxDim)
+    return NVFP4_ERR_SHAPE;
+  if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
+  if (!aligned(W, 4) || !aligned(h, 16) || !aligned(S, 4) || !aligned(codes, 8))
+    return NVFP4_ERR_ALIGN;
+  if (empty) return NVFP4_OK;
+  const int sms = current_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorNoDevice);
+  return cuda_status(nvfp4::launch_sweep_f32(W, out, in, ldw, h, S, lo, hi, codes, scales, sms,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 size_t nvfp4_quantize_layers_workspace_size(const nvfp4_layer* layers, int n_layers) {
   std::vector<nvfp4_layer_weight> w;
   std::vector<nvfp4_layer_input> x;

@@ -55,7 +55,8 @@ typedef enum nvfp4_status {
     NVFP4_ERR_NONFINITE = -5,    /* written to a device status word: Inf/NaN in W       */
     NVFP4_ERR_CUDA = -6,         /* a CUDA runtime call or kernel launch failed         */
     NVFP4_ERR_WORKSPACE = -7,    /* workspace NULL or smaller than the queried size     */
-    NVFP4_ERR_CAPTURE = -8       /* a call that stages host tables, on a capturing stream */
+    NVFP4_ERR_CAPTURE = -8,      /* a call that stages host tables, on a capturing stream */
+    NVFP4_ERR_NUMERIC = -9       /* written to a device status word: a Cholesky failed  */
 } nvfp4_status;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -374,6 +375,56 @@ size_t nvfp4_quantize_layers_workspace_size(const nvfp4_layer* layers, int n_lay
 int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, int lo, int hi,
                           void* workspace, size_t workspace_bytes, void* const* sweep_events,
                           void* stream);
+
+/* ------------------------------------------------------------------------
+ * H-Scale as GPTQ's local quantizer (H-Scale summary, sec. B "Implementation"
+ * and "GPTQ Integration": H-Scale replaces only the local quantization call;
+ * GPTQ's inverse-Cholesky processing, error computation and propagation are
+ * unchanged).  GPTQ in the given column order on W with the calibration
+ * inputs X:
+ *   H = X^T X; a column whose diagonal is 0 gets H_jj = 1 and zero weights;
+ *   H += damp * mean(diag H) * I (GPTQ's usual damp is 0.01);
+ *   U = the upper Cholesky factor of H^-1;
+ *   column by column: quantize w_j, err = (w_j - q_j) / U_jj, and w_k -= err U_jk
+ *   for every later column k.
+ * The local call: at the first column of each 16-column group, every row's
+ * scale code for the group is the windowed sweep's choice (weighted by
+ * h = diag(X^T X), or plain MSE if weighted == 0) on the group's current,
+ * error-updated FP32 weights, with S = the global scale of the original W;
+ * each column of the group is then quantized at its turn with that scale.
+ *
+ *   W        bf16 [out, ldw]; in % 16 == 0; out, in > 0; in < 2^31.
+ *   X        bf16 [tokens, ldx], tokens >= 0, ldx >= in.
+ *   codes, scales, S, h  the NVFP4 result ([out, in/2], [out, in/16]), the
+ *            global scale and diag(X^T X) (as nvfp4_diag_hessian writes it).
+ *   status   nullable device int: 0, NVFP4_ERR_NONFINITE (W holds Inf/NaN), or
+ *            NVFP4_ERR_NUMERIC (the damped Hessian's Cholesky failed in FP32).
+ *   workspace  nvfp4_gptq_workspace_size(out, in, tokens) bytes, 256-byte
+ *            aligned (it holds H, an FP32 copy of W and the solver's scratch:
+ *            about 4 (in^2 + out in) bytes).
+ * Steps: h, S and the GPTQ batches are this library's kernels; X^T X and the
+ * batches' updates of later columns are GEMMs (cuBLAS), the Cholesky factor
+ * and inverse come from cuSOLVER.  The first call on a device creates the
+ * library's cuBLAS and cuSOLVER handles there, which hold a little device
+ * memory until the process exits; every call's scratch is the caller's
+ * workspace.  Calls are serialised on the host; asynchronous on `stream`.
+ * Results are FP32 GPTQ: they follow an FP64 evaluation of the same steps
+ * until a quantization decision flips, which a row then carries into its
+ * later columns.
+ * ------------------------------------------------------------------------ */
+size_t nvfp4_gptq_workspace_size(int64_t out, int64_t in, int64_t tokens);
+int nvfp4_gptq_quantize(const void* W, int64_t out, int64_t in, int64_t ldw, const void* X,
+                        int64_t tokens, int64_t ldx, float q_max, int lo, int hi, float damp,
+                        int weighted, uint8_t* codes, uint8_t* scales, float* S, float* h,
+                        int* status, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The local call of nvfp4_gptq_quantize on its own: the windowed sweep of an
+ * FP32 matrix W [out, ldw] (in % 16 == 0; h NULL = plain MSE; S a device
+ * scalar), each group quantized at its chosen scale -- the same device code
+ * GPTQ runs on its error-updated columns.  codes 8-byte aligned. */
+int nvfp4_scale_sweep_quantize_f32(const float* W, int64_t out, int64_t in, int64_t ldw,
+                                   const float* h, const float* S, int lo, int hi,
+                                   uint8_t* codes, uint8_t* scales, void* stream);
 
 /* ------------------------------------------------------------------------
  * A mixture-of-experts layer in one call: two batches of expert matrices, each

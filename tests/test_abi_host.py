@@ -341,7 +341,7 @@ def test_every_launching_entry_point_opens_an_nvtx_range():
                "nvfp4_debug_checks_compiled", "nvfp4_debug_checks",
                "nvfp4_quantize_grouped_layer_order", "nvfp4_debug_row_counters"}
     launching = {k: v for k, v in found.items() if k not in queries}
-    assert len(launching) == 14, sorted(launching)
+    assert len(launching) == 16, sorted(launching)
     for name, first in launching.items():
         assert first == f'NVFP4_RANGE("{name}");', (name, first)
 
