@@ -18,10 +18,13 @@
 //   * h and S: this library's diagonal-Hessian and global-scale kernels;
 //   * H = X^T X: one cuBLAS GEMM (bf16 in, FP32 accumulate; a plain GEMM);
 //   * the dead-column rule and the damping: gptq_prep_kernel;
-//   * Cholesky of H, its inverse, and the Cholesky factor of that: cuSOLVER
-//     (potrf, potri, potrf, all on the lower triangle, in FP32).  The last
-//     factor L (lower, column-major) with H^-1 = L L^T is U^T, so read
-//     row-major the same array holds U: U[j][k] = L(k, j) at j * in + k;
+//   * U without forming H^-1: with J the order-reversing permutation, the
+//     lower Cholesky factor L' of J H J gives H = R R^T with R = J L' J upper,
+//     so H^-1 = (R^-1)^T R^-1 and U = R^-1 = J L'^-1 J.  cuSOLVER factors
+//     (potrf) and inverts (trtri) in FP32 on the lower triangle; the
+//     reflection of the n x n array about its anti-diagonal, done in place
+//     before (J H J, H symmetric) and after, turns the column-major L'^-1
+//     into U row-major: U[j][k] at j * in + k;
 //   * GPTQ's lazy batches of 128 columns: gptq_block_kernel runs the columns of
 //     one batch for 64 rows per CTA -- local call, quantization, in-batch
 //     propagation -- with the batch's triangle of U and the rows' weights in
@@ -247,8 +250,24 @@ gptq_wcopy_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t in, int64
   }
 }
 
-// A failed Cholesky (devInfo != 0: the damped Hessian is not positive
-// definite in FP32) is reported through the status word.
+// In place: a[r][c] <-> a[n-1-c][n-1-r] (reflection about the anti-diagonal),
+// one thread per pair r + c < n - 1.
+__global__ void __launch_bounds__(256)
+antitranspose_kernel(float* __restrict__ a, int64_t n) {
+  const int64_t total = n * n;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / n, c = i - r * n;
+    if (r + c >= n - 1) continue;
+    const int64_t o = (n - 1 - c) * n + (n - 1 - r);
+    const float t = a[i];
+    a[i] = a[o];
+    a[o] = t;
+  }
+}
+
+// A failed Cholesky or inverse (devInfo != 0: the damped Hessian is not
+// positive definite in FP32) is reported through the status word.
 __global__ void gptq_status_kernel(const int* __restrict__ info, int n, int* status) {
   int bad = 0;
   for (int i = 0; i < n; ++i) bad |= info[i] != 0;
@@ -345,6 +364,7 @@ bool handles_for_current_device(Handles** out) {
 struct GptqLayout {
   size_t h_ws = 0, s_ws = 0, H = 0, Wf = 0, Err = 0, dead = 0, info = 0, lapack = 0, blas = 0;
   size_t bytes = 0;
+  size_t lapack_bytes = 0, host_bytes = 0;
   int lwork = 0;
   LanePlan dplan, gplan;
 };
@@ -354,14 +374,18 @@ constexpr size_t kBlasWorkspace = 32u << 20;
 bool gptq_layout(int64_t out, int64_t in, int64_t tokens, int sms, Handles* hd, GptqLayout* L) {
   L->dplan = diag_hessian_plan(tokens, in, sms);
   L->gplan = global_scale_plan(out, in, sms);
-  int lw1 = 0, lw2 = 0;
+  int lw1 = 0;
   if (cusolverDnSpotrf_bufferSize(hd->solver, CUBLAS_FILL_MODE_LOWER, static_cast<int>(in),
                                   nullptr, static_cast<int>(in), &lw1) != CUSOLVER_STATUS_SUCCESS)
     return false;
-  if (cusolverDnSpotri_bufferSize(hd->solver, CUBLAS_FILL_MODE_LOWER, static_cast<int>(in),
-                                  nullptr, static_cast<int>(in), &lw2) != CUSOLVER_STATUS_SUCCESS)
+  size_t dev_b = 0, host_b = 0;
+  if (cusolverDnXtrtri_bufferSize(hd->solver, CUBLAS_FILL_MODE_LOWER, CUBLAS_DIAG_NON_UNIT, in,
+                                  CUDA_R_32F, nullptr, in, &dev_b, &host_b) !=
+      CUSOLVER_STATUS_SUCCESS)
     return false;
-  L->lwork = std::max(lw1, lw2);
+  L->lwork = lw1;
+  L->lapack_bytes = std::max(static_cast<size_t>(lw1) * sizeof(float), dev_b);
+  L->host_bytes = host_b;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -375,7 +399,7 @@ bool gptq_layout(int64_t out, int64_t in, int64_t tokens, int sms, Handles* hd, 
   L->Err = take(static_cast<size_t>(out) * kGB * sizeof(float));
   L->dead = take(static_cast<size_t>(in));
   L->info = take(3 * sizeof(int));
-  L->lapack = take(static_cast<size_t>(L->lwork) * sizeof(float));
+  L->lapack = take(L->lapack_bytes);
   L->blas = take(kBlasWorkspace);
   L->bytes = off;
   return true;
@@ -454,9 +478,11 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
   auto lapack_ok = [](cusolverStatus_t s) { return s == CUSOLVER_STATUS_SUCCESS; };
   if (!blas_ok(cublasSetStream(hd->blas, stream)) ||
       !blas_ok(cublasSetWorkspace(hd->blas, ws + L.blas, kBlasWorkspace)) ||
-      !blas_ok(cublasSetMathMode(hd->blas, CUBLAS_DEFAULT_MATH)) ||
       !lapack_ok(cusolverDnSetStream(hd->solver, stream)))
     return cudaErrorUnknown;
+  // plain FP32 GEMMs (no TF32 or emulated paths: the same arithmetic whichever
+  // cuBLAS build the process has loaded)
+  if (!blas_ok(cublasSetMathMode(hd->blas, CUBLAS_DEFAULT_MATH))) return cudaErrorUnknown;
   // h and S with this library's kernels
   if ((e = launch_diag_hessian(X, tokens, in, ldx, h, 0, reinterpret_cast<float*>(ws + L.h_ws),
                                L.dplan, stream)) != cudaSuccess)
@@ -488,18 +514,27 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
     gptq_wcopy_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(W, out, in, ldw, dead, Wf);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // U: Cholesky of H, inverse from it, Cholesky of the inverse (lower, FP32)
+  // U = J L'^-1 J, L' the lower Cholesky factor of J H J (FP32)
   const int n = static_cast<int>(in);
+  auto reflect = [&]() {
+    int64_t blocks = (in * in + 255) / 256;
+    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
+    antitranspose_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(H, in);
+    return cudaGetLastError();
+  };
+  std::vector<char> host_scratch(L.host_bytes);
+  if ((e = reflect()) != cudaSuccess) return e;
   if (!lapack_ok(cusolverDnSpotrf(hd->solver, CUBLAS_FILL_MODE_LOWER, n, H, n, lapack, L.lwork,
                                   info)) ||
-      !lapack_ok(cusolverDnSpotri(hd->solver, CUBLAS_FILL_MODE_LOWER, n, H, n, lapack, L.lwork,
-                                  info + 1)) ||
-      !lapack_ok(cusolverDnSpotrf(hd->solver, CUBLAS_FILL_MODE_LOWER, n, H, n, lapack, L.lwork,
-                                  info + 2)))
+      !lapack_ok(cusolverDnXtrtri(hd->solver, CUBLAS_FILL_MODE_LOWER, CUBLAS_DIAG_NON_UNIT, in,
+                                  CUDA_R_32F, H, in, lapack, L.lapack_bytes,
+                                  host_scratch.empty() ? nullptr : host_scratch.data(),
+                                  L.host_bytes, info + 1)))
     return cudaErrorUnknown;
-  gptq_status_kernel<<<1, 1, 0, stream>>>(info, 3, status);
+  if ((e = reflect()) != cudaSuccess) return e;
+  gptq_status_kernel<<<1, 1, 0, stream>>>(info, 2, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const float* U = H;  // row-major view: U[j][k] = L(k, j) for k >= j
+  const float* U = H;  // row-major U[j][k] for k >= j (the reflected L'^-1)
   const int K = hi - lo + 1;
   const float minus_one = -1.0f;
   for (int64_t j0 = 0; j0 < in; j0 += kGB) {
