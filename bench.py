@@ -827,6 +827,76 @@ def run_activations(args, nv, rank, local, ws, dev):
         print(json.dumps(out), flush=True)
 
 
+GPTQ_WORKLOAD = ("gptq_llama33_70b_gate: GPTQ with the H-Scale local call on the 70B-shaped gate "
+                 "projection, W 28672x8192 bf16 N(0,0.015) 0.1% x10, X 65536x8192 bf16 "
+                 "lognormal(1.5) channel scales; damping 0.01; window [-9,+6]")
+
+
+def run_gptq(args, nv, rank, local, ws, dev):
+    """One step = one nvfp4_gptq_quantize call: h, S, X^T X, the inverse-Cholesky
+    factor and GPTQ's column loop with the H-Scale local call.  Graded on the
+    propagation's FP32 work (out * in^2 multiply-adds in GPTQ's column updates)
+    against the FP32 lane peak."""
+    import torch
+    import workloads
+    W = workloads.weight(28672, 8192, 0.015, 0.001, 10.0, 401 + 97 * rank, dev)
+    X = workloads.calib(65536, 8192, 1.5, 441 + 97 * rank, dev)
+    out, n = W.shape
+    codes = torch.empty(out, n // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(out, n // 16, dtype=torch.uint8, device=dev)
+    S = torch.empty(1, dtype=torch.float32, device=dev)
+    h = torch.empty(n, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    nb = nv.nvfp4_gptq_workspace_size(out, n, X.shape[0])
+    wsb = torch.empty(nb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nv.nvfp4_gptq_quantize(W, out, n, n, X, X.shape[0], n, 448.0, LO, HI, 0.01, True, codes,
+                               scales, S, h, status, wsb, nb, stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(ws)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(ws)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler.mark_start()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    barrier(ws)
+    sampler.mark_end()
+    clocks = sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, ws)
+    assert int(status.item()) == 0, "GPTQ status"
+    el = out * n
+    clk = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = SMS * LANES_PER_SM * 2 * clk * 1e6 / 1e12
+    achieved = 2.0 * out * n * n / (ms * 1e-3) / 1e12
+    roofline = {"kernel": "gptq (whole call)", "bound": "alu", "achieved": round(achieved, 2),
+                "peak": round(peak, 2), "unit": "TFLOP/s",
+                "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {clk:.0f} MHz (sampled SM clock)",
+                "frac": round(achieved / peak, 4),
+                "ops_per_unit": "2 * in FP32 flops per weight element (GPTQ's column updates)",
+                "traffic": None}
+    if rank == 0:
+        out_line = {"metric": "GPTQ + H-Scale local call: weight elems/s", "value": el * ws / (ms * 1e-3),
+                    "unit": "elem/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                    "config": {"workload": GPTQ_WORKLOAD, "window": [LO, HI], "q_max": 448.0,
+                               "l2": "inputs 1.54 GB per rank > 126 MB L2; no flush",
+                               "parallelism": f"weak: {ws} rank(s), one projection per rank"},
+                    "roofline": roofline, "e2e": None, "gpu_launches": None,
+                    "cpu_baseline": None, "clocks": clocks}
+        print(json.dumps(out_line), flush=True)
+
+
 # ------------------------------------------------------------------ main
 
 def init_dist():
@@ -1000,7 +1070,7 @@ def main():
                          "calls with later weights' S and h on a second stream; auto: layer "
                          "(nvfp4_quantize_grouped_layer for the MoE layer)")
     ap.add_argument("--workload", default="llama33_70b_mlp",
-                    choices=list(WORKLOADS) + ["act_llama33_70b"])
+                    choices=list(WORKLOADS) + ["act_llama33_70b", "gptq_llama33_70b_gate"])
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1014,8 +1084,9 @@ def main():
     rank, local, ws = init_dist()
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
-    if args.workload == "act_llama33_70b":
-        run_activations(args, nv, rank, local, ws, dev)
+    if args.workload in ("act_llama33_70b", "gptq_llama33_70b_gate"):
+        (run_activations if args.workload == "act_llama33_70b" else run_gptq)(
+            args, nv, rank, local, ws, dev)
         if ws > 1:
             import torch.distributed as dist
             dist.barrier()
