@@ -791,10 +791,6 @@ def run_activations(args, nv, rank, local, ws, dev):
             hC.copy_(codes, non_blocking=True)
             hK.copy_(scales, non_blocking=True)
 
-        # the per-step calls pipeline with the copies (each waits for its own
-        # inputs); the one-call form would wait for all of them
-        layer_mode = getattr(step, "layer", False)
-        step.layer = False
         e2e_step()
         barrier(ws)
         a = torch.cuda.Event(enable_timing=True)
@@ -804,7 +800,6 @@ def run_activations(args, nv, rank, local, ws, dev):
             e2e_step()
         b.record(stream)
         barrier(ws)
-        step.layer = layer_mode
         e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, ws)
         e2e = {"value": el * ws / (e_ms * 1e-3), "unit": "elem/s", "ms_per_step": round(e_ms, 3),
                "h2d_bytes_per_step": int(hA.numel() * 2),
