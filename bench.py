@@ -830,8 +830,8 @@ GPTQ_WORKLOAD = ("gptq_llama33_70b_gate: GPTQ with the H-Scale local call on the
 def run_gptq(args, nv, rank, local, ws, dev):
     """One step = one nvfp4_gptq_quantize call: h, S, X^T X, the inverse-Cholesky
     factor and GPTQ's column loop with the H-Scale local call.  Graded on the
-    propagation's FP32 work (out * in^2 multiply-adds in GPTQ's column updates)
-    against the FP32 lane peak."""
+    propagation's FP32 work (out * in^2 / 2 multiply-adds in GPTQ's column
+    updates) against the FP32 lane peak."""
     import torch
     import workloads
     W = workloads.weight(28672, 8192, 0.015, 0.001, 10.0, 401 + 97 * rank, dev)
@@ -872,12 +872,13 @@ def run_gptq(args, nv, rank, local, ws, dev):
     el = out * n
     clk = (clocks or {}).get("sm_mhz") or 1965.0
     peak = SMS * LANES_PER_SM * 2 * clk * 1e6 / 1e12
-    achieved = 2.0 * out * n * n / (ms * 1e-3) / 1e12
+    achieved = 1.0 * out * n * n / (ms * 1e-3) / 1e12   # out * n(n-1)/2 multiply-adds
     roofline = {"kernel": "gptq (whole call)", "bound": "alu", "achieved": round(achieved, 2),
                 "peak": round(peak, 2), "unit": "TFLOP/s",
                 "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {clk:.0f} MHz (sampled SM clock)",
                 "frac": round(achieved / peak, 4),
-                "ops_per_unit": "2 * in FP32 flops per weight element (GPTQ's column updates)",
+                "ops_per_unit": "in FP32 flops per weight element (GPTQ's column updates: "
+                                "in/2 multiply-adds each)",
                 "traffic": None}
     if rank == 0:
         out_line = {"metric": "GPTQ + H-Scale local call: weight elems/s", "value": el * ws / (ms * 1e-3),
