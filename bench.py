@@ -1001,9 +1001,12 @@ def kernel_table(ev, steps, wl):
     return kern
 
 
-def dominant_roofline(kern, wl, clocks, traffic_key=None):
+def dominant_roofline(kern, wl, clocks, traffic_key=None, inst_key="scale_sweep"):
     """Roofline object of the kernel with the most time per step.  traffic_key:
-    the traffic record to report (default: the kernel's own kind)."""
+    the traffic record to report (default: the kernel's own kind); inst_key:
+    the record whose instruction count per element gives the sweep's issue
+    fraction (the plain sweep kernel's, or the batched one's for expert
+    layers)."""
     kb = kernel_bytes(wl)
     peak, peak_kind, _ = measured_peaks()
     dom = max(kern, key=lambda k: kern[k]["ms_per_step"])
@@ -1018,7 +1021,7 @@ def dominant_roofline(kern, wl, clocks, traffic_key=None):
         # the older model of 5 FP32 lane operations per element and candidate.
         achieved = kb[dom] / launches / per_launch_s / 1e9
         clk = (clocks or {}).get("sm_mhz") or 1965.0
-        wi = profiled_warp_inst(dom, wl.weight_elems / launches)
+        wi = profiled_warp_inst(inst_key, wl.weight_elems / launches)
         issue_slots = SMS * ISSUE_PER_SM * clk * 1e6 * per_launch_s
         ops = SWEEP_OPS_PER_ELEM_CAND * (HI - LO + 1) * wl.weight_elems / launches
         peak_top = SMS * LANES_PER_SM * clk * 1e6 / 1e12
@@ -1028,8 +1031,8 @@ def dominant_roofline(kern, wl, clocks, traffic_key=None):
                 "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                 "binding_resource": "instruction issue (FP32 FMA and ALU pipes)",
                 "issue_frac": None if wi is None else round(wi / issue_slots, 4),
-                "issue_note": ("warp instructions per launch from the committed ncu capture "
-                               "(sm__inst_executed.sum per weight element x elements) / "
+                "issue_note": (f"warp instructions per launch from the committed ncu capture of "
+                               f"{inst_key} (sm__inst_executed.sum per weight element x elements) / "
                                f"(148 SMs x {ISSUE_PER_SM} issue slots x {clk:.0f} MHz sampled "
                                "x launch time); null once the sweep's sources change"),
                 "alu_model": {"achieved_top_s": round(ops / per_launch_s / 1e12, 2),
@@ -1208,7 +1211,8 @@ def main():
 
     # ---- roofline of the dominant kernel, as timed in the region above
     in_layer = getattr(step, "layer", False) and not getattr(step, "serial", True)
-    roofline = dominant_roofline(kern, wl, clocks)
+    inst_key = "scale_sweep_batched" if isinstance(step, GroupedStep) else "scale_sweep"
+    roofline = dominant_roofline(kern, wl, clocks, inst_key=inst_key)
     layer_info = None
     if in_layer:
         # the carrying sweeps stream every reduction but the first ones: their
@@ -1264,7 +1268,7 @@ def main():
         barrier(ws)
         step.serial = False
         kern_iso = kernel_table(ev_iso, n_iso, wl)
-        roof_iso = dominant_roofline(kern_iso, wl, clocks)
+        roof_iso = dominant_roofline(kern_iso, wl, clocks, inst_key=inst_key)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
