@@ -297,8 +297,9 @@ int flatten_layers(const nvfp4_layer* layers, int n_layers, std::vector<nvfp4_la
 extern "C" {
 
 size_t nvfp4_gptq_workspace_size(int64_t out, int64_t in, int64_t tokens) {
-  if (out <= 0 || in <= 0 || tokens < 0 || in % 16 != 0 || in >= (int64_t{1} << 31) ||
-      out > kMaxDim || tokens > kMaxDim)
+  constexpr int64_t kIntMax = (int64_t{1} << 31) - 1;
+  if (out <= 0 || in <= 0 || tokens < 0 || in % 16 != 0 || in > kIntMax || out > kIntMax ||
+      tokens > kIntMax)
     return 0;
   const int sms = current_sm_count();
   if (sms <= 0) return 0;
@@ -315,8 +316,10 @@ int nvfp4_gptq_quantize(const void* W, int64_t out, int64_t in, int64_t ldw, con
     return NVFP4_ERR_INVALID_ARG;
   if (out <= 0 || in <= 0 || tokens < 0 || (weighted != 0 && weighted != 1))
     return NVFP4_ERR_INVALID_ARG;
-  if (in % 16 != 0 || ldw < in || ldx < in || in >= (int64_t{1} << 31) || out > kMaxDim ||
-      tokens > kMaxDim || ldw > kMaxDim || ldx > kMaxDim || tokens * ldx > (int64_t{1} << 31) * 64)
+  // cuBLAS and cuSOLVER take int sizes and leading dimensions
+  constexpr int64_t kIntMax = (int64_t{1} << 31) - 1;
+  if (in % 16 != 0 || ldw < in || ldx < in || in > kIntMax || out > kIntMax || tokens > kIntMax ||
+      ldw > kMaxDim || ldx > kIntMax)
     return NVFP4_ERR_SHAPE;
   if (!std::isfinite(q_max) || !(q_max > 0.0f) || !std::isfinite(damp) || damp < 0.0f)
     return NVFP4_ERR_INVALID_ARG;

@@ -393,8 +393,9 @@ int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, 
  * error-updated FP32 weights, with S = the global scale of the original W;
  * each column of the group is then quantized at its turn with that scale.
  *
- *   W        bf16 [out, ldw]; in % 16 == 0; out, in > 0; in < 2^31.
- *   X        bf16 [tokens, ldx], tokens >= 0, ldx >= in.
+ *   W        bf16 [out, ldw]; in % 16 == 0; out, in > 0; out, in < 2^31.
+ *   X        bf16 [tokens, ldx], 16-byte aligned, ldx % 8 == 0; tokens >= 0,
+ *            ldx >= in; tokens, ldx < 2^31 (the GEMM's int sizes).
  *   codes, scales, S, h  the NVFP4 result ([out, in/2], [out, in/16]), the
  *            global scale and diag(X^T X) (as nvfp4_diag_hessian writes it).
  *   status   nullable device int: 0, NVFP4_ERR_NONFINITE (W holds Inf/NaN), or

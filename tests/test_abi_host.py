@@ -361,3 +361,36 @@ def test_checked_build_loads_and_exports_the_same_entry_points():
     assert Lp.nvfp4_debug_checks(C.byref(first), C.byref(count), 0) == 0
     assert first.value == 0 and count.value == 0            # nothing recorded without checks
     assert Lp.nvfp4_debug_checks(None, C.byref(count), 0) == -1
+
+
+def test_gptq_validation(L):
+    """GPTQ's arguments are checked before anything runs (no device needed)."""
+    import block_scale_search_b200 as nv
+    f = L.nvfp4_gptq_quantize
+    ok = dict(W=P, out=64, inp=256, ldw=256, X=P, tokens=128, ldx=256, q=448.0, lo=-9, hi=6,
+              damp=0.01, w=1, codes=P, scales=P, S=P, h=P, st=None, ws=P, nb=1 << 30)
+
+    def call(**k):
+        a = {**ok, **k}
+        return f(a["W"], a["out"], a["inp"], a["ldw"], a["X"], a["tokens"], a["ldx"], a["q"], a["lo"],
+                 a["hi"], a["damp"], a["w"], a["codes"], a["scales"], a["S"], a["h"], a["st"], a["ws"],
+                 a["nb"], None)
+
+    assert call(W=None) == -1 and call(h=None) == -1 and call(X=None) == -1
+    assert call(out=0) == -1 and call(w=2) == -1 and call(damp=-1.0) == -1
+    assert call(q=float("inf")) == -1
+    assert call(inp=250, ldw=256, ldx=256) == -2            # in % 16
+    assert call(ldx=128) == -2                                # ldx < in
+    assert call(tokens=1 << 31) == -2                        # beyond the GEMM's int sizes
+    assert call(lo=-10) == -4
+    assert call(X=P + 8) == -3 and call(codes=P + 4) == -3 and call(h=P + 4) == -3
+    assert call(ws=None) == -7 and call(ws=P + 64) == -3
+    assert L.nvfp4_gptq_workspace_size(64, 250, 128) == 0
+    g = L.nvfp4_scale_sweep_quantize_f32
+    assert g(P, 4, 250, 256, None, P, -9, 6, P, P, None) == -2
+    assert g(P, 4, 256, 256, None, P, -10, 6, P, P, None) == -4
+    assert g(P + 2, 4, 256, 256, None, P, -9, 6, P, P, None) == -3
+    assert g(None, 0, 256, 256, None, None, -9, 6, None, None, None) == 0     # empty
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == -6 and L.nvfp4_gptq_workspace_size(64, 256, 128) == 0
