@@ -96,16 +96,20 @@ def _correlated(n, tokens, seed):
     return (Z @ mix).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("out,n,tokens,seed", [(256, 512, 2048, 81), (128, 1024, 4096, 82)])
-def test_correlated_inputs_follow_the_oracle(orc, nv, parity_report, out, n, tokens, seed):
+@pytest.mark.parametrize("out,n,tokens,seed,weighted,lo,hi", [
+    (256, 512, 2048, 81, True, -9, 6), (128, 1024, 4096, 82, True, -9, 6),
+    (192, 512, 2048, 83, False, -3, 7), (160, 768, 3072, 84, True, -8, 7)])
+def test_correlated_inputs_follow_the_oracle(orc, nv, parity_report, out, n, tokens, seed,
+                                             weighted, lo, hi):
     import workloads
     from oracle import gptq
     W = workloads.weight(out, n, 0.02, 0.005, 10.0, seed)
     X = _correlated(n, tokens, seed + 1)
-    codes, scales, S, h, status = nv.gptq_quantize(W.to(DEV), X.to(DEV))
+    codes, scales, S, h, status = nv.gptq_quantize(W.to(DEV), X.to(DEV), lo=lo, hi=hi,
+                                                   weighted=weighted)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    oc, os_, oS, Q, oh = gptq.gptq_hscale(W, X)
+    oc, os_, oS, Q, oh = gptq.gptq_hscale(W, X, lo=lo, hi=hi, weighted=weighted)
     assert np.float32(S.item()) == oS
     Wf = gptq.bf16_to_f64(orc._bf16_bits(W))
     Xf = gptq.bf16_to_f64(orc._bf16_bits(X))
@@ -115,11 +119,12 @@ def test_correlated_inputs_follow_the_oracle(orc, nv, parity_report, out, n, tok
     gc = codes.cpu().numpy().reshape(-1, 8)
     gs = scales.cpu().numpy().reshape(-1)
     same = float(((gs == os_.reshape(-1)) & np.all(gc == oc.reshape(-1, 8), axis=1)).mean())
-    # the standalone sweep on the same h, for the gain GPTQ brings
-    rc, rs, _ = orc.sweep_quantize(W, oh, float(oS), -9, 6)
+    # the standalone sweep with the same objective, for the gain GPTQ brings
+    rc, rs, _ = orc.sweep_quantize(W, oh if weighted else None, float(oS), lo, hi)
     e_sweep = np.sum((Xf @ (Wf - _decoded(rc, rs, oS, out, n)).T) ** 2)
-    parity_report(f"gptq {out}x{n}, {tokens} tokens: output error GPU/oracle {e_gpu / e_orc:.5f}, "
-                  f"groups equal {same:.4f}, GPTQ/sweep-alone {e_orc / e_sweep:.3f}")
+    parity_report(f"gptq {out}x{n}, {tokens} tokens, {'WMSE' if weighted else 'MSE'} [{lo},{hi}]: "
+                  f"output error GPU/oracle {e_gpu / e_orc:.5f}, groups equal {same:.4f}, "
+                  f"GPTQ/sweep-alone {e_orc / e_sweep:.3f}")
     # Tolerances (FP32 against FP64 GPTQ): a flipped decision changes one
     # element's reconstruction by a grid step and the row's later columns
     # re-fit around it, so a row's tail can differ while the layer error
