@@ -23,6 +23,8 @@ import sys
 import threading
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -1270,6 +1272,28 @@ def main():
         kern_iso = kernel_table(ev_iso, n_iso, wl)
         roof_iso = dominant_roofline(kern_iso, wl, clocks, inst_key=inst_key)
 
+    # ---- which offsets the sweep chose (outside the timed region): the
+    # H-Scale summary's direction statistic (larger / kept / smaller than the
+    # max-abs base scale) on this synthetic layer
+    offsets = None
+    if not isinstance(step, GroupedStep):
+        hist = np.zeros(HI - LO + 1, np.int64)
+        zero = 0
+        for m in wl.matrices:
+            h = step.h[m.x_key]
+            _, sc_, of = nv.scale_sweep_quantize(Ws[m.name], h, step.S[m.name], LO, HI,
+                                                 want_offsets=True)
+            o = of.cpu().numpy().reshape(-1)
+            zero += int((sc_.cpu().numpy().reshape(-1) == 0).sum())
+            hist += np.bincount(o.astype(np.int64) - LO, minlength=HI - LO + 1)
+        hist[-LO] -= zero                      # all-zero groups report offset 0
+        tot = max(1, int(hist.sum()))
+        offsets = {"window": [LO, HI], "histogram": hist.tolist(),
+                   "larger": round(float(hist[1 - LO:].sum()) / tot, 4),
+                   "kept": round(float(hist[-LO]) / tot, 4),
+                   "smaller": round(float(hist[:-LO].sum()) / tot, 4),
+                   "zero_groups": zero}
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, info = oracle_sample_rate(wl, Ws, Xs, single_thread=True)
@@ -1310,7 +1334,7 @@ def main():
             "kernels": kern, "roofline": roofline,
             "kernels_isolated": kern_iso, "roofline_isolated": roof_iso, "e2e": e2e,
             "gpu_launches": step.launches_per_step * args.steps,
-            "cpu_baseline": cpu, "clocks": clocks,
+            "cpu_baseline": cpu, "clocks": clocks, "offsets": offsets,
         }
         print(json.dumps(out), flush=True)
     if ws > 1:
