@@ -98,7 +98,8 @@ def _correlated(n, tokens, seed):
 
 @pytest.mark.parametrize("out,n,tokens,seed,weighted,lo,hi", [
     (256, 512, 2048, 81, True, -9, 6), (128, 1024, 4096, 82, True, -9, 6),
-    (192, 512, 2048, 83, False, -3, 7), (160, 768, 3072, 84, True, -8, 7)])
+    (192, 512, 2048, 83, False, -3, 7), (160, 768, 3072, 84, True, -8, 7),
+    (96, 528, 2048, 85, True, -9, 6)])   # a last batch of 16 columns
 def test_correlated_inputs_follow_the_oracle(orc, nv, parity_report, out, n, tokens, seed,
                                              weighted, lo, hi):
     import workloads
