@@ -221,3 +221,25 @@ def test_two_layers_in_one_call(orc, nv):
             gc, gs = c.cpu().numpy(), s.cpu().numpy()
             w, hh, _, _ = matrix_groups(bits, gc, gs, h)
             assert_parity(compare_groups(orc, w, hh, float(S.item()), gc, gs, rcodes, rscales))
+
+
+def test_layers_with_mse_weights_and_unused_inputs(nv):
+    """nvfp4_quantize_layers over layers of different make-up -- a plain-MSE
+    weight, an input no weight reads, a layer of one weight -- writes the
+    per-step calls' bytes."""
+    import workloads
+    L1 = ([workloads.weight(2048, 4096, 0.02, 0.001, 8.0, 111, DEV),
+           workloads.weight(1536, 4096, 0.02, 0.001, 8.0, 112, DEV)],
+          [workloads.calib(1024, 1024, 1.0, 113, DEV), workloads.calib(2048, 4096, 1.0, 114, DEV)],
+          [-1, 1])
+    L2 = ([workloads.weight(4096, 2048, 0.02, 0.001, 8.0, 121, DEV)],
+          [workloads.calib(3000, 2048, 1.0, 122, DEV)], [0])
+    got = nv.quantize_layers_many([L1, L2], q_max=256.0, lo=-8, hi=7, want_offsets=True)
+    torch.cuda.synchronize()
+    for (Ws, Xs, inputs), (outs, hs) in zip([L1, L2], got):
+        ref, href = _per_step(nv, Ws, Xs, inputs, 256.0, -8, 7)
+        for a, b in zip(hs, href):
+            assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+        for (c, s, S, o, st), (rc, rs, rS, ro, rst) in zip(outs, ref):
+            assert torch.equal(S.view(torch.int32), rS.view(torch.int32))
+            assert torch.equal(c, rc) and torch.equal(s, rs) and torch.equal(o, ro)
