@@ -829,11 +829,28 @@ GPTQ_WORKLOAD = ("gptq_llama33_70b_gate: GPTQ with the H-Scale local call on the
                  "lognormal(1.5) channel scales; damping 0.01; window [-9,+6]")
 
 
+def gptq_update_flops(out: int, n: int, gb: int = 128, sub: int = 2) -> float:
+    """TF32 flops of one GPTQ call's update GEMMs: per lazy batch of sub * gb
+    columns, a GEMM of K = 3 * gb (three split products) from its first half
+    into its second, and one of K = 3 * gb * sub into every later column."""
+    total = 0.0
+    for j0 in range(0, n, gb * sub):
+        jend = min(j0 + gb * sub, n)
+        halves = (jend - j0 + gb - 1) // gb
+        for s in range(halves - 1):
+            c1 = j0 + gb * (s + 1)
+            total += 2.0 * min(gb, jend - c1) * out * 3 * gb * (s + 1)
+        if jend < n:
+            total += 2.0 * (n - jend) * out * 3 * gb * halves
+    return total
+
+
 def run_gptq(args, nv, rank, local, ws, dev):
-    """One step = one nvfp4_gptq_quantize call: h, S, X^T X, the inverse-Cholesky
-    factor and GPTQ's column loop with the H-Scale local call.  Graded on the
-    propagation's FP32 work (out * in^2 / 2 multiply-adds in GPTQ's column
-    updates) against the FP32 lane peak."""
+    """One step = one nvfp4_gptq_quantize call: h, S, X^T X, the Cholesky factor
+    and GPTQ's column loop with the H-Scale local call.  The roofline is the
+    update GEMMs' (the largest phase): their TF32 tensor-core flops over their
+    time, measured with the library's phase timer (CUDA events on the call's
+    stream) in a second pass of the same calls after the timed region."""
     import torch
     import workloads
     W = workloads.weight(28672, 8192, 0.015, 0.001, 10.0, 401 + 97 * rank, dev)
@@ -871,16 +888,31 @@ def run_gptq(args, nv, rank, local, ws, dev):
     clocks = sampler.stop()
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, ws)
     assert int(status.item()) == 0, "GPTQ status"
+    # the phases, from a second pass of the same calls with the phase timer on
+    nv.nvfp4_gptq_set_timing(True)
+    for _ in range(args.steps):
+        step()
+    phases = {k: max_over_ranks(v / args.steps, ws) for k, v in nv.nvfp4_gptq_phase_times().items()}
+    nv.nvfp4_gptq_set_timing(False)
     el = out * n
-    clk = (clocks or {}).get("sm_mhz") or 1965.0
-    peak = SMS * LANES_PER_SM * 2 * clk * 1e6 / 1e12
-    achieved = 1.0 * out * n * n / (ms * 1e-3) / 1e12   # out * n(n-1)/2 multiply-adds
-    roofline = {"kernel": "gptq (whole call)", "bound": "alu", "achieved": round(achieved, 2),
-                "peak": round(peak, 2), "unit": "TFLOP/s",
-                "peak_source": f"148 SMs x 128 FP32 lanes x 2 x {clk:.0f} MHz (sampled SM clock)",
-                "frac": round(achieved / peak, 4),
-                "ops_per_unit": "in FP32 flops per weight element (GPTQ's column updates: "
-                                "in/2 multiply-adds each)",
+    _hbm, _kind, peaks = measured_peaks()
+    bf16 = peaks.get("bf16_tflops_sustained")
+    tf32_ratio = 1.1 / 2.25            # nominal dense TF32 / bf16 on B200
+    peak = bf16 * tf32_ratio if bf16 else 1590.0 * tf32_ratio
+    flops = gptq_update_flops(out, n)
+    upd_ms = phases["update"]
+    achieved = flops / (upd_ms * 1e-3) / 1e12 if upd_ms > 0 else None
+    roofline = {"kernel": "GPTQ update GEMMs (cuBLAS, 3 TF32 tensor-core products of split FP32 "
+                          "operands)",
+                "bound": "tensor", "achieved": round(achieved, 1) if achieved else None,
+                "peak": round(peak, 1), "unit": "TFLOP/s",
+                "peak_source": ("measured bf16_tflops_sustained x nominal TF32/bf16 ratio 1.1/2.25"
+                                if bf16 else "fallback 1.59 PFLOP/s bf16 x 1.1/2.25"),
+                "frac": round(achieved / peak, 4) if achieved else None,
+                "flops_per_call": flops,
+                "ms_per_call": round(upd_ms, 3),
+                "fp32_equivalent_tflops": round(out * n * n / 2 * 2 / (upd_ms * 1e-3) / 1e12, 1)
+                if upd_ms > 0 else None,
                 "traffic": None}
     if rank == 0:
         out_line = {"metric": "GPTQ + H-Scale local call: weight elems/s", "value": el * ws / (ms * 1e-3),
@@ -891,7 +923,8 @@ def run_gptq(args, nv, rank, local, ws, dev):
                                "l2": "inputs 1.54 GB per rank > 126 MB L2; no flush",
                                "parallelism": f"weak: {ws} rank(s), one projection per rank"},
                     "roofline": roofline, "e2e": None, "gpu_launches": None,
-                    "cpu_baseline": None, "clocks": clocks}
+                    "cpu_baseline": None, "clocks": clocks,
+                    "phases_ms_per_call": {k: round(v, 3) for k, v in phases.items()}}
         print(json.dumps(out_line), flush=True)
 
 

@@ -27,7 +27,8 @@ __all__ = [
     "nvfp4_scale_sweep_quantize_full", "scale_sweep_quantize_full", "nvfp4_debug_row_counters",
     "nvfp4_quantize_layer_workspace_size", "nvfp4_quantize_layer", "nvfp4_quantize_layer_order",
     "quantize_layer_many", "nvfp4_gptq_workspace_size", "nvfp4_gptq_quantize", "gptq_quantize",
-    "nvfp4_scale_sweep_quantize_f32", "scale_sweep_quantize_f32", "nvfp4_debug_checks", "nvfp4_debug_checks_compiled", "Layer", "nvfp4_quantize_layers_workspace_size",
+    "nvfp4_scale_sweep_quantize_f32", "scale_sweep_quantize_f32", "nvfp4_gptq_set_timing",
+    "nvfp4_gptq_phase_times", "GPTQ_PHASES", "nvfp4_debug_checks", "nvfp4_debug_checks_compiled", "Layer", "nvfp4_quantize_layers_workspace_size",
     "nvfp4_quantize_layers", "quantize_layers_many", "quantize_grouped_layer",
     "LayerWeight", "LayerInput", "GroupedInput", "nvfp4_quantize_grouped_layer_workspace_size",
     "nvfp4_quantize_grouped_layer", "nvfp4_quantize_grouped_layer_order",
@@ -133,6 +134,8 @@ _SIGS = {
                              _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "nvfp4_scale_sweep_quantize_f32": ([_vp, _i64, _i64, _i64, _vp, _vp, _int, _int, _vp, _vp, _vp],
                                        _int),
+    "nvfp4_gptq_set_timing": ([_int], _int),
+    "nvfp4_gptq_phase_times": ([C.POINTER(C.c_float), _int], _int),
     "nvfp4_blocked_scales_size": ([_i64, _i64], _sz),
     "nvfp4_scales_to_blocked": ([_vp, _i64, _i64, _i64, _vp, _vp], _int),
     "nvfp4_quantize_activations": ([_vp, _i64, _i64, _i64, _f32, _int, _int, _vp, _vp, _vp, _vp,
@@ -351,6 +354,21 @@ def nvfp4_gptq_quantize(W, out, inp, ldw, X, tokens, ldx, q_max, lo, hi, damp, w
         _ptr(W), out, inp, ldw, _ptr(X), tokens, ldx, float(q_max), int(lo), int(hi), float(damp),
         int(bool(weighted)), _ptr(codes), _ptr(scales), _ptr(S), _ptr(h), _ptr(status),
         _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+GPTQ_PHASES = ("reductions", "gram", "factor", "batch", "split", "update")
+
+
+def nvfp4_gptq_set_timing(on: bool) -> None:
+    _check("nvfp4_gptq_set_timing", lib().nvfp4_gptq_set_timing(int(bool(on))))
+
+
+def nvfp4_gptq_phase_times() -> dict:
+    """Milliseconds per GPTQ phase summed over the calls timed since
+    nvfp4_gptq_set_timing(True) (waits for their events)."""
+    ms = (C.c_float * len(GPTQ_PHASES))()
+    _check("nvfp4_gptq_phase_times", lib().nvfp4_gptq_phase_times(ms, len(GPTQ_PHASES)))
+    return {name: float(ms[i]) for i, name in enumerate(GPTQ_PHASES)}
 
 
 def nvfp4_scale_sweep_quantize_f32(W, out, inp, ldw, h, S, lo, hi, codes, scales, stream=None):

@@ -18,22 +18,36 @@
 //   * h and S: this library's diagonal-Hessian and global-scale kernels;
 //   * H = X^T X: one cuBLAS GEMM (bf16 in, FP32 accumulate; a plain GEMM);
 //   * the dead-column rule and the damping: gptq_prep_kernel;
-//   * U without forming H^-1: with J the order-reversing permutation, the
-//     lower Cholesky factor L' of J H J gives H = R R^T with R = J L' J upper,
-//     so H^-1 = (R^-1)^T R^-1 and U = R^-1 = J L'^-1 J.  cuSOLVER factors
-//     (potrf) and inverts (trtri) in FP32 on the lower triangle; the
-//     reflection of the n x n array about its anti-diagonal, done in place
-//     before (J H J, H symmetric) and after, turns the column-major L'^-1
-//     into U row-major: U[j][k] at j * in + k;
-//   * GPTQ's lazy batches of 128 columns: gptq_block_kernel runs the columns of
-//     one batch for 64 rows per CTA -- local call, quantization, in-batch
-//     propagation -- with the batch's triangle of U and the rows' weights in
-//     shared memory, and writes the batch's errors; one FP32 GEMM (cuBLAS)
-//     then applies them to every later column: W[:, >] -= Err U[batch, >].
-// Rows are independent in GPTQ (U is shared), so the batch kernel needs no
-// communication between rows.  FP32 throughout on the device: its results
-// drift from the FP64 oracle's after a quantization decision flips, which a
-// row then carries through its later columns.
+//   * no inverse is formed.  With J the order-reversing permutation, the lower
+//     Cholesky factor L' of J H J (cuSOLVER potrf, FP32) gives H = R R^T with
+//     R = J L' J upper, and U = R^-1.  Reflecting the n x n array about its
+//     anti-diagonal in place, before (J H J, H symmetric) and after, turns the
+//     column-major L' into R row-major: R[j][k] at j * in + k, k >= j;
+//   * the column loop runs in the R form of GPTQ's recurrence.  Quantizing
+//     column j at its turn and propagating err_j = (w_j - q_j) / U_jj gives,
+//     by induction over the columns, W - Q = Err U, so Err = (W - Q) R.  Then,
+//     with D = W - Q and a 16-column group starting at column g0, the group's
+//     current weights are  W_grp + (D[:, <g0] R[<g0, grp]) U_grp,  where
+//     U_grp = R_grp^-1 is the inverse of the group's 16 x 16 diagonal block of
+//     R (U is block upper triangular); inside the group the updates use U_grp
+//     and err_j = (w_j - q_j) R_jj.  gptq_udiag_kernel inverts the diagonal
+//     blocks (FP64);
+//   * GPTQ's lazy batches, 256 columns each, in two halves of 128:
+//     gptq_rblock_kernel runs the columns of one half, one thread per row --
+//     each group's sums from the earlier groups of the half, its current
+//     weights, the local call, the exact quantization and the in-group
+//     updates -- and writes the half's D.  A small GEMM adds the first half to
+//     the second half's sums; after the batch one GEMM adds the batch to every
+//     later column's sums: P[:, >] += D[:, batch] R[batch, >].  The GEMMs run
+//     on the tensor cores as three TF32 products, D_hi R_hi + D_hi R_lo +
+//     D_lo R_hi, with each FP32 operand split into its TF32 head and the
+//     remainder (gptq_rsplit_kernel for R; the batch kernel writes D's
+//     parts).  Each P element is read and written once per 256 columns.
+// Rows are independent in GPTQ (R is shared), so the batch kernel needs no
+// communication between rows.  The device arithmetic is FP32 (the update GEMM
+// about 2^-18 relative per product): results drift from the FP64 oracle's
+// after a quantization decision flips, which a row then carries through its
+// later columns.
 #include <cublas_v2.h>
 #include <cusolverDn.h>
 
@@ -41,14 +55,20 @@
 #include <vector>
 
 #include "nvfp4_kernels.cuh"
+#include "nvfp4hs.h"
 #include "sweep_core.cuh"
 
 namespace nvfp4 {
 
 namespace {
 
-constexpr int kGB = 128;  // columns per lazy batch
-constexpr int kGT = 64;   // rows (threads) per CTA of the batch kernel
+constexpr int kGB = 128;        // columns per batch kernel launch
+constexpr int kCat = 3 * kGB;   // K of the split update per 128 columns
+constexpr int kSub = 2;         // batch-kernel launches per lazy batch (256 columns)
+constexpr int kDs = kGB + 4;    // a row's D in shared memory (16-byte rows)
+// R's blocks above the diagonal blocks of one batch: for group b, the rows of
+// the batch's earlier groups (16 b of them) by the group's 16 columns.
+constexpr int kRsFloats = 256 * (kGB / 16) * (kGB / 16 - 1) / 2;
 
 size_t al256(size_t x) { return (x + 255) & ~size_t{255}; }
 
@@ -100,11 +120,9 @@ __device__ int local_sweep_f32(const float* w, const float* h16, const ScaleCons
   const float S = sc.S;
   const int b = clamp_code(e4m3_code_rne_sat(__fdiv_rn(__fdiv_rn(a, 6.0f), S)));
   const CandEntry* ce = tab + (b + lo + kTabOffset);
-  float Lf[16];
   uint32_t kbest = 0xFFFFFFFFu, ksec = 0xFFFFFFFFu;
   auto cand = [&](int i) {
     const float Li = fast_candidate_loss<kWeighted>(y2, h2, ce[i]);
-    Lf[i] = Li;
     const uint32_t key = (__float_as_uint(Li) & ~0xFu) | static_cast<uint32_t>(i);
     ksec = min(ksec, max(kbest, key));
     kbest = min(kbest, key);
@@ -141,7 +159,8 @@ __device__ int local_sweep_f32(const float* w, const float* h16, const ScaleCons
     double bestd = __longlong_as_double(0x7FF0000000000000ll);
     int bid = bi;
     for (int i = 0; i < K; ++i) {
-      if (Lf[i] > T) continue;
+      // the fast loss again (flagged groups are rare; no per-candidate array)
+      if (fast_candidate_loss<kWeighted>(y2, h2, ce[i]) > T) continue;
       const CandEntry t = ce[i];
       const float ivl = t.iv * (1.0f - 0x1p-20f);
       const double vS = __dmul_rn(static_cast<double>(t.v), static_cast<double>(S));
@@ -239,31 +258,26 @@ gptq_prep_kernel(float* __restrict__ H, int64_t in, float damp, uint8_t* __restr
   for (int64_t j = threadIdx.x; j < in; j += blockDim.x) H[j * in + j] += lam;
 }
 
-// FP32 working copy of W (row stride in), dead columns zero.
-__global__ void __launch_bounds__(256)
-gptq_wcopy_kernel(const uint16_t* __restrict__ W, int64_t out, int64_t in, int64_t ldw,
-                  const uint8_t* __restrict__ dead, float* __restrict__ Wf) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < out * in;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / in, j = i - r * in;
-    Wf[i] = dead[j] ? 0.0f : bf16_lo(W[r * ldw + j]);
-  }
-}
-
-// In place: a[r][c] <-> a[n-1-c][n-1-r] (reflection about the anti-diagonal),
-// one thread per pair r + c < n - 1.
+// In place: a[r][c] <-> a[n-1-c][n-1-r] (reflection about the anti-diagonal;
+// n a multiple of 16).  One 16 x 16 thread block per pair of 16 x 16 tiles:
+// tile (bi, bj) pairs with tile (t-1-bj, t-1-bi), t = n / 16, so element
+// (y, x) of the first is element (15-x, 15-y) of the second; blocks with
+// bi + bj > t - 1 have nothing to do.  Both tiles are read and written in
+// 16-float row segments through shared memory.
 __global__ void __launch_bounds__(256)
 antitranspose_kernel(float* __restrict__ a, int64_t n) {
-  const int64_t total = n * n;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / n, c = i - r * n;
-    if (r + c >= n - 1) continue;
-    const int64_t o = (n - 1 - c) * n + (n - 1 - r);
-    const float t = a[i];
-    a[i] = a[o];
-    a[o] = t;
-  }
+  __shared__ float ta[16][17], tb[16][17];
+  const int64_t t = n / 16;
+  const int64_t bi = blockIdx.y, bj = blockIdx.x;
+  if (bi + bj > t - 1) return;
+  const int x = threadIdx.x & 15, y = threadIdx.x >> 4;
+  float* A = a + (16 * bi + y) * n + 16 * bj + x;
+  float* B = a + (16 * (t - 1 - bj) + y) * n + 16 * (t - 1 - bi) + x;
+  ta[y][x] = *A;
+  tb[y][x] = *B;
+  __syncthreads();
+  *A = tb[15 - x][15 - y];
+  if (bi + bj < t - 1) *B = ta[15 - x][15 - y];
 }
 
 // A failed Cholesky or inverse (devInfo != 0: the damped Hessian is not
@@ -274,56 +288,225 @@ __global__ void gptq_status_kernel(const int* __restrict__ info, int n, int* sta
   if (bad && status) *status = -9;  // NVFP4_ERR_NUMERIC
 }
 
-// One lazy batch [j0, j0 + nb) of GPTQ's columns for kGT rows per CTA.
-// Dynamic shared memory: U's batch triangle [kGB][kGB] then the rows'
-// weights [kGT][kGB + 1].
-template <bool kWeighted, int kK>
-__global__ void __launch_bounds__(kGT)
-gptq_block_kernel(const float* __restrict__ Wf, int64_t out, int64_t in, int64_t j0, int nb,
-                  const float* __restrict__ U, const float* __restrict__ h,
-                  const float* __restrict__ Sp, int lo, int hi, uint8_t* __restrict__ codes,
-                  uint8_t* __restrict__ scales, float* __restrict__ Err) {
+// The inverses of R's 16 x 16 diagonal blocks (upper triangular), FP64 back
+// substitution, one thread per column of an inverse: Ud[blk][i][k] =
+// (R_blk^-1)[i][k], zero below the diagonal.  R row-major with stride in;
+// entries below R's diagonal are not read.
+__global__ void __launch_bounds__(128)
+gptq_udiag_kernel(const float* __restrict__ R, int64_t in, float* __restrict__ Ud) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= in) return;  // in / 16 blocks x 16 columns
+  const int64_t blk = idx >> 4;
+  const int k = static_cast<int>(idx & 15);
+  const float* Rb = R + blk * 16 * in + blk * 16;
+  double x[16];
+#pragma unroll
+  for (int i = 15; i >= 0; --i) {
+    if (i > k) {
+      x[i] = 0.0;
+    } else {
+      double s = i == k ? 1.0 : 0.0;
+#pragma unroll
+      for (int l = i + 1; l < 16; ++l)
+        if (l <= k) s -= static_cast<double>(Rb[i * in + l]) * x[l];
+      x[i] = s / static_cast<double>(Rb[i * in + i]);
+    }
+  }
+  float* o = Ud + blk * 256 + k;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o[i * 16] = static_cast<float>(x[i]);
+}
+
+// The TF32 head of an FP32 value (10 explicit mantissa bits, rounded to
+// nearest; truncated where rounding would overflow); x - head is exact.
+__device__ __forceinline__ float tf32_head(float x) {
+  const uint32_t u = __float_as_uint(x);
+  uint32_t hbits = (u + 0x1000u) & 0xFFFFE000u;
+  if ((hbits & 0x7F800000u) == 0x7F800000u) hbits = u & 0xFFFFE000u;
+  return __uint_as_float(hbits);
+}
+
+// One 128-row slice of the B operand of a split update GEMM: rows
+// [r0, r0 + kGB) of R, columns [c0, c0 + m), as [R_hi; R_lo; R_hi] (kCat rows
+// of Rcat, row stride ldr).  blockIdx.y is the row.
+__global__ void __launch_bounds__(256)
+gptq_rsplit_kernel(const float* __restrict__ R, int64_t in, int64_t r0, int64_t c0, int64_t m,
+                   float* __restrict__ Rcat, int64_t ldr) {
+  const int64_t rr = blockIdx.y;
+  const float* src = R + (r0 + rr) * in + c0;
+  float* dst = Rcat + rr * ldr;
+  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < m;
+       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float x = src[c];
+    const float hd = tf32_head(x);
+    dst[c] = hd;
+    dst[kGB * ldr + c] = x - hd;
+    dst[2 * kGB * ldr + c] = hd;
+  }
+}
+
+// One lazy batch [j0, j0 + nb) of GPTQ's columns in the R form, one thread per
+// row, kT rows per CTA.  Per 16-column group at g0 the thread
+//   * sums v = P[r, grp] + D[r, j0:g0] R[j0:g0, grp] (P holds the earlier
+//     batches' sums, D the batch's earlier groups, in shared memory);
+//   * forms the current weights w = W[r, grp] + v U_grp;
+//   * runs the local call on w (the group's E4M3 scale code);
+//   * quantizes each column at its turn -- exact E2M1 decision, D = W - q,
+//     err = (w - q) R_jj -- and updates the group's later columns by
+//     w_k -= err U_jk;
+// and writes the batch's D as [D_hi | D_hi | D_lo] (kCat columns from Dcat,
+// row stride ldd) for the split update GEMMs.  Dynamic shared memory: R's blocks above the diagonal
+// blocks (kRsFloats), the groups' U blocks (8 x 256), the rows' D (kT x kDs).
+template <bool kWeighted, int kK, int kT>
+__global__ void __launch_bounds__(kT)
+gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* __restrict__ dead,
+                   int64_t out, int64_t in, int64_t j0, int nb, const float* __restrict__ P,
+                   const float* __restrict__ R, const float* __restrict__ Ud,
+                   const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
+                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                   float* __restrict__ Dcat, int64_t ldd) {
   extern __shared__ __align__(16) float gsm[];
   __shared__ CandEntry tab[kTabSize];
   __shared__ float hb[kGB];
-  float* Ub = gsm;
-  float* wr = gsm + kGB * kGB;
+  __shared__ float rdiag[kGB];
+  __shared__ uint8_t deadb[kGB];
+  float* Rs = gsm;
+  float* Us = gsm + kRsFloats;
+  float* Ds = Us + (kGB / 16) * 256;
   fill_candidate_table(tab);
   const int t = threadIdx.x;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kGT;
-  for (int idx = t; idx < nb * nb; idx += kGT) {
-    const int i = idx / nb, k = idx - i * nb;
-    Ub[i * kGB + k] = k >= i ? U[(j0 + i) * in + j0 + k] : 0.0f;
+  const int ng = nb / 16;
+  // group b's block: R[j0 + i][j0 + 16 b + k], i < 16 b, at Rs + 128 b (b - 1) + 16 i + k.
+  // Every copy is a 16-byte cp.async (R's rows and Ud are 64-byte aligned:
+  // in % 16 == 0, j0 % 128 == 0), all in flight before one wait.
+  for (int b = 1; b < ng; ++b) {
+    float* dst = Rs + 128 * b * (b - 1);
+    for (int c = t; c < 64 * b; c += kT) {  // 16 b rows x 4 chunks
+      const int i = c >> 2, q = c & 3;
+      cp_async16(dst + 16 * i + 4 * q, R + (j0 + i) * in + j0 + 16 * b + 4 * q);
+    }
   }
-  for (int idx = t; idx < kGT * nb; idx += kGT) {
-    const int rr = idx / nb, k = idx - rr * nb;
-    const int64_t r = r0 + rr;
-    wr[rr * (kGB + 1) + k] = r < out ? Wf[r * in + j0 + k] : 0.0f;
+  for (int c = t; c < ng * 64; c += kT) cp_async16(Us + 4 * c, Ud + (j0 / 16) * 256 + 4 * c);
+  cp_async_commit();
+  for (int k = t; k < nb; k += kT) {
+    rdiag[k] = R[(j0 + k) * in + j0 + k];
+    deadb[k] = dead[j0 + k];
+    if (kWeighted) hb[k] = h[j0 + k];
   }
-  if (kWeighted)
-    for (int k = t; k < nb; k += kGT) hb[k] = h[j0 + k];
+  cp_async_wait<0>();
   __syncthreads();
-  const int64_t r = r0 + t;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * kT + t;
   if (r >= out) return;  // after the kernel's only barrier
   const ScaleConsts sc = scale_consts(*Sp);
   const int K = hi - lo + 1;
-  float* w = wr + t * (kGB + 1);
+  float* ds = Ds + t * kDs;
+  const float* prow = P + r * in + j0;
+  const uint16_t* wrow = W + r * ldw + j0;
+  float* dcat = Dcat + r * ldd;
   const int64_t G = in / 16;
-  for (int g = 0; g < nb / 16; ++g) {
-    float wg[16];
+  // A group's P (16 floats) and W (16 bf16, as 8 pairs) are loaded one group
+  // ahead, so their latency hides behind the previous group's sweep.  W takes
+  // two 16-byte loads where its rows allow, else 16 two-byte loads.
+  const bool w_vec = (reinterpret_cast<uintptr_t>(W) & 15u) == 0 && ldw % 8 == 0;
+  float4 pn[4];
+  uint32_t wn[8];
+  auto load_group = [&](int g) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) wg[j] = w[16 * g + j];
-    const int code = local_sweep_f32<kWeighted, kK>(wg, kWeighted ? hb + 16 * g : nullptr, sc,
+    for (int q = 0; q < 4; ++q) pn[q] = reinterpret_cast<const float4*>(prow + 16 * g)[q];
+    if (w_vec) {
+      const uint4 a = reinterpret_cast<const uint4*>(wrow + 16 * g)[0];
+      const uint4 b = reinterpret_cast<const uint4*>(wrow + 16 * g)[1];
+      wn[0] = a.x; wn[1] = a.y; wn[2] = a.z; wn[3] = a.w;
+      wn[4] = b.x; wn[5] = b.y; wn[6] = b.z; wn[7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        wn[i] = static_cast<uint32_t>(wrow[16 * g + 2 * i]) |
+                (static_cast<uint32_t>(wrow[16 * g + 2 * i + 1]) << 16);
+    }
+  };
+  load_group(0);
+  for (int g = 0; g < ng; ++g) {
+    f32x2_t v2[8];
+    uint32_t wc[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      v2[2 * q] = f2_pack(pn[q].x, pn[q].y);
+      v2[2 * q + 1] = f2_pack(pn[q].z, pn[q].w);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wc[i] = wn[i];
+    if (g + 1 < ng) load_group(g + 1);
+    const float* rs = Rs + 128 * g * (g - 1);
+    for (int i = 0; i < 16 * g; i += 4) {
+      const float4 d4 = *reinterpret_cast<const float4*>(ds + i);
+      const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const f32x2_t d2 = f2_pack(dv[u], dv[u]);
+        const float4* rr = reinterpret_cast<const float4*>(rs + (i + u) * 16);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 x = rr[q];
+          v2[2 * q] = f2_fma(d2, f2_pack(x.x, x.y), v2[2 * q]);
+          v2[2 * q + 1] = f2_fma(d2, f2_pack(x.z, x.w), v2[2 * q + 1]);
+        }
+      }
+    }
+    float v[16], w[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f2_unpack(v2[i], v[2 * i], v[2 * i + 1]);
+    // the group's original weights (dead columns zero), kept as bf16 pairs
+    auto w0 = [&](int j) {
+      const float wj = (j & 1) ? bf16_hi(wc[j >> 1]) : bf16_lo(wc[j >> 1]);
+      return deadb[16 * g + j] ? 0.0f : wj;
+    };
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = w0(j);
+    const float* ug = Us + 256 * g;
+    // row i of the group's U block, columns 4 * (i / 4) .. 15, as float4 loads
+    auto urow = [&](int i, float (&u)[16]) {
+#pragma unroll
+      for (int q = i / 4; q < 4; ++q) {
+        const float4 x = reinterpret_cast<const float4*>(ug + i * 16)[q];
+        u[4 * q] = x.x;
+        u[4 * q + 1] = x.y;
+        u[4 * q + 2] = x.z;
+        u[4 * q + 3] = x.w;
+      }
+    };
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float u[16];
+      urow(i, u);
+#pragma unroll
+      for (int k = i; k < 16; ++k) w[k] = fmaf(v[i], u[k], w[k]);
+    }
+    const int code = local_sweep_f32<kWeighted, kK>(w, kWeighted ? hb + 16 * g : nullptr, sc,
                                                     tab, lo, K);
     uint32_t packed[2] = {0u, 0u};
-    for (int i = 0; i < 16; ++i) {
-      const int j = 16 * g + i;
-      const float wv = w[j];
+    float dl[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
       float q;
-      packed[i >> 3] |= quantize_one(wv, code, sc, tab, q) << (4 * (i & 7));
-      const float err = (wv - q) / Ub[j * kGB + j];
-      Err[r * kGB + j] = err;
-      for (int k = j + 1; k < nb; ++k) w[k] = fmaf(-err, Ub[j * kGB + k], w[k]);
+      packed[j >> 3] |= quantize_one(w[j], code, sc, tab, q) << (4 * (j & 7));
+      dl[j] = w0(j) - q;
+      const float err = (w[j] - q) * rdiag[16 * g + j];
+      float u[16];
+      urow(j, u);
+#pragma unroll
+      for (int k = j + 1; k < 16; ++k) w[k] = fmaf(-err, u[k], w[k]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 d4 = make_float4(dl[4 * q], dl[4 * q + 1], dl[4 * q + 2], dl[4 * q + 3]);
+      *reinterpret_cast<float4*>(ds + 16 * g + 4 * q) = d4;
+      const float4 hd = make_float4(tf32_head(d4.x), tf32_head(d4.y), tf32_head(d4.z),
+                                    tf32_head(d4.w));
+      const float4 tl = make_float4(d4.x - hd.x, d4.y - hd.y, d4.z - hd.z, d4.w - hd.w);
+      *reinterpret_cast<float4*>(dcat + 16 * g + 4 * q) = hd;
+      *reinterpret_cast<float4*>(dcat + kGB + 16 * g + 4 * q) = hd;
+      *reinterpret_cast<float4*>(dcat + 2 * kGB + 16 * g + 4 * q) = tl;
     }
     const int64_t gg = j0 / 16 + g;
     *reinterpret_cast<uint2*>(codes + r * (G * 8) + gg * 8) = make_uint2(packed[0], packed[1]);
@@ -361,10 +544,61 @@ bool handles_for_current_device(Handles** out) {
   return true;
 }
 
+// Opt-in phase timing: CUDA event pairs recorded on the call's stream around
+// its phases, summed per phase when read.  Process-wide, guarded by the
+// handles' mutex; events are created on the device of the first timed call,
+// and calls on another device are not timed.
+struct PhaseTimer {
+  bool on = false;
+  int device = -1;
+  struct Pair {
+    cudaEvent_t a = nullptr, b = nullptr;
+    int phase = 0;
+  };
+  std::vector<Pair> pairs;
+  size_t used = 0;
+  bool overflow = false;
+};
+PhaseTimer g_timer;
+constexpr size_t kTimerPairs = 8192;
+
+// Starts interval `phase` on `s`; returns its index, or -1 when not timing.
+int timer_begin(int phase, cudaStream_t s) {
+  PhaseTimer& T = g_timer;
+  if (!T.on) return -1;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != T.device) return -1;
+  if (T.used == T.pairs.size()) {
+    if (T.pairs.size() >= kTimerPairs) {
+      T.overflow = true;
+      return -1;
+    }
+    PhaseTimer::Pair p;
+    if (cudaEventCreate(&p.a) != cudaSuccess || cudaEventCreate(&p.b) != cudaSuccess) {
+      cudaGetLastError();
+      T.overflow = true;
+      return -1;
+    }
+    T.pairs.push_back(p);
+  }
+  PhaseTimer::Pair& p = T.pairs[T.used];
+  p.phase = phase;
+  if (cudaEventRecord(p.a, s) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return static_cast<int>(T.used++);
+}
+
+void timer_end(int idx, cudaStream_t s) {
+  if (idx < 0) return;
+  if (cudaEventRecord(g_timer.pairs[idx].b, s) != cudaSuccess) cudaGetLastError();
+}
+
 struct GptqLayout {
-  size_t h_ws = 0, s_ws = 0, H = 0, Wf = 0, Err = 0, dead = 0, info = 0, lapack = 0, blas = 0;
+  size_t h_ws = 0, s_ws = 0, H = 0, P = 0, Dcat = 0, Rbig = 0, Rsmall = 0, Ud = 0, dead = 0,
+         info = 0, lapack = 0, blas = 0;
   size_t bytes = 0;
-  size_t lapack_bytes = 0, host_bytes = 0;
   int lwork = 0;
   LanePlan dplan, gplan;
 };
@@ -374,51 +608,69 @@ constexpr size_t kBlasWorkspace = 32u << 20;
 bool gptq_layout(int64_t out, int64_t in, int64_t tokens, int sms, Handles* hd, GptqLayout* L) {
   L->dplan = diag_hessian_plan(tokens, in, sms);
   L->gplan = global_scale_plan(out, in, sms);
-  int lw1 = 0;
+  int lw = 0;
   if (cusolverDnSpotrf_bufferSize(hd->solver, CUBLAS_FILL_MODE_LOWER, static_cast<int>(in),
-                                  nullptr, static_cast<int>(in), &lw1) != CUSOLVER_STATUS_SUCCESS)
+                                  nullptr, static_cast<int>(in), &lw) != CUSOLVER_STATUS_SUCCESS)
     return false;
-  size_t dev_b = 0, host_b = 0;
-  if (cusolverDnXtrtri_bufferSize(hd->solver, CUBLAS_FILL_MODE_LOWER, CUBLAS_DIAG_NON_UNIT, in,
-                                  CUDA_R_32F, nullptr, in, &dev_b, &host_b) !=
-      CUSOLVER_STATUS_SUCCESS)
-    return false;
-  L->lwork = lw1;
-  L->lapack_bytes = std::max(static_cast<size_t>(lw1) * sizeof(float), dev_b);
-  L->host_bytes = host_b;
+  L->lwork = lw;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off = al256(off + std::max<size_t>(bytes, 4));
     return o;
   };
+  const size_t n = static_cast<size_t>(in), o = static_cast<size_t>(out);
   L->h_ws = take(diag_hessian_workspace_bytes(L->dplan, in));
   L->s_ws = take(global_scale_workspace_bytes(L->gplan));
-  L->H = take(static_cast<size_t>(in) * static_cast<size_t>(in) * sizeof(float));
-  L->Wf = take(static_cast<size_t>(out) * static_cast<size_t>(in) * sizeof(float));
-  L->Err = take(static_cast<size_t>(out) * kGB * sizeof(float));
-  L->dead = take(static_cast<size_t>(in));
-  L->info = take(3 * sizeof(int));
-  L->lapack = take(L->lapack_bytes);
+  L->H = take(n * n * sizeof(float));
+  L->P = take(o * n * sizeof(float));
+  L->Dcat = take(o * kCat * kSub * sizeof(float));
+  L->Rbig = take(static_cast<size_t>(kCat) * kSub * n * sizeof(float));
+  L->Rsmall = take(static_cast<size_t>(kCat) * (kSub - 1) * kGB * sizeof(float));
+  L->Ud = take(n * 16 * sizeof(float));
+  L->dead = take(n);
+  L->info = take(sizeof(int));
+  L->lapack = take(static_cast<size_t>(lw) * sizeof(float));
   L->blas = take(kBlasWorkspace);
   L->bytes = off;
   return true;
 }
 
-template <bool kW, int kKK>
-cudaError_t launch_block(const float* Wf, int64_t out, int64_t in, int64_t j0, int nb,
-                         const float* U, const float* h, const float* S, int lo, int hi,
-                         uint8_t* codes, uint8_t* scales, float* Err, cudaStream_t s) {
-  constexpr size_t smem = (static_cast<size_t>(kGB) * kGB + static_cast<size_t>(kGT) * (kGB + 1)) *
-                          sizeof(float);
+// Rows per CTA of the batch kernel: 128 (two CTAs per SM) when that still
+// fills every SM, else 32.
+constexpr size_t rblock_smem(int rows) {
+  return (static_cast<size_t>(kRsFloats) + (kGB / 16) * 256 + static_cast<size_t>(rows) * kDs) *
+         sizeof(float);
+}
+
+template <bool kW, int kKK, int kT>
+cudaError_t launch_rblock_t(const uint16_t* W, int64_t ldw, const uint8_t* dead, int64_t out,
+                            int64_t in, int64_t j0, int nb, const float* P, const float* R,
+                            const float* Ud, const float* h, const float* S, int lo, int hi,
+                            uint8_t* codes, uint8_t* scales, float* Dcat, int64_t ldd,
+                            cudaStream_t s) {
+  constexpr size_t smem = rblock_smem(kT);
   static const cudaError_t attr = cudaFuncSetAttribute(
-      reinterpret_cast<const void*>(&gptq_block_kernel<kW, kKK>),
+      reinterpret_cast<const void*>(&gptq_rblock_kernel<kW, kKK, kT>),
       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (attr != cudaSuccess) return attr;
-  const unsigned blocks = static_cast<unsigned>((out + kGT - 1) / kGT);
-  gptq_block_kernel<kW, kKK><<<blocks, kGT, smem, s>>>(Wf, out, in, j0, nb, U, h, S, lo, hi, codes,
-                                                       scales, Err);
+  const unsigned blocks = static_cast<unsigned>((out + kT - 1) / kT);
+  gptq_rblock_kernel<kW, kKK, kT><<<blocks, kT, smem, s>>>(W, ldw, dead, out, in, j0, nb, P, R, Ud,
+                                                           h, S, lo, hi, codes, scales, Dcat, ldd);
   return cudaGetLastError();
+}
+
+template <bool kW, int kKK>
+cudaError_t launch_rblock(const uint16_t* W, int64_t ldw, const uint8_t* dead, int64_t out,
+                          int64_t in, int64_t j0, int nb, const float* P, const float* R,
+                          const float* Ud, const float* h, const float* S, int lo, int hi,
+                          uint8_t* codes, uint8_t* scales, float* Dcat, int64_t ldd, int sms,
+                          cudaStream_t s) {
+  if ((out + 127) / 128 >= static_cast<int64_t>(sms))
+    return launch_rblock_t<kW, kKK, 128>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi,
+                                         codes, scales, Dcat, ldd, s);
+  return launch_rblock_t<kW, kKK, 32>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi, codes,
+                                      scales, Dcat, ldd, s);
 }
 
 }  // namespace
@@ -468,8 +720,11 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
   if (workspace_bytes < L.bytes) return cudaErrorInvalidValue;
   char* ws = static_cast<char*>(workspace);
   float* H = reinterpret_cast<float*>(ws + L.H);
-  float* Wf = reinterpret_cast<float*>(ws + L.Wf);
-  float* Err = reinterpret_cast<float*>(ws + L.Err);
+  float* P = reinterpret_cast<float*>(ws + L.P);
+  float* Dcat = reinterpret_cast<float*>(ws + L.Dcat);
+  float* Rbig = reinterpret_cast<float*>(ws + L.Rbig);
+  float* Rsmall = reinterpret_cast<float*>(ws + L.Rsmall);
+  float* Ud = reinterpret_cast<float*>(ws + L.Ud);
   uint8_t* dead = reinterpret_cast<uint8_t*>(ws + L.dead);
   int* info = reinterpret_cast<int*>(ws + L.info);
   float* lapack = reinterpret_cast<float*>(ws + L.lapack);
@@ -480,10 +735,10 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
       !blas_ok(cublasSetWorkspace(hd->blas, ws + L.blas, kBlasWorkspace)) ||
       !lapack_ok(cusolverDnSetStream(hd->solver, stream)))
     return cudaErrorUnknown;
-  // plain FP32 GEMMs (no TF32 or emulated paths: the same arithmetic whichever
-  // cuBLAS build the process has loaded)
+  // the compute types are given per call; the handle's math mode stays the default
   if (!blas_ok(cublasSetMathMode(hd->blas, CUBLAS_DEFAULT_MATH))) return cudaErrorUnknown;
   // h and S with this library's kernels
+  int tm = timer_begin(NVFP4_GPTQ_PHASE_REDUCTIONS, stream);
   if ((e = launch_diag_hessian(X, tokens, in, ldx, h, 0, reinterpret_cast<float*>(ws + L.h_ws),
                                L.dplan, stream)) != cudaSuccess)
     return e;
@@ -491,70 +746,147 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
                                reinterpret_cast<uint32_t*>(ws + L.s_ws), L.gplan, stream)) !=
       cudaSuccess)
     return e;
+  timer_end(tm, stream);
+  tm = timer_begin(NVFP4_GPTQ_PHASE_GRAM, stream);
   // H = X^T X: X row-major [tokens, ldx] is column-major [ldx, tokens], so
-  // H = X_cm X_cm^T, bf16 products exact, FP32 accumulation
+  // H = X_cm X_cm^T, bf16 products exact, FP32 accumulation.  Only H's
+  // column-major lower triangle is read later (the reflection keeps each
+  // triangle in place and potrf reads the lower one), so for in >= 4096 H is
+  // built from the 10 blocks (I, J), I >= J, of a 4 x 4 split -- 10/16 of the
+  // products; the blocks above the diagonal are left unwritten.
   const float one = 1.0f, zero = 0.0f;
   if (tokens > 0) {
-    if (!blas_ok(cublasGemmEx(hd->blas, CUBLAS_OP_N, CUBLAS_OP_T, static_cast<int>(in),
-                              static_cast<int>(in), static_cast<int>(tokens), &one, X, CUDA_R_16BF,
-                              static_cast<int>(ldx), X, CUDA_R_16BF, static_cast<int>(ldx), &zero,
-                              H, CUDA_R_32F, static_cast<int>(in), CUBLAS_COMPUTE_32F,
-                              CUBLAS_GEMM_DEFAULT)))
-      return cudaErrorUnknown;
+    const int nsplit = in >= 4096 ? 4 : 1;
+    int64_t edge[5];
+    for (int k = 0; k <= nsplit; ++k) edge[k] = (in * k / nsplit) / 16 * 16;
+    edge[nsplit] = in;
+    for (int bi = 0; bi < nsplit; ++bi)
+      for (int bj = 0; bj <= bi; ++bj) {
+        const int64_t i0 = edge[bi], j0 = edge[bj];
+        if (!blas_ok(cublasGemmEx(hd->blas, CUBLAS_OP_N, CUBLAS_OP_T,
+                                  static_cast<int>(edge[bi + 1] - i0),
+                                  static_cast<int>(edge[bj + 1] - j0), static_cast<int>(tokens),
+                                  &one, X + i0, CUDA_R_16BF, static_cast<int>(ldx), X + j0,
+                                  CUDA_R_16BF, static_cast<int>(ldx), &zero, H + i0 + j0 * in,
+                                  CUDA_R_32F, static_cast<int>(in), CUBLAS_COMPUTE_32F,
+                                  CUBLAS_GEMM_DEFAULT)))
+          return cudaErrorUnknown;
+      }
   } else if ((e = cudaMemsetAsync(H, 0, static_cast<size_t>(in) * in * sizeof(float), stream)) !=
              cudaSuccess) {
     return e;
   }
+  timer_end(tm, stream);
+  tm = timer_begin(NVFP4_GPTQ_PHASE_FACTOR, stream);
   gptq_prep_kernel<<<1, 256, 0, stream>>>(H, in, damp, dead);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  {
-    const int64_t n = out * in;
-    int64_t blocks = (n + 255) / 256;
-    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
-    gptq_wcopy_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(W, out, in, ldw, dead, Wf);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  // U = J L'^-1 J, L' the lower Cholesky factor of J H J (FP32)
+  // R = J L' J row-major, L' the lower Cholesky factor of J H J (FP32)
   const int n = static_cast<int>(in);
   auto reflect = [&]() {
-    int64_t blocks = (in * in + 255) / 256;
-    if (blocks > static_cast<int64_t>(sms) * 16) blocks = static_cast<int64_t>(sms) * 16;
-    antitranspose_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(H, in);
+    const dim3 grid(static_cast<unsigned>(in / 16), static_cast<unsigned>(in / 16));
+    antitranspose_kernel<<<grid, 256, 0, stream>>>(H, in);
     return cudaGetLastError();
   };
-  std::vector<char> host_scratch(L.host_bytes);
   if ((e = reflect()) != cudaSuccess) return e;
   if (!lapack_ok(cusolverDnSpotrf(hd->solver, CUBLAS_FILL_MODE_LOWER, n, H, n, lapack, L.lwork,
-                                  info)) ||
-      !lapack_ok(cusolverDnXtrtri(hd->solver, CUBLAS_FILL_MODE_LOWER, CUBLAS_DIAG_NON_UNIT, in,
-                                  CUDA_R_32F, H, in, lapack, L.lapack_bytes,
-                                  host_scratch.empty() ? nullptr : host_scratch.data(),
-                                  L.host_bytes, info + 1)))
+                                  info)))
     return cudaErrorUnknown;
   if ((e = reflect()) != cudaSuccess) return e;
-  gptq_status_kernel<<<1, 1, 0, stream>>>(info, 2, status);
+  gptq_status_kernel<<<1, 1, 0, stream>>>(info, 1, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const float* U = H;  // row-major U[j][k] for k >= j (the reflected L'^-1)
+  const float* R = H;  // row-major R[j][k] for k >= j
+  gptq_udiag_kernel<<<static_cast<unsigned>((in + 127) / 128), 128, 0, stream>>>(R, in, Ud);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(P, 0, static_cast<size_t>(out) * in * sizeof(float), stream)) !=
+      cudaSuccess)
+    return e;
+  timer_end(tm, stream);
   const int K = hi - lo + 1;
-  const float minus_one = -1.0f;
-  for (int64_t j0 = 0; j0 < in; j0 += kGB) {
-    const int nb = static_cast<int>(std::min<int64_t>(kGB, in - j0));
+  const uint8_t* dd = dead;
+  const int64_t ldd = static_cast<int64_t>(kCat) * kSub;
+  auto block_t = [&](int64_t c0, int nb, float* dcat) {
     if (weighted)
-      e = K == 16 ? launch_block<true, 16>(Wf, out, in, j0, nb, U, h, S, lo, hi, codes, scales, Err, stream)
-                  : launch_block<true, 0>(Wf, out, in, j0, nb, U, h, S, lo, hi, codes, scales, Err, stream);
-    else
-      e = K == 16 ? launch_block<false, 16>(Wf, out, in, j0, nb, U, nullptr, S, lo, hi, codes, scales, Err, stream)
-                  : launch_block<false, 0>(Wf, out, in, j0, nb, U, nullptr, S, lo, hi, codes, scales, Err, stream);
-    if (e != cudaSuccess) return e;
-    const int64_t j1 = j0 + nb;
-    if (j1 < in) {
-      // W[:, j1:] -= Err[:, :nb] U[j0:j1, j1:], all row-major: in column-major
-      // terms C^T (n2 x out) -= U_blk^T (n2 x nb) Err^T (nb x out)
-      if (!blas_ok(cublasSgemm(hd->blas, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(in - j1),
-                               static_cast<int>(out), nb, &minus_one, U + j0 * in + j1, n, Err,
-                               kGB, &one, Wf + j1, n)))
-        return cudaErrorUnknown;
+      return K == 16 ? launch_rblock<true, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, dcat, ldd, sms, stream)
+                     : launch_rblock<true, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, dcat, ldd, sms, stream);
+    return K == 16 ? launch_rblock<false, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, dcat, ldd, sms, stream)
+                   : launch_rblock<false, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, dcat, ldd, sms, stream);
+  };
+  auto block = [&](int64_t c0, int nb, float* dcat) {
+    const int t = timer_begin(NVFP4_GPTQ_PHASE_BATCH, stream);
+    const cudaError_t r = block_t(c0, nb, dcat);
+    timer_end(t, stream);
+    return r;
+  };
+  auto split = [&](int64_t r0, int64_t c0, int64_t m, float* rcat, int64_t ldr) {
+    const int t = timer_begin(NVFP4_GPTQ_PHASE_SPLIT, stream);
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>((m + 255) / 256, 8)), kGB);
+    gptq_rsplit_kernel<<<grid, 256, 0, stream>>>(R, in, r0, c0, m, rcat, ldr);
+    timer_end(t, stream);
+    return cudaGetLastError();
+  };
+  // P[:, c0 : c0 + m] += Dcat[:, :k] Rcat[:k, :m], all row-major: in
+  // column-major terms P^T (m x out) += Rcat^T (m x k) Dcat^T (k x out)
+  auto update = [&](int64_t c0, int64_t m, int k, const float* rcat, int64_t ldr) {
+    const int t = timer_begin(NVFP4_GPTQ_PHASE_UPDATE, stream);
+    const bool ok = blas_ok(cublasGemmEx(hd->blas, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(m),
+                                static_cast<int>(out), k, &one, rcat, CUDA_R_32F,
+                                static_cast<int>(ldr), Dcat, CUDA_R_32F, static_cast<int>(ldd), &one,
+                                P + c0, CUDA_R_32F, n, CUBLAS_COMPUTE_32F_FAST_TF32,
+                                CUBLAS_GEMM_DEFAULT));
+    timer_end(t, stream);
+    return ok;
+  };
+  constexpr int64_t kBatch = static_cast<int64_t>(kGB) * kSub;
+  for (int64_t j0 = 0; j0 < in; j0 += kBatch) {
+    const int64_t jend = std::min(j0 + kBatch, in);
+    const int nsub = static_cast<int>((jend - j0 + kGB - 1) / kGB);
+    for (int sb = 0; sb < nsub; ++sb) {
+      const int64_t c0 = j0 + static_cast<int64_t>(kGB) * sb;
+      const int nb = static_cast<int>(std::min<int64_t>(kGB, jend - c0));
+      if ((e = block(c0, nb, Dcat + static_cast<int64_t>(kCat) * sb)) != cudaSuccess) return e;
+      if (sb + 1 < nsub) {  // the batch's later half takes this half's columns
+        const int64_t c1 = c0 + nb;  // nb == kGB: only a batch's last half can be narrower
+        const int64_t m = std::min<int64_t>(kGB, jend - c1);
+        for (int s0 = 0; s0 <= sb; ++s0)
+          if ((e = split(j0 + static_cast<int64_t>(kGB) * s0, c1, m,
+                         Rsmall + static_cast<int64_t>(kCat) * s0 * kGB, kGB)) != cudaSuccess)
+            return e;
+        if (!update(c1, m, kCat * (sb + 1), Rsmall, kGB)) return cudaErrorUnknown;
+      }
     }
+    if (jend < in) {  // every later column takes the whole batch (all halves full)
+      for (int s0 = 0; s0 < nsub; ++s0)
+        if ((e = split(j0 + static_cast<int64_t>(kGB) * s0, jend, in - jend,
+                       Rbig + static_cast<int64_t>(kCat) * s0 * in, in)) != cudaSuccess)
+          return e;
+      if (!update(jend, in - jend, kCat * nsub, Rbig, in)) return cudaErrorUnknown;
+    }
+  }
+  return cudaSuccess;
+}
+
+void gptq_set_timing(bool on) {
+  std::lock_guard<std::mutex> lock(g_handles_mutex);
+  g_timer.on = on;
+  g_timer.used = 0;
+  g_timer.overflow = false;
+  if (on && g_timer.device < 0 && cudaGetDevice(&g_timer.device) != cudaSuccess) {
+    cudaGetLastError();
+    g_timer.on = false;
+  }
+}
+
+cudaError_t gptq_phase_times(float* ms, int n, bool* overflow) {
+  std::lock_guard<std::mutex> lock(g_handles_mutex);
+  for (int i = 0; i < n; ++i) ms[i] = 0.0f;
+  *overflow = g_timer.overflow;
+  for (size_t i = 0; i < g_timer.used; ++i) {
+    const PhaseTimer::Pair& p = g_timer.pairs[i];
+    cudaError_t e = cudaEventSynchronize(p.b);
+    float t = 0.0f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, p.a, p.b);
+    if (e != cudaSuccess) return e;
+    if (p.phase >= 0 && p.phase < n) ms[p.phase] += t;
   }
   return cudaSuccess;
 }

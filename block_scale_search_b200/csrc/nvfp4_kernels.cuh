@@ -163,6 +163,9 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               cudaStream_t stream);
 
 // H-Scale as GPTQ's local quantizer (gptq.cu).
+// Opt-in phase timing of launch_gptq (see nvfp4_gptq_set_timing).
+void gptq_set_timing(bool on);
+cudaError_t gptq_phase_times(float* ms, int n, bool* overflow);
 size_t gptq_workspace_bytes(int64_t out, int64_t in, int64_t tokens, int sms);
 cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw, const uint16_t* X,
                         int64_t tokens, int64_t ldx, float q_max, int lo, int hi, float damp,

@@ -298,7 +298,7 @@ extern "C" {
 
 size_t nvfp4_gptq_workspace_size(int64_t out, int64_t in, int64_t tokens) {
   constexpr int64_t kIntMax = (int64_t{1} << 31) - 1;
-  if (out <= 0 || in <= 0 || tokens < 0 || in % 16 != 0 || in > kIntMax || out > kIntMax ||
+  if (out <= 0 || in <= 0 || tokens < 0 || in % 16 != 0 || in > 16 * 65535 || out > kIntMax ||
       tokens > kIntMax)
     return 0;
   const int sms = current_sm_count();
@@ -318,8 +318,9 @@ int nvfp4_gptq_quantize(const void* W, int64_t out, int64_t in, int64_t ldw, con
     return NVFP4_ERR_INVALID_ARG;
   // cuBLAS and cuSOLVER take int sizes and leading dimensions
   constexpr int64_t kIntMax = (int64_t{1} << 31) - 1;
-  if (in % 16 != 0 || ldw < in || ldx < in || in > kIntMax || out > kIntMax || tokens > kIntMax ||
-      ldw > kMaxDim || ldx > kIntMax)
+  // in / 16 is also a grid dimension of the factor's reflection
+  if (in % 16 != 0 || ldw < in || ldx < in || in > 16 * 65535 || out > kIntMax ||
+      tokens > kIntMax || ldw > kMaxDim || ldx > kIntMax)
     return NVFP4_ERR_SHAPE;
   if (!std::isfinite(q_max) || !(q_max > 0.0f) || !std::isfinite(damp) || damp < 0.0f)
     return NVFP4_ERR_INVALID_ARG;
@@ -338,6 +339,20 @@ int nvfp4_gptq_quantize(const void* W, int64_t out, int64_t in, int64_t ldw, con
       static_cast<const uint16_t*>(W), out, in, ldw, static_cast<const uint16_t*>(X), tokens, ldx,
       q_max, lo, hi, damp, weighted != 0, codes, scales, S, h, status, workspace, workspace_bytes,
       sms, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_gptq_set_timing(int on) {
+  if (on != 0 && on != 1) return NVFP4_ERR_INVALID_ARG;
+  nvfp4::gptq_set_timing(on != 0);
+  return NVFP4_OK;
+}
+
+int nvfp4_gptq_phase_times(float* ms, int n) {
+  if (ms == nullptr || n < 0 || n > NVFP4_GPTQ_PHASES) return NVFP4_ERR_INVALID_ARG;
+  bool overflow = false;
+  const cudaError_t e = nvfp4::gptq_phase_times(ms, n, &overflow);
+  if (e != cudaSuccess) return cuda_status(e);
+  return overflow ? NVFP4_ERR_WORKSPACE : NVFP4_OK;
 }
 
 int nvfp4_scale_sweep_quantize_f32(const float* W, int64_t out, int64_t in, int64_t ldw,

@@ -393,7 +393,8 @@ int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, 
  * error-updated FP32 weights, with S = the global scale of the original W;
  * each column of the group is then quantized at its turn with that scale.
  *
- *   W        bf16 [out, ldw]; in % 16 == 0; out, in > 0; out, in < 2^31.
+ *   W        bf16 [out, ldw]; in % 16 == 0; out, in > 0; out < 2^31,
+ *            in <= 16 * 65535.
  *   X        bf16 [tokens, ldx], 16-byte aligned, ldx % 8 == 0; tokens >= 0,
  *            ldx >= in; tokens, ldx < 2^31 (the GEMM's int sizes).
  *   codes, scales, S, h  the NVFP4 result ([out, in/2], [out, in/16]), the
@@ -401,11 +402,19 @@ int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, 
  *   status   nullable device int: 0, NVFP4_ERR_NONFINITE (W holds Inf/NaN), or
  *            NVFP4_ERR_NUMERIC (the damped Hessian's Cholesky failed in FP32).
  *   workspace  nvfp4_gptq_workspace_size(out, in, tokens) bytes, 256-byte
- *            aligned (it holds H, an FP32 copy of W and the solver's scratch:
- *            about 4 (in^2 + out in) bytes).
- * Steps: h, S and the GPTQ batches are this library's kernels; X^T X and the
- * batches' updates of later columns are GEMMs (cuBLAS), the Cholesky factor
- * and inverse come from cuSOLVER.  The first call on a device creates the
+ *            aligned (it holds H and its Cholesky factor, the FP32 sums P
+ *            [out, in] of the propagated errors, a batch's errors and
+ *            factor rows for the update GEMMs and the solver's scratch:
+ *            about 4 (in^2 + out (in + 768) + 800 in) bytes).
+ * Steps: no inverse is formed.  The lower Cholesky factor of the reversed H
+ * gives H = R R^T with R upper (U = R^-1), and the columns run in the
+ * equivalent R form: W - Q = Err U, so Err = (W - Q) R, and a group's current
+ * weights are W_grp + ((W - Q)[:, <grp] R[<grp, grp]) R_grp^-1 with R_grp the
+ * group's 16 x 16 diagonal block.  h, S, the block inverses and the batches
+ * of columns are this library's kernels; X^T X and the batches' updates of
+ * later columns' sums are GEMMs (cuBLAS; the updates as three TF32
+ * tensor-core products of split FP32 operands), the Cholesky factor comes
+ * from cuSOLVER.  The first call on a device creates the
  * library's cuBLAS and cuSOLVER handles there, which hold a little device
  * memory until the process exits; every call's scratch is the caller's
  * workspace.  Calls are serialised on the host; asynchronous on `stream`.
@@ -418,6 +427,30 @@ int nvfp4_gptq_quantize(const void* W, int64_t out, int64_t in, int64_t ldw, con
                         int64_t tokens, int64_t ldx, float q_max, int lo, int hi, float damp,
                         int weighted, uint8_t* codes, uint8_t* scales, float* S, float* h,
                         int* status, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Opt-in phase timing of nvfp4_gptq_quantize, for profiling without external
+ * tools.  nvfp4_gptq_set_timing(1) starts it (and clears what was recorded);
+ * each later call records CUDA event pairs on its own stream around its
+ * phases (a few hundred per call, up to 8192 pairs in all; the events are
+ * created on the device current at the first nvfp4_gptq_set_timing(1) of the
+ * process, and calls on other devices are not timed).  nvfp4_gptq_phase_times waits for the recorded
+ * events and writes ms[p], the milliseconds spent in phase p summed over
+ * the timed calls, for p < n (at most NVFP4_GPTQ_PHASES); it returns
+ * NVFP4_ERR_WORKSPACE if the pairs ran out (the sums are then partial).
+ * nvfp4_gptq_set_timing(0) stops recording.  Host calls, serialised with
+ * nvfp4_gptq_quantize. */
+enum nvfp4_gptq_phase {
+    NVFP4_GPTQ_PHASE_REDUCTIONS = 0,  /* h and S                                    */
+    NVFP4_GPTQ_PHASE_GRAM = 1,        /* X^T X                                      */
+    NVFP4_GPTQ_PHASE_FACTOR = 2,      /* damping, Cholesky factor, block inverses   */
+    NVFP4_GPTQ_PHASE_BATCH = 3,       /* batch kernels: local call, quantization,
+                                         propagation inside a batch                 */
+    NVFP4_GPTQ_PHASE_SPLIT = 4,       /* TF32 splits of the factor's rows           */
+    NVFP4_GPTQ_PHASE_UPDATE = 5,      /* update GEMMs of later columns' sums        */
+    NVFP4_GPTQ_PHASES = 6
+};
+int nvfp4_gptq_set_timing(int on);
+int nvfp4_gptq_phase_times(float* ms, int n);
 
 /* The local call of nvfp4_gptq_quantize on its own: the windowed sweep of an
  * FP32 matrix W [out, ldw] (in % 16 == 0; h NULL = plain MSE; S a device

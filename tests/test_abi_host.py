@@ -339,7 +339,8 @@ def test_every_launching_entry_point_opens_an_nvtx_range():
             found[m.group(1)] = m.group(2).strip()
     queries = {"nvfp4_version", "nvfp4_last_cuda_error", "nvfp4_quantize_layer_order",
                "nvfp4_debug_checks_compiled", "nvfp4_debug_checks",
-               "nvfp4_quantize_grouped_layer_order", "nvfp4_debug_row_counters"}
+               "nvfp4_quantize_grouped_layer_order", "nvfp4_debug_row_counters",
+               "nvfp4_gptq_set_timing", "nvfp4_gptq_phase_times"}
     launching = {k: v for k, v in found.items() if k not in queries}
     assert len(launching) == 16, sorted(launching)
     for name, first in launching.items():
@@ -382,10 +383,16 @@ def test_gptq_validation(L):
     assert call(inp=250, ldw=256, ldx=256) == -2            # in % 16
     assert call(ldx=128) == -2                                # ldx < in
     assert call(tokens=1 << 31) == -2                        # beyond the GEMM's int sizes
+    assert call(inp=16 * 65536, ldw=16 * 65536, ldx=16 * 65536) == -2   # in / 16 > 65535
     assert call(lo=-10) == -4
     assert call(X=P + 8) == -3 and call(codes=P + 4) == -3 and call(h=P + 4) == -3
     assert call(ws=None) == -7 and call(ws=P + 64) == -3
     assert L.nvfp4_gptq_workspace_size(64, 250, 128) == 0
+    ms = (C.c_float * 6)()
+    assert L.nvfp4_gptq_set_timing(2) == -1
+    assert L.nvfp4_gptq_phase_times(None, 6) == -1 and L.nvfp4_gptq_phase_times(ms, 7) == -1
+    assert L.nvfp4_gptq_phase_times(ms, -1) == -1
+    assert L.nvfp4_gptq_workspace_size(64, 16 * 65536, 128) == 0
     g = L.nvfp4_scale_sweep_quantize_f32
     assert g(P, 4, 250, 256, None, P, -9, 6, P, P, None) == -2
     assert g(P, 4, 256, 256, None, P, -10, 6, P, P, None) == -4

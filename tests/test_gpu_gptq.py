@@ -99,7 +99,8 @@ def _correlated(n, tokens, seed):
 @pytest.mark.parametrize("out,n,tokens,seed,weighted,lo,hi", [
     (256, 512, 2048, 81, True, -9, 6), (128, 1024, 4096, 82, True, -9, 6),
     (192, 512, 2048, 83, False, -3, 7), (160, 768, 3072, 84, True, -8, 7),
-    (96, 528, 2048, 85, True, -9, 6)])   # a last batch of 16 columns
+    (96, 528, 2048, 85, True, -9, 6),    # a last lazy batch of 16 columns
+    (112, 400, 2048, 86, True, -9, 6)])  # a last lazy batch of 128 + 16 columns
 def test_correlated_inputs_follow_the_oracle(orc, nv, parity_report, out, n, tokens, seed,
                                              weighted, lo, hi):
     import workloads
@@ -154,3 +155,28 @@ def test_dead_columns_and_repeat_calls(nv):
     nib = _nibbles(codes.cpu().numpy(), 128, n)
     assert np.all(nib[:, 10] == 0) and np.all(nib[:, 32:48] == 0)
     assert torch.all(scales[:, 2] == 0)                # the group of all-dead columns
+
+
+def test_phase_timer_covers_the_call(nv):
+    """With the phase timer on, every phase of a GPTQ call records time, the
+    phases sum to no more than the calls' own event-timed span, and turning
+    the timer off clears it."""
+    import workloads
+    W = workloads.weight(256, 1024, 0.02, 0.005, 10.0, 91).to(DEV)
+    X = _correlated(1024, 2048, 92).to(DEV)
+    nv.gptq_quantize(W, X)                       # first call: handles, module load
+    torch.cuda.synchronize()
+    nv.nvfp4_gptq_set_timing(True)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(2):
+        nv.gptq_quantize(W, X)
+    t1.record()
+    torch.cuda.synchronize()
+    p = nv.nvfp4_gptq_phase_times()
+    nv.nvfp4_gptq_set_timing(False)
+    assert set(p) == set(nv.GPTQ_PHASES)
+    assert all(v > 0.0 for v in p.values()), p
+    assert sum(p.values()) <= t0.elapsed_time(t1) * 1.02, (p, t0.elapsed_time(t1))
+    assert sum(nv.nvfp4_gptq_phase_times().values()) == 0.0
