@@ -824,9 +824,20 @@ def run_activations(args, nv, rank, local, ws, dev):
         print(json.dumps(out), flush=True)
 
 
-GPTQ_WORKLOAD = ("gptq_llama33_70b_gate: GPTQ with the H-Scale local call on the 70B-shaped gate "
-                 "projection, W 28672x8192 bf16 N(0,0.015) 0.1% x10, X 65536x8192 bf16 "
-                 "lognormal(1.5) channel scales; damping 0.01; window [-9,+6]")
+GPTQ_WORKLOADS = {
+    # name: (out, in, tokens, description)
+    "gptq_llama33_70b_gate": (28672, 8192, 65536,
+                              "gptq_llama33_70b_gate: GPTQ with the H-Scale local call on the "
+                              "70B-shaped gate projection, W 28672x8192 bf16 N(0,0.015) 0.1% x10, "
+                              "X 65536x8192 bf16 lognormal(1.5) channel scales; damping 0.01; "
+                              "window [-9,+6]"),
+    # profiling size: the gate's rows (so the batch kernel's grid is the same), a
+    # quarter of its columns, an eighth of its tokens
+    "gptq_slice": (28672, 2048, 8192,
+                   "gptq_slice: GPTQ with the H-Scale local call, W 28672x2048 bf16 N(0,0.015) "
+                   "0.1% x10, X 8192x2048 bf16 lognormal(1.5) channel scales; damping 0.01; "
+                   "window [-9,+6] (profiling size)"),
+}
 
 
 def gptq_update_flops(out: int, n: int, gb: int = 128, sub: int = 2) -> float:
@@ -853,8 +864,9 @@ def run_gptq(args, nv, rank, local, ws, dev):
     stream) in a second pass of the same calls after the timed region."""
     import torch
     import workloads
-    W = workloads.weight(28672, 8192, 0.015, 0.001, 10.0, 401 + 97 * rank, dev)
-    X = workloads.calib(65536, 8192, 1.5, 441 + 97 * rank, dev)
+    o_, n_, t_, desc = GPTQ_WORKLOADS[args.workload]
+    W = workloads.weight(o_, n_, 0.015, 0.001, 10.0, 401 + 97 * rank, dev)
+    X = workloads.calib(t_, n_, 1.5, 441 + 97 * rank, dev)
     out, n = W.shape
     codes = torch.empty(out, n // 2, dtype=torch.uint8, device=dev)
     scales = torch.empty(out, n // 16, dtype=torch.uint8, device=dev)
@@ -919,8 +931,9 @@ def run_gptq(args, nv, rank, local, ws, dev):
                     "unit": "elem/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
                     "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
                     "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                    "config": {"workload": GPTQ_WORKLOAD, "window": [LO, HI], "q_max": 448.0,
-                               "l2": "inputs 1.54 GB per rank > 126 MB L2; no flush",
+                    "config": {"workload": desc, "window": [LO, HI], "q_max": 448.0,
+                               "l2": f"inputs {(out * n + t_ * n) * 2 / 1e9:.2f} GB per rank "
+                                     "> 126 MB L2; no flush",
                                "parallelism": f"weak: {ws} rank(s), one projection per rank"},
                     "roofline": roofline, "e2e": None, "gpu_launches": None,
                     "cpu_baseline": None, "clocks": clocks,
@@ -1104,7 +1117,7 @@ def main():
                          "calls with later weights' S and h on a second stream; auto: layer "
                          "(nvfp4_quantize_grouped_layer for the MoE layer)")
     ap.add_argument("--workload", default="llama33_70b_mlp",
-                    choices=list(WORKLOADS) + ["act_llama33_70b", "gptq_llama33_70b_gate"])
+                    choices=list(WORKLOADS) + ["act_llama33_70b"] + list(GPTQ_WORKLOADS))
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1118,7 +1131,7 @@ def main():
     rank, local, ws = init_dist()
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
-    if args.workload in ("act_llama33_70b", "gptq_llama33_70b_gate"):
+    if args.workload == "act_llama33_70b" or args.workload in GPTQ_WORKLOADS:
         (run_activations if args.workload == "act_llama33_70b" else run_gptq)(
             args, nv, rank, local, ws, dev)
         if ws > 1:

@@ -60,19 +60,23 @@ def decode(nib: np.ndarray, scale: np.ndarray, S: float) -> np.ndarray:
 
 
 def gptq_hscale(W, X, q_max: float = 448.0, lo: int = -9, hi: int = 6, damp: float = 0.01,
-                weighted: bool = True, trace=None):
+                weighted: bool = True, trace=None, S=None):
     """GPTQ with the H-Scale local call.  W: bf16 [out, in] (bits or torch);
     X: bf16 [tokens, in].  Returns (codes [out, in/2], scales [out, in/16], S,
     Q [out, in] the FP64 dequantized weights, h [in]).  trace(j, W, Q) is called
     after column j's error has been propagated, with the current FP64 weights
-    and the columns quantized so far."""
+    and the columns quantized so far.  S, if given, is the global scale to use
+    instead of W's own: rows are independent in GPTQ given H, so some rows of a
+    larger matrix run alone with that matrix's S give that matrix's rows."""
     Wb = _bf16_bits(W)
     Xb = _bf16_bits(X)
     out, n = Wb.shape
     assert n % 16 == 0 and Xb.shape[1] == n
-    S, _amax, st = global_scale(Wb, q_max)
-    if st != 0:
-        raise ValueError("non-finite weights")
+    if S is None:
+        S, _amax, st = global_scale(Wb, q_max)
+        if st != 0:
+            raise ValueError("non-finite weights")
+    S = np.float32(S)
     h = diag_hessian(Xb)
     U, dead, _H = inverse_cholesky_upper(Xb, damp)
     Wc = bf16_to_f64(Wb)
