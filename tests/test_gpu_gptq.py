@@ -157,6 +157,28 @@ def test_dead_columns_and_repeat_calls(nv):
     assert torch.all(scales[:, 2] == 0)                # the group of all-dead columns
 
 
+def test_cholesky_failure_is_reported_and_the_next_call_is_clean(nv):
+    """With no damping, calibration inputs of rank one make H = X^T X singular:
+    entries +-c_j (c_j with two significant bits) over 256 tokens give
+    H = 256 c c^T exactly in FP32, the factorization's second pivot is exactly
+    0, and the status word reads NVFP4_ERR_NUMERIC.  The outputs are then
+    undefined, but nothing faults, and the next call is unaffected."""
+    import workloads
+    n = 64
+    g = torch.Generator().manual_seed(93)
+    z = torch.where(torch.rand(256, 1, generator=g) < 0.5, -1.0, 1.0)
+    c = torch.tensor([1.0, 1.5, 2.0, 3.0]).repeat(n // 4).reshape(1, n)
+    X = (z * c).to(torch.bfloat16)
+    assert torch.equal(X.float(), z * c)                  # exactly rank one
+    W = workloads.weight(32, n, 0.02, 0.0, 1.0, 94, DEV)
+    *_, status = nv.gptq_quantize(W, X.to(DEV), damp=0.0)
+    torch.cuda.synchronize()
+    assert int(status.item()) == -9                      # NVFP4_ERR_NUMERIC
+    *_, status = nv.gptq_quantize(W, X.to(DEV), damp=0.01)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
 def test_phase_timer_covers_the_call(nv):
     """With the phase timer on, every phase of a GPTQ call records time, the
     phases sum to no more than the calls' own event-timed span, and turning
