@@ -840,10 +840,11 @@ GPTQ_WORKLOADS = {
 }
 
 
-def gptq_update_flops(out: int, n: int, gb: int = 128, sub: int = 2) -> float:
-    """TF32 flops of one GPTQ call's update GEMMs: per lazy batch of sub * gb
-    columns, a GEMM of K = 3 * gb (three split products) from its first half
-    into its second, and one of K = 3 * gb * sub into every later column."""
+def gptq_update_flops(out: int, n: int, gb: int = 128, sub: int = 4) -> float:
+    """Tensor-core flops of one GPTQ call's update GEMMs (three split FP16
+    products each): per lazy batch of sub parts of gb columns, after part s a
+    GEMM of K = 3 * gb * (s + 1) from the parts so far into the next part, and
+    after the batch one of K = 3 * gb * sub into every later column."""
     total = 0.0
     for j0 in range(0, n, gb * sub):
         jend = min(j0 + gb * sub, n)
@@ -909,17 +910,16 @@ def run_gptq(args, nv, rank, local, ws, dev):
     el = out * n
     _hbm, _kind, peaks = measured_peaks()
     bf16 = peaks.get("bf16_tflops_sustained")
-    tf32_ratio = 1.1 / 2.25            # nominal dense TF32 / bf16 on B200
-    peak = bf16 * tf32_ratio if bf16 else 1590.0 * tf32_ratio
+    peak = bf16 if bf16 else 1590.0    # dense FP16 runs at the bf16 rate on B200
     flops = gptq_update_flops(out, n)
     upd_ms = phases["update"]
     achieved = flops / (upd_ms * 1e-3) / 1e12 if upd_ms > 0 else None
-    roofline = {"kernel": "GPTQ update GEMMs (cuBLAS, 3 TF32 tensor-core products of split FP32 "
-                          "operands)",
+    roofline = {"kernel": "GPTQ update GEMMs (cuBLAS, 3 FP16 tensor-core products of split, "
+                          "scaled FP32 operands, FP32 accumulation)",
                 "bound": "tensor", "achieved": round(achieved, 1) if achieved else None,
                 "peak": round(peak, 1), "unit": "TFLOP/s",
-                "peak_source": ("measured bf16_tflops_sustained x nominal TF32/bf16 ratio 1.1/2.25"
-                                if bf16 else "fallback 1.59 PFLOP/s bf16 x 1.1/2.25"),
+                "peak_source": ("measured bf16_tflops_sustained (dense FP16 = bf16 rate)"
+                                if bf16 else "fallback 1.59 PFLOP/s bf16 (dense FP16 = bf16 rate)"),
                 "frac": round(achieved / peak, 4) if achieved else None,
                 "flops_per_call": flops,
                 "ms_per_call": round(upd_ms, 3),

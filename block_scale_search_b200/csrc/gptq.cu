@@ -32,20 +32,25 @@
 //     R (U is block upper triangular); inside the group the updates use U_grp
 //     and err_j = (w_j - q_j) R_jj.  gptq_udiag_kernel inverts the diagonal
 //     blocks (FP64);
-//   * GPTQ's lazy batches, 256 columns each, in two halves of 128:
-//     gptq_rblock_kernel runs the columns of one half, one thread per row --
-//     each group's sums from the earlier groups of the half, its current
+//   * GPTQ's lazy batches, 512 columns each, in four parts of 128:
+//     gptq_rblock_kernel runs the columns of one part, one thread per row --
+//     each group's sums from the earlier groups of the part, its current
 //     weights, the local call, the exact quantization and the in-group
-//     updates -- and writes the half's D.  A small GEMM adds the first half to
-//     the second half's sums; after the batch one GEMM adds the batch to every
-//     later column's sums: P[:, >] += D[:, batch] R[batch, >].  The GEMMs run
-//     on the tensor cores as three TF32 products, D_hi R_hi + D_hi R_lo +
-//     D_lo R_hi, with each FP32 operand split into its TF32 head and the
-//     remainder (gptq_rsplit_kernel for R; the batch kernel writes D's
-//     parts).  Each P element is read and written once per 256 columns.
+//     updates -- and writes the part's D.  After each part a small GEMM adds
+//     the batch's parts so far to the next part's sums; after the batch one
+//     GEMM adds the batch to every later column's sums:
+//     P[:, >] += D[:, batch] R[batch, >].  The GEMMs run
+//     on the tensor cores as three FP16 products with FP32 accumulation,
+//     D_hi R_hi + D_hi R_lo + D_lo R_hi: each FP32 operand, scaled by a power
+//     of two that keeps it inside FP16's range, is split into its FP16
+//     rounding and the FP16 rounding of the remainder (gptq_rsplit_kernel for
+//     R; the batch kernel writes D's parts); the GEMM's alpha undoes the
+//     scales exactly.  Each P element is read and written once per 512
+//     columns, and the GEMM's K (3 x 512) keeps its FP32 read-modify-write of
+//     P shorter than its products.
 // Rows are independent in GPTQ (R is shared), so the batch kernel needs no
 // communication between rows.  The device arithmetic is FP32 (the update GEMM
-// about 2^-18 relative per product): results drift from the FP64 oracle's
+// about 2^-21 relative per product): results drift from the FP64 oracle's
 // after a quantization decision flips, which a row then carries through its
 // later columns.
 #include <cublas_v2.h>
@@ -64,7 +69,7 @@ namespace {
 
 constexpr int kGB = 128;        // columns per batch kernel launch
 constexpr int kCat = 3 * kGB;   // K of the split update per 128 columns
-constexpr int kSub = 2;         // batch-kernel launches per lazy batch (256 columns)
+constexpr int kSub = 4;         // batch-kernel launches per lazy batch (512 columns)
 constexpr int kDs = kGB + 4;    // a row's D in shared memory (16-byte rows)
 // R's blocks above the diagonal blocks of one batch: for group b, the rows of
 // the batch's earlier groups (16 b of them) by the group's 16 columns.
@@ -235,10 +240,24 @@ sweep_f32_kernel(const float* __restrict__ W, int64_t out, int64_t G, int64_t ld
 }
 
 // Dead columns, damping: one CTA.  H is symmetric (row- or column-major alike).
+// Also the FP16 scales of the split update GEMMs, gs = {s_D, s_R, alpha, 1}:
+// powers of two with |D| s_D <= 2^14 and |R| s_R <= 2^14, where |D| = |W - q|
+// <= amax + 6 * 448 * S (amax ~ S * 6 q_max) and every entry of row i of R is
+// at most sqrt(H_ii) (H = R R^T); alpha = 1 / (s_D s_R).
+__device__ __forceinline__ int pow2_floor_exp(float ratio) {
+  if (!(ratio > 0.0f) || !isfinite(ratio)) return 0;
+  int e;
+  frexpf(ratio, &e);  // ratio in [2^(e-1), 2^e)
+  return max(-60, min(60, e - 1));
+}
+
 __global__ void __launch_bounds__(256)
-gptq_prep_kernel(float* __restrict__ H, int64_t in, float damp, uint8_t* __restrict__ dead) {
+gptq_prep_kernel(float* __restrict__ H, int64_t in, float damp, uint8_t* __restrict__ dead,
+                 const float* __restrict__ Sp, float q_max, float* __restrict__ gs) {
   __shared__ double part[256];
+  __shared__ float mx[256];
   double s = 0.0;
+  float m = 0.0f;
   for (int64_t j = threadIdx.x; j < in; j += blockDim.x) {
     float d = H[j * in + j];
     dead[j] = d == 0.0f ? 1 : 0;
@@ -247,15 +266,30 @@ gptq_prep_kernel(float* __restrict__ H, int64_t in, float damp, uint8_t* __restr
       H[j * in + j] = 1.0f;
     }
     s += static_cast<double>(d);
+    m = fmaxf(m, d);
   }
   part[threadIdx.x] = s;
+  mx[threadIdx.x] = m;
   __syncthreads();
   for (int o = 128; o > 0; o >>= 1) {
-    if (threadIdx.x < o) part[threadIdx.x] += part[threadIdx.x + o];
+    if (threadIdx.x < o) {
+      part[threadIdx.x] += part[threadIdx.x + o];
+      mx[threadIdx.x] = fmaxf(mx[threadIdx.x], mx[threadIdx.x + o]);
+    }
     __syncthreads();
   }
   const float lam = static_cast<float>(static_cast<double>(damp) * part[0] / static_cast<double>(in));
   for (int64_t j = threadIdx.x; j < in; j += blockDim.x) H[j * in + j] += lam;
+  if (threadIdx.x == 0) {
+    const float S = *Sp;
+    const float dmax = S * (6.0f * q_max + 2688.0f) * (1.0f + 0x1p-10f);
+    const float rmax = sqrtf(mx[0] + lam) * (1.0f + 0x1p-10f);
+    const int kd = pow2_floor_exp(16384.0f / dmax), kr = pow2_floor_exp(16384.0f / rmax);
+    gs[0] = ldexpf(1.0f, kd);
+    gs[1] = ldexpf(1.0f, kr);
+    gs[2] = ldexpf(1.0f, -kd - kr);
+    gs[3] = 1.0f;
+  }
 }
 
 // In place: a[r][c] <-> a[n-1-c][n-1-r] (reflection about the anti-diagonal;
@@ -317,31 +351,33 @@ gptq_udiag_kernel(const float* __restrict__ R, int64_t in, float* __restrict__ U
   for (int i = 0; i < 16; ++i) o[i * 16] = static_cast<float>(x[i]);
 }
 
-// The TF32 head of an FP32 value (10 explicit mantissa bits, rounded to
-// nearest; truncated where rounding would overflow); x - head is exact.
-__device__ __forceinline__ float tf32_head(float x) {
-  const uint32_t u = __float_as_uint(x);
-  uint32_t hbits = (u + 0x1000u) & 0xFFFFE000u;
-  if ((hbits & 0x7F800000u) == 0x7F800000u) hbits = u & 0xFFFFE000u;
-  return __uint_as_float(hbits);
+// x scaled by the power of two s, as its FP16 rounding and the FP16 rounding
+// of the (exact FP32) remainder.
+__device__ __forceinline__ void f16_split(float x, float s, __half& hi, __half& lo) {
+  const float y = x * s;
+  hi = __float2half_rn(y);
+  lo = __float2half_rn(y - __half2float(hi));
 }
 
-// One 128-row slice of the B operand of a split update GEMM: rows
-// [r0, r0 + kGB) of R, columns [c0, c0 + m), as [R_hi; R_lo; R_hi] (kCat rows
-// of Rcat, row stride ldr).  blockIdx.y is the row.
+// The B operand of a batch's split update GEMMs: for each part p of the batch
+// (rows [r0 + kGB p, r0 + kGB (p + 1)) of R) and columns [c0, c0 + m), R scaled
+// by s_R = gs[1], as [R_hi; R_lo; R_hi] in FP16 at rows kCat p .. of Rcat (row
+// stride ldr).  blockIdx.y is the row of R within the batch.  Columns left of
+// a row's diagonal are copied too and never read.
 __global__ void __launch_bounds__(256)
 gptq_rsplit_kernel(const float* __restrict__ R, int64_t in, int64_t r0, int64_t c0, int64_t m,
-                   float* __restrict__ Rcat, int64_t ldr) {
-  const int64_t rr = blockIdx.y;
-  const float* src = R + (r0 + rr) * in + c0;
-  float* dst = Rcat + rr * ldr;
+                   const float* __restrict__ gs, __half* __restrict__ Rcat, int64_t ldr) {
+  const int64_t part = blockIdx.y / kGB, rr = blockIdx.y % kGB;
+  const float sr = gs[1];
+  const float* src = R + (r0 + blockIdx.y) * in + c0;
+  __half* dst = Rcat + (part * kCat + rr) * ldr;
   for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < m;
        c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float x = src[c];
-    const float hd = tf32_head(x);
-    dst[c] = hd;
-    dst[kGB * ldr + c] = x - hd;
-    dst[2 * kGB * ldr + c] = hd;
+    __half hi, lo;
+    f16_split(src[c], sr, hi, lo);
+    dst[c] = hi;
+    dst[kGB * ldr + c] = lo;
+    dst[2 * kGB * ldr + c] = hi;
   }
 }
 
@@ -354,8 +390,8 @@ gptq_rsplit_kernel(const float* __restrict__ R, int64_t in, int64_t r0, int64_t 
 //   * quantizes each column at its turn -- exact E2M1 decision, D = W - q,
 //     err = (w - q) R_jj -- and updates the group's later columns by
 //     w_k -= err U_jk;
-// and writes the batch's D as [D_hi | D_hi | D_lo] (kCat columns from Dcat,
-// row stride ldd) for the split update GEMMs.  Dynamic shared memory: R's blocks above the diagonal
+// and writes the batch's D, scaled by s_D = gs[0], as [D_hi | D_hi | D_lo] in
+// FP16 (kCat columns from Dcat, row stride ldd) for the split update GEMMs.  Dynamic shared memory: R's blocks above the diagonal
 // blocks (kRsFloats), the groups' U blocks (8 x 256), the rows' D (kT x kDs).
 template <bool kWeighted, int kK, int kT>
 __global__ void __launch_bounds__(kT)
@@ -364,7 +400,7 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
                    const float* __restrict__ R, const float* __restrict__ Ud,
                    const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                   float* __restrict__ Dcat, int64_t ldd) {
+                   const float* __restrict__ gs, __half* __restrict__ Dcat, int64_t ldd) {
   extern __shared__ __align__(16) float gsm[];
   __shared__ CandEntry tab[kTabSize];
   __shared__ float hb[kGB];
@@ -402,10 +438,11 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
   float* ds = Ds + t * kDs;
   const float* prow = P + r * in + j0;
   const uint16_t* wrow = W + r * ldw + j0;
-  float* dcat = Dcat + r * ldd;
+  __half* dcat = Dcat + r * ldd;
+  const float sd = gs[0];
   const int64_t G = in / 16;
   // A group's P (16 floats) and W (16 bf16, as 8 pairs) are loaded one group
-  // ahead, so their latency hides behind the previous group's sweep.  W takes
+  // ahead, so their latency hides behind the previous group's column loop.  W takes
   // two 16-byte loads where its rows allow, else 16 two-byte loads.
   const bool w_vec = (reinterpret_cast<uintptr_t>(W) & 15u) == 0 && ldw % 8 == 0;
   float4 pn[4];
@@ -436,7 +473,6 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) wc[i] = wn[i];
-    if (g + 1 < ng) load_group(g + 1);
     const float* rs = Rs + 128 * g * (g - 1);
     for (int i = 0; i < 16 * g; i += 4) {
       const float4 d4 = *reinterpret_cast<const float4*>(ds + i);
@@ -484,6 +520,7 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
     }
     const int code = local_sweep_f32<kWeighted, kK>(w, kWeighted ? hb + 16 * g : nullptr, sc,
                                                     tab, lo, K);
+    if (g + 1 < ng) load_group(g + 1);  // in flight during the column loop
     uint32_t packed[2] = {0u, 0u};
     float dl[16];
 #pragma unroll
@@ -498,15 +535,27 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
       for (int k = j + 1; k < 16; ++k) w[k] = fmaf(-err, u[k], w[k]);
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 d4 = make_float4(dl[4 * q], dl[4 * q + 1], dl[4 * q + 2], dl[4 * q + 3]);
-      *reinterpret_cast<float4*>(ds + 16 * g + 4 * q) = d4;
-      const float4 hd = make_float4(tf32_head(d4.x), tf32_head(d4.y), tf32_head(d4.z),
-                                    tf32_head(d4.w));
-      const float4 tl = make_float4(d4.x - hd.x, d4.y - hd.y, d4.z - hd.z, d4.w - hd.w);
-      *reinterpret_cast<float4*>(dcat + 16 * g + 4 * q) = hd;
-      *reinterpret_cast<float4*>(dcat + kGB + 16 * g + 4 * q) = hd;
-      *reinterpret_cast<float4*>(dcat + 2 * kGB + 16 * g + 4 * q) = tl;
+    for (int q = 0; q < 4; ++q)
+      *reinterpret_cast<float4*>(ds + 16 * g + 4 * q) =
+          make_float4(dl[4 * q], dl[4 * q + 1], dl[4 * q + 2], dl[4 * q + 3]);
+    uint32_t hw[8], lw[8];  // FP16 pairs, element 2i in the low half
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      __half h0, l0, h1, l1;
+      f16_split(dl[2 * i], sd, h0, l0);
+      f16_split(dl[2 * i + 1], sd, h1, l1);
+      hw[i] = static_cast<uint32_t>(__half_as_ushort(h0)) |
+              (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
+      lw[i] = static_cast<uint32_t>(__half_as_ushort(l0)) |
+              (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 hv = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
+      const uint4 lv = make_uint4(lw[4 * q], lw[4 * q + 1], lw[4 * q + 2], lw[4 * q + 3]);
+      reinterpret_cast<uint4*>(dcat + 16 * g)[q] = hv;
+      reinterpret_cast<uint4*>(dcat + kGB + 16 * g)[q] = hv;
+      reinterpret_cast<uint4*>(dcat + 2 * kGB + 16 * g)[q] = lv;
     }
     const int64_t gg = j0 / 16 + g;
     *reinterpret_cast<uint2*>(codes + r * (G * 8) + gg * 8) = make_uint2(packed[0], packed[1]);
@@ -596,7 +645,7 @@ void timer_end(int idx, cudaStream_t s) {
 }
 
 struct GptqLayout {
-  size_t h_ws = 0, s_ws = 0, H = 0, P = 0, Dcat = 0, Rbig = 0, Rsmall = 0, Ud = 0, dead = 0,
+  size_t h_ws = 0, s_ws = 0, H = 0, P = 0, Dcat = 0, Rcat = 0, gs = 0, Ud = 0, dead = 0,
          info = 0, lapack = 0, blas = 0;
   size_t bytes = 0;
   int lwork = 0;
@@ -624,9 +673,9 @@ bool gptq_layout(int64_t out, int64_t in, int64_t tokens, int sms, Handles* hd, 
   L->s_ws = take(global_scale_workspace_bytes(L->gplan));
   L->H = take(n * n * sizeof(float));
   L->P = take(o * n * sizeof(float));
-  L->Dcat = take(o * kCat * kSub * sizeof(float));
-  L->Rbig = take(static_cast<size_t>(kCat) * kSub * n * sizeof(float));
-  L->Rsmall = take(static_cast<size_t>(kCat) * (kSub - 1) * kGB * sizeof(float));
+  L->Dcat = take(o * kCat * kSub * sizeof(__half));
+  L->Rcat = take(static_cast<size_t>(kCat) * kSub * n * sizeof(__half));
+  L->gs = take(4 * sizeof(float));
   L->Ud = take(n * 16 * sizeof(float));
   L->dead = take(n);
   L->info = take(sizeof(int));
@@ -647,7 +696,7 @@ template <bool kW, int kKK, int kT>
 cudaError_t launch_rblock_t(const uint16_t* W, int64_t ldw, const uint8_t* dead, int64_t out,
                             int64_t in, int64_t j0, int nb, const float* P, const float* R,
                             const float* Ud, const float* h, const float* S, int lo, int hi,
-                            uint8_t* codes, uint8_t* scales, float* Dcat, int64_t ldd,
+                            uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat, int64_t ldd,
                             cudaStream_t s) {
   constexpr size_t smem = rblock_smem(kT);
   static const cudaError_t attr = cudaFuncSetAttribute(
@@ -656,7 +705,7 @@ cudaError_t launch_rblock_t(const uint16_t* W, int64_t ldw, const uint8_t* dead,
   if (attr != cudaSuccess) return attr;
   const unsigned blocks = static_cast<unsigned>((out + kT - 1) / kT);
   gptq_rblock_kernel<kW, kKK, kT><<<blocks, kT, smem, s>>>(W, ldw, dead, out, in, j0, nb, P, R, Ud,
-                                                           h, S, lo, hi, codes, scales, Dcat, ldd);
+                                                           h, S, lo, hi, codes, scales, gs, Dcat, ldd);
   return cudaGetLastError();
 }
 
@@ -664,13 +713,13 @@ template <bool kW, int kKK>
 cudaError_t launch_rblock(const uint16_t* W, int64_t ldw, const uint8_t* dead, int64_t out,
                           int64_t in, int64_t j0, int nb, const float* P, const float* R,
                           const float* Ud, const float* h, const float* S, int lo, int hi,
-                          uint8_t* codes, uint8_t* scales, float* Dcat, int64_t ldd, int sms,
+                          uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat, int64_t ldd, int sms,
                           cudaStream_t s) {
   if ((out + 127) / 128 >= static_cast<int64_t>(sms))
     return launch_rblock_t<kW, kKK, 128>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi,
-                                         codes, scales, Dcat, ldd, s);
+                                         codes, scales, gs, Dcat, ldd, s);
   return launch_rblock_t<kW, kKK, 32>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi, codes,
-                                      scales, Dcat, ldd, s);
+                                      scales, gs, Dcat, ldd, s);
 }
 
 }  // namespace
@@ -721,9 +770,9 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
   char* ws = static_cast<char*>(workspace);
   float* H = reinterpret_cast<float*>(ws + L.H);
   float* P = reinterpret_cast<float*>(ws + L.P);
-  float* Dcat = reinterpret_cast<float*>(ws + L.Dcat);
-  float* Rbig = reinterpret_cast<float*>(ws + L.Rbig);
-  float* Rsmall = reinterpret_cast<float*>(ws + L.Rsmall);
+  __half* Dcat = reinterpret_cast<__half*>(ws + L.Dcat);
+  __half* Rcat = reinterpret_cast<__half*>(ws + L.Rcat);
+  float* gs = reinterpret_cast<float*>(ws + L.gs);
   float* Ud = reinterpret_cast<float*>(ws + L.Ud);
   uint8_t* dead = reinterpret_cast<uint8_t*>(ws + L.dead);
   int* info = reinterpret_cast<int*>(ws + L.info);
@@ -736,7 +785,15 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
       !lapack_ok(cusolverDnSetStream(hd->solver, stream)))
     return cudaErrorUnknown;
   // the compute types are given per call; the handle's math mode stays the default
-  if (!blas_ok(cublasSetMathMode(hd->blas, CUBLAS_DEFAULT_MATH))) return cudaErrorUnknown;
+  if (!blas_ok(cublasSetMathMode(hd->blas, CUBLAS_DEFAULT_MATH)) ||
+      !blas_ok(cublasSetPointerMode(hd->blas, CUBLAS_POINTER_MODE_HOST)))
+    return cudaErrorUnknown;
+  // the update GEMMs take alpha and beta from device memory; host mode again
+  // on every way out of this call
+  struct PointerModeGuard {
+    cublasHandle_t h;
+    ~PointerModeGuard() { cublasSetPointerMode(h, CUBLAS_POINTER_MODE_HOST); }
+  } pointer_mode_guard{hd->blas};
   // h and S with this library's kernels
   int tm = timer_begin(NVFP4_GPTQ_PHASE_REDUCTIONS, stream);
   if ((e = launch_diag_hessian(X, tokens, in, ldx, h, 0, reinterpret_cast<float*>(ws + L.h_ws),
@@ -778,7 +835,7 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
   }
   timer_end(tm, stream);
   tm = timer_begin(NVFP4_GPTQ_PHASE_FACTOR, stream);
-  gptq_prep_kernel<<<1, 256, 0, stream>>>(H, in, damp, dead);
+  gptq_prep_kernel<<<1, 256, 0, stream>>>(H, in, damp, dead, S, q_max, gs);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // R = J L' J row-major, L' the lower Cholesky factor of J H J (FP32)
   const int n = static_cast<int>(in);
@@ -804,63 +861,66 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
   const int K = hi - lo + 1;
   const uint8_t* dd = dead;
   const int64_t ldd = static_cast<int64_t>(kCat) * kSub;
-  auto block_t = [&](int64_t c0, int nb, float* dcat) {
+  auto block_t = [&](int64_t c0, int nb, __half* dcat) {
     if (weighted)
-      return K == 16 ? launch_rblock<true, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, dcat, ldd, sms, stream)
-                     : launch_rblock<true, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, dcat, ldd, sms, stream);
-    return K == 16 ? launch_rblock<false, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, dcat, ldd, sms, stream)
-                   : launch_rblock<false, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, dcat, ldd, sms, stream);
+      return K == 16 ? launch_rblock<true, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream)
+                     : launch_rblock<true, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream);
+    return K == 16 ? launch_rblock<false, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream)
+                   : launch_rblock<false, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream);
   };
-  auto block = [&](int64_t c0, int nb, float* dcat) {
+  auto block = [&](int64_t c0, int nb, __half* dcat) {
     const int t = timer_begin(NVFP4_GPTQ_PHASE_BATCH, stream);
     const cudaError_t r = block_t(c0, nb, dcat);
     timer_end(t, stream);
     return r;
   };
-  auto split = [&](int64_t r0, int64_t c0, int64_t m, float* rcat, int64_t ldr) {
+  // one split per batch: every full part's rows, columns [c0, in)
+  auto split = [&](int64_t r0, int parts, int64_t c0) {
     const int t = timer_begin(NVFP4_GPTQ_PHASE_SPLIT, stream);
-    const dim3 grid(static_cast<unsigned>(std::min<int64_t>((m + 255) / 256, 8)), kGB);
-    gptq_rsplit_kernel<<<grid, 256, 0, stream>>>(R, in, r0, c0, m, rcat, ldr);
+    const int64_t m = in - c0;
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>((m + 255) / 256, 8)),
+                    static_cast<unsigned>(kGB * parts));
+    gptq_rsplit_kernel<<<grid, 256, 0, stream>>>(R, in, r0, c0, m, gs, Rcat, in);
     timer_end(t, stream);
     return cudaGetLastError();
   };
   // P[:, c0 : c0 + m] += Dcat[:, :k] Rcat[:k, :m], all row-major: in
   // column-major terms P^T (m x out) += Rcat^T (m x k) Dcat^T (k x out)
-  auto update = [&](int64_t c0, int64_t m, int k, const float* rcat, int64_t ldr) {
+  // alpha = 1 / (s_D s_R) and beta = 1 are device scalars (gs[2], gs[3])
+  auto update = [&](int64_t c0, int64_t m, int k, const __half* rcat, int64_t ldr) {
     const int t = timer_begin(NVFP4_GPTQ_PHASE_UPDATE, stream);
     const bool ok = blas_ok(cublasGemmEx(hd->blas, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(m),
-                                static_cast<int>(out), k, &one, rcat, CUDA_R_32F,
-                                static_cast<int>(ldr), Dcat, CUDA_R_32F, static_cast<int>(ldd), &one,
-                                P + c0, CUDA_R_32F, n, CUBLAS_COMPUTE_32F_FAST_TF32,
+                                static_cast<int>(out), k, gs + 2, rcat, CUDA_R_16F,
+                                static_cast<int>(ldr), Dcat, CUDA_R_16F, static_cast<int>(ldd),
+                                gs + 3, P + c0, CUDA_R_32F, n, CUBLAS_COMPUTE_32F,
                                 CUBLAS_GEMM_DEFAULT));
     timer_end(t, stream);
     return ok;
   };
+  if (!blas_ok(cublasSetPointerMode(hd->blas, CUBLAS_POINTER_MODE_DEVICE)))
+    return cudaErrorUnknown;
   constexpr int64_t kBatch = static_cast<int64_t>(kGB) * kSub;
   for (int64_t j0 = 0; j0 < in; j0 += kBatch) {
     const int64_t jend = std::min(j0 + kBatch, in);
     const int nsub = static_cast<int>((jend - j0 + kGB - 1) / kGB);
+    // R's rows of the batch's full parts (only the last part can be narrower,
+    // and its rows are never an operand), columns from the second part on
+    const int64_t col0 = j0 + kGB;
+    const int full = static_cast<int>((jend - j0) / kGB);
+    if (col0 < in && full > 0 && (e = split(j0, full, col0)) != cudaSuccess) return e;
     for (int sb = 0; sb < nsub; ++sb) {
       const int64_t c0 = j0 + static_cast<int64_t>(kGB) * sb;
       const int nb = static_cast<int>(std::min<int64_t>(kGB, jend - c0));
       if ((e = block(c0, nb, Dcat + static_cast<int64_t>(kCat) * sb)) != cudaSuccess) return e;
-      if (sb + 1 < nsub) {  // the batch's later half takes this half's columns
-        const int64_t c1 = c0 + nb;  // nb == kGB: only a batch's last half can be narrower
+      if (sb + 1 < nsub) {  // the next part takes the batch's parts so far
+        const int64_t c1 = c0 + nb;  // nb == kGB: only a batch's last part can be narrower
         const int64_t m = std::min<int64_t>(kGB, jend - c1);
-        for (int s0 = 0; s0 <= sb; ++s0)
-          if ((e = split(j0 + static_cast<int64_t>(kGB) * s0, c1, m,
-                         Rsmall + static_cast<int64_t>(kCat) * s0 * kGB, kGB)) != cudaSuccess)
-            return e;
-        if (!update(c1, m, kCat * (sb + 1), Rsmall, kGB)) return cudaErrorUnknown;
+        if (!update(c1, m, kCat * (sb + 1), Rcat + (c1 - col0), in)) return cudaErrorUnknown;
       }
     }
-    if (jend < in) {  // every later column takes the whole batch (all halves full)
-      for (int s0 = 0; s0 < nsub; ++s0)
-        if ((e = split(j0 + static_cast<int64_t>(kGB) * s0, jend, in - jend,
-                       Rbig + static_cast<int64_t>(kCat) * s0 * in, in)) != cudaSuccess)
-          return e;
-      if (!update(jend, in - jend, kCat * nsub, Rbig, in)) return cudaErrorUnknown;
-    }
+    if (jend < in &&  // every later column takes the whole batch (all parts full)
+        !update(jend, in - jend, kCat * nsub, Rcat + (jend - col0), in))
+      return cudaErrorUnknown;
   }
   return cudaSuccess;
 }
