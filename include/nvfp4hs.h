@@ -404,16 +404,18 @@ int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, 
  *   workspace  nvfp4_gptq_workspace_size(out, in, tokens) bytes, 256-byte
  *            aligned (it holds H and its Cholesky factor, the FP32 sums P
  *            [out, in] of the propagated errors, a batch's errors and
- *            factor rows for the update GEMMs and the solver's scratch:
- *            about 4 (in^2 + out (in + 768) + 800 in) bytes).
+ *            factor rows for the update GEMMs in FP16 and the solver's
+ *            scratch: about 4 in^2 + out (4 in + 3072) + 3200 in bytes plus
+ *            32 MiB).
  * Steps: no inverse is formed.  The lower Cholesky factor of the reversed H
  * gives H = R R^T with R upper (U = R^-1), and the columns run in the
  * equivalent R form: W - Q = Err U, so Err = (W - Q) R, and a group's current
  * weights are W_grp + ((W - Q)[:, <grp] R[<grp, grp]) R_grp^-1 with R_grp the
  * group's 16 x 16 diagonal block.  h, S, the block inverses and the batches
  * of columns are this library's kernels; X^T X and the batches' updates of
- * later columns' sums are GEMMs (cuBLAS; the updates as three TF32
- * tensor-core products of split FP32 operands), the Cholesky factor comes
+ * later columns' sums are GEMMs (cuBLAS; the updates as three FP16
+ * tensor-core products of split, power-of-two-scaled FP32 operands with FP32
+ * accumulation, about 2^-21 relative per product), the Cholesky factor comes
  * from cuSOLVER.  The first call on a device creates the
  * library's cuBLAS and cuSOLVER handles there, which hold a little device
  * memory until the process exits; every call's scratch is the caller's
@@ -445,7 +447,7 @@ enum nvfp4_gptq_phase {
     NVFP4_GPTQ_PHASE_FACTOR = 2,      /* damping, Cholesky factor, block inverses   */
     NVFP4_GPTQ_PHASE_BATCH = 3,       /* batch kernels: local call, quantization,
                                          propagation inside a batch                 */
-    NVFP4_GPTQ_PHASE_SPLIT = 4,       /* TF32 splits of the factor's rows           */
+    NVFP4_GPTQ_PHASE_SPLIT = 4,       /* FP16 splits of the factor's rows           */
     NVFP4_GPTQ_PHASE_UPDATE = 5,      /* update GEMMs of later columns' sums        */
     NVFP4_GPTQ_PHASES = 6
 };

@@ -96,13 +96,16 @@ def _correlated(n, tokens, seed):
     return (Z @ mix).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("out,n,tokens,seed,weighted,lo,hi", [
-    (256, 512, 2048, 81, True, -9, 6), (128, 1024, 4096, 82, True, -9, 6),
-    (192, 512, 2048, 83, False, -3, 7), (160, 768, 3072, 84, True, -8, 7),
-    (96, 528, 2048, 85, True, -9, 6),    # a last lazy batch of 16 columns
-    (112, 400, 2048, 86, True, -9, 6)])  # a last lazy batch of 128 + 16 columns
+@pytest.mark.parametrize("out,n,tokens,seed,weighted,lo,hi,min_same", [
+    (256, 512, 2048, 81, True, -9, 6, 0.97), (128, 1024, 4096, 82, True, -9, 6, 0.97),
+    (192, 512, 2048, 83, False, -3, 7, 0.97), (160, 768, 3072, 84, True, -8, 7, 0.97),
+    (96, 528, 2048, 85, True, -9, 6, 0.97),     # a last lazy batch of 16 columns
+    (112, 400, 2048, 86, True, -9, 6, 0.97),    # a last lazy batch of 128 + 16 columns
+    # a long row over strongly correlated inputs (damped H's condition number
+    # about 1.7e4): see the note on the bars below
+    (64, 4112, 8192, 87, True, -9, 6, 0.80)])
 def test_correlated_inputs_follow_the_oracle(orc, nv, parity_report, out, n, tokens, seed,
-                                             weighted, lo, hi):
+                                             weighted, lo, hi, min_same):
     import workloads
     from oracle import gptq
     W = workloads.weight(out, n, 0.02, 0.005, 10.0, seed)
@@ -130,11 +133,17 @@ def test_correlated_inputs_follow_the_oracle(orc, nv, parity_report, out, n, tok
     # Tolerances (FP32 against FP64 GPTQ): a flipped decision changes one
     # element's reconstruction by a grid step and the row's later columns
     # re-fit around it, so a row's tail can differ while the layer error
-    # barely moves.  Measured on a B200: output error ratios 1.0007 and
-    # 1.0002, 99.3% and 99.4% of groups equal; the bars below leave about 7x
-    # and 4x of that.
+    # barely moves.  Measured on a B200: output error ratios within 0.999 to
+    # 1.002 and 98.4% to 100% of groups equal on the first six layers; the
+    # bars leave about 2x and 1.5x of that.  On the ill-conditioned 4112-wide
+    # layer the output error stays within 0.3% of the oracle's but only 86%
+    # to 90% of the groups are equal: X^T X from bf16 tensor-core GEMMs is
+    # summed less precisely (2-3e-6 of sqrt(H_ii H_jj), against 8e-7 for an
+    # FP32 CPU GEMM), and on this H that moves the Cholesky factor enough to
+    # flip about a tenth of the decisions; an FP32 CPU GPTQ given the
+    # device's factor flips the same ones.
     assert abs(e_gpu / e_orc - 1.0) < 0.005
-    assert same > 0.97
+    assert same > min_same
     assert e_gpu < 0.95 * e_sweep
 
 
