@@ -16,8 +16,10 @@
 //
 // On the device:
 //   * h and S: this library's diagonal-Hessian and global-scale kernels;
-//   * H = X^T X: one cuBLAS GEMM (bf16 in, FP32 accumulate; a plain GEMM);
-//   * the dead-column rule and the damping: gptq_prep_kernel;
+//   * H = X^T X: cuBLAS GEMMs (bf16 in, FP32 accumulate), only the lower
+//     blocks of a 4 x 4 split for in >= 4096 (the factorization reads one
+//     triangle);
+//   * the dead-column rule, the damping and the FP16 scales: gptq_prep_kernel;
 //   * no inverse is formed.  With J the order-reversing permutation, the lower
 //     Cholesky factor L' of J H J (cuSOLVER potrf, FP32) gives H = R R^T with
 //     R = J L' J upper, and U = R^-1.  Reflecting the n x n array about its
@@ -71,8 +73,8 @@ constexpr int kGB = 128;        // columns per batch kernel launch
 constexpr int kCat = 3 * kGB;   // K of the split update per 128 columns
 constexpr int kSub = 4;         // batch-kernel launches per lazy batch (512 columns)
 constexpr int kDs = kGB + 4;    // a row's D in shared memory (16-byte rows)
-// R's blocks above the diagonal blocks of one batch: for group b, the rows of
-// the batch's earlier groups (16 b of them) by the group's 16 columns.
+// R's blocks above the diagonal blocks of one part: for group b, the rows of
+// the part's earlier groups (16 b of them) by the group's 16 columns.
 constexpr int kRsFloats = 256 * (kGB / 16) * (kGB / 16 - 1) / 2;
 
 size_t al256(size_t x) { return (x + 255) & ~size_t{255}; }
@@ -314,7 +316,7 @@ antitranspose_kernel(float* __restrict__ a, int64_t n) {
   if (bi + bj < t - 1) *B = ta[15 - x][15 - y];
 }
 
-// A failed Cholesky or inverse (devInfo != 0: the damped Hessian is not
+// A failed Cholesky factorization (devInfo != 0: the damped Hessian is not
 // positive definite in FP32) is reported through the status word.
 __global__ void gptq_status_kernel(const int* __restrict__ info, int n, int* status) {
   int bad = 0;
@@ -381,18 +383,19 @@ gptq_rsplit_kernel(const float* __restrict__ R, int64_t in, int64_t r0, int64_t 
   }
 }
 
-// One lazy batch [j0, j0 + nb) of GPTQ's columns in the R form, one thread per
-// row, kT rows per CTA.  Per 16-column group at g0 the thread
+// One part [j0, j0 + nb) of a lazy batch of GPTQ's columns in the R form, one
+// thread per row, kT rows per CTA.  Per 16-column group at g0 the thread
 //   * sums v = P[r, grp] + D[r, j0:g0] R[j0:g0, grp] (P holds the earlier
-//     batches' sums, D the batch's earlier groups, in shared memory);
+//     parts' sums, D the part's earlier groups, in shared memory);
 //   * forms the current weights w = W[r, grp] + v U_grp;
 //   * runs the local call on w (the group's E4M3 scale code);
 //   * quantizes each column at its turn -- exact E2M1 decision, D = W - q,
 //     err = (w - q) R_jj -- and updates the group's later columns by
 //     w_k -= err U_jk;
-// and writes the batch's D, scaled by s_D = gs[0], as [D_hi | D_hi | D_lo] in
-// FP16 (kCat columns from Dcat, row stride ldd) for the split update GEMMs.  Dynamic shared memory: R's blocks above the diagonal
-// blocks (kRsFloats), the groups' U blocks (8 x 256), the rows' D (kT x kDs).
+// and writes the part's D, scaled by s_D = gs[0], as [D_hi | D_hi | D_lo] in
+// FP16 (kCat columns from Dcat, row stride ldd) for the split update GEMMs.
+// Dynamic shared memory: R's blocks above the diagonal blocks (kRsFloats), the
+// groups' U blocks (8 x 256), the rows' D (kT x kDs).
 template <bool kWeighted, int kK, int kT>
 __global__ void __launch_bounds__(kT)
 gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* __restrict__ dead,
