@@ -444,26 +444,18 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
   __half* dcat = Dcat + r * ldd;
   const float sd = gs[0];
   const int64_t G = in / 16;
-  // A group's P (16 floats) and W (16 bf16, as 8 pairs) are loaded one group
-  // ahead, so their latency hides behind the previous group's column loop.  W takes
-  // two 16-byte loads where its rows allow, else 16 two-byte loads.
-  const bool w_vec = (reinterpret_cast<uintptr_t>(W) & 15u) == 0 && ldw % 8 == 0;
+  // A group's P (16 floats) and W (16 bf16, as 8 pairs, two 16-byte loads: W
+  // is 16-byte aligned and ldw % 8 == 0) are loaded one group ahead, so their
+  // latency hides behind the previous group's column loop.
   float4 pn[4];
   uint32_t wn[8];
   auto load_group = [&](int g) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) pn[q] = reinterpret_cast<const float4*>(prow + 16 * g)[q];
-    if (w_vec) {
-      const uint4 a = reinterpret_cast<const uint4*>(wrow + 16 * g)[0];
-      const uint4 b = reinterpret_cast<const uint4*>(wrow + 16 * g)[1];
-      wn[0] = a.x; wn[1] = a.y; wn[2] = a.z; wn[3] = a.w;
-      wn[4] = b.x; wn[5] = b.y; wn[6] = b.z; wn[7] = b.w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        wn[i] = static_cast<uint32_t>(wrow[16 * g + 2 * i]) |
-                (static_cast<uint32_t>(wrow[16 * g + 2 * i + 1]) << 16);
-    }
+    const uint4 a = reinterpret_cast<const uint4*>(wrow + 16 * g)[0];
+    const uint4 b = reinterpret_cast<const uint4*>(wrow + 16 * g)[1];
+    wn[0] = a.x; wn[1] = a.y; wn[2] = a.z; wn[3] = a.w;
+    wn[4] = b.x; wn[5] = b.y; wn[6] = b.z; wn[7] = b.w;
   };
   load_group(0);
   for (int g = 0; g < ng; ++g) {

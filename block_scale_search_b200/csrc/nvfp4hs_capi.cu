@@ -325,8 +325,9 @@ int nvfp4_gptq_quantize(const void* W, int64_t out, int64_t in, int64_t ldw, con
   if (!std::isfinite(q_max) || !(q_max > 0.0f) || !std::isfinite(damp) || damp < 0.0f)
     return NVFP4_ERR_INVALID_ARG;
   if (lo < -16 || lo > 0 || hi < 0 || hi > 15 || hi - lo > 15) return NVFP4_ERR_WINDOW;
-  if (!aligned(W, 2) || !aligned(X, 16) || ldx % 8 != 0 || !aligned(codes, 8) || !aligned(S, 4) ||
-      !aligned(h, 16) || !aligned(status, 4))
+  // W's rows are read in 16-byte vectors (its global scale, the batch kernel)
+  if (!aligned(W, 16) || ldw % 8 != 0 || !aligned(X, 16) || ldx % 8 != 0 || !aligned(codes, 8) ||
+      !aligned(S, 4) || !aligned(h, 16) || !aligned(status, 4))
     return NVFP4_ERR_ALIGN;
   if (workspace == nullptr) return NVFP4_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return NVFP4_ERR_ALIGN;

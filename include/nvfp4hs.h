@@ -393,8 +393,8 @@ int nvfp4_quantize_layers(const nvfp4_layer* layers, int n_layers, float q_max, 
  * error-updated FP32 weights, with S = the global scale of the original W;
  * each column of the group is then quantized at its turn with that scale.
  *
- *   W        bf16 [out, ldw]; in % 16 == 0; out, in > 0; out < 2^31,
- *            in <= 16 * 65535.
+ *   W        bf16 [out, ldw], 16-byte aligned, ldw % 8 == 0; in % 16 == 0;
+ *            out, in > 0; out < 2^31, in <= 16 * 65535.
  *   X        bf16 [tokens, ldx], 16-byte aligned, ldx % 8 == 0; tokens >= 0,
  *            ldx >= in; tokens, ldx < 2^31 (the GEMM's int sizes).
  *   codes, scales, S, h  the NVFP4 result ([out, in/2], [out, in/16]), the

@@ -386,6 +386,8 @@ def test_gptq_validation(L):
     assert call(inp=16 * 65536, ldw=16 * 65536, ldx=16 * 65536) == -2   # in / 16 > 65535
     assert call(lo=-10) == -4
     assert call(X=P + 8) == -3 and call(codes=P + 4) == -3 and call(h=P + 4) == -3
+    assert call(W=P + 2) == -3 and call(W=P + 8) == -3        # W's rows are read 16 bytes at a time
+    assert call(ldw=260) == -3                                # ldw % 8 != 0
     assert call(ws=None) == -7 and call(ws=P + 64) == -3
     assert L.nvfp4_gptq_workspace_size(64, 250, 128) == 0
     ms = (C.c_float * 6)()

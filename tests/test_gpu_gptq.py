@@ -250,3 +250,24 @@ def test_benchmarked_call_on_sampled_rows_follows_the_oracle(orc, nv, parity_rep
     # Measured on a B200: ratio 1.00000, every group of the eight rows equal.
     assert abs(e_gpu / e_orc - 1.0) < 0.005
     assert same > 0.97
+
+
+@pytest.mark.parametrize("pad_w,pad_x", [(8, 8), (32, 40)])
+def test_padded_leading_dimensions_give_the_same_bytes(nv, pad_w, pad_x):
+    """W and X as views into wider rows (leading dimensions in + 8 and in + 32
+    for W, in + 8 and in + 40 for X); every output byte equals the contiguous
+    call's."""
+    import workloads
+    out, n, tokens = 96, 528, 2048
+    W = workloads.weight(out, n, 0.02, 0.005, 10.0, 95, DEV)
+    X = _correlated(n, tokens, 96).to(DEV)
+    Wp = torch.zeros(out, n + pad_w, dtype=torch.bfloat16, device=DEV)
+    Xp = torch.zeros(tokens, n + pad_x, dtype=torch.bfloat16, device=DEV)
+    Wp[:, :n] = W
+    Xp[:, :n] = X
+    a = nv.gptq_quantize(W, X)
+    b = nv.gptq_quantize(Wp[:, :n], Xp[:, :n])
+    torch.cuda.synchronize()
+    assert b[0].shape == a[0].shape
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
