@@ -110,3 +110,71 @@ def test_dead_columns_quantize_to_zero():
     assert np.all(Q[:, 17] == 0) and np.all(Q[:, 40:48] == 0)
     nib = np.stack([codes & 15, codes >> 4], -1).reshape(32, n)
     assert np.all(nib[:, 17] == 0) and np.all(nib[:, 40:48] == 0)
+
+
+def _r_form(W, X, lo=-9, hi=6, damp=0.01, part=128, parts=4):
+    """GPTQ restated in the form the device runs, FP64, no inverse of H: H =
+    R R^T with R upper (R = J L J, L the lower Cholesky factor of J H J, J the
+    order reversal); since W - Q = Err U with U = R^-1, a group's current
+    weights are W_grp + (D[:, <g0] R[<g0, grp]) R_grp^-1 with D = W - Q; the
+    later columns' sums P are brought up to date in lazy batches of `parts`
+    parts of `part` columns (after each part for the next one, after each
+    batch for all later columns)."""
+    from oracle import e2m1_quantize_list, sweep_group_f32_list
+    Wb, Xb = oracle._bf16_bits(W), oracle._bf16_bits(X)
+    out, n = Wb.shape
+    S, _, _ = oracle.global_scale(Wb, 448.0)
+    h = oracle.diag_hessian(Xb)
+    Xf = gptq.bf16_to_f64(Xb)
+    H = Xf.T @ Xf
+    dead = np.diag(H) == 0.0
+    H[dead, dead] = 1.0
+    H += damp * np.mean(np.diag(H)) * np.eye(n)
+    J = np.eye(n)[::-1]
+    R = J @ np.linalg.cholesky(J @ H @ J) @ J
+    W0 = gptq.bf16_to_f64(Wb)
+    W0[:, dead] = 0.0
+    P, D = np.zeros((out, n)), np.zeros((out, n))
+    nib = np.zeros((out, n), np.uint8)
+    scales = np.zeros((out, n // 16), np.uint8)
+    for j0 in range(0, n, part * parts):
+        jend = min(j0 + part * parts, n)
+        for c0 in range(j0, jend, part):
+            c1 = min(c0 + part, jend)
+            for g0 in range(c0, c1, 16):
+                gs = slice(g0, g0 + 16)
+                Ug = np.linalg.inv(R[gs, gs])
+                w = W0[:, gs] + (P[:, gs] + D[:, c0:g0] @ R[c0:g0, gs]) @ Ug
+                _, sc, _, _ = sweep_group_f32_list(
+                    w.astype(np.float32), np.broadcast_to(h[gs], (out, 16)), float(S), lo, hi)
+                scales[:, g0 // 16] = sc
+                vS = gptq._V[sc] * np.float64(S)
+                for i in range(16):
+                    j = g0 + i
+                    nib[:, j] = e2m1_quantize_list(w[:, i].astype(np.float32), vS)
+                    q = gptq.decode(nib[:, j], sc, S)
+                    w[:, i + 1:] -= np.outer((w[:, i] - q) * R[j, j], Ug[i, i + 1:])
+                    D[:, j] = W0[:, j] - q
+            if c1 < jend:
+                P[:, c1:c1 + part] += D[:, j0:c1] @ R[j0:c1, c1:c1 + part]
+        if jend < n:
+            P[:, jend:] += D[:, j0:jend] @ R[j0:jend, jend:]
+    return (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8), scales
+
+
+@pytest.mark.parametrize("n", [272, 400, 656])
+def test_the_devices_r_form_gives_the_oracles_bytes(n):
+    """The rearrangement the device runs (no inverse, lazy batches of 512 in
+    parts of 128; here parts of 32 so that small widths cross several parts
+    and batches) takes the same decisions as the oracle's U form in FP64: the
+    two differ only in rounding order."""
+    import torch
+    rng = np.random.default_rng(n)
+    W = _w(24, n, 50 + n)
+    base = rng.normal(size=(768, 8)) @ rng.normal(size=(8, n))
+    X = torch.from_numpy(base + 0.3 * rng.normal(size=(768, n)) * np.exp(rng.normal(size=n)))
+    X = X.to(torch.bfloat16)
+    oc, os_, *_ = gptq.gptq_hscale(W, X)
+    rc, rs = _r_form(W, X, part=32, parts=4)
+    np.testing.assert_array_equal(rs, os_)
+    np.testing.assert_array_equal(rc, oc)
