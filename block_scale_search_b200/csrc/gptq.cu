@@ -513,9 +513,24 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
 #pragma unroll
       for (int k = i; k < 16; ++k) w[k] = fmaf(v[i], u[k], w[k]);
     }
-    const int code = local_sweep_f32<kWeighted, kK>(w, kWeighted ? hb + 16 * g : nullptr, sc,
-                                                    tab, lo, K);
+    // w waits in the row's D slots of this group (written only after the
+    // column loop) while the sweep runs, which frees 16 registers there
+    float* wpark = ds + 16 * g;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      reinterpret_cast<float4*>(wpark)[q] =
+          make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    const int code = local_sweep_f32<kWeighted, kK>(wpark, kWeighted ? hb + 16 * g : nullptr,
+                                                    sc, tab, lo, K);
     if (g + 1 < ng) load_group(g + 1);  // in flight during the column loop
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 x = reinterpret_cast<const float4*>(wpark)[q];
+      w[4 * q] = x.x;
+      w[4 * q + 1] = x.y;
+      w[4 * q + 2] = x.z;
+      w[4 * q + 3] = x.w;
+    }
     uint32_t packed[2] = {0u, 0u};
     float dl[16];
 #pragma unroll
