@@ -101,6 +101,9 @@ def _correlated(n, tokens, seed):
     (192, 512, 2048, 83, False, -3, 7, 0.97), (160, 768, 3072, 84, True, -8, 7, 0.97),
     (96, 528, 2048, 85, True, -9, 6, 0.97),     # a last lazy batch of 16 columns
     (112, 400, 2048, 86, True, -9, 6, 0.97),    # a last lazy batch of 128 + 16 columns
+    (100, 512, 2048, 88, True, -9, 6, 0.97),    # rows not filling the last CTA
+    (64, 48, 1024, 89, True, -9, 6, 0.97),      # one part of 48 columns, no update GEMM
+    (64, 144, 1024, 90, False, -3, 7, 0.97),    # one part of 128 and one of 16
     # a long row over strongly correlated inputs (damped H's condition number
     # about 1.7e4): see the note on the bars below
     (64, 4112, 8192, 87, True, -9, 6, 0.80)])
