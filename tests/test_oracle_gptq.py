@@ -178,3 +178,79 @@ def test_the_devices_r_form_gives_the_oracles_bytes(n):
     rc, rs = _r_form(W, X, part=32, parts=4)
     np.testing.assert_array_equal(rs, os_)
     np.testing.assert_array_equal(rc, oc)
+
+
+# --- direct pins of the FP32 forms the GPTQ oracle uses ----------------------
+
+_GRID = [0, 1, 2, 3, 4, 6, 8, 12]   # E2M1 magnitudes times 2 (exact integers)
+
+
+def _nearest_e2m1(a, vS):
+    """Index of the E2M1 magnitude nearest to a / vS, exact ties to the even
+    index, by exact rational arithmetic (the E2M1 definition, brute force)."""
+    from fractions import Fraction
+    x = Fraction(a) / Fraction(vS) * 2
+    best = min(range(8), key=lambda k: (abs(x - _GRID[k]), k & 1))
+    return best
+
+
+def test_e2m1_quantize_list_is_the_nearest_grid_value():
+    """Nibbles of FP32 values at their own exact scales: the nearest E2M1 value
+    by exact arithmetic, ties to the even code, saturating at 6, sign in bit 3
+    except for a zero magnitude -- on random values and on exact midpoints."""
+    rng = np.random.default_rng(11)
+    v = np.array([oracle.e4m3_value(c) for c in rng.integers(1, 127, 600)])
+    S = np.float32(2.0 ** -7)
+    vS = v * np.float64(S)                                   # exact
+    w = (rng.standard_normal(600) * 4 * vS).astype(np.float32)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.5])
+    k = rng.integers(0, 8, 400)
+    vm = vS[:400]
+    wm = (mids[k] * vm * rng.choice([-1.0, 1.0], 400)).astype(np.float32)
+    assert np.all(wm.astype(np.float64) == mids[k] * vm * np.sign(wm))   # exact midpoints
+    W = np.concatenate([w, wm, np.float32([0.0, -0.0, 1e-30, -1e-30])])
+    VS = np.concatenate([vS, vm, vS[:4]])
+    got = oracle.e2m1_quantize_list(W, VS)
+    for x, s, g in zip(W, VS, got):
+        m = _nearest_e2m1(abs(float(x)), float(s))
+        want = m | (8 if (x < 0 and m != 0) else 0)
+        assert g == want, (float(x), float(s), int(g), want)
+
+
+def test_fp32_base_code_is_the_e4m3_rounding_of_two_fp32_divisions():
+    """A one-candidate window returns the base code: E4M3 round-to-nearest-even
+    (torch's float8_e4m3fn cast, saturated at 448) of fl32(fl32(a/6)/S), a the
+    group's largest magnitude, clamped to [1, 126]; 0 for a zero group."""
+    import torch
+    rng = np.random.default_rng(12)
+    w = (rng.standard_normal((500, 16)) * np.exp(rng.normal(0, 3, (500, 1)))).astype(np.float32)
+    w[7] = 0.0
+    S = np.float32(0.01)
+    _, scales, _, _ = oracle.sweep_group_f32_list(w, None, float(S), 0, 0)
+    a = np.abs(w).max(axis=1).astype(np.float32)
+    t = (a / np.float32(6.0)).astype(np.float32) / S
+    t = np.minimum(t.astype(np.float32), np.float32(448.0))
+    code = torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy().astype(int)
+    want = np.where(a > 0, np.clip(code, 1, 126), 0)
+    np.testing.assert_array_equal(scales.astype(int), want)
+
+
+def test_fp32_group_loss_is_the_exact_weighted_error():
+    """orc_group_loss_f32 against the weighted squared error computed in exact
+    rational arithmetic from the brute-force nearest grid values (FP64 sums of
+    exact terms: agreement to 1e-13)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(13)
+    S = np.float32(3e-4)
+    for _ in range(40):
+        w = (rng.standard_normal(16) * 0.02).astype(np.float32)
+        h = rng.lognormal(0.0, 1.0, 16).astype(np.float32)
+        code = int(rng.integers(40, 110))
+        vS = oracle.e4m3_value(code) * float(S)
+        exact = Fraction(0)
+        for x, hx in zip(w, h):
+            k = _nearest_e2m1(abs(float(x)), vS)
+            e = Fraction(abs(float(x))) - Fraction(_GRID[k], 2) * Fraction(vS)
+            exact += Fraction(float(hx)) * e * e
+        got = oracle.group_loss_f32(w, h, float(S), code)
+        assert abs(got - float(exact)) <= 1e-13 * float(exact), (got, float(exact))
