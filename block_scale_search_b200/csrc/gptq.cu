@@ -188,6 +188,101 @@ __device__ int local_sweep_f32(const float* w, const float* h16, const ScaleCons
   return clamp_code(b + lo + bi);
 }
 
+// local_sweep_f32 shared by the two lanes of a pair (lanes 2k and 2k + 1 of a
+// warp, both holding the same 16 weights w): lane `half` scores candidates
+// half, half + 2, ..., and the pair's smallest and second-smallest keys are
+// combined by shuffles, so both lanes take the same decision as one lane
+// scoring them all.  pm holds whole pairs and every lane in it must call this.
+template <bool kWeighted, int kK>
+__device__ int local_sweep_f32_pair(const float* w, const float* h16, const ScaleConsts& sc,
+                                    const CandEntry* tab, int lo, int K, int half, unsigned pm) {
+  float a = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(w[j]));
+  f32x2_t h2[8];
+  float hs = 1.0f, hsum = 16.0f;
+  if constexpr (kWeighted) {
+    weights_from(h16, h2, hs, hsum);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h2[i] = f2_pack(1.0f, 1.0f);
+  }
+  f32x2_t y2[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f32x2_t a2 = f2_pack(w[2 * i], w[2 * i + 1]);
+    if (sc.tiny_s) a2 = f2_mul(a2, f2_pack(sc.p, sc.p));
+    y2[i] = f2_mul(a2, f2_pack(sc.inv_sp, sc.inv_sp));
+  }
+  const float S = sc.S;
+  const int b = clamp_code(e4m3_code_rne_sat(__fdiv_rn(__fdiv_rn(a, 6.0f), S)));
+  const CandEntry* ce = tab + (b + lo + kTabOffset);
+  uint32_t kbest = 0xFFFFFFFFu, ksec = 0xFFFFFFFFu;
+  auto cand = [&](int i) {
+    const float Li = fast_candidate_loss<kWeighted>(y2, h2, ce[i]);
+    const uint32_t key = (__float_as_uint(Li) & ~0xFu) | static_cast<uint32_t>(i);
+    ksec = min(ksec, max(kbest, key));
+    kbest = min(kbest, key);
+  };
+  if constexpr (kK > 0) {
+#pragma unroll
+    for (int m = 0; m < kK; m += 2) cand(m + half);
+  } else {
+    for (int i = half; i < K; i += 2) cand(i);
+  }
+  {  // the pair's two smallest keys
+    const uint32_t ob = __shfl_xor_sync(pm, kbest, 1), os = __shfl_xor_sync(pm, ksec, 1);
+    ksec = min(min(ksec, os), max(kbest, ob));
+    kbest = min(kbest, ob);
+  }
+  if (!(a > 0.0f)) return 0;
+  int bi = static_cast<int>(kbest & 0xFu);
+  const float best = __uint_as_float(kbest & ~0xFu) * (1.0f + 0x1p-18f);
+  const float second = __uint_as_float(ksec & ~0xFu);
+  constexpr float c1 = 0x1p-19f, c2 = 0x1p-15f;
+  constexpr float k2 = 1.0f / (2.0f * (1.0f - c2));
+  auto threshold = [&](float A) {
+    const float ca = c1 * sqrt_approx(A);
+    const float sr = (ca + sqrt_approx(fmaf(ca, ca, 4.0f * (1.0f - c2) * best))) * k2;
+    return sr * sr * (1.0f + 0x1p-16f);
+  };
+  const float ymax = (sc.tiny_s ? a * sc.p : a) * sc.inv_sp;
+  float T = threshold(hsum * ymax * ymax);
+  bool flagged = second <= T;
+  if (flagged) {
+    f32x2_t A2 = f2_pack(0.0f, 0.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) A2 = f2_fma(kWeighted ? f2_mul(h2[i], y2[i]) : y2[i], y2[i], A2);
+    float A0, A1;
+    f2_unpack(A2, A0, A1);
+    T = threshold(A0 + A1);
+    flagged = second <= T;
+  }
+  if (flagged) {  // rare: both lanes run the definition's own arithmetic on every candidate
+    double bestd = __longlong_as_double(0x7FF0000000000000ll);
+    int bid = bi;
+    for (int i = 0; i < K; ++i) {
+      if (fast_candidate_loss<kWeighted>(y2, h2, ce[i]) > T) continue;
+      const CandEntry t = ce[i];
+      const float ivl = t.iv * (1.0f - 0x1p-20f);
+      const double vS = __dmul_rn(static_cast<double>(t.v), static_cast<double>(S));
+      double Ld = 0.0;
+      for (int j = 0; j < 16; ++j) {
+        const float aj = fabsf(w[j]);
+        const float yj = (sc.tiny_s ? aj * sc.p : aj) * sc.inv_sp;
+        const uint32_t k = exact_e2m1_one(yj * ivl, aj, t.v, S);
+        const double q = static_cast<double>(e2m1_nibble_value(k));
+        const double d = fma(-q, vS, static_cast<double>(aj));  // exact
+        const double hj = kWeighted ? static_cast<double>(h16[j]) : 1.0;
+        Ld = __dadd_rn(Ld, __dmul_rn(hj, __dmul_rn(d, d)));
+      }
+      if (Ld < bestd) { bestd = Ld; bid = i; }
+    }
+    bi = bid;
+  }
+  return clamp_code(b + lo + bi);
+}
+
 // One FP32 weight quantized at E4M3 code `code` (0: the group is all zero):
 // its nibble (sign << 3 | E2M1 index, +0 for a zero magnitude) and its
 // reconstruction sign * g * v * S (one rounding).  The E2M1 decision is exact
@@ -383,27 +478,33 @@ gptq_rsplit_kernel(const float* __restrict__ R, int64_t in, int64_t r0, int64_t 
   }
 }
 
-// One part [j0, j0 + nb) of a lazy batch of GPTQ's columns in the R form, one
-// thread per row, kT rows per CTA.  Per 16-column group at g0 the thread
+// One part [j0, j0 + nb) of a lazy batch of GPTQ's columns in the R form, two
+// threads (a pair of adjacent lanes) per row, kR rows per CTA.  Per 16-column
+// group at g0 the pair
 //   * sums v = P[r, grp] + D[r, j0:g0] R[j0:g0, grp] (P holds the earlier
-//     parts' sums, D the part's earlier groups, in shared memory);
-//   * forms the current weights w = W[r, grp] + v U_grp;
-//   * runs the local call on w (the group's E4M3 scale code);
+//     parts' sums, D the part's earlier groups, in shared memory), each lane
+//     8 of the 16 columns, and swaps halves;
+//   * forms the current weights w = W[r, grp] + v U_grp (both lanes);
+//   * runs the local call on w, each lane half of the candidates
+//     (local_sweep_f32_pair);
 //   * quantizes each column at its turn -- exact E2M1 decision, D = W - q,
 //     err = (w - q) R_jj -- and updates the group's later columns by
-//     w_k -= err U_jk;
-// and writes the part's D, scaled by s_D = gs[0], as [D_hi | D_hi | D_lo] in
-// FP16 (kCat columns from Dcat, row stride ldd) for the split update GEMMs.
-// Dynamic shared memory: R's blocks above the diagonal blocks (kRsFloats), the
-// groups' U blocks (8 x 256), the rows' D (kT x kDs).
-template <bool kWeighted, int kK, int kT>
-__global__ void __launch_bounds__(kT)
+//     w_k -= err U_jk (both lanes, the same arithmetic);
+// and each lane writes its 8 columns of D, scaled by s_D = gs[0], as
+// [D_hi | D_hi | D_lo] in FP16 (kCat columns from Dcat, row stride ldd) for
+// the split update GEMMs.  Every sum is taken in the order one lane alone
+// would take it, so the bytes do not depend on the pairing.  Dynamic shared
+// memory: R's blocks above the diagonal blocks (kRsFloats), the groups' U
+// blocks (8 x 256), the rows' D (kR x kDs).
+template <bool kWeighted, int kK, int kR>
+__global__ void __launch_bounds__(2 * kR)
 gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* __restrict__ dead,
                    int64_t out, int64_t in, int64_t j0, int nb, const float* __restrict__ P,
                    const float* __restrict__ R, const float* __restrict__ Ud,
                    const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                    const float* __restrict__ gs, __half* __restrict__ Dcat, int64_t ldd) {
+  constexpr int kT = 2 * kR;
   extern __shared__ __align__(16) float gsm[];
   __shared__ CandEntry tab[kTabSize];
   __shared__ float hb[kGB];
@@ -434,24 +535,26 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
   }
   cp_async_wait<0>();
   __syncthreads();
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * kT + t;
-  if (r >= out) return;  // after the kernel's only barrier
+  const int lr = t >> 1, half = t & 1;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * kR + lr;
+  if (r >= out) return;  // both lanes of a pair, after the kernel's only barrier
+  const unsigned pm = __activemask();  // whole pairs
   const ScaleConsts sc = scale_consts(*Sp);
   const int K = hi - lo + 1;
-  float* ds = Ds + t * kDs;
-  const float* prow = P + r * in + j0;
+  float* ds = Ds + lr * kDs;
+  const float* prow = P + r * in + j0 + 8 * half;
   const uint16_t* wrow = W + r * ldw + j0;
-  __half* dcat = Dcat + r * ldd;
+  __half* dcat = Dcat + r * ldd + 8 * half;
   const float sd = gs[0];
   const int64_t G = in / 16;
-  // A group's P (16 floats) and W (16 bf16, as 8 pairs, two 16-byte loads: W
-  // is 16-byte aligned and ldw % 8 == 0) are loaded one group ahead, so their
-  // latency hides behind the previous group's column loop.
-  float4 pn[4];
+  // A group's P (this lane's 8 floats) and W (16 bf16, as 8 pairs, two 16-byte
+  // loads: W is 16-byte aligned and ldw % 8 == 0) are loaded one group ahead,
+  // so their latency hides behind the previous group's column loop.
+  float4 pn[2];
   uint32_t wn[8];
   auto load_group = [&](int g) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) pn[q] = reinterpret_cast<const float4*>(prow + 16 * g)[q];
+    for (int q = 0; q < 2; ++q) pn[q] = reinterpret_cast<const float4*>(prow + 16 * g)[q];
     const uint4 a = reinterpret_cast<const uint4*>(wrow + 16 * g)[0];
     const uint4 b = reinterpret_cast<const uint4*>(wrow + 16 * g)[1];
     wn[0] = a.x; wn[1] = a.y; wn[2] = a.z; wn[3] = a.w;
@@ -459,16 +562,16 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
   };
   load_group(0);
   for (int g = 0; g < ng; ++g) {
-    f32x2_t v2[8];
+    f32x2_t v2[4];  // this lane's 8 columns, 8 * half .. 8 * half + 7
     uint32_t wc[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
       v2[2 * q] = f2_pack(pn[q].x, pn[q].y);
       v2[2 * q + 1] = f2_pack(pn[q].z, pn[q].w);
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) wc[i] = wn[i];
-    const float* rs = Rs + 128 * g * (g - 1);
+    const float* rs = Rs + 128 * g * (g - 1) + 8 * half;
     for (int i = 0; i < 16 * g; i += 4) {
       const float4 d4 = *reinterpret_cast<const float4*>(ds + i);
       const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
@@ -477,7 +580,7 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
         const f32x2_t d2 = f2_pack(dv[u], dv[u]);
         const float4* rr = reinterpret_cast<const float4*>(rs + (i + u) * 16);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           const float4 x = rr[q];
           v2[2 * q] = f2_fma(d2, f2_pack(x.x, x.y), v2[2 * q]);
           v2[2 * q + 1] = f2_fma(d2, f2_pack(x.z, x.w), v2[2 * q + 1]);
@@ -485,8 +588,17 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
       }
     }
     float v[16], w[16];
+    {
+      float mine[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) f2_unpack(v2[i], v[2 * i], v[2 * i + 1]);
+      for (int i = 0; i < 4; ++i) f2_unpack(v2[i], mine[2 * i], mine[2 * i + 1]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float other = __shfl_xor_sync(pm, mine[k], 1);
+        v[k] = half ? other : mine[k];
+        v[8 + k] = half ? mine[k] : other;
+      }
+    }
     // the group's original weights (dead columns zero), kept as bf16 pairs
     auto w0 = [&](int j) {
       const float wj = (j & 1) ? bf16_hi(wc[j >> 1]) : bf16_lo(wc[j >> 1]);
@@ -514,14 +626,18 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
       for (int k = i; k < 16; ++k) w[k] = fmaf(v[i], u[k], w[k]);
     }
     // w waits in the row's D slots of this group (written only after the
-    // column loop) while the sweep runs, which frees 16 registers there
+    // column loop) while the sweep runs, which frees 16 registers there;
+    // each lane parks its half, both read all 16
     float* wpark = ds + 16 * g;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      reinterpret_cast<float4*>(wpark)[q] =
-          make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-    const int code = local_sweep_f32<kWeighted, kK>(wpark, kWeighted ? hb + 16 * g : nullptr,
-                                                    sc, tab, lo, K);
+    for (int q = 0; q < 2; ++q) {
+      const float4 lo4 = make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      const float4 hi4 = make_float4(w[8 + 4 * q], w[9 + 4 * q], w[10 + 4 * q], w[11 + 4 * q]);
+      reinterpret_cast<float4*>(wpark + 8 * half)[q] = half ? hi4 : lo4;
+    }
+    __syncwarp(pm);
+    const int code = local_sweep_f32_pair<kWeighted, kK>(
+        wpark, kWeighted ? hb + 16 * g : nullptr, sc, tab, lo, K, half, pm);
     if (g + 1 < ng) load_group(g + 1);  // in flight during the column loop
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -544,32 +660,36 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
 #pragma unroll
       for (int k = j + 1; k < 16; ++k) w[k] = fmaf(-err, u[k], w[k]);
     }
+    __syncwarp(pm);  // both lanes have read the parked w before D overwrites it
+    float dh[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      *reinterpret_cast<float4*>(ds + 16 * g + 4 * q) =
-          make_float4(dl[4 * q], dl[4 * q + 1], dl[4 * q + 2], dl[4 * q + 3]);
-    uint32_t hw[8], lw[8];  // FP16 pairs, element 2i in the low half
+    for (int k = 0; k < 8; ++k) dh[k] = half ? dl[8 + k] : dl[k];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int q = 0; q < 2; ++q)
+      *reinterpret_cast<float4*>(ds + 16 * g + 8 * half + 4 * q) =
+          make_float4(dh[4 * q], dh[4 * q + 1], dh[4 * q + 2], dh[4 * q + 3]);
+    uint32_t hw[4], lw[4];  // FP16 pairs, element 2i in the low half
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
       __half h0, l0, h1, l1;
-      f16_split(dl[2 * i], sd, h0, l0);
-      f16_split(dl[2 * i + 1], sd, h1, l1);
+      f16_split(dh[2 * i], sd, h0, l0);
+      f16_split(dh[2 * i + 1], sd, h1, l1);
       hw[i] = static_cast<uint32_t>(__half_as_ushort(h0)) |
               (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
       lw[i] = static_cast<uint32_t>(__half_as_ushort(l0)) |
               (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
     }
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint4 hv = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
-      const uint4 lv = make_uint4(lw[4 * q], lw[4 * q + 1], lw[4 * q + 2], lw[4 * q + 3]);
-      reinterpret_cast<uint4*>(dcat + 16 * g)[q] = hv;
-      reinterpret_cast<uint4*>(dcat + kGB + 16 * g)[q] = hv;
-      reinterpret_cast<uint4*>(dcat + 2 * kGB + 16 * g)[q] = lv;
+    const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    const uint4 lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    *reinterpret_cast<uint4*>(dcat + 16 * g) = hv;
+    *reinterpret_cast<uint4*>(dcat + kGB + 16 * g) = hv;
+    *reinterpret_cast<uint4*>(dcat + 2 * kGB + 16 * g) = lv;
+    if (half == 0) {
+      const int64_t gg = j0 / 16 + g;
+      *reinterpret_cast<uint2*>(codes + r * (G * 8) + gg * 8) = make_uint2(packed[0], packed[1]);
+      scales[r * G + gg] = static_cast<uint8_t>(code);
     }
-    const int64_t gg = j0 / 16 + g;
-    *reinterpret_cast<uint2*>(codes + r * (G * 8) + gg * 8) = make_uint2(packed[0], packed[1]);
-    scales[r * G + gg] = static_cast<uint8_t>(code);
+    __syncwarp(pm);  // the next group reads the partner's D
   }
 }
 
@@ -695,27 +815,28 @@ bool gptq_layout(int64_t out, int64_t in, int64_t tokens, int sms, Handles* hd, 
   return true;
 }
 
-// Rows per CTA of the batch kernel: 128 (two CTAs per SM) when that still
-// fills every SM, else 32.
+// Rows per CTA of the batch kernel (two threads each): 208 -- one CTA per SM,
+// 416 threads, so that a 28672-row matrix fits in one wave of 138 CTAs --
+// when that keeps at least two thirds of the SMs busy, else 32.
 constexpr size_t rblock_smem(int rows) {
   return (static_cast<size_t>(kRsFloats) + (kGB / 16) * 256 + static_cast<size_t>(rows) * kDs) *
          sizeof(float);
 }
 
-template <bool kW, int kKK, int kT>
+template <bool kW, int kKK, int kR>
 cudaError_t launch_rblock_t(const uint16_t* W, int64_t ldw, const uint8_t* dead, int64_t out,
                             int64_t in, int64_t j0, int nb, const float* P, const float* R,
                             const float* Ud, const float* h, const float* S, int lo, int hi,
-                            uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat, int64_t ldd,
-                            cudaStream_t s) {
-  constexpr size_t smem = rblock_smem(kT);
+                            uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat,
+                            int64_t ldd, cudaStream_t s) {
+  constexpr size_t smem = rblock_smem(kR);
   static const cudaError_t attr = cudaFuncSetAttribute(
-      reinterpret_cast<const void*>(&gptq_rblock_kernel<kW, kKK, kT>),
+      reinterpret_cast<const void*>(&gptq_rblock_kernel<kW, kKK, kR>),
       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (attr != cudaSuccess) return attr;
-  const unsigned blocks = static_cast<unsigned>((out + kT - 1) / kT);
-  gptq_rblock_kernel<kW, kKK, kT><<<blocks, kT, smem, s>>>(W, ldw, dead, out, in, j0, nb, P, R, Ud,
-                                                           h, S, lo, hi, codes, scales, gs, Dcat, ldd);
+  const unsigned blocks = static_cast<unsigned>((out + kR - 1) / kR);
+  gptq_rblock_kernel<kW, kKK, kR><<<blocks, 2 * kR, smem, s>>>(
+      W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, Dcat, ldd);
   return cudaGetLastError();
 }
 
@@ -723,10 +844,10 @@ template <bool kW, int kKK>
 cudaError_t launch_rblock(const uint16_t* W, int64_t ldw, const uint8_t* dead, int64_t out,
                           int64_t in, int64_t j0, int nb, const float* P, const float* R,
                           const float* Ud, const float* h, const float* S, int lo, int hi,
-                          uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat, int64_t ldd, int sms,
-                          cudaStream_t s) {
-  if ((out + 127) / 128 >= static_cast<int64_t>(sms))
-    return launch_rblock_t<kW, kKK, 128>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi,
+                          uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat,
+                          int64_t ldd, int sms, cudaStream_t s) {
+  if (3 * ((out + 207) / 208) >= 2 * static_cast<int64_t>(sms))
+    return launch_rblock_t<kW, kKK, 208>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi,
                                          codes, scales, gs, Dcat, ldd, s);
   return launch_rblock_t<kW, kKK, 32>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi, codes,
                                       scales, gs, Dcat, ldd, s);
