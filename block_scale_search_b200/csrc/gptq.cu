@@ -35,7 +35,7 @@
 //     and err_j = (w_j - q_j) R_jj.  gptq_udiag_kernel inverts the diagonal
 //     blocks (FP64);
 //   * GPTQ's lazy batches, 512 columns each, in four parts of 128:
-//     gptq_rblock_kernel runs the columns of one part, one thread per row --
+//     gptq_rblock_kernel runs the columns of one part, two threads per row --
 //     each group's sums from the earlier groups of the part, its current
 //     weights, the local call, the exact quantization and the in-group
 //     updates -- and writes the part's D.  After each part a small GEMM adds
