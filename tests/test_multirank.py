@@ -55,3 +55,14 @@ def test_two_gloo_ranks_weak_scaling():
     assert set(r0[0]).isdisjoint(r1[0])        # but independent layers (seeds)
     assert r0[2] == r1[2] == 1.0               # step time = max over ranks
     assert r0[3] != r1[3]                      # different data, different scales
+
+
+@pytest.mark.parametrize("out,n", [(28672, 8192), (100, 400), (64, 48), (64, 144), (7, 4112)])
+def test_gptq_update_flops_count_every_cross_part_column_pair(out, n):
+    """The GPTQ bench line's flop count: the update GEMMs make one multiply-add
+    per row for every column pair i < k in different 128-column parts (pairs
+    inside a part are the batch kernel's), three split products each."""
+    import bench
+    sizes = [min(128, n - i) for i in range(0, n, 128)]
+    pairs = (n * n - sum(s * s for s in sizes)) // 2
+    assert bench.gptq_update_flops(out, n) == 6.0 * out * pairs
