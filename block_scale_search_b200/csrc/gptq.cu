@@ -337,7 +337,7 @@ sweep_f32_kernel(const float* __restrict__ W, int64_t out, int64_t G, int64_t ld
 }
 
 // Dead columns, damping: one CTA.  H is symmetric (row- or column-major alike).
-// Also the FP16 scales of the split update GEMMs, gs = {s_D, s_R, alpha, 1}:
+// Also the FP16 scales of the split update GEMMs, gs = {s_D, s_R, alpha, 1, 0}:
 // powers of two with |D| s_D <= 2^14 and |R| s_R <= 2^14, where |D| = |W - q|
 // <= amax + 6 * 448 * S (amax ~ S * 6 q_max) and every entry of row i of R is
 // at most sqrt(H_ii) (H = R R^T); alpha = 1 / (s_D s_R).
@@ -386,6 +386,7 @@ gptq_prep_kernel(float* __restrict__ H, int64_t in, float damp, uint8_t* __restr
     gs[1] = ldexpf(1.0f, kr);
     gs[2] = ldexpf(1.0f, -kd - kr);
     gs[3] = 1.0f;
+    gs[4] = 0.0f;
   }
 }
 
@@ -493,7 +494,8 @@ gptq_rsplit_kernel(const float* __restrict__ R, int64_t in, int64_t r0, int64_t 
 // and each lane writes its 8 columns of D, scaled by s_D = gs[0], as
 // [D_hi | D_hi | D_lo] in FP16 (kCat columns from Dcat, row stride ldd) for
 // the split update GEMMs.  Every sum is taken in the order one lane alone
-// would take it, so the bytes do not depend on the pairing.  Dynamic shared
+// would take it, so the bytes do not depend on the pairing.  p_zero: the
+// part's sums are zero (the first part of the first batch) and P is not read.  Dynamic shared
 // memory: R's blocks above the diagonal blocks (kRsFloats), the groups' U
 // blocks (8 x 256), the rows' D (kR x kDs).
 template <bool kWeighted, int kK, int kR>
@@ -503,7 +505,8 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
                    const float* __restrict__ R, const float* __restrict__ Ud,
                    const float* __restrict__ h, const float* __restrict__ Sp, int lo, int hi,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                   const float* __restrict__ gs, __half* __restrict__ Dcat, int64_t ldd) {
+                   const float* __restrict__ gs, __half* __restrict__ Dcat, int64_t ldd,
+                   bool p_zero) {
   constexpr int kT = 2 * kR;
   extern __shared__ __align__(16) float gsm[];
   __shared__ CandEntry tab[kTabSize];
@@ -554,7 +557,9 @@ gptq_rblock_kernel(const uint16_t* __restrict__ W, int64_t ldw, const uint8_t* _
   uint32_t wn[8];
   auto load_group = [&](int g) {
 #pragma unroll
-    for (int q = 0; q < 2; ++q) pn[q] = reinterpret_cast<const float4*>(prow + 16 * g)[q];
+    for (int q = 0; q < 2; ++q)
+      pn[q] = p_zero ? make_float4(0.0f, 0.0f, 0.0f, 0.0f)
+                     : reinterpret_cast<const float4*>(prow + 16 * g)[q];
     const uint4 a = reinterpret_cast<const uint4*>(wrow + 16 * g)[0];
     const uint4 b = reinterpret_cast<const uint4*>(wrow + 16 * g)[1];
     wn[0] = a.x; wn[1] = a.y; wn[2] = a.z; wn[3] = a.w;
@@ -805,7 +810,7 @@ bool gptq_layout(int64_t out, int64_t in, int64_t tokens, int sms, Handles* hd, 
   L->P = take(o * n * sizeof(float));
   L->Dcat = take(o * kCat * kSub * sizeof(__half));
   L->Rcat = take(static_cast<size_t>(kCat) * kSub * n * sizeof(__half));
-  L->gs = take(4 * sizeof(float));
+  L->gs = take(5 * sizeof(float));
   L->Ud = take(n * 16 * sizeof(float));
   L->dead = take(n);
   L->info = take(sizeof(int));
@@ -828,7 +833,7 @@ cudaError_t launch_rblock_t(const uint16_t* W, int64_t ldw, const uint8_t* dead,
                             int64_t in, int64_t j0, int nb, const float* P, const float* R,
                             const float* Ud, const float* h, const float* S, int lo, int hi,
                             uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat,
-                            int64_t ldd, cudaStream_t s) {
+                            int64_t ldd, bool p_zero, cudaStream_t s) {
   constexpr size_t smem = rblock_smem(kR);
   static const cudaError_t attr = cudaFuncSetAttribute(
       reinterpret_cast<const void*>(&gptq_rblock_kernel<kW, kKK, kR>),
@@ -836,7 +841,7 @@ cudaError_t launch_rblock_t(const uint16_t* W, int64_t ldw, const uint8_t* dead,
   if (attr != cudaSuccess) return attr;
   const unsigned blocks = static_cast<unsigned>((out + kR - 1) / kR);
   gptq_rblock_kernel<kW, kKK, kR><<<blocks, 2 * kR, smem, s>>>(
-      W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, Dcat, ldd);
+      W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, Dcat, ldd, p_zero);
   return cudaGetLastError();
 }
 
@@ -845,12 +850,12 @@ cudaError_t launch_rblock(const uint16_t* W, int64_t ldw, const uint8_t* dead, i
                           int64_t in, int64_t j0, int nb, const float* P, const float* R,
                           const float* Ud, const float* h, const float* S, int lo, int hi,
                           uint8_t* codes, uint8_t* scales, const float* gs, __half* Dcat,
-                          int64_t ldd, int sms, cudaStream_t s) {
+                          int64_t ldd, bool p_zero, int sms, cudaStream_t s) {
   if (3 * ((out + 207) / 208) >= 2 * static_cast<int64_t>(sms))
     return launch_rblock_t<kW, kKK, 208>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi,
-                                         codes, scales, gs, Dcat, ldd, s);
+                                         codes, scales, gs, Dcat, ldd, p_zero, s);
   return launch_rblock_t<kW, kKK, 32>(W, ldw, dead, out, in, j0, nb, P, R, Ud, h, S, lo, hi, codes,
-                                      scales, gs, Dcat, ldd, s);
+                                      scales, gs, Dcat, ldd, p_zero, s);
 }
 
 }  // namespace
@@ -985,19 +990,16 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
   const float* R = H;  // row-major R[j][k] for k >= j
   gptq_udiag_kernel<<<static_cast<unsigned>((in + 127) / 128), 128, 0, stream>>>(R, in, Ud);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(P, 0, static_cast<size_t>(out) * in * sizeof(float), stream)) !=
-      cudaSuccess)
-    return e;
   timer_end(tm, stream);
   const int K = hi - lo + 1;
   const uint8_t* dd = dead;
   const int64_t ldd = static_cast<int64_t>(kCat) * kSub;
   auto block_t = [&](int64_t c0, int nb, __half* dcat) {
     if (weighted)
-      return K == 16 ? launch_rblock<true, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream)
-                     : launch_rblock<true, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream);
-    return K == 16 ? launch_rblock<false, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream)
-                   : launch_rblock<false, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, gs, dcat, ldd, sms, stream);
+      return K == 16 ? launch_rblock<true, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, dcat, ldd, c0 == 0, sms, stream)
+                     : launch_rblock<true, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, h, S, lo, hi, codes, scales, gs, dcat, ldd, c0 == 0, sms, stream);
+    return K == 16 ? launch_rblock<false, 16>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, gs, dcat, ldd, c0 == 0, sms, stream)
+                   : launch_rblock<false, 0>(W, ldw, dd, out, in, c0, nb, P, R, Ud, nullptr, S, lo, hi, codes, scales, gs, dcat, ldd, c0 == 0, sms, stream);
   };
   auto block = [&](int64_t c0, int nb, __half* dcat) {
     const int t = timer_begin(NVFP4_GPTQ_PHASE_BATCH, stream);
@@ -1017,13 +1019,16 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
   };
   // P[:, c0 : c0 + m] += Dcat[:, :k] Rcat[:k, :m], all row-major: in
   // column-major terms P^T (m x out) += Rcat^T (m x k) Dcat^T (k x out)
-  // alpha = 1 / (s_D s_R) and beta = 1 are device scalars (gs[2], gs[3])
-  auto update = [&](int64_t c0, int64_t m, int k, const __half* rcat, int64_t ldr) {
+  // alpha = 1 / (s_D s_R) and beta are device scalars (gs[2]; gs[3] = 1, or
+  // gs[4] = 0 where the GEMM writes its columns of P first: every update of
+  // the first batch -- P is never cleared, and the first part reads none of it)
+  auto update = [&](int64_t c0, int64_t m, int k, const __half* rcat, int64_t ldr, bool first) {
     const int t = timer_begin(NVFP4_GPTQ_PHASE_UPDATE, stream);
     const bool ok = blas_ok(cublasGemmEx(hd->blas, CUBLAS_OP_N, CUBLAS_OP_N, static_cast<int>(m),
                                 static_cast<int>(out), k, gs + 2, rcat, CUDA_R_16F,
                                 static_cast<int>(ldr), Dcat, CUDA_R_16F, static_cast<int>(ldd),
-                                gs + 3, P + c0, CUDA_R_32F, n, CUBLAS_COMPUTE_32F,
+                                first ? gs + 4 : gs + 3, P + c0, CUDA_R_32F, n,
+                                CUBLAS_COMPUTE_32F,
                                 CUBLAS_GEMM_DEFAULT));
     timer_end(t, stream);
     return ok;
@@ -1046,11 +1051,12 @@ cudaError_t launch_gptq(const uint16_t* W, int64_t out, int64_t in, int64_t ldw,
       if (sb + 1 < nsub) {  // the next part takes the batch's parts so far
         const int64_t c1 = c0 + nb;  // nb == kGB: only a batch's last part can be narrower
         const int64_t m = std::min<int64_t>(kGB, jend - c1);
-        if (!update(c1, m, kCat * (sb + 1), Rcat + (c1 - col0), in)) return cudaErrorUnknown;
+        if (!update(c1, m, kCat * (sb + 1), Rcat + (c1 - col0), in, j0 == 0))
+          return cudaErrorUnknown;
       }
     }
     if (jend < in &&  // every later column takes the whole batch (all parts full)
-        !update(jend, in - jend, kCat * nsub, Rcat + (jend - col0), in))
+        !update(jend, in - jend, kCat * nsub, Rcat + (jend - col0), in, j0 == 0))
       return cudaErrorUnknown;
   }
   return cudaSuccess;
